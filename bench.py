@@ -1,0 +1,435 @@
+"""Benchmark of the fused 4-bit dequantize + skinny GEMM on B200.
+
+One step = one decode pass through the four 4-bit linear layers of a
+70B-class transformer block at M = 1 (K8192/N10240, K8192/N28672,
+K28672/N8192, K8192/N8192; blocksize 64, bf16 activations, normal-quantile
+code table).  Metric: effective HBM bandwidth
+    (M*K*2 + N*K/2 + 4*N*K/bs + M*N*2 bytes) / time
+summed over the step, and its fraction of the measured B200 peak.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                  [--workload decode70b|square4096|msweep|variants|aspect]
+
+For N > 1 it runs under torchrun, one process per GPU, each GPU running the
+same step on its own replica of the weights (the path has no exchange step:
+"replicas only", weak scaling); the time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from bit_weight_dequant_b200 import binding as q4  # noqa: E402
+from bit_weight_dequant_b200 import inputs  # noqa: E402
+
+METRIC = "fused 4-bit dequant-GEMM effective HBM GB/s and % of B200 peak, per M=1..16"
+FALLBACK_HBM_GBS = 6650.0
+L2_BYTES = 126 * 1024 * 1024
+CHUNK_STEPS = 100          # steps per captured CUDA graph
+
+
+def log(*a):
+    print(*a, file=sys.stderr, flush=True)
+
+
+def hbm_peak():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            v = float(json.load(f)["hbm_gbs"])
+        return v, "measured (MEASURED_PEAKS.json hbm_gbs: STREAM-style copy)"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback 6.65 TB/s (no MEASURED_PEAKS.json)"
+
+
+def gemm_kernel_hash() -> str:
+    h = hashlib.sha256()
+    for f in ("q4_gemm.cu", "q4_device.cuh", "q4_plan.cuh"):
+        with open(os.path.join(ROOT, "bit_weight_dequant_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(workload: str):
+    """DRAM bytes per launch of the GEMM kernel from the committed ncu
+    summary, if it was taken on the current kernel source; else None."""
+    p = os.path.join(ROOT, "profiles", "gemm_dram_traffic.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        if d.get("kernel_hash") != gemm_kernel_hash():
+            return None
+        return d.get("bytes_per_launch", {}).get(workload)
+    except Exception:
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu = gpu_id
+        self.proc = None
+        self.path = os.path.join("/tmp", f"q4_clocks_{os.getpid()}.csv")
+
+    def start(self):
+        try:
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=self.fh, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        self.proc.wait()
+        self.fh.close()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    smax.append(float(parts[2]))
+                except ValueError:
+                    continue
+                for nm, v in zip(names, parts[5:9]):
+                    if v.lower().startswith("active"):
+                        reasons.add(nm)
+        os.unlink(self.path)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return world, rank, local
+
+
+def max_over_ranks(v: float, world: int, device) -> float:
+    if world == 1:
+        return v
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ---------------------------------------------------------------------------
+# Our arm
+# ---------------------------------------------------------------------------
+
+class Layer:
+    """One 4-bit linear layer resident on the device, with its C-ABI call
+    arguments prepared once (the timed loop only makes the call)."""
+
+    def __init__(self, case: inputs.Case, seed: int, device):
+        self.case = case
+        dt = torch.bfloat16 if case.act == "bf16" else torch.float16
+        code = inputs.CODE_TABLES[case.table]()
+        self.code = torch.from_numpy(code).to(device)
+        W = inputs.weights_device(case.N, case.K, seed, device, case.outliers)
+        self.packed, self.absmax = q4.q4_quantize_blockwise(W.reshape(-1), case.blocksize, self.code)
+        del W
+        self.A_host = inputs.activations(case.M, case.K, dt, seed).pin_memory()
+        self.A = self.A_host.to(device)
+        self.out = torch.empty((case.M, case.N), dtype=dt, device=device)
+        self.out_host = torch.empty((case.M, case.N), dtype=dt).pin_memory()
+        self.ws_bytes = q4.q4_gemm_workspace_size(case.M, case.N, case.K, case.blocksize, dt)
+        self.ws = torch.zeros(max(self.ws_bytes, 16), dtype=torch.uint8, device=device)
+        self.act = q4.Q4_BF16 if case.act == "bf16" else q4.Q4_FP16
+        self.plan = q4.q4_gemm_plan(case.M, case.N, case.K, case.blocksize, dt)
+        import ctypes
+        P = ctypes.c_void_p
+        self._args = (P(self.A.data_ptr()), P(self.packed.data_ptr()), P(self.absmax.data_ptr()),
+                      P(self.code.data_ptr()), case.M, case.N, case.K, case.blocksize, self.act,
+                      P(self.out.data_ptr()), P(self.ws.data_ptr()), self.ws.numel())
+        self.bytes = case.algorithmic_bytes()
+
+    def launch(self, stream_handle):
+        import ctypes
+        rc = q4.lib().q4_gemm_skinny(*self._args, ctypes.c_void_p(stream_handle))
+        if rc != 0:
+            raise q4.Q4Error(rc, "q4_gemm_skinny")
+
+    def launch_public(self):
+        """The public Python API call a user makes (binding marshals the tensors)."""
+        return q4.q4_gemm_skinny(self.A, self.packed, self.absmax, self.code, self.case.N, self.case.K,
+                                 self.case.blocksize, out=self.out)
+
+
+def run_ours(args, world, rank, local):
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    wl = inputs.workloads()[args.workload]
+    peak, peak_src = hbm_peak()
+    layers = [Layer(c, inputs.seed_for(wl.index, c.M) + i, device) for i, c in enumerate(wl.cases)]
+    torch.cuda.synchronize()
+    step_bytes = sum(L.bytes for L in layers)
+    stream = torch.cuda.Stream(device)
+
+    # Warm-up (eager launches through the C ABI; sets kernel attributes).
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            for L in layers:
+                L.launch(stream.cuda_stream)
+    stream.synchronize()
+
+    # Capture CHUNK steps per graph, with one timing event after every launch.
+    def capture(nsteps):
+        g = torch.cuda.CUDAGraph()
+        evs = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(nsteps * len(layers) + 1)]
+        with torch.cuda.graph(g, stream=stream, capture_error_mode="relaxed"):
+            s = torch.cuda.current_stream()
+            evs[0].record(s)
+            k = 1
+            for _ in range(nsteps):
+                for L in layers:
+                    L.launch(s.cuda_stream)
+                    evs[k].record(s)
+                    k += 1
+        return g, evs
+
+    chunk = min(CHUNK_STEPS, args.steps)
+    g_main, ev_main = capture(chunk)
+    nfull, rem = divmod(args.steps, chunk)
+    g_rem, _ = capture(rem) if rem else (None, None)
+    g_main.replay()           # graph warm-up (not timed)
+    stream.synchronize()
+
+    uuid = str(getattr(torch.cuda.get_device_properties(device), "uuid", ""))
+    sampler = ClockSampler(("GPU-" + uuid) if uuid and not uuid.startswith("GPU-") else (uuid or str(local)))
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    sampler.start()
+    time.sleep(0.3)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(nfull):
+            g_main.replay()
+        if g_rem is not None:
+            g_rem.replay()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    barrier(world)
+    ms_total = e0.elapsed_time(e1)
+    ms_total = max_over_ranks(ms_total, world, device)
+    ms_step = ms_total / args.steps
+    value = world * step_bytes * args.steps / (ms_total * 1e-3) / 1e9
+
+    # Per-launch durations from the last replay of the main graph.
+    per = {L.case.tag: [] for L in layers}
+    for k in range(chunk * len(layers)):
+        per[layers[k % len(layers)].case.tag].append(ev_main[k].elapsed_time(ev_main[k + 1]))
+    per_shape = []
+    tot_bytes = tot_ms = 0.0
+    for L in layers:
+        us = statistics.mean(per[L.case.tag]) * 1e3
+        gbs = L.bytes / (us * 1e-6) / 1e9
+        bf16_roof_us = (L.case.M * L.case.K * 2 + 2 * L.case.N * L.case.K + L.case.M * L.case.N * 2) / (peak * 1e3)
+        per_shape.append({"shape": f"M{L.case.M} K{L.case.K} N{L.case.N} bs{L.case.blocksize}", "tag": L.case.tag,
+                          "us": round(us, 3), "GB/s": round(gbs, 1), "frac_of_peak": round(gbs / peak, 4),
+                          "bytes": L.bytes, "bf16_weight_roofline_us": round(bf16_roof_us, 3),
+                          "plan": {k: L.plan[k] for k in ("ctas", "warps", "m_pad", "sub_block", "units")}})
+        tot_bytes += L.bytes
+        tot_ms += us * 1e-3
+    achieved = tot_bytes / (tot_ms * 1e-3) / 1e9
+    del g_main, g_rem
+
+    # End to end through the public Python API: per step, H2D of the
+    # activations from pinned memory, the four calls, D2H of the outputs.
+    e2e_steps = max(1, min(args.steps, 2000))
+    torch.cuda.synchronize()
+    barrier(world)
+    t0 = time.perf_counter()
+    for _ in range(e2e_steps):
+        for L in layers:
+            L.A.copy_(L.A_host, non_blocking=True)
+            L.launch_public()
+            L.out_host.copy_(L.out, non_blocking=True)
+    torch.cuda.synchronize()
+    e2e_s = max_over_ranks(time.perf_counter() - t0, world, device)
+    e2e_value = world * step_bytes * e2e_steps / e2e_s / 1e9
+    h2d = sum(L.A_host.numel() * L.A_host.element_size() for L in layers)
+    d2h = sum(L.out_host.numel() * L.out_host.element_size() for L in layers)
+
+    if rank != 0:
+        return None
+    cpu = cpu_baseline(wl, args.cpu_seconds) if (world == 1 and not args.no_cpu_baseline) else None
+    total_weight_bytes = sum(L.packed.numel() + 4 * L.absmax.numel() for L in layers)
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_step, 5), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": wl.name, "M": sorted({c.M for c in wl.cases}), "blocksize": 64,
+                   "code_table": "normal-quantile", "activations": "bf16 ~N(0,1)", "weights": "N(0,0.02^2) fp32 -> 4-bit",
+                   "l2": f"inputs larger than L2: {total_weight_bytes / 1e6:.0f} MB of packed weights per step "
+                         f"vs {L2_BYTES / 2**20:.0f} MiB L2, no flush",
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "timing": f"CUDA graphs of {chunk} steps, CUDA events, device time"},
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                     "frac": round(achieved / peak, 4), "traffic": ncu_traffic(args.workload),
+                     "peak_source": peak_src, "kernel": "q4_gemm_mma_kernel",
+                     "per_unit": "0.5 B per weight (codes) + 4/bs B (absmax) + A and C once"},
+        "per_shape": per_shape,
+        "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "steps": e2e_steps,
+                "api": "bit_weight_dequant_b200.q4_gemm_skinny (ctypes -> libq4 C ABI), wall clock"},
+        "gpu_launches": args.steps * len(layers),
+        "clocks": clocks,
+        "cpu_baseline": cpu,
+    }
+    return line
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle (baseline leg and the reference arm)
+# ---------------------------------------------------------------------------
+
+SAMPLE_ROWS_MAX = 1024
+
+
+def _oracle_sample(case: inputs.Case, rows: int, seed: int):
+    """The first `rows` weight rows of a layer, quantized by the oracle, and
+    its activations (bf16 bit patterns)."""
+    import oracle
+    code = inputs.CODE_TABLES[case.table]()
+    W = inputs.weight_rows(case.K, seed, 0, rows, case.outliers)
+    packed, absmax = oracle.quantize(W, case.blocksize, code)
+    A = inputs.activations(case.M, case.K, torch.bfloat16, seed)
+    abits = A.view(torch.int16).numpy().view(np.uint16)
+    return (abits, packed, absmax, code)
+
+
+def _oracle_time(case, rows, prepared):
+    import oracle
+    abits, packed, absmax, code = prepared
+    t0 = time.perf_counter()
+    oracle.gemm(abits, oracle.BF16, packed, absmax, code, case.M, rows, case.K, case.blocksize, want_s=False)
+    return time.perf_counter() - t0
+
+
+def cpu_baseline(wl, seconds: float) -> dict:
+    """The oracle's GEMM as it stands (plain C loops, one thread), on the
+    first rows of each layer, called repeatedly for about `seconds` in all."""
+    tot_bytes = tot_s = 0.0
+    desc = []
+    for i, c in enumerate(wl.cases):
+        rows = min(c.N, SAMPLE_ROWS_MAX)
+        prep = _oracle_sample(c, rows, inputs.seed_for(wl.index, c.M) + i)
+        spent, reps = 0.0, 0
+        while reps == 0 or spent < seconds / len(wl.cases):
+            spent += _oracle_time(c, rows, prep)
+            reps += 1
+        tot_s += spent
+        tot_bytes += reps * inputs.Case(c.M, rows, c.K, c.blocksize).algorithmic_bytes()
+        desc.append(f"{reps}x {rows}/{c.N} rows of K{c.K}N{c.N}")
+    return {"value": round(tot_bytes / tot_s / 1e9, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "sample": "; ".join(desc) + f" (M={wl.cases[0].M}; {tot_s:.1f} s single-threaded)"}
+
+
+def run_reference(args, world, rank):
+    """Reference arm: the CPU oracle as it stands, each step a bounded
+    sample of the same workload (the first rows of each layer), sized so the
+    whole run takes about --reference-seconds."""
+    if rank != 0:
+        return None
+    wl = inputs.workloads()[args.workload]
+    per_row = []
+    for i, c in enumerate(wl.cases):
+        prep = _oracle_sample(c, 2, inputs.seed_for(wl.index, c.M) + i)
+        per_row.append(_oracle_time(c, 2, prep) / 2)
+    step_s = args.reference_seconds / max(1, args.steps + args.warmup)
+    rows = [int(max(1, min(c.N, SAMPLE_ROWS_MAX, step_s / len(wl.cases) / max(pr, 1e-9))))
+            for c, pr in zip(wl.cases, per_row)]
+    preps = [_oracle_sample(c, r, inputs.seed_for(wl.index, c.M) + i) for i, (c, r) in enumerate(zip(wl.cases, rows))]
+    for _ in range(args.warmup):
+        for c, r, p in zip(wl.cases, rows, preps):
+            _oracle_time(c, r, p)
+    tot_s = 0.0
+    for _ in range(args.steps):
+        for c, r, p in zip(wl.cases, rows, preps):
+            tot_s += _oracle_time(c, r, p)
+    step_bytes = sum(inputs.Case(c.M, r, c.K, c.blocksize).algorithmic_bytes() for c, r in zip(wl.cases, rows))
+    value = step_bytes * args.steps / tot_s / 1e9
+    sample = "; ".join(f"{r}/{c.N} rows of K{c.K}N{c.N}" for c, r in zip(wl.cases, rows))
+    return {"impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(tot_s / args.steps * 1e3, 4),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": wl.name, "parallelism": "CPU oracle, one thread"},
+            "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+                             "sample": sample + " per step"},
+            "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20000)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="decode70b", choices=list(inputs.workloads()))
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--reference-seconds", type=float, default=60.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        log("note: warm-up raised to 3 steps (minimum)")
+        args.warmup = 3
+    world, rank, local = dist_setup()
+    try:
+        if args.impl == "reference":
+            line = run_reference(args, world, rank)
+        else:
+            line = run_ours(args, world, rank, local)
+        if rank == 0 and line is not None:
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,173 @@
+"""Thin ctypes binding over libq4.so (the C ABI of include/q4.h).
+
+Argument marshalling only: every step of the computation runs in the CUDA
+kernels of libq4.  PyTorch supplies device memory and the current stream.
+The library must be built (``python -m bit_weight_dequant_b200.build``);
+there is no fallback of any kind, a missing library raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libq4.so")
+HEADER = os.path.join(os.path.dirname(_HERE), "include", "q4.h")
+
+Q4_OK, Q4_ERR_INVALID_ARG, Q4_ERR_UNSUPPORTED, Q4_ERR_MISALIGNED, Q4_ERR_CUDA, Q4_ERR_WORKSPACE = range(6)
+Q4_BF16, Q4_FP16, Q4_FP32 = 0, 1, 2
+
+_TORCH_TO_Q4 = {torch.bfloat16: Q4_BF16, torch.float16: Q4_FP16, torch.float32: Q4_FP32}
+_Q4_TO_TORCH = {v: k for k, v in _TORCH_TO_Q4.items()}
+
+
+class Q4Error(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {status_string(status)}")
+
+
+class q4_gemm_plan_t(ctypes.Structure):
+    _fields_ = [("math", ctypes.c_int), ("sub_block", ctypes.c_int), ("m_pad", ctypes.c_int),
+                ("rows_per_tile", ctypes.c_int), ("warps", ctypes.c_int), ("ctas", ctypes.c_int),
+                ("tiles", ctypes.c_int), ("units", ctypes.c_int64), ("smem_bytes", ctypes.c_size_t),
+                ("workspace_bytes", ctypes.c_size_t)]
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libq4.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"libq4.so is not built ({LIB_PATH}); run `python -m bit_weight_dequant_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        P, i64, ci, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
+        L.q4_status_string.argtypes = [ci]
+        L.q4_status_string.restype = ctypes.c_char_p
+        L.q4_quantize_blockwise.argtypes = [P, i64, ci, P, P, P, P]
+        L.q4_dequantize_blockwise.argtypes = [P, P, P, i64, ci, ci, P, P]
+        L.q4_gemm_workspace_size.argtypes = [ci, ci, ci, ci, ci, ctypes.POINTER(sz)]
+        L.q4_gemm_skinny.argtypes = [P, P, P, P, ci, ci, ci, ci, ci, P, P, sz, P]
+        L.q4_gemm_skinny_ex.argtypes = [P, P, P, P, ci, ci, ci, ci, ci, P, P, sz, P, ci, ci, ci]
+        L.q4_gemm_plan.argtypes = [ci, ci, ci, ci, ci, ci, ctypes.POINTER(q4_gemm_plan_t)]
+        L.q4_partition_start.argtypes = [i64, ci, ci]
+        L.q4_partition_start.restype = i64
+        L.q4_partition_owner.argtypes = [i64, ci, i64]
+        for f in ("q4_quantize_blockwise", "q4_dequantize_blockwise", "q4_gemm_workspace_size",
+                  "q4_gemm_skinny", "q4_gemm_skinny_ex", "q4_gemm_plan", "q4_partition_owner"):
+            getattr(L, f).restype = ci
+        _lib = L
+    return _lib
+
+
+def declared_functions() -> list:
+    """Names of the functions include/q4.h declares."""
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(q4_\w+)\s*\(", text)))
+
+
+def status_string(status: int) -> str:
+    return lib().q4_status_string(status).decode()
+
+
+def _check(rc: int, what: str):
+    if rc != Q4_OK:
+        raise Q4Error(rc, what)
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else None
+
+
+def _stream(device) -> ctypes.c_void_p:
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def q4_quantize_blockwise(W: torch.Tensor, blocksize: int, code: torch.Tensor):
+    """Quantize a CUDA fp32 tensor blockwise; returns (packed uint8, absmax fp32)."""
+    assert W.is_cuda and W.dtype == torch.float32 and W.is_contiguous()
+    n = W.numel()
+    packed = torch.empty((n + 1) // 2, dtype=torch.uint8, device=W.device)
+    absmax = torch.empty((n + blocksize - 1) // blocksize, dtype=torch.float32, device=W.device)
+    rc = lib().q4_quantize_blockwise(_ptr(W), n, blocksize, _ptr(code), _ptr(packed), _ptr(absmax),
+                                     _stream(W.device))
+    _check(rc, "q4_quantize_blockwise")
+    return packed, absmax
+
+
+def q4_dequantize_blockwise(packed: torch.Tensor, absmax: torch.Tensor, code: torch.Tensor, n: int,
+                            blocksize: int, out_dtype: torch.dtype = torch.bfloat16,
+                            out: torch.Tensor | None = None) -> torch.Tensor:
+    """Dequantize to bf16/fp16/fp32 (CUDA tensor of n elements)."""
+    if out is None:
+        out = torch.empty(n, dtype=out_dtype, device=packed.device)
+    rc = lib().q4_dequantize_blockwise(_ptr(packed), _ptr(absmax), _ptr(code), n, blocksize,
+                                       _TORCH_TO_Q4[out.dtype], _ptr(out), _stream(packed.device))
+    _check(rc, "q4_dequantize_blockwise")
+    return out
+
+
+def q4_gemm_workspace_size(M: int, N: int, K: int, blocksize: int, act_dtype: torch.dtype) -> int:
+    v = ctypes.c_size_t(0)
+    _check(lib().q4_gemm_workspace_size(M, N, K, blocksize, _TORCH_TO_Q4[act_dtype], ctypes.byref(v)),
+           "q4_gemm_workspace_size")
+    return v.value
+
+
+def q4_gemm_plan(M: int, N: int, K: int, blocksize: int, act_dtype: torch.dtype = torch.bfloat16,
+                 num_sms: int = 0) -> dict:
+    pl = q4_gemm_plan_t()
+    _check(lib().q4_gemm_plan(M, N, K, blocksize, _TORCH_TO_Q4[act_dtype], num_sms, ctypes.byref(pl)),
+           "q4_gemm_plan")
+    return {f: getattr(pl, f) for f, _ in q4_gemm_plan_t._fields_}
+
+
+class Workspace:
+    """Zero-filled device scratch for q4_gemm_skinny, grown on demand.
+
+    The library returns it zero-filled after every call; one per stream."""
+
+    def __init__(self, device):
+        self.device = torch.device(device)
+        self.buf = torch.zeros(0, dtype=torch.uint8, device=self.device)
+
+    def get(self, nbytes: int) -> torch.Tensor:
+        if self.buf.numel() < nbytes:
+            self.buf = torch.zeros(max(nbytes, 2 * self.buf.numel()), dtype=torch.uint8, device=self.device)
+        return self.buf
+
+
+_workspaces: dict = {}
+
+
+def _default_workspace(device) -> Workspace:
+    key = (torch.device(device), torch.cuda.current_stream(device).cuda_stream)
+    ws = _workspaces.get(key)
+    if ws is None:
+        ws = _workspaces[key] = Workspace(device)
+    return ws
+
+
+def q4_gemm_skinny(A: torch.Tensor, Wpacked: torch.Tensor, absmax: torch.Tensor, code: torch.Tensor, N: int,
+                   K: int, blocksize: int, out: torch.Tensor | None = None, workspace: Workspace | None = None,
+                   math: int = 0, ctas: int = 0, warps: int = 0) -> torch.Tensor:
+    """out[M, N] = A[M, K] . dequant(W)[N, K]^T on the GPU (fused kernel)."""
+    M = A.shape[0] if A.dim() == 2 else 1
+    if out is None:
+        out = torch.empty((M, N), dtype=A.dtype, device=A.device)
+    act = _TORCH_TO_Q4[A.dtype]
+    need = ctypes.c_size_t(0)
+    _check(lib().q4_gemm_workspace_size(M, N, K, blocksize, act, ctypes.byref(need)), "q4_gemm_workspace_size")
+    ws = (workspace or _default_workspace(A.device)).get(need.value) if need.value else None
+    rc = lib().q4_gemm_skinny_ex(_ptr(A), _ptr(Wpacked), _ptr(absmax), _ptr(code), M, N, K, blocksize, act,
+                                 _ptr(out), _ptr(ws), ws.numel() if ws is not None else 0, _stream(A.device),
+                                 math, ctas, warps)
+    _check(rc, "q4_gemm_skinny")
+    return out

@@ -1,0 +1,241 @@
+// q4_api.cu -- extern "C" entry points of libq4 (declared in include/q4.h):
+// argument validation, the M- and shape-keyed launch table, workspace sizing
+// and error reporting.  Every function validates before it enqueues anything
+// and returns a q4_status; a failed launch drains the runtime's last error.
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+#include <unordered_map>
+
+#include "../../include/q4.h"
+#include "q4_internal.h"
+#include "q4_plan.cuh"
+
+namespace q4 {
+
+static constexpr int kMaxDevices = 64;
+
+int device_sm_count(int* sms) {
+    static std::atomic<int> cache[kMaxDevices];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+        cudaGetLastError();
+        return 1;
+    }
+    int v = cache[dev].load(std::memory_order_relaxed);
+    if (v <= 0) {
+        if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0) {
+            cudaGetLastError();
+            return 1;
+        }
+        cache[dev].store(v, std::memory_order_relaxed);
+    }
+    *sms = v;
+    return 0;
+}
+
+cudaError_t ensure_smem_attr(const void* kernel, size_t bytes) {
+    static std::mutex mu;
+    static std::unordered_map<const void*, uint64_t> done;  // kernel -> bitmask of devices
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    std::lock_guard<std::mutex> lock(mu);
+    uint64_t& mask = done[kernel];
+    const uint64_t bit = (dev >= 0 && dev < 64) ? (uint64_t(1) << dev) : 0;
+    if (bit && (mask & bit)) return cudaSuccess;
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+    if (e == cudaSuccess) mask |= bit;
+    return e;
+}
+
+static bool is_pow2_blocksize(int bs) { return bs >= 32 && bs <= 4096 && (bs & (bs - 1)) == 0; }
+
+static bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+// Host-side fault injection for tests: Q4_TEST_FAIL_LAUNCH set to a
+// non-empty value other than "0" makes every entry point report Q4_ERR_CUDA
+// instead of launching (nothing reaches the GPU).
+static bool injected_failure() {
+    const char* v = std::getenv("Q4_TEST_FAIL_LAUNCH");
+    return v && v[0] && std::strcmp(v, "0") != 0;
+}
+
+static int from_cuda(cudaError_t e) {
+    if (e == cudaSuccess) return Q4_OK;
+    cudaGetLastError();  // drain: leave no error of ours pending
+    return Q4_ERR_CUDA;
+}
+
+static size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+// Validates a GEMM request.  Returns Q4_OK and fills `out` with the launch
+// table's choice (and the problem's unit counts) when it can run.
+static int gemm_choose(int M, int N, int K, int blocksize, int act_dtype, int num_sms, int math, int ctas,
+                       int warps, GemmChoice* ch, int* tiles, int64_t* units, size_t* ws_bytes) {
+    if (M < 0 || N < 0 || K < 0) return Q4_ERR_INVALID_ARG;
+    if (!is_pow2_blocksize(blocksize)) return Q4_ERR_INVALID_ARG;
+    if (act_dtype != Q4_BF16 && act_dtype != Q4_FP16 && act_dtype != Q4_FP32) return Q4_ERR_INVALID_ARG;
+    if (math < 0 || math > 2 || ctas < 0 || warps < 0) return Q4_ERR_INVALID_ARG;
+    if (M > 16 || act_dtype == Q4_FP32 || K % blocksize != 0) return Q4_ERR_UNSUPPORTED;
+    GemmChoice c{};
+    c.math = 1;
+    if (math == 2) return Q4_ERR_UNSUPPORTED;  // CUDA-core variant not built in this library version
+    c.sub_block = blocksize < 64 ? blocksize : 64;
+    c.m_pad = M <= 8 ? 8 : 16;
+    c.rows_per_tile = 64;
+    c.warps = c.m_pad == 8 ? 16 : 8;
+    if (warps > 0) {
+        if (!(warps == 8 || (warps == 16 && c.m_pad == 8))) return Q4_ERR_UNSUPPORTED;
+        c.warps = warps;
+    }
+    const int t = N > 0 ? (N + c.rows_per_tile - 1) / c.rows_per_tile : 0;
+    const int64_t u = (int64_t)t * (K / c.sub_block);
+    int sms = num_sms;
+    if (sms <= 0 && device_sm_count(&sms) != 0) return Q4_ERR_CUDA;
+    int64_t g = ctas > 0 ? ctas : sms;
+    if (g > u) g = u;  // every CTA owns at least one unit
+    if (g < 1) g = 1;
+    c.ctas = (int)g;
+    *ch = c;
+    *tiles = t;
+    *units = u;
+    // Workspace: a counter per tile (256-B aligned), then two partial slots per CTA.
+    *ws_bytes = (c.ctas > 1 && u > 0)
+                    ? align_up((size_t)t * sizeof(int), 256) + (size_t)c.ctas * 2 * gemm_slot_floats(c.m_pad) * 4
+                    : 0;
+    return Q4_OK;
+}
+
+}  // namespace q4
+
+using namespace q4;
+
+extern "C" {
+
+const char* q4_status_string(int status) {
+    switch (status) {
+        case Q4_OK: return "Q4_OK";
+        case Q4_ERR_INVALID_ARG: return "Q4_ERR_INVALID_ARG: null pointer, negative size, bad blocksize or dtype";
+        case Q4_ERR_UNSUPPORTED: return "Q4_ERR_UNSUPPORTED: valid request outside this library's fused path";
+        case Q4_ERR_MISALIGNED: return "Q4_ERR_MISALIGNED: pointer misses its required alignment";
+        case Q4_ERR_CUDA: return "Q4_ERR_CUDA: CUDA call or kernel launch failed";
+        case Q4_ERR_WORKSPACE: return "Q4_ERR_WORKSPACE: GEMM workspace missing or too small";
+        default: return "unknown q4 status";
+    }
+}
+
+int q4_quantize_blockwise(const float* W, int64_t n, int blocksize, const float* code, uint8_t* packed,
+                          float* absmax, void* stream) {
+    if (!W || !code || !packed || !absmax || n < 0 || !is_pow2_blocksize(blocksize)) return Q4_ERR_INVALID_ARG;
+    if (!aligned(W, 16) || !aligned(code, 4) || !aligned(absmax, 4)) return Q4_ERR_MISALIGNED;
+    if (n == 0) return Q4_OK;
+    if (injected_failure()) return Q4_ERR_CUDA;
+    return from_cuda(quantize_launch(W, n, blocksize, code, packed, absmax, (cudaStream_t)stream));
+}
+
+int q4_dequantize_blockwise(const uint8_t* packed, const float* absmax, const float* code, int64_t n,
+                            int blocksize, int out_dtype, void* out, void* stream) {
+    if (!packed || !absmax || !code || !out || n < 0 || !is_pow2_blocksize(blocksize)) return Q4_ERR_INVALID_ARG;
+    if (out_dtype != Q4_BF16 && out_dtype != Q4_FP16 && out_dtype != Q4_FP32) return Q4_ERR_INVALID_ARG;
+    if (!aligned(packed, 16) || !aligned(out, 16) || !aligned(absmax, 4) || !aligned(code, 4))
+        return Q4_ERR_MISALIGNED;
+    if (n == 0) return Q4_OK;
+    if (injected_failure()) return Q4_ERR_CUDA;
+    return from_cuda(dequantize_launch(packed, absmax, code, n, blocksize, out_dtype, out, (cudaStream_t)stream));
+}
+
+int q4_gemm_plan(int M, int N, int K, int blocksize, int act_dtype, int num_sms, q4_gemm_plan_t* plan) {
+    if (!plan) return Q4_ERR_INVALID_ARG;
+    GemmChoice ch;
+    int tiles = 0;
+    int64_t units = 0;
+    size_t ws = 0;
+    const int rc = gemm_choose(M, N, K, blocksize, act_dtype, num_sms, 0, 0, 0, &ch, &tiles, &units, &ws);
+    if (rc != Q4_OK) return rc;
+    plan->math = ch.math;
+    plan->sub_block = ch.sub_block;
+    plan->m_pad = ch.m_pad;
+    plan->rows_per_tile = ch.rows_per_tile;
+    plan->warps = ch.warps;
+    plan->ctas = ch.ctas;
+    plan->tiles = tiles;
+    plan->units = units;
+    plan->smem_bytes = gemm_smem_bytes(ch.sub_block, ch.m_pad, ch.warps);
+    plan->workspace_bytes = ws;
+    return Q4_OK;
+}
+
+int q4_gemm_workspace_size(int M, int N, int K, int blocksize, int act_dtype, size_t* bytes) {
+    if (!bytes) return Q4_ERR_INVALID_ARG;
+    GemmChoice ch;
+    int tiles = 0;
+    int64_t units = 0;
+    const int rc = gemm_choose(M, N, K, blocksize, act_dtype, 0, 0, 0, 0, &ch, &tiles, &units, bytes);
+    return rc;
+}
+
+int q4_gemm_skinny_ex(const void* A, const uint8_t* Wpacked, const float* absmax, const float* code, int M, int N,
+                      int K, int blocksize, int act_dtype, void* out, void* workspace, size_t workspace_bytes,
+                      void* stream, int math, int ctas, int warps) {
+    if (!A || !Wpacked || !absmax || !code || !out) return Q4_ERR_INVALID_ARG;
+    GemmChoice ch;
+    int tiles = 0;
+    int64_t units = 0;
+    size_t need = 0;
+    int rc = gemm_choose(M, N, K, blocksize, act_dtype, 0, math, ctas, warps, &ch, &tiles, &units, &need);
+    if (rc != Q4_OK) return rc;
+    if (!aligned(A, 16) || !aligned(Wpacked, 16) || !aligned(out, 16) || !aligned(absmax, 4) || !aligned(code, 4))
+        return Q4_ERR_MISALIGNED;
+    if (need > 0 && (!workspace || workspace_bytes < need)) return Q4_ERR_WORKSPACE;
+    if (workspace && !aligned(workspace, 16)) return Q4_ERR_MISALIGNED;
+    if (M == 0 || N == 0) return Q4_OK;
+    if (injected_failure()) return Q4_ERR_CUDA;
+    cudaStream_t st = (cudaStream_t)stream;
+    if (K == 0)  // empty contraction: all-zero output (0x0000 is +0 in bf16 and fp16)
+        return from_cuda(cudaMemsetAsync(out, 0, (size_t)M * N * 2, st));
+    GemmParams p{};
+    p.A = A;
+    p.Wp = Wpacked;
+    p.absmax = absmax;
+    p.code = code;
+    p.out = out;
+    p.counters = static_cast<int*>(workspace);
+    p.partials = workspace ? reinterpret_cast<float*>(static_cast<char*>(workspace) +
+                                                      align_up((size_t)tiles * sizeof(int), 256))
+                           : nullptr;
+    p.M = M;
+    p.N = N;
+    p.K = K;
+    p.kb_per_tile = K / ch.sub_block;
+    int sh = 0;
+    while ((ch.sub_block << sh) < blocksize) ++sh;
+    p.am_shift = sh;
+    p.am_per_row = K / blocksize;
+    p.tiles = tiles;
+    p.ctas = ch.ctas;
+    p.units = units;
+    return from_cuda(gemm_launch(ch, act_dtype, p, st));
+}
+
+int q4_gemm_skinny(const void* A, const uint8_t* Wpacked, const float* absmax, const float* code, int M, int N,
+                   int K, int blocksize, int act_dtype, void* out, void* workspace, size_t workspace_bytes,
+                   void* stream) {
+    return q4_gemm_skinny_ex(A, Wpacked, absmax, code, M, N, K, blocksize, act_dtype, out, workspace,
+                             workspace_bytes, stream, 0, 0, 0);
+}
+
+int64_t q4_partition_start(int64_t total, int parts, int part) {
+    if (total < 0 || parts <= 0 || part < 0 || part > parts) return -1;
+    return part_start(total, parts, part);
+}
+
+int q4_partition_owner(int64_t total, int parts, int64_t u) {
+    if (total <= 0 || parts <= 0 || u < 0 || u >= total) return -1;
+    return part_owner(total, parts, u);
+}
+
+}  // extern "C"

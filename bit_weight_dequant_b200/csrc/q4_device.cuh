@@ -1,0 +1,155 @@
+// q4_device.cuh -- small device-side helpers shared by the libq4 kernels:
+// cache-hinted global loads, shared-memory access by 32-bit window address,
+// byte permutes, 16-bit float packing and the m16n8k16 tensor-core MMA.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <stdint.h>
+
+namespace q4 {
+
+// ---------------------------------------------------------------------------
+// Global loads.  Weights and absmax are read exactly once per call: stream
+// them past L1 (no_allocate) through the read-only path.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint2 ldg_stream_v2(const void* p) {
+    uint2 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0, %1}, [%2];"
+                 : "=r"(v.x), "=r"(v.y)
+                 : "l"(p));
+    return v;
+}
+
+__device__ __forceinline__ uint32_t ldg_stream_u32(const void* p) {
+    uint32_t v;
+    asm volatile("ld.global.nc.L1::no_allocate.u32 %0, [%1];" : "=r"(v) : "l"(p));
+    return v;
+}
+
+__device__ __forceinline__ float ldg_stream_f32(const float* p) {
+    float v;
+    asm volatile("ld.global.nc.L1::no_allocate.f32 %0, [%1];" : "=f"(v) : "l"(p));
+    return v;
+}
+
+__device__ __forceinline__ uint4 ldg_stream_v4(const void* p) {
+    uint4 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p));
+    return v;
+}
+
+// Activations are re-read by several warps of an SM: keep them in L1.
+__device__ __forceinline__ uint4 ldg_v4(const void* p) {
+    uint4 v;
+    asm volatile("ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p));
+    return v;
+}
+
+// L2-coherent load (bypasses L1): for data other CTAs wrote in this launch.
+__device__ __forceinline__ float ldg_cg_f32(const float* p) {
+    float v;
+    asm volatile("ld.global.cg.f32 %0, [%1];" : "=f"(v) : "l"(p));
+    return v;
+}
+
+// ---------------------------------------------------------------------------
+// Shared memory by 32-bit shared-window address.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ uint32_t lds_u32(uint32_t addr) {
+    uint32_t v;
+    asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(addr));
+    return v;
+}
+
+__device__ __forceinline__ float lds_f32(uint32_t addr) {
+    float v;
+    asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(addr));
+    return v;
+}
+
+__device__ __forceinline__ void sts_f32(uint32_t addr, float v) {
+    asm volatile("st.shared.f32 [%0], %1;" ::"r"(addr), "f"(v));
+}
+
+__device__ __forceinline__ void sts_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d));
+}
+
+// ---------------------------------------------------------------------------
+// Byte permute: result byte i = byte sel_i of the 8-byte value {hi:lo}.
+// ---------------------------------------------------------------------------
+template <uint32_t SEL>
+__device__ __forceinline__ uint32_t prmt(uint32_t lo, uint32_t hi) {
+    uint32_t r;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(lo), "r"(hi), "n"(SEL));
+    return r;
+}
+
+// ---------------------------------------------------------------------------
+// 16-bit activation types.
+// ---------------------------------------------------------------------------
+template <typename T>
+struct Act;
+
+template <>
+struct Act<__nv_bfloat16> {
+    // Two floats -> packed pair, each rounded to nearest even; `first` in the
+    // low 16 bits.
+    __device__ __forceinline__ static uint32_t pack(float first, float second) {
+        __nv_bfloat162 h = __floats2bfloat162_rn(first, second);
+        return *reinterpret_cast<uint32_t*>(&h);
+    }
+    __device__ __forceinline__ static __nv_bfloat16 from_float(float v) { return __float2bfloat16_rn(v); }
+};
+
+template <>
+struct Act<__half> {
+    __device__ __forceinline__ static uint32_t pack(float first, float second) {
+        __half2 h = __floats2half2_rn(first, second);
+        return *reinterpret_cast<uint32_t*>(&h);
+    }
+    __device__ __forceinline__ static __half from_float(float v) { return __float2half_rn(v); }
+};
+
+// ---------------------------------------------------------------------------
+// D = A(16x16, row) * B(16x8, col) + C, fp32 accumulate.
+// Fragment ownership (g = lane/4, t = lane%4):
+//   a0: A[g][2t..2t+1]   a1: A[g+8][2t..2t+1]   a2: A[g][2t+8..2t+9]   a3: A[g+8][2t+8..2t+9]
+//   b0: B[2t..2t+1][g]   b1: B[2t+8..2t+9][g]
+//   d0,d1: D[g][2t..2t+1]   d2,d3: D[g+8][2t..2t+1]
+// ---------------------------------------------------------------------------
+template <typename T>
+__device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                         uint32_t b0, uint32_t b1, const float (&c)[4]);
+
+template <>
+__device__ __forceinline__ void mma16816<__nv_bfloat16>(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                                        uint32_t a3, uint32_t b0, uint32_t b1,
+                                                        const float (&c)[4]) {
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+        "{%8, %9}, {%10, %11, %12, %13};"
+        : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(c[0]), "f"(c[1]), "f"(c[2]),
+          "f"(c[3]));
+}
+
+template <>
+__device__ __forceinline__ void mma16816<__half>(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                                 uint32_t a3, uint32_t b0, uint32_t b1, const float (&c)[4]) {
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+        "{%8, %9}, {%10, %11, %12, %13};"
+        : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(c[0]), "f"(c[1]), "f"(c[2]),
+          "f"(c[3]));
+}
+
+}  // namespace q4

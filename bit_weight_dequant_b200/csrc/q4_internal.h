@@ -1,0 +1,37 @@
+// q4_internal.h -- declarations shared by the libq4 translation units
+// (launchers, launch-table choice, per-device attribute cache).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "q4_plan.cuh"
+
+namespace q4 {
+
+// One launch-table decision for the GEMM.
+struct GemmChoice {
+    int math;       // 1 = tensor-core MMA, 2 = CUDA-core FMA
+    int sub_block;  // 32 or 64
+    int m_pad;      // 8 or 16
+    int warps;      // warps per CTA
+    int ctas;       // persistent CTAs
+    int rows_per_tile;
+};
+
+// Sets cudaFuncAttributeMaxDynamicSharedMemorySize once per (kernel, device).
+cudaError_t ensure_smem_attr(const void* kernel, size_t bytes);
+
+cudaError_t gemm_launch(const GemmChoice& ch, int act_dtype, const GemmParams& p, cudaStream_t stream);
+size_t gemm_smem_bytes(int sub_block, int m_pad, int warps);
+size_t gemm_slot_floats(int m_pad);
+
+cudaError_t quantize_launch(const float* W, int64_t n, int blocksize, const float* code, uint8_t* packed,
+                            float* absmax, cudaStream_t stream);
+cudaError_t dequantize_launch(const uint8_t* packed, const float* absmax, const float* code, int64_t n,
+                              int blocksize, int out_dtype, void* out, cudaStream_t stream);
+
+int device_sm_count(int* sms);  // current device; returns 0 on success
+
+}  // namespace q4

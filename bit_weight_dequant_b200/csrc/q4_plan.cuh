@@ -1,0 +1,65 @@
+// q4_plan.cuh -- work decomposition of the fused dequantize + skinny GEMM.
+//
+// The weight matrix W[N,K] is cut into work units of `rows_per_tile` rows by
+// `sub_block` columns (one absmax block, or a part of one).  Units are
+// numbered tile-major: unit u covers tile u / kb_per_tile, column block
+// u % kb_per_tile.  A persistent grid of `ctas` CTAs splits the unit range
+// into equal contiguous ranges (stream-K style), and each CTA splits its
+// range again over its warps.  A tile cut by a warp boundary is combined in
+// shared memory; a tile cut by a CTA boundary is combined through a small
+// global workspace by whichever CTA arrives last.  Every SM gets the same
+// number of weight bytes to within one unit, whatever N and K are.
+#pragma once
+
+#include <stdint.h>
+
+namespace q4 {
+
+// First unit of part p when `total` units are split into `parts` ranges.
+__host__ __device__ __forceinline__ int64_t part_start(int64_t total, int parts, int p) {
+    return (total * (int64_t)p) / parts;
+}
+
+// The unique part p with part_start(p) <= u < part_start(p + 1).
+// part_start(p) <= u  <=>  total*p < (u+1)*parts  <=>  p <= ((u+1)*parts - 1) / total.
+__host__ __device__ __forceinline__ int part_owner(int64_t total, int parts, int64_t u) {
+    return (int)(((u + 1) * (int64_t)parts - 1) / total);
+}
+
+// Compile-time shape of one GEMM kernel variant.
+template <int SB_, int MPAD_, int TW_, int NW_>
+struct GemmShape {
+    static constexpr int SB = SB_;      // k-width of a unit (32 or 64)
+    static constexpr int MPAD = MPAD_;  // M padded to 8 or 16 (MMA columns)
+    static constexpr int NJ = MPAD_ / 8;
+    static constexpr int TW = TW_;      // 16-row MMA tiles per unit
+    static constexpr int TR = 16 * TW_; // rows per unit
+    static constexpr int NW = NW_;      // warps per CTA
+    static constexpr int SLOT_REGS = TW_ * NJ * 4;     // accumulator registers per lane
+    static constexpr int SLOT_FLOATS = SLOT_REGS * 32; // one warp's partial tile
+    static constexpr uint32_t LUT_BYTES = 256u * 256u; // 256 byte values x 32 lanes x 4 B, 256-B rows
+    static constexpr uint32_t SLOT_BYTES = (uint32_t)NW_ * 2u * SLOT_FLOATS * 4u;
+    // Dynamic shared memory: up to 64 KiB of padding so the LUT starts on a
+    // 64 KiB boundary of the shared window, the LUT, and the warp slots.
+    static constexpr uint32_t SMEM_BYTES = 65536u + LUT_BYTES + SLOT_BYTES;
+};
+
+// Runtime parameters of one GEMM launch.
+struct GemmParams {
+    const void* A;
+    const uint8_t* Wp;
+    const float* absmax;
+    const float* code;
+    void* out;
+    float* partials;   // [ctas][2][SLOT_FLOATS]
+    int* counters;     // [tiles], zero between calls
+    int M, N, K;
+    int kb_per_tile;   // K / SB
+    int am_shift;      // log2(blocksize / SB): absmax column of unit column kb = kb >> am_shift
+    int am_per_row;    // K / blocksize
+    int tiles;
+    int ctas;
+    int64_t units;
+};
+
+}  // namespace q4

@@ -1,0 +1,194 @@
+// q4_quant.cu -- blockwise 4-bit quantize and dequantize kernels.
+//
+// Dequantize is the building block of the split "dequantize + GEMM" path
+// that bitsandbytes PR #1920 ("Fused path support for M > 1") compares the
+// fused kernel against; quantize produces the packed format the fused
+// kernel reads.  Both are memory-bound streams; both must match the
+// definition exactly (codes and absmax equal, dequantized values bit-equal),
+// so every floating-point step is an explicitly rounded intrinsic.
+#include <cuda_runtime.h>
+
+#include "q4_device.cuh"
+#include "q4_internal.h"
+
+namespace q4 {
+
+// Index of the nearest code: argmin_j |x - code[j]| on binary32
+// differences, lowest j on ties (strict "<" while scanning upward).
+__device__ __forceinline__ int nearest_code(float x, const float (&c)[16]) {
+    int best = 0;
+    float bd = fabsf(__fsub_rn(x, c[0]));
+#pragma unroll
+    for (int j = 1; j < 16; ++j) {
+        const float d = fabsf(__fsub_rn(x, c[j]));
+        if (d < bd) {
+            bd = d;
+            best = j;
+        }
+    }
+    return best;
+}
+
+// One warp per block of `bs` elements (grid-stride over blocks).  Pairs of
+// elements map to one output byte (even element -> high nibble); blocks
+// start at even indices because bs is even, so pairs never straddle blocks.
+__global__ void __launch_bounds__(256) q4_quantize_kernel(const float* __restrict__ W, int64_t n, int bs_shift,
+                                                          const float* __restrict__ code,
+                                                          uint8_t* __restrict__ packed,
+                                                          float* __restrict__ absmax, int64_t nblocks) {
+    float c[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) c[j] = __ldg(code + j);
+    const int lane = threadIdx.x & 31;
+    const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+    for (int64_t b = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; b < nblocks; b += nwarps) {
+        const int64_t lo = b << bs_shift;
+        const int64_t rem = n - lo;
+        const int cnt = rem < ((int64_t)1 << bs_shift) ? (int)rem : (1 << bs_shift);
+        const float* wb = W + lo;
+        float amax = 0.f;
+        for (int p = lane; 2 * p < cnt; p += 32) {
+            if (2 * p + 1 < cnt) {
+                const float2 v = __ldg(reinterpret_cast<const float2*>(wb) + p);
+                amax = fmaxf(amax, fmaxf(fabsf(v.x), fabsf(v.y)));
+            } else {
+                amax = fmaxf(amax, fabsf(__ldg(wb + 2 * p)));
+            }
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+        if (lane == 0) absmax[b] = amax;
+        for (int p = lane; 2 * p < cnt; p += 32) {
+            float w0, w1 = 0.f;
+            const bool has1 = 2 * p + 1 < cnt;
+            if (has1) {
+                const float2 v = __ldg(reinterpret_cast<const float2*>(wb) + p);
+                w0 = v.x;
+                w1 = v.y;
+            } else {
+                w0 = __ldg(wb + 2 * p);
+            }
+            const int i0 = nearest_code(amax > 0.f ? __fdiv_rn(w0, amax) : 0.f, c);
+            const int i1 = has1 ? nearest_code(amax > 0.f ? __fdiv_rn(w1, amax) : 0.f, c) : 0;
+            packed[(lo >> 1) + p] = (uint8_t)((i0 << 4) | i1);
+        }
+    }
+}
+
+template <int OUT>
+struct DequantOut;
+
+template <>
+struct DequantOut<0> {  // bf16
+    __device__ __forceinline__ static uint32_t pair(float a, float b) { return Act<__nv_bfloat16>::pack(a, b); }
+    __device__ __forceinline__ static void one(void* out, int64_t i, float v) {
+        static_cast<__nv_bfloat16*>(out)[i] = __float2bfloat16_rn(v);
+    }
+};
+
+template <>
+struct DequantOut<1> {  // fp16
+    __device__ __forceinline__ static uint32_t pair(float a, float b) { return Act<__half>::pack(a, b); }
+    __device__ __forceinline__ static void one(void* out, int64_t i, float v) {
+        static_cast<__half*>(out)[i] = __float2half_rn(v);
+    }
+};
+
+// One thread per 32 elements (16 packed bytes -> one 128-bit load); a chunk
+// never straddles an absmax block because blocksize is a multiple of 32.
+template <int OUT>
+__global__ void __launch_bounds__(256) q4_dequant_kernel(const uint8_t* __restrict__ packed,
+                                                         const float* __restrict__ absmax,
+                                                         const float* __restrict__ code, int64_t n, int bs_shift,
+                                                         void* __restrict__ out) {
+    __shared__ float sc[16];
+    if (threadIdx.x < 16) sc[threadIdx.x] = code[threadIdx.x];
+    __syncthreads();
+    const int64_t nchunks = n >> 5;
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    const int64_t t0 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    for (int64_t q = t0; q < nchunks; q += stride) {
+        const uint4 v = ldg_stream_v4(packed + 16 * q);
+        const float am = __ldg(absmax + ((q << 5) >> bs_shift));
+        const uint32_t words[4] = {v.x, v.y, v.z, v.w};
+        if constexpr (OUT == 2) {
+            float4* o = reinterpret_cast<float4*>(static_cast<float*>(out) + (q << 5));
+#pragma unroll
+            for (int w = 0; w < 4; ++w) {
+                float f[8];
+#pragma unroll
+                for (int by = 0; by < 4; ++by) {
+                    const uint32_t b = (words[w] >> (8 * by)) & 0xFFu;
+                    f[2 * by] = __fmul_rn(sc[b >> 4], am);
+                    f[2 * by + 1] = __fmul_rn(sc[b & 15u], am);
+                }
+                o[2 * w] = make_float4(f[0], f[1], f[2], f[3]);
+                o[2 * w + 1] = make_float4(f[4], f[5], f[6], f[7]);
+            }
+        } else {
+            uint4* o = reinterpret_cast<uint4*>(static_cast<uint16_t*>(out) + (q << 5));
+#pragma unroll
+            for (int w = 0; w < 4; ++w) {
+                uint32_t r[4];
+#pragma unroll
+                for (int by = 0; by < 4; ++by) {
+                    const uint32_t b = (words[w] >> (8 * by)) & 0xFFu;
+                    r[by] = DequantOut<OUT>::pair(__fmul_rn(sc[b >> 4], am), __fmul_rn(sc[b & 15u], am));
+                }
+                o[w] = make_uint4(r[0], r[1], r[2], r[3]);
+            }
+        }
+    }
+    // Ragged tail (n % 32 elements): one element per thread.
+    for (int64_t i = (nchunks << 5) + t0; i < n; i += stride) {
+        const uint32_t byte = packed[i >> 1];
+        const uint32_t idx = (i & 1) ? (byte & 15u) : (byte >> 4);
+        const float v = __fmul_rn(sc[idx], __ldg(absmax + (i >> bs_shift)));
+        if constexpr (OUT == 2)
+            static_cast<float*>(out)[i] = v;
+        else
+            DequantOut<OUT>::one(out, i, v);
+    }
+}
+
+static int log2_exact(int v) {
+    int s = 0;
+    while ((1 << s) < v) ++s;
+    return s;
+}
+
+static int grid_for(int64_t work_items, int threads, int per_sm) {
+    int sms = 148;
+    device_sm_count(&sms);
+    int64_t blocks = (work_items + threads - 1) / threads;
+    const int64_t cap = (int64_t)sms * per_sm;
+    if (blocks > cap) blocks = cap;
+    if (blocks < 1) blocks = 1;
+    return (int)blocks;
+}
+
+cudaError_t quantize_launch(const float* W, int64_t n, int blocksize, const float* code, uint8_t* packed,
+                            float* absmax, cudaStream_t stream) {
+    const int64_t nblocks = (n + blocksize - 1) / blocksize;
+    const int threads = 256;
+    const int grid = grid_for(nblocks * 32, threads, 8);
+    q4_quantize_kernel<<<grid, threads, 0, stream>>>(W, n, log2_exact(blocksize), code, packed, absmax, nblocks);
+    return cudaGetLastError();
+}
+
+cudaError_t dequantize_launch(const uint8_t* packed, const float* absmax, const float* code, int64_t n,
+                              int blocksize, int out_dtype, void* out, cudaStream_t stream) {
+    const int threads = 256;
+    const int64_t items = (n >> 5) > 0 ? (n >> 5) : 1;
+    const int grid = grid_for(items, threads, 8);
+    const int sh = log2_exact(blocksize);
+    if (out_dtype == 0)
+        q4_dequant_kernel<0><<<grid, threads, 0, stream>>>(packed, absmax, code, n, sh, out);
+    else if (out_dtype == 1)
+        q4_dequant_kernel<1><<<grid, threads, 0, stream>>>(packed, absmax, code, n, sh, out);
+    else
+        q4_dequant_kernel<2><<<grid, threads, 0, stream>>>(packed, absmax, code, n, sh, out);
+    return cudaGetLastError();
+}
+
+}  // namespace q4

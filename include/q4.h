@@ -1,0 +1,177 @@
+/*
+ * q4.h -- C ABI of libq4: blockwise 4-bit weight quantization,
+ * dequantization and the fused dequantize + skinny matmul
+ *     C[M,N] = A[M,K] . dequant(W)[N,K]^T,   1 <= M <= 16,
+ * the decode-time hot path of a 4-bit quantized linear layer, hand-written
+ * for NVIDIA B200 (sm_100a).
+ *
+ * Source of the method: bitsandbytes PR #1920, "[ROCm] Optimize
+ * kgemm_4bit_inference_naive for ROCm, use it for batch sizes other than 1":
+ *   - "Technical details / Kernel optimization": the fused dequantize +
+ *     matmul kernel streams packed 4-bit weights and dequantizes them on the
+ *     fly;
+ *   - "Fused path support for M > 1": the op receives the real number of
+ *     activation rows M and runs the fused kernel for small M > 1 instead of
+ *     only the vector case; split dequantize + GEMM takes over past a
+ *     GPU-specific crossover;
+ *   - the maintainer's reply: weights index a 16-entry "NF4/FP4 dtype LUT",
+ *     blocksize 64 is the default and other blocksizes are supported,
+ *     accumulation is fp32, only the torch inference ("TN") layout W[N,K]
+ *     is supported, activations fp16/bf16 (fp32 for the SIMT kernel).
+ *
+ * Data format (the pages print no byte layout; this is the plainest
+ * reading they support):
+ *   - W is row-major [N, K], flattened to n = N*K elements;
+ *   - absmax: one fp32 per contiguous block of `blocksize` flattened
+ *     elements (ceil(n / blocksize) values); the last block may be short;
+ *   - packed: ceil(n / 2) bytes, two 4-bit codes per byte, the HIGH nibble
+ *     holds the even element;
+ *   - code: 16 fp32 values (the lookup table), caller supplied.
+ *   - a weight is w[i] = code[idx[i]] * absmax[i / blocksize] (fp32).
+ *
+ * Conventions for every entry point:
+ *   - All pointers are caller-owned DEVICE memory unless stated otherwise;
+ *     the library allocates nothing and keeps no state besides a per-device
+ *     cache of kernel attributes.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream); calls are
+ *     asynchronous on it.  Argument errors are reported synchronously by
+ *     the return value before anything is enqueued.
+ *   - Return value: a q4_status.  A launch failure returns Q4_ERR_CUDA after
+ *     draining the runtime's last-error state, so no error the library
+ *     caused is left pending for the caller.  Kernels never trap and never
+ *     wait on other kernels.
+ *   - Q4_ERR_UNSUPPORTED means "valid request this library does not run";
+ *     it is the caller's cue to use a split dequantize + dense GEMM path.
+ */
+#ifndef Q4_H_
+#define Q4_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    Q4_OK = 0,
+    Q4_ERR_INVALID_ARG = 1, /* null pointer, negative size, bad blocksize or dtype */
+    Q4_ERR_UNSUPPORTED = 2, /* M > 16, K % blocksize != 0, fp32 activations     */
+    Q4_ERR_MISALIGNED = 3,  /* a pointer misses the alignment stated below      */
+    Q4_ERR_CUDA = 4,        /* a CUDA call or kernel launch failed              */
+    Q4_ERR_WORKSPACE = 5    /* GEMM workspace missing or smaller than required  */
+} q4_status;
+
+typedef enum { Q4_BF16 = 0, Q4_FP16 = 1, Q4_FP32 = 2 } q4_dtype;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* q4_status_string(int status);
+
+/*
+ * Blockwise 4-bit quantization (inverse of the dequantize step the fused
+ * kernel performs; the pages quantize offline).
+ *   W       fp32 [n], 16-byte aligned
+ *   n       number of elements, >= 0 (0 is a no-op)
+ *   blocksize  power of two in [32, 4096]
+ *   code    fp32 [16], 4-byte aligned; any values (a strict table order is
+ *           not required)
+ *   packed  uint8 [ceil(n/2)] output; for odd n the final low nibble is 0
+ *   absmax  fp32 [ceil(n/blocksize)] output, 4-byte aligned
+ * Per block: absmax = max|w| (exact); x = w / absmax, one correctly rounded
+ * fp32 division (x = 0 for an all-zero block); idx = argmin_j |x - code[j]|
+ * on fp32 differences, ties to the lowest j.  Non-finite W is undefined.
+ */
+int q4_quantize_blockwise(const float* W, int64_t n, int blocksize, const float* code,
+                          uint8_t* packed, float* absmax, void* stream);
+
+/*
+ * Blockwise 4-bit dequantization (the building block of the split path of
+ * PR #1920, "split dequantize + GEMM").
+ *   packed  uint8 [ceil(n/2)], 16-byte aligned
+ *   absmax  fp32 [ceil(n/blocksize)], 4-byte aligned
+ *   code    fp32 [16], 4-byte aligned
+ *   n, blocksize  as for quantize
+ *   out_dtype  Q4_BF16, Q4_FP16 or Q4_FP32
+ *   out     [n] elements of out_dtype, 16-byte aligned
+ * out[i] = round_to_nearest_even_out_dtype(code[idx_i] * absmax[i/blocksize])
+ * with the product formed once in fp32 (bit-exact, -0.0 kept).
+ */
+int q4_dequantize_blockwise(const uint8_t* packed, const float* absmax, const float* code,
+                            int64_t n, int blocksize, int out_dtype, void* out, void* stream);
+
+/*
+ * Bytes of device workspace q4_gemm_skinny needs for this problem on the
+ * CURRENT device (host-only query; never enqueues work).  Writes 0 when no
+ * workspace is needed.  Same argument rules as q4_gemm_skinny.
+ */
+int q4_gemm_workspace_size(int M, int N, int K, int blocksize, int act_dtype, size_t* bytes);
+
+/*
+ * Fused dequantize + skinny matmul (PR #1920's kgemm_4bit_inference_naive
+ * generalised to M > 1, "Fused path support for M > 1"):
+ *     out[m, n] = round_rn_act( sum_k A[m,k] * code[idx(n,k)] * absmax(n,k) )
+ * accumulated in fp32 (codes enter the tensor-core contraction rounded to
+ * the activation dtype; the per-block absmax scale is applied in fp32).
+ *   A        [M, K] act_dtype, row-major contiguous, 16-byte aligned
+ *   Wpacked  uint8 [N*K/2] (rows of K/2 bytes), 16-byte aligned
+ *   absmax   fp32 [N*K/blocksize], 4-byte aligned
+ *   code     fp32 [16], 4-byte aligned
+ *   M        0..16 (0 is a no-op; > 16 -> Q4_ERR_UNSUPPORTED)
+ *   N, K     >= 0; K % blocksize == 0 (else Q4_ERR_UNSUPPORTED); N = 0 is
+ *            a no-op; K = 0 writes zeros
+ *   blocksize  power of two in [32, 4096]
+ *   act_dtype  Q4_BF16 or Q4_FP16 (Q4_FP32 -> Q4_ERR_UNSUPPORTED)
+ *   out      [M, N] act_dtype, row-major, 16-byte aligned
+ *   workspace  device scratch of at least q4_gemm_workspace_size() bytes,
+ *            16-byte aligned, ZERO-FILLED before its first use; every call
+ *            leaves it zero-filled again.  Calls that share a workspace
+ *            must not overlap on the GPU (use one per stream).
+ * The result is deterministic: partial sums are combined in a fixed order.
+ */
+int q4_gemm_skinny(const void* A, const uint8_t* Wpacked, const float* absmax, const float* code,
+                   int M, int N, int K, int blocksize, int act_dtype, void* out, void* workspace,
+                   size_t workspace_bytes, void* stream);
+
+/* Launch-table entry chosen for a GEMM problem (host-only, for reporting and
+ * tests).  `num_sms` <= 0 means "the current device's SM count". */
+typedef struct {
+    int math;          /* 1 = tensor-core (mma.sync m16n8k16), 2 = CUDA-core FMA */
+    int sub_block;     /* k-width of one work unit: min(blocksize, 64)           */
+    int m_pad;         /* M padded to the MMA column count: 8 or 16              */
+    int rows_per_tile; /* weight rows per work unit                              */
+    int warps;         /* warps per CTA                                          */
+    int ctas;          /* persistent CTAs (<= SM count, <= number of units)      */
+    int tiles;         /* ceil(N / rows_per_tile)                                */
+    int64_t units;     /* tiles * (K / sub_block)                                */
+    size_t smem_bytes; /* dynamic shared memory per CTA                          */
+    size_t workspace_bytes;
+} q4_gemm_plan_t;
+
+int q4_gemm_plan(int M, int N, int K, int blocksize, int act_dtype, int num_sms,
+                 q4_gemm_plan_t* plan);
+
+/*
+ * Same as q4_gemm_skinny with explicit launch-table overrides; any field
+ * <= 0 keeps the table's choice.  math: 1 tensor-core, 2 CUDA-core FMA
+ * (M <= 4 only).  Used to measure the choices the launch table makes.
+ */
+int q4_gemm_skinny_ex(const void* A, const uint8_t* Wpacked, const float* absmax,
+                      const float* code, int M, int N, int K, int blocksize, int act_dtype,
+                      void* out, void* workspace, size_t workspace_bytes, void* stream, int math,
+                      int ctas, int warps);
+
+/*
+ * Work partition used by the GEMM (host-callable so it can be checked
+ * without a GPU): `total` units split into `parts` contiguous ranges,
+ * part p owning [q4_partition_start(total, parts, p),
+ *                q4_partition_start(total, parts, p + 1)).
+ * q4_partition_owner returns the part owning unit u (0 <= u < total).
+ */
+int64_t q4_partition_start(int64_t total, int parts, int part);
+int q4_partition_owner(int64_t total, int parts, int64_t u);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* Q4_H_ */

@@ -1,0 +1,113 @@
+"""Host-only checks of libq4's C ABI (no GPU work is enqueued here).
+
+* the library loads and exports every function include/q4.h declares;
+* argument validation answers before any CUDA call;
+* the launch table and the stream-K work partition keep their invariants.
+"""
+import ctypes
+import os
+
+import pytest
+
+from bit_weight_dequant_b200 import binding as b
+from bit_weight_dequant_b200 import inputs
+
+pytestmark = pytest.mark.skipif(not os.path.exists(b.LIB_PATH), reason="libq4.so not built")
+
+
+def test_exports_every_declared_symbol():
+    names = b.declared_functions()
+    assert {"q4_quantize_blockwise", "q4_dequantize_blockwise", "q4_gemm_skinny"} <= set(names)
+    L = b.lib()
+    for n in names:
+        assert hasattr(L, n), f"libq4.so does not export {n}"
+
+
+def test_status_strings():
+    for s in range(6):
+        assert b.status_string(s).startswith("Q4_")
+    assert b.status_string(99) == "unknown q4 status"
+
+
+ALIGNED = ctypes.c_void_p(1 << 20)      # never dereferenced: every call below returns before launching
+MISALIGNED = ctypes.c_void_p((1 << 20) + 4)
+
+
+def test_quantize_validation():
+    L = b.lib()
+    q = L.q4_quantize_blockwise
+    assert q(None, 16, 64, ALIGNED, ALIGNED, ALIGNED, None) == b.Q4_ERR_INVALID_ARG
+    assert q(ALIGNED, -1, 64, ALIGNED, ALIGNED, ALIGNED, None) == b.Q4_ERR_INVALID_ARG
+    for bs in (0, 16, 48, 8192):
+        assert q(ALIGNED, 16, bs, ALIGNED, ALIGNED, ALIGNED, None) == b.Q4_ERR_INVALID_ARG
+    assert q(MISALIGNED, 16, 64, ALIGNED, ALIGNED, ALIGNED, None) == b.Q4_ERR_MISALIGNED
+    assert q(ALIGNED, 0, 64, ALIGNED, ALIGNED, ALIGNED, None) == b.Q4_OK   # empty input: no-op
+
+
+def test_dequantize_validation():
+    d = b.lib().q4_dequantize_blockwise
+    assert d(ALIGNED, ALIGNED, ALIGNED, 16, 64, 3, ALIGNED, None) == b.Q4_ERR_INVALID_ARG
+    assert d(ALIGNED, ALIGNED, ALIGNED, 16, 64, 0, None, None) == b.Q4_ERR_INVALID_ARG
+    assert d(MISALIGNED, ALIGNED, ALIGNED, 16, 64, 0, ALIGNED, None) == b.Q4_ERR_MISALIGNED
+    assert d(ALIGNED, ALIGNED, ALIGNED, 16, 64, 0, MISALIGNED, None) == b.Q4_ERR_MISALIGNED
+    assert d(ALIGNED, ALIGNED, ALIGNED, 0, 64, 1, ALIGNED, None) == b.Q4_OK
+
+
+def test_injected_launch_failure_reports_cuda_error(monkeypatch):
+    monkeypatch.setenv("Q4_TEST_FAIL_LAUNCH", "1")
+    L = b.lib()
+    assert L.q4_quantize_blockwise(ALIGNED, 16, 64, ALIGNED, ALIGNED, ALIGNED, None) == b.Q4_ERR_CUDA
+    assert L.q4_dequantize_blockwise(ALIGNED, ALIGNED, ALIGNED, 16, 64, 0, ALIGNED, None) == b.Q4_ERR_CUDA
+    monkeypatch.setenv("Q4_TEST_FAIL_LAUNCH", "0")
+    assert L.q4_quantize_blockwise(ALIGNED, 0, 64, ALIGNED, ALIGNED, ALIGNED, None) == b.Q4_OK
+
+
+def test_gemm_validation_before_cuda():
+    g = b.lib().q4_gemm_skinny
+    args = [ALIGNED] * 4
+    # (M, N, K, bs, dtype) -> status; all decided before the device is queried
+    cases = {(17, 64, 4096, 64, 0): b.Q4_ERR_UNSUPPORTED,
+             (1, 64, 4000, 64, 0): b.Q4_ERR_UNSUPPORTED,
+             (1, 64, 4096, 64, 2): b.Q4_ERR_UNSUPPORTED,
+             (-1, 64, 4096, 64, 0): b.Q4_ERR_INVALID_ARG,
+             (1, -5, 4096, 64, 0): b.Q4_ERR_INVALID_ARG,
+             (1, 64, 4096, 96, 0): b.Q4_ERR_INVALID_ARG,
+             (1, 64, 4096, 64, 7): b.Q4_ERR_INVALID_ARG}
+    for (M, N, K, bs, dt), want in cases.items():
+        assert g(*args, M, N, K, bs, dt, ALIGNED, None, 0, None) == want, (M, N, K, bs, dt)
+    assert g(None, *args[1:], 1, 64, 4096, 64, 0, ALIGNED, None, 0, None) == b.Q4_ERR_INVALID_ARG
+    ex = b.lib().q4_gemm_skinny_ex
+    assert ex(*args, 1, 64, 4096, 64, 0, ALIGNED, None, 0, None, 3, 0, 0) == b.Q4_ERR_INVALID_ARG
+    assert ex(*args, 12, 64, 4096, 64, 0, ALIGNED, None, 0, None, 0, 0, 16) == b.Q4_ERR_UNSUPPORTED
+
+
+@pytest.mark.parametrize("wl", list(inputs.workloads()))
+def test_launch_table_invariants(wl):
+    for c in inputs.workloads()[wl].cases:
+        p = b.q4_gemm_plan(c.M, c.N, c.K, c.blocksize, num_sms=148)
+        assert p["math"] == 1
+        assert p["sub_block"] == min(c.blocksize, 64)
+        assert p["m_pad"] == (8 if c.M <= 8 else 16)
+        assert p["tiles"] == -(-c.N // p["rows_per_tile"])
+        assert p["units"] == p["tiles"] * (c.K // p["sub_block"])
+        assert 1 <= p["ctas"] <= min(148, p["units"])
+        assert p["smem_bytes"] <= 227 * 1024
+        slot = p["rows_per_tile"] * p["m_pad"] * 4
+        want_ws = 0 if p["ctas"] == 1 else (-(-p["tiles"] * 4 // 256) * 256 + p["ctas"] * 2 * slot)
+        assert p["workspace_bytes"] == want_ws
+
+
+@pytest.mark.parametrize("total,parts", [(1, 1), (1, 16), (7, 3), (40, 148), (4096, 148), (57344, 148),
+                                         (155200, 148), (13, 16), (1000003, 2368)])
+def test_partition_invariants(total, parts):
+    L = b.lib()
+    starts = [L.q4_partition_start(total, parts, p) for p in range(parts + 1)]
+    assert starts[0] == 0 and starts[-1] == total
+    sizes = [starts[p + 1] - starts[p] for p in range(parts)]
+    assert min(sizes) >= 0 and max(sizes) - min(sizes) <= 1, "ranges must be balanced to one unit"
+    probe = sorted({0, total - 1, total // 2, total // 3} | set(s for s in starts if s < total) |
+                   set(s - 1 for s in starts if 0 < s <= total))
+    for u in probe:
+        p = L.q4_partition_owner(total, parts, u)
+        assert starts[p] <= u < starts[p + 1], (u, p)
+    assert L.q4_partition_owner(total, parts, total) == -1

@@ -1,0 +1,132 @@
+"""GPU parity of the fused dequantize + skinny GEMM against the oracle at
+sizes the oracle finishes quickly: every output element must satisfy
+|gpu - y| <= 1e-2 * sum_k |a w| + ulp(y).  The operation is the fused path of
+bitsandbytes PR #1920 ("Fused path support for M > 1")."""
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from bit_weight_dequant_b200 import binding as q4
+from bit_weight_dequant_b200 import inputs
+from bit_weight_dequant_b200.inputs import Case
+from parity import TORCH_ACT, bits_of, run_case
+
+pytestmark = pytest.mark.gpu
+
+SHAPES = [(1, 64), (12, 2560), (64, 64), (65, 128), (100, 320), (513, 1024), (320, 1280), (257, 4096), (130, 192)]
+
+
+@pytest.mark.parametrize("M", [1, 2, 3, 4, 5, 8, 9, 12, 16])
+@pytest.mark.parametrize("N,K", SHAPES)
+def test_gemm_bf16_normal(cuda_device, M, N, K):
+    run_case(Case(M, N, K), seed=1000 + M * 7 + N + K, device=cuda_device)
+
+
+@pytest.mark.parametrize("M", [1, 4, 13])
+@pytest.mark.parametrize("bs", [32, 128, 256, 1024])
+def test_gemm_blocksizes(cuda_device, M, bs):
+    run_case(Case(M, 200, 2048, blocksize=bs), seed=2000 + bs + M, device=cuda_device)
+
+
+@pytest.mark.parametrize("M", [1, 5, 16])
+@pytest.mark.parametrize("act,table", [("fp16", "normal"), ("bf16", "uniform"), ("fp16", "uniform")])
+def test_gemm_dtypes_tables(cuda_device, M, act, table):
+    run_case(Case(M, 300, 1536, act=act, table=table), seed=3000 + M, device=cuda_device)
+
+
+@pytest.mark.parametrize("M", [1, 8])
+def test_gemm_outliers(cuda_device, M):
+    run_case(Case(M, 256, 2048, outliers=True), seed=4000 + M, device=cuda_device)
+
+
+# Launch-table overrides: tiles cut between CTAs (global fix-up) and between
+# warps (shared-memory combine), empty warp ranges, single CTA.
+@pytest.mark.parametrize("ctas", [1, 2, 3, 7, 64, 148])
+@pytest.mark.parametrize("warps", [8, 16])
+@pytest.mark.parametrize("M", [1, 6])
+def test_gemm_partition_overrides(cuda_device, ctas, warps, M):
+    run_case(Case(M, 257, 1280), seed=5000 + ctas, device=cuda_device, check_quantizer=False, ctas=ctas, warps=warps)
+
+
+@pytest.mark.parametrize("ctas", [1, 5, 33])
+@pytest.mark.parametrize("M", [9, 16])
+def test_gemm_partition_overrides_m16(cuda_device, ctas, M):
+    run_case(Case(M, 190, 960), seed=6000 + ctas, device=cuda_device, check_quantizer=False, ctas=ctas, warps=8)
+
+
+def _problem(device, M=3, N=300, K=1024, bs=64, seed=7):
+    code = inputs.code_normal_quantile()
+    W = inputs.weights(N, K, seed)
+    packed, absmax = oracle.quantize(W, bs, code)
+    A = inputs.activations(M, K, torch.bfloat16, seed).to(device)
+    return (A, torch.from_numpy(packed).to(device), torch.from_numpy(absmax).to(device),
+            torch.from_numpy(code).to(device), N, K, bs)
+
+
+def test_deterministic_and_workspace_left_zero(cuda_device):
+    A, P, Am, C, N, K, bs = _problem(cuda_device)
+    ws = q4.Workspace(cuda_device)
+    outs = [q4.q4_gemm_skinny(A, P, Am, C, N, K, bs, workspace=ws, ctas=5) for _ in range(3)]
+    torch.cuda.synchronize()
+    for o in outs[1:]:
+        assert torch.equal(o.view(torch.int16), outs[0].view(torch.int16))
+    assert ws.buf.numel() > 0 and int(ws.buf.count_nonzero()) == 0
+
+
+def test_empty_and_degenerate(cuda_device):
+    A, P, Am, C, N, K, bs = _problem(cuda_device)
+    out = q4.q4_gemm_skinny(A[:0], P, Am, C, N, K, bs)          # M = 0
+    assert out.shape == (0, N)
+    out = q4.q4_gemm_skinny(A, P, Am, C, 0, K, bs)             # N = 0
+    assert out.shape == (A.shape[0], 0)
+    z = torch.empty((A.shape[0], 0), dtype=A.dtype, device=cuda_device)
+    out = torch.full((A.shape[0], N), 7.0, dtype=A.dtype, device=cuda_device)
+    q4.q4_gemm_skinny(z, P, Am, C, N, 0, bs, out=out)          # K = 0 -> zeros
+    torch.cuda.synchronize()
+    assert int(out.count_nonzero()) == 0
+
+
+def test_error_paths_leave_no_sticky_error(cuda_device, monkeypatch):
+    A, P, Am, C, N, K, bs = _problem(cuda_device)
+    ref = q4.q4_gemm_skinny(A, P, Am, C, N, K, bs)
+    Amis = torch.zeros(A.numel() + 1, dtype=A.dtype, device=cuda_device)[1:].view_as(A)
+    with pytest.raises(q4.Q4Error) as e:
+        q4.q4_gemm_skinny(Amis, P, Am, C, N, K, bs)
+    assert e.value.status == q4.Q4_ERR_MISALIGNED
+    L = q4.lib()
+    out = torch.empty_like(ref)
+    ptr = lambda t: ctypes.c_void_p(t.data_ptr())
+    need = q4.q4_gemm_workspace_size(A.shape[0], N, K, bs, A.dtype)
+    if need:
+        assert L.q4_gemm_skinny(ptr(A), ptr(P), ptr(Am), ptr(C), A.shape[0], N, K, bs, 0, ptr(out), None, 0,
+                                None) == q4.Q4_ERR_WORKSPACE
+    monkeypatch.setenv("Q4_TEST_FAIL_LAUNCH", "1")
+    with pytest.raises(q4.Q4Error) as e:
+        q4.q4_gemm_skinny(A, P, Am, C, N, K, bs)
+    assert e.value.status == q4.Q4_ERR_CUDA
+    monkeypatch.delenv("Q4_TEST_FAIL_LAUNCH")
+    again = q4.q4_gemm_skinny(A, P, Am, C, N, K, bs)
+    torch.cuda.synchronize()
+    assert torch.equal(again.view(torch.int16), ref.view(torch.int16))
+
+
+def test_one_hot_activation_selects_dequantized_column(cuda_device):
+    """A = e_k: out[0, n] = w[n, k] up to the kernel's rounding of the code to
+    bf16 before the MMA (relative 2^-9) and the final bf16 rounding, i.e.
+    within one bf16 ulp of the oracle's bf16(w[n, k])."""
+    M, N, K, bs = 1, 300, 1024, 64
+    code = inputs.code_normal_quantile()
+    packed, absmax = oracle.quantize(inputs.weights(N, K, 7), bs, code)
+    want_all = oracle.decode(oracle.dequantize(packed, absmax, code, N * K, bs, oracle.BF16), oracle.BF16)
+    want_all = want_all.reshape(N, K)
+    P, Am, C = (torch.from_numpy(x).to(cuda_device) for x in (packed, absmax, code))
+    for k in (0, 17, 64, K - 1):
+        e = torch.zeros((1, K), dtype=torch.bfloat16, device=cuda_device)
+        e[0, k] = 1.0
+        out = q4.q4_gemm_skinny(e, P, Am, C, N, K, bs)
+        want = want_all[:, k]
+        got = out[0].to(torch.float64).cpu().numpy()
+        assert np.all(np.abs(got - want) <= oracle.ulp(want, oracle.BF16)), k
