@@ -201,7 +201,10 @@ def run_ours(args, world, rank, local):
     torch.cuda.set_device(device)
     wl = inputs.workloads()[args.workload]
     peak, peak_src = hbm_peak()
-    layers = [Layer(c, inputs.seed_for(wl.index, c.M) + i, device) for i, c in enumerate(wl.cases)]
+    cases = [(i, c) for i, c in enumerate(wl.cases) if not args.only or c.tag in args.only.split(",")]
+    if not cases:
+        raise SystemExit(f"--only {args.only!r} matches no case of {args.workload}")
+    layers = [Layer(c, inputs.seed_for(wl.index, c.M) + i, device) for i, c in cases]
     torch.cuda.synchronize()
     step_bytes = sum(L.bytes for L in layers)
     stream = torch.cuda.Stream(device)
@@ -279,7 +282,7 @@ def run_ours(args, world, rank, local):
 
     # End to end through the public Python API: per step, H2D of the
     # activations from pinned memory, the four calls, D2H of the outputs.
-    e2e_steps = max(1, min(args.steps, 2000))
+    e2e_steps = 0 if args.no_e2e else max(1, min(args.steps, 2000))
     torch.cuda.synchronize()
     barrier(world)
     t0 = time.perf_counter()
@@ -290,7 +293,7 @@ def run_ours(args, world, rank, local):
             L.out_host.copy_(L.out, non_blocking=True)
     torch.cuda.synchronize()
     e2e_s = max_over_ranks(time.perf_counter() - t0, world, device)
-    e2e_value = world * step_bytes * e2e_steps / e2e_s / 1e9
+    e2e_value = world * step_bytes * e2e_steps / e2e_s / 1e9 if e2e_steps else None
     h2d = sum(L.A_host.numel() * L.A_host.element_size() for L in layers)
     d2h = sum(L.out_host.numel() * L.out_host.element_size() for L in layers)
 
@@ -302,7 +305,7 @@ def run_ours(args, world, rank, local):
         "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms_step, 5), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": wl.name, "M": sorted({c.M for c in wl.cases}), "blocksize": 64,
+        "config": {"workload": wl.name + (f" [only {args.only}]" if args.only else ""), "M": sorted({c.M for c in wl.cases}), "blocksize": 64,
                    "code_table": "normal-quantile", "activations": "bf16 ~N(0,1)", "weights": "N(0,0.02^2) fp32 -> 4-bit",
                    "l2": f"inputs larger than L2: {total_weight_bytes / 1e6:.0f} MB of packed weights per step "
                          f"vs {L2_BYTES / 2**20:.0f} MiB L2, no flush",
@@ -313,7 +316,7 @@ def run_ours(args, world, rank, local):
                      "peak_source": peak_src, "kernel": "q4_gemm_mma_kernel",
                      "per_unit": "0.5 B per weight (codes) + 4/bs B (absmax) + A and C once"},
         "per_shape": per_shape,
-        "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d,
+        "e2e": {"value": round(e2e_value, 2) if e2e_value else None, "unit": "GB/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "steps": e2e_steps,
                 "api": "bit_weight_dequant_b200.q4_gemm_skinny (ctypes -> libq4 C ABI), wall clock"},
         "gpu_launches": args.steps * len(layers),
@@ -413,6 +416,8 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--reference-seconds", type=float, default=60.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end leg (profiling runs)")
+    ap.add_argument("--only", default="", help="comma-separated case tags of the workload to run (profiling)")
     args = ap.parse_args()
     if args.warmup < 3:
         log("note: warm-up raised to 3 steps (minimum)")

@@ -33,8 +33,8 @@ class Q4Error(RuntimeError):
 class q4_gemm_plan_t(ctypes.Structure):
     _fields_ = [("math", ctypes.c_int), ("sub_block", ctypes.c_int), ("m_pad", ctypes.c_int),
                 ("rows_per_tile", ctypes.c_int), ("warps", ctypes.c_int), ("ctas", ctypes.c_int),
-                ("tiles", ctypes.c_int), ("units", ctypes.c_int64), ("smem_bytes", ctypes.c_size_t),
-                ("workspace_bytes", ctypes.c_size_t)]
+                ("depth", ctypes.c_int), ("l2_prefetch", ctypes.c_int), ("tiles", ctypes.c_int),
+                ("units", ctypes.c_int64), ("smem_bytes", ctypes.c_size_t), ("workspace_bytes", ctypes.c_size_t)]
 
 
 _lib = None
@@ -54,7 +54,7 @@ def lib() -> ctypes.CDLL:
         L.q4_dequantize_blockwise.argtypes = [P, P, P, i64, ci, ci, P, P]
         L.q4_gemm_workspace_size.argtypes = [ci, ci, ci, ci, ci, ctypes.POINTER(sz)]
         L.q4_gemm_skinny.argtypes = [P, P, P, P, ci, ci, ci, ci, ci, P, P, sz, P]
-        L.q4_gemm_skinny_ex.argtypes = [P, P, P, P, ci, ci, ci, ci, ci, P, P, sz, P, ci, ci, ci]
+        L.q4_gemm_skinny_ex.argtypes = [P, P, P, P, ci, ci, ci, ci, ci, P, P, sz, P, ctypes.POINTER(q4_gemm_plan_t)]
         L.q4_gemm_plan.argtypes = [ci, ci, ci, ci, ci, ci, ctypes.POINTER(q4_gemm_plan_t)]
         L.q4_partition_start.argtypes = [i64, ci, ci]
         L.q4_partition_start.restype = i64
@@ -132,7 +132,8 @@ def q4_gemm_plan(M: int, N: int, K: int, blocksize: int, act_dtype: torch.dtype 
 class Workspace:
     """Zero-filled device scratch for q4_gemm_skinny, grown on demand.
 
-    The library returns it zero-filled after every call; one per stream."""
+    Every call returns the workspace's tile counters to zero, so it is
+    zero-filled once, at allocation; one per stream."""
 
     def __init__(self, device):
         self.device = torch.device(device)
@@ -146,6 +147,15 @@ class Workspace:
 
 _workspaces: dict = {}
 
+MAX_SLOT_BYTES = 4096     # partial-sum slot of the largest variant (64 rows x 16 columns x fp32)
+
+
+def workspace_counter_offset(device) -> int:
+    """Byte offset of the per-tile counters inside a GEMM workspace (two
+    partial-sum slots per SM come first; see q4_gemm_skinny in q4.h)."""
+    return torch.cuda.get_device_properties(device).multi_processor_count * 2 * MAX_SLOT_BYTES
+
+
 
 def _default_workspace(device) -> Workspace:
     key = (torch.device(device), torch.cuda.current_stream(device).cuda_stream)
@@ -155,19 +165,35 @@ def _default_workspace(device) -> Workspace:
     return ws
 
 
+def overrides(**kw) -> q4_gemm_plan_t | None:
+    """Launch-table overrides (math, warps, ctas, depth, l2_prefetch); None if empty."""
+    kw = {k: v for k, v in kw.items() if v}
+    if not kw:
+        return None
+    ov = q4_gemm_plan_t()
+    for k, v in kw.items():
+        setattr(ov, k, int(v))
+    return ov
+
+
 def q4_gemm_skinny(A: torch.Tensor, Wpacked: torch.Tensor, absmax: torch.Tensor, code: torch.Tensor, N: int,
                    K: int, blocksize: int, out: torch.Tensor | None = None, workspace: Workspace | None = None,
-                   math: int = 0, ctas: int = 0, warps: int = 0) -> torch.Tensor:
-    """out[M, N] = A[M, K] . dequant(W)[N, K]^T on the GPU (fused kernel)."""
+                   **launch) -> torch.Tensor:
+    """out[M, N] = A[M, K] . dequant(W)[N, K]^T on the GPU (fused kernel).
+
+    ``launch`` may hold launch-table overrides (math, warps, ctas, depth,
+    l2_prefetch) for measurements; by default the table decides."""
     M = A.shape[0] if A.dim() == 2 else 1
     if out is None:
         out = torch.empty((M, N), dtype=A.dtype, device=A.device)
     act = _TORCH_TO_Q4[A.dtype]
     need = ctypes.c_size_t(0)
     _check(lib().q4_gemm_workspace_size(M, N, K, blocksize, act, ctypes.byref(need)), "q4_gemm_workspace_size")
-    ws = (workspace or _default_workspace(A.device)).get(need.value) if need.value else None
+    nbytes = need.value
+    ws = (workspace or _default_workspace(A.device)).get(nbytes) if nbytes else None
+    ov = overrides(**launch)
     rc = lib().q4_gemm_skinny_ex(_ptr(A), _ptr(Wpacked), _ptr(absmax), _ptr(code), M, N, K, blocksize, act,
                                  _ptr(out), _ptr(ws), ws.numel() if ws is not None else 0, _stream(A.device),
-                                 math, ctas, warps)
+                                 ctypes.byref(ov) if ov is not None else None)
     _check(rc, "q4_gemm_skinny")
     return out

@@ -72,41 +72,51 @@ static int from_cuda(cudaError_t e) {
 
 static size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
-// Validates a GEMM request.  Returns Q4_OK and fills `out` with the launch
-// table's choice (and the problem's unit counts) when it can run.
-static int gemm_choose(int M, int N, int K, int blocksize, int act_dtype, int num_sms, int math, int ctas,
-                       int warps, GemmChoice* ch, int* tiles, int64_t* units, size_t* ws_bytes) {
+// Workspace layout: [partial slots: sms x 2 x kMaxSlotBytes][counters: one int per tile].
+// The counters sit at an offset that depends only on the SM count, so
+// scratch written by a call of one shape never lands on another shape's
+// counters; each call returns the counters it used to zero.
+static size_t ws_counter_offset(int sms) { return (size_t)sms * 2 * kMaxSlotBytes; }
+
+// Validates a GEMM request.  Returns Q4_OK and fills `ch` with the launch
+// table's choice (with `ov` applied) and the problem's unit counts.
+static int gemm_choose(int M, int N, int K, int blocksize, int act_dtype, int num_sms, const q4_gemm_plan_t* ov,
+                       GemmChoice* ch, int* tiles, int64_t* units, size_t* ws_bytes, int* sms_out) {
     if (M < 0 || N < 0 || K < 0) return Q4_ERR_INVALID_ARG;
     if (!is_pow2_blocksize(blocksize)) return Q4_ERR_INVALID_ARG;
     if (act_dtype != Q4_BF16 && act_dtype != Q4_FP16 && act_dtype != Q4_FP32) return Q4_ERR_INVALID_ARG;
-    if (math < 0 || math > 2 || ctas < 0 || warps < 0) return Q4_ERR_INVALID_ARG;
+    if (ov && (ov->math > 2 || ov->l2_prefetch > 256)) return Q4_ERR_INVALID_ARG;
     if (M > 16 || act_dtype == Q4_FP32 || K % blocksize != 0) return Q4_ERR_UNSUPPORTED;
     GemmChoice c{};
     c.math = 1;
-    if (math == 2) return Q4_ERR_UNSUPPORTED;  // CUDA-core variant not built in this library version
     c.sub_block = blocksize < 64 ? blocksize : 64;
     c.m_pad = M <= 8 ? 8 : 16;
     c.rows_per_tile = 64;
     c.warps = c.m_pad == 8 ? 16 : 8;
-    if (warps > 0) {
-        if (!(warps == 8 || (warps == 16 && c.m_pad == 8))) return Q4_ERR_UNSUPPORTED;
-        c.warps = warps;
+    c.depth = 1;
+    c.l2pf = 128;
+    if (ov) {
+        if (ov->math > 0) c.math = ov->math;
+        if (ov->warps > 0) c.warps = ov->warps;
+        if (ov->depth > 0) c.depth = ov->depth;
+        if (ov->l2_prefetch > 0) c.l2pf = ov->l2_prefetch == 1 ? 0 : ov->l2_prefetch;
     }
-    const int t = N > 0 ? (N + c.rows_per_tile - 1) / c.rows_per_tile : 0;
-    const int64_t u = (int64_t)t * (K / c.sub_block);
+    if (c.math != 1 || !gemm_variant_exists(act_dtype, c)) return Q4_ERR_UNSUPPORTED;
     int sms = num_sms;
     if (sms <= 0 && device_sm_count(&sms) != 0) return Q4_ERR_CUDA;
-    int64_t g = ctas > 0 ? ctas : sms;
+    if (ov && ov->ctas > sms) return Q4_ERR_INVALID_ARG;
+    const int t = N > 0 ? (N + c.rows_per_tile - 1) / c.rows_per_tile : 0;
+    const int64_t u = (int64_t)t * (K / c.sub_block);
+    int64_t g = (ov && ov->ctas > 0) ? ov->ctas : sms;
     if (g > u) g = u;  // every CTA owns at least one unit
     if (g < 1) g = 1;
     c.ctas = (int)g;
     *ch = c;
     *tiles = t;
     *units = u;
-    // Workspace: a counter per tile (256-B aligned), then two partial slots per CTA.
-    *ws_bytes = (c.ctas > 1 && u > 0)
-                    ? align_up((size_t)t * sizeof(int), 256) + (size_t)c.ctas * 2 * gemm_slot_floats(c.m_pad) * 4
-                    : 0;
+    *sms_out = sms;
+    // A problem of one unit never splits a tile, so it needs no workspace.
+    *ws_bytes = u > 1 ? ws_counter_offset(sms) + align_up((size_t)t * sizeof(int), 256) : 0;
     return Q4_OK;
 }
 
@@ -151,10 +161,10 @@ int q4_dequantize_blockwise(const uint8_t* packed, const float* absmax, const fl
 int q4_gemm_plan(int M, int N, int K, int blocksize, int act_dtype, int num_sms, q4_gemm_plan_t* plan) {
     if (!plan) return Q4_ERR_INVALID_ARG;
     GemmChoice ch;
-    int tiles = 0;
+    int tiles = 0, sms = 0;
     int64_t units = 0;
     size_t ws = 0;
-    const int rc = gemm_choose(M, N, K, blocksize, act_dtype, num_sms, 0, 0, 0, &ch, &tiles, &units, &ws);
+    const int rc = gemm_choose(M, N, K, blocksize, act_dtype, num_sms, nullptr, &ch, &tiles, &units, &ws, &sms);
     if (rc != Q4_OK) return rc;
     plan->math = ch.math;
     plan->sub_block = ch.sub_block;
@@ -162,9 +172,11 @@ int q4_gemm_plan(int M, int N, int K, int blocksize, int act_dtype, int num_sms,
     plan->rows_per_tile = ch.rows_per_tile;
     plan->warps = ch.warps;
     plan->ctas = ch.ctas;
+    plan->depth = ch.depth;
+    plan->l2_prefetch = ch.l2pf == 0 ? 1 : ch.l2pf;
     plan->tiles = tiles;
     plan->units = units;
-    plan->smem_bytes = gemm_smem_bytes(ch.sub_block, ch.m_pad, ch.warps);
+    plan->smem_bytes = gemm_smem_bytes(act_dtype == Q4_FP32 ? Q4_BF16 : act_dtype, ch);
     plan->workspace_bytes = ws;
     return Q4_OK;
 }
@@ -172,21 +184,20 @@ int q4_gemm_plan(int M, int N, int K, int blocksize, int act_dtype, int num_sms,
 int q4_gemm_workspace_size(int M, int N, int K, int blocksize, int act_dtype, size_t* bytes) {
     if (!bytes) return Q4_ERR_INVALID_ARG;
     GemmChoice ch;
-    int tiles = 0;
+    int tiles = 0, sms = 0;
     int64_t units = 0;
-    const int rc = gemm_choose(M, N, K, blocksize, act_dtype, 0, 0, 0, 0, &ch, &tiles, &units, bytes);
-    return rc;
+    return gemm_choose(M, N, K, blocksize, act_dtype, 0, nullptr, &ch, &tiles, &units, bytes, &sms);
 }
 
 int q4_gemm_skinny_ex(const void* A, const uint8_t* Wpacked, const float* absmax, const float* code, int M, int N,
                       int K, int blocksize, int act_dtype, void* out, void* workspace, size_t workspace_bytes,
-                      void* stream, int math, int ctas, int warps) {
+                      void* stream, const q4_gemm_plan_t* overrides) {
     if (!A || !Wpacked || !absmax || !code || !out) return Q4_ERR_INVALID_ARG;
     GemmChoice ch;
-    int tiles = 0;
+    int tiles = 0, sms = 0;
     int64_t units = 0;
     size_t need = 0;
-    int rc = gemm_choose(M, N, K, blocksize, act_dtype, 0, math, ctas, warps, &ch, &tiles, &units, &need);
+    int rc = gemm_choose(M, N, K, blocksize, act_dtype, 0, overrides, &ch, &tiles, &units, &need, &sms);
     if (rc != Q4_OK) return rc;
     if (!aligned(A, 16) || !aligned(Wpacked, 16) || !aligned(out, 16) || !aligned(absmax, 4) || !aligned(code, 4))
         return Q4_ERR_MISALIGNED;
@@ -203,10 +214,8 @@ int q4_gemm_skinny_ex(const void* A, const uint8_t* Wpacked, const float* absmax
     p.absmax = absmax;
     p.code = code;
     p.out = out;
-    p.counters = static_cast<int*>(workspace);
-    p.partials = workspace ? reinterpret_cast<float*>(static_cast<char*>(workspace) +
-                                                      align_up((size_t)tiles * sizeof(int), 256))
-                           : nullptr;
+    p.partials = static_cast<float*>(workspace);
+    p.counters = workspace ? reinterpret_cast<int*>(static_cast<char*>(workspace) + ws_counter_offset(sms)) : nullptr;
     p.M = M;
     p.N = N;
     p.K = K;
@@ -225,7 +234,7 @@ int q4_gemm_skinny(const void* A, const uint8_t* Wpacked, const float* absmax, c
                    int K, int blocksize, int act_dtype, void* out, void* workspace, size_t workspace_bytes,
                    void* stream) {
     return q4_gemm_skinny_ex(A, Wpacked, absmax, code, M, N, K, blocksize, act_dtype, out, workspace,
-                             workspace_bytes, stream, 0, 0, 0);
+                             workspace_bytes, stream, nullptr);
 }
 
 int64_t q4_partition_start(int64_t total, int parts, int part) {

@@ -21,6 +21,48 @@ __device__ __forceinline__ uint2 ldg_stream_v2(const void* p) {
     return v;
 }
 
+// Same, with an L2 fetch-size hint: the L2 brings in the whole 128/256-byte
+// span around the 8 bytes requested (the following units of the same rows).
+template <int L2PF>
+__device__ __forceinline__ uint2 ldg_stream_v2_pf(const void* p) {
+    uint2 v;
+    if constexpr (L2PF == 256)
+        asm volatile("ld.global.nc.L1::no_allocate.L2::256B.v2.u32 {%0, %1}, [%2];"
+                     : "=r"(v.x), "=r"(v.y)
+                     : "l"(p));
+    else if constexpr (L2PF == 128)
+        asm volatile("ld.global.nc.L1::no_allocate.L2::128B.v2.u32 {%0, %1}, [%2];"
+                     : "=r"(v.x), "=r"(v.y)
+                     : "l"(p));
+    else
+        asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "l"(p));
+    return v;
+}
+
+template <int L2PF>
+__device__ __forceinline__ uint32_t ldg_stream_u32_pf(const void* p) {
+    uint32_t v;
+    if constexpr (L2PF == 256)
+        asm volatile("ld.global.nc.L1::no_allocate.L2::256B.u32 %0, [%1];" : "=r"(v) : "l"(p));
+    else if constexpr (L2PF == 128)
+        asm volatile("ld.global.nc.L1::no_allocate.L2::128B.u32 %0, [%1];" : "=r"(v) : "l"(p));
+    else
+        asm volatile("ld.global.nc.L1::no_allocate.u32 %0, [%1];" : "=r"(v) : "l"(p));
+    return v;
+}
+
+template <int L2PF>
+__device__ __forceinline__ float ldg_stream_f32_pf(const float* p) {
+    float v;
+    if constexpr (L2PF == 256)
+        asm volatile("ld.global.nc.L1::no_allocate.L2::256B.f32 %0, [%1];" : "=f"(v) : "l"(p));
+    else if constexpr (L2PF == 128)
+        asm volatile("ld.global.nc.L1::no_allocate.L2::128B.f32 %0, [%1];" : "=f"(v) : "l"(p));
+    else
+        asm volatile("ld.global.nc.L1::no_allocate.f32 %0, [%1];" : "=f"(v) : "l"(p));
+    return v;
+}
+
 __device__ __forceinline__ uint32_t ldg_stream_u32(const void* p) {
     uint32_t v;
     asm volatile("ld.global.nc.L1::no_allocate.u32 %0, [%1];" : "=r"(v) : "l"(p));

@@ -60,13 +60,13 @@ __device__ __forceinline__ void load_unit(Unit<S>& u, const GemmParams& p, int t
             const int n = min(tile * S::TR + 16 * i + g + 8 * r, p.N - 1);  // rows past N: clamp, never stored
             const uint8_t* wp = p.Wp + (size_t)n * row_bytes + kbyte;
             if constexpr (S::SB == 64) {
-                const uint2 v = ldg_stream_v2(wp);
+                const uint2 v = ldg_stream_v2_pf<S::L2PF>(wp);
                 u.w[i][r][0] = v.x;
                 u.w[i][r][1] = v.y;
             } else {
-                u.w[i][r][0] = ldg_stream_u32(wp);
+                u.w[i][r][0] = ldg_stream_u32_pf<S::L2PF>(wp);
             }
-            u.am[i][r] = ldg_stream_f32(p.absmax + (size_t)n * p.am_per_row + am_col);
+            u.am[i][r] = ldg_stream_f32_pf<S::L2PF>(p.absmax + (size_t)n * p.am_per_row + am_col);
         }
     }
     const T* A = static_cast<const T*>(p.A);
@@ -260,24 +260,30 @@ __global__ void __launch_bounds__(S::NW * 32, 1) q4_gemm_mma_kernel(const GemmPa
         c.kb = (int)(ws - (int64_t)c.tile * p.kb_per_tile);
         c.from_start = (c.kb == 0);
         c.first_tile = true;
-        int lt = c.tile, lk = c.kb;  // load cursor, one unit ahead
-        Unit<S> b0, b1;
-        load_unit<T, S>(b0, p, lt, lk, g, tq);
-        advance(lt, lk, p.kb_per_tile);
-        for (int i = 0; i < nunits; i += 2) {
-            if (i + 1 < nunits) {
-                load_unit<T, S>(b1, p, lt, lk, g, tq);
+        // Ring of DEPTH + 1 unit buffers: the loads of DEPTH units are in
+        // flight while one unit is computed.
+        constexpr int R = S::DEPTH + 1;
+        int lt = c.tile, lk = c.kb;  // load cursor
+        Unit<S> buf[R];
+#pragma unroll
+        for (int d = 0; d < S::DEPTH; ++d) {
+            if (d < nunits) {
+                load_unit<T, S>(buf[d], p, lt, lk, g, tq);
                 advance(lt, lk, p.kb_per_tile);
             }
-            mma_unit<T, S>(acc, b0, lane4);
-            finish_unit<T, S>(acc, c, i + 1 == nunits, p, slots, warp, lane, g, tq);
-            if (i + 1 >= nunits) break;
-            if (i + 2 < nunits) {
-                load_unit<T, S>(b0, p, lt, lk, g, tq);
-                advance(lt, lk, p.kb_per_tile);
+        }
+        for (int i = 0; i < nunits; i += R) {
+#pragma unroll
+            for (int r = 0; r < R; ++r) {
+                if (i + r < nunits) {
+                    if (i + r + S::DEPTH < nunits) {
+                        load_unit<T, S>(buf[(r + S::DEPTH) % R], p, lt, lk, g, tq);
+                        advance(lt, lk, p.kb_per_tile);
+                    }
+                    mma_unit<T, S>(acc, buf[r], lane4);
+                    finish_unit<T, S>(acc, c, i + r + 1 == nunits, p, slots, warp, lane, g, tq);
+                }
             }
-            mma_unit<T, S>(acc, b1, lane4);
-            finish_unit<T, S>(acc, c, i + 2 == nunits, p, slots, warp, lane, g, tq);
         }
     }
     __syncthreads();
@@ -337,7 +343,7 @@ __global__ void __launch_bounds__(S::NW * 32, 1) q4_gemm_mma_kernel(const GemmPa
 }
 
 // ---------------------------------------------------------------------------
-// Host launchers.
+// Host launchers: the table of compiled variants.
 // ---------------------------------------------------------------------------
 template <typename T, class S>
 static cudaError_t launch_mma(const GemmParams& p, cudaStream_t stream) {
@@ -348,32 +354,56 @@ static cudaError_t launch_mma(const GemmParams& p, cudaStream_t stream) {
     return cudaGetLastError();
 }
 
-template <typename T>
-static cudaError_t dispatch_mma(const GemmChoice& ch, const GemmParams& p, cudaStream_t stream) {
-    if (ch.sub_block == 64) {
-        if (ch.m_pad == 8)
-            return ch.warps == 8 ? launch_mma<T, GemmShape<64, 8, 4, 8>>(p, stream)
-                                 : launch_mma<T, GemmShape<64, 8, 4, 16>>(p, stream);
-        return launch_mma<T, GemmShape<64, 16, 4, 8>>(p, stream);
+struct Variant {
+    int act, sub_block, m_pad, warps, depth, l2pf;
+    size_t smem;
+    cudaError_t (*launch)(const GemmParams&, cudaStream_t);
+};
+
+#define Q4_VARIANT(ACT, T, SB, MP, NW, D, PF)                                                  \
+    Variant {                                                                                 \
+        ACT, SB, MP, NW, D, PF, GemmShape<SB, MP, 4, NW, D, PF>::SMEM_BYTES,                  \
+            &launch_mma<T, GemmShape<SB, MP, 4, NW, D, PF>>                                   \
     }
-    if (ch.m_pad == 8)
-        return ch.warps == 8 ? launch_mma<T, GemmShape<32, 8, 4, 8>>(p, stream)
-                             : launch_mma<T, GemmShape<32, 8, 4, 16>>(p, stream);
-    return launch_mma<T, GemmShape<32, 16, 4, 8>>(p, stream);
+
+#define Q4_VARIANTS_FOR(ACT, T)                                                                \
+    Q4_VARIANT(ACT, T, 64, 8, 16, 1, 128), Q4_VARIANT(ACT, T, 64, 8, 8, 2, 128),               \
+        Q4_VARIANT(ACT, T, 64, 16, 8, 1, 128), Q4_VARIANT(ACT, T, 32, 8, 16, 1, 128),         \
+        Q4_VARIANT(ACT, T, 32, 16, 8, 1, 128)
+
+static const Variant kVariants[] = {
+    Q4_VARIANTS_FOR(0, __nv_bfloat16),
+    Q4_VARIANTS_FOR(1, __half),
+    // measurement-only variants of the main M<=8, blocksize-64, bf16 case
+    Q4_VARIANT(0, __nv_bfloat16, 64, 8, 16, 1, 0),
+    Q4_VARIANT(0, __nv_bfloat16, 64, 8, 16, 1, 256),
+    Q4_VARIANT(0, __nv_bfloat16, 64, 8, 16, 2, 128),
+    Q4_VARIANT(0, __nv_bfloat16, 64, 8, 8, 1, 128),
+    Q4_VARIANT(0, __nv_bfloat16, 64, 8, 8, 2, 0),
+    Q4_VARIANT(0, __nv_bfloat16, 64, 8, 8, 2, 256),
+    Q4_VARIANT(0, __nv_bfloat16, 64, 8, 8, 3, 128),
+    Q4_VARIANT(0, __nv_bfloat16, 64, 16, 8, 2, 128),
+};
+
+static const Variant* find_variant(int act, const GemmChoice& ch) {
+    for (const Variant& v : kVariants)
+        if (v.act == act && v.sub_block == ch.sub_block && v.m_pad == ch.m_pad && v.warps == ch.warps &&
+            v.depth == ch.depth && v.l2pf == ch.l2pf)
+            return &v;
+    return nullptr;
+}
+
+bool gemm_variant_exists(int act_dtype, const GemmChoice& ch) { return find_variant(act_dtype, ch) != nullptr; }
+
+size_t gemm_smem_bytes(int act_dtype, const GemmChoice& ch) {
+    const Variant* v = find_variant(act_dtype, ch);
+    return v ? v->smem : 0;
 }
 
 cudaError_t gemm_launch(const GemmChoice& ch, int act_dtype, const GemmParams& p, cudaStream_t stream) {
-    if (act_dtype == 0) return dispatch_mma<__nv_bfloat16>(ch, p, stream);
-    return dispatch_mma<__half>(ch, p, stream);
-}
-
-size_t gemm_smem_bytes(int sub_block, int m_pad, int warps) {
-    if (sub_block == 64) {
-        if (m_pad == 8) return warps == 8 ? GemmShape<64, 8, 4, 8>::SMEM_BYTES : GemmShape<64, 8, 4, 16>::SMEM_BYTES;
-        return GemmShape<64, 16, 4, 8>::SMEM_BYTES;
-    }
-    if (m_pad == 8) return warps == 8 ? GemmShape<32, 8, 4, 8>::SMEM_BYTES : GemmShape<32, 8, 4, 16>::SMEM_BYTES;
-    return GemmShape<32, 16, 4, 8>::SMEM_BYTES;
+    const Variant* v = find_variant(act_dtype, ch);
+    if (!v) return cudaErrorInvalidConfiguration;
+    return v->launch(p, stream);
 }
 
 size_t gemm_slot_floats(int m_pad) { return (size_t)4 * (m_pad / 8) * 4 * 32; }

@@ -18,13 +18,16 @@ struct GemmChoice {
     int warps;      // warps per CTA
     int ctas;       // persistent CTAs
     int rows_per_tile;
+    int depth;      // units in flight ahead of the one being computed
+    int l2pf;       // L2 fetch-size hint on weight loads: 0 (none), 128, 256
 };
 
 // Sets cudaFuncAttributeMaxDynamicSharedMemorySize once per (kernel, device).
 cudaError_t ensure_smem_attr(const void* kernel, size_t bytes);
 
 cudaError_t gemm_launch(const GemmChoice& ch, int act_dtype, const GemmParams& p, cudaStream_t stream);
-size_t gemm_smem_bytes(int sub_block, int m_pad, int warps);
+bool gemm_variant_exists(int act_dtype, const GemmChoice& ch);
+size_t gemm_smem_bytes(int act_dtype, const GemmChoice& ch);
 size_t gemm_slot_floats(int m_pad);
 
 cudaError_t quantize_launch(const float* W, int64_t n, int blocksize, const float* code, uint8_t* packed,

@@ -27,7 +27,7 @@ __host__ __device__ __forceinline__ int part_owner(int64_t total, int parts, int
 }
 
 // Compile-time shape of one GEMM kernel variant.
-template <int SB_, int MPAD_, int TW_, int NW_>
+template <int SB_, int MPAD_, int TW_, int NW_, int DEPTH_, int L2PF_>
 struct GemmShape {
     static constexpr int SB = SB_;      // k-width of a unit (32 or 64)
     static constexpr int MPAD = MPAD_;  // M padded to 8 or 16 (MMA columns)
@@ -35,6 +35,8 @@ struct GemmShape {
     static constexpr int TW = TW_;      // 16-row MMA tiles per unit
     static constexpr int TR = 16 * TW_; // rows per unit
     static constexpr int NW = NW_;      // warps per CTA
+    static constexpr int DEPTH = DEPTH_;  // units in flight ahead of the one being computed
+    static constexpr int L2PF = L2PF_;    // L2 fetch-size hint for weight loads (0, 128, 256 bytes)
     static constexpr int SLOT_REGS = TW_ * NJ * 4;     // accumulator registers per lane
     static constexpr int SLOT_FLOATS = SLOT_REGS * 32; // one warp's partial tile
     static constexpr uint32_t LUT_BYTES = 256u * 256u; // 256 byte values x 32 lanes x 4 B, 256-B rows
@@ -43,6 +45,11 @@ struct GemmShape {
     // 64 KiB boundary of the shared window, the LUT, and the warp slots.
     static constexpr uint32_t SMEM_BYTES = 65536u + LUT_BYTES + SLOT_BYTES;
 };
+
+// Largest partial-sum slot of any variant (TW = 4, MPAD = 16): the GEMM
+// workspace reserves this much per slot so its counters sit at an offset
+// that depends only on the device's SM count.
+static constexpr size_t kMaxSlotBytes = 4 * 2 * 4 * 32 * 4;
 
 // Runtime parameters of one GEMM launch.
 struct GemmParams {

@@ -123,9 +123,12 @@ int q4_gemm_workspace_size(int M, int N, int K, int blocksize, int act_dtype, si
  *   act_dtype  Q4_BF16 or Q4_FP16 (Q4_FP32 -> Q4_ERR_UNSUPPORTED)
  *   out      [M, N] act_dtype, row-major, 16-byte aligned
  *   workspace  device scratch of at least q4_gemm_workspace_size() bytes,
- *            16-byte aligned, ZERO-FILLED before its first use; every call
- *            leaves it zero-filled again.  Calls that share a workspace
- *            must not overlap on the GPU (use one per stream).
+ *            16-byte aligned, ZERO-FILLED before its first use.  It holds
+ *            one counter per weight tile (every call returns the counters
+ *            it used to zero) after a fixed-size region of partial sums
+ *            (scratch), so one workspace serves every problem size on a
+ *            device.  Calls that share a workspace must not overlap on the
+ *            GPU (use one per stream).
  * The result is deterministic: partial sums are combined in a fixed order.
  */
 int q4_gemm_skinny(const void* A, const uint8_t* Wpacked, const float* absmax, const float* code,
@@ -135,15 +138,17 @@ int q4_gemm_skinny(const void* A, const uint8_t* Wpacked, const float* absmax, c
 /* Launch-table entry chosen for a GEMM problem (host-only, for reporting and
  * tests).  `num_sms` <= 0 means "the current device's SM count". */
 typedef struct {
-    int math;          /* 1 = tensor-core (mma.sync m16n8k16), 2 = CUDA-core FMA */
-    int sub_block;     /* k-width of one work unit: min(blocksize, 64)           */
-    int m_pad;         /* M padded to the MMA column count: 8 or 16              */
-    int rows_per_tile; /* weight rows per work unit                              */
-    int warps;         /* warps per CTA                                          */
-    int ctas;          /* persistent CTAs (<= SM count, <= number of units)      */
-    int tiles;         /* ceil(N / rows_per_tile)                                */
-    int64_t units;     /* tiles * (K / sub_block)                                */
-    size_t smem_bytes; /* dynamic shared memory per CTA                          */
+    int math;          /* 1 = tensor-core (mma.sync m16n8k16), 2 = CUDA-core FMA  */
+    int sub_block;     /* k-width of one work unit: min(blocksize, 64)            */
+    int m_pad;         /* M padded to the MMA column count: 8 or 16               */
+    int rows_per_tile; /* weight rows per work unit                               */
+    int warps;         /* warps per CTA                                           */
+    int ctas;          /* persistent CTAs (<= SM count, <= number of units)       */
+    int depth;         /* work units each warp has in flight ahead of its compute */
+    int l2_prefetch;   /* L2 fetch-size hint on weight loads: 1 none, 128, 256 B  */
+    int tiles;         /* ceil(N / rows_per_tile)                                 */
+    int64_t units;     /* tiles * (K / sub_block)                                 */
+    size_t smem_bytes; /* dynamic shared memory per CTA                           */
     size_t workspace_bytes;
 } q4_gemm_plan_t;
 
@@ -151,14 +156,17 @@ int q4_gemm_plan(int M, int N, int K, int blocksize, int act_dtype, int num_sms,
                  q4_gemm_plan_t* plan);
 
 /*
- * Same as q4_gemm_skinny with explicit launch-table overrides; any field
- * <= 0 keeps the table's choice.  math: 1 tensor-core, 2 CUDA-core FMA
- * (M <= 4 only).  Used to measure the choices the launch table makes.
+ * Same as q4_gemm_skinny with explicit launch-table overrides, used to
+ * measure the choices the table makes.  `overrides` may be NULL; in it,
+ * math, warps, ctas, depth and l2_prefetch override the table when > 0 (all
+ * other fields are ignored).  A combination that was not compiled returns
+ * Q4_ERR_UNSUPPORTED; ctas above the SM count returns Q4_ERR_INVALID_ARG.
+ * The workspace size needed does not depend on the overrides.
  */
 int q4_gemm_skinny_ex(const void* A, const uint8_t* Wpacked, const float* absmax,
                       const float* code, int M, int N, int K, int blocksize, int act_dtype,
-                      void* out, void* workspace, size_t workspace_bytes, void* stream, int math,
-                      int ctas, int warps);
+                      void* out, void* workspace, size_t workspace_bytes, void* stream,
+                      const q4_gemm_plan_t* overrides);
 
 /*
  * Work partition used by the GEMM (host-callable so it can be checked

@@ -77,8 +77,10 @@ def test_gemm_validation_before_cuda():
         assert g(*args, M, N, K, bs, dt, ALIGNED, None, 0, None) == want, (M, N, K, bs, dt)
     assert g(None, *args[1:], 1, 64, 4096, 64, 0, ALIGNED, None, 0, None) == b.Q4_ERR_INVALID_ARG
     ex = b.lib().q4_gemm_skinny_ex
-    assert ex(*args, 1, 64, 4096, 64, 0, ALIGNED, None, 0, None, 3, 0, 0) == b.Q4_ERR_INVALID_ARG
-    assert ex(*args, 12, 64, 4096, 64, 0, ALIGNED, None, 0, None, 0, 0, 16) == b.Q4_ERR_UNSUPPORTED
+    assert ex(*args, 1, 64, 4096, 64, 0, ALIGNED, None, 0, None, b.overrides(math=3)) == b.Q4_ERR_INVALID_ARG
+    assert ex(*args, 12, 64, 4096, 64, 0, ALIGNED, None, 0, None, b.overrides(warps=16)) == b.Q4_ERR_UNSUPPORTED
+    assert ex(*args, 1, 64, 4096, 64, 0, ALIGNED, None, 0, None, b.overrides(depth=7)) == b.Q4_ERR_UNSUPPORTED
+    assert ex(*args, 1, 64, 4096, 64, 0, ALIGNED, None, 0, None, b.overrides(math=2)) == b.Q4_ERR_UNSUPPORTED
 
 
 @pytest.mark.parametrize("wl", list(inputs.workloads()))
@@ -92,9 +94,10 @@ def test_launch_table_invariants(wl):
         assert p["units"] == p["tiles"] * (c.K // p["sub_block"])
         assert 1 <= p["ctas"] <= min(148, p["units"])
         assert p["smem_bytes"] <= 227 * 1024
-        slot = p["rows_per_tile"] * p["m_pad"] * 4
-        want_ws = 0 if p["ctas"] == 1 else (-(-p["tiles"] * 4 // 256) * 256 + p["ctas"] * 2 * slot)
+        # workspace: 2 slots of 4 KiB per SM, then one int per tile (256-B granules)
+        want_ws = 0 if p["units"] == 1 else 148 * 2 * 4096 + -(-p["tiles"] * 4 // 256) * 256
         assert p["workspace_bytes"] == want_ws
+        assert p["depth"] >= 1 and p["l2_prefetch"] in (1, 128, 256)
 
 
 @pytest.mark.parametrize("total,parts", [(1, 1), (1, 16), (7, 3), (40, 148), (4096, 148), (57344, 148),

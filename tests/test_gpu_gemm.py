@@ -12,7 +12,7 @@ import oracle
 from bit_weight_dequant_b200 import binding as q4
 from bit_weight_dequant_b200 import inputs
 from bit_weight_dequant_b200.inputs import Case
-from parity import TORCH_ACT, bits_of, run_case
+from parity import TORCH_ACT, bits_of, check_gemm, run_case
 
 pytestmark = pytest.mark.gpu
 
@@ -66,14 +66,44 @@ def _problem(device, M=3, N=300, K=1024, bs=64, seed=7):
             torch.from_numpy(code).to(device), N, K, bs)
 
 
-def test_deterministic_and_workspace_left_zero(cuda_device):
+def test_deterministic_and_counters_left_zero(cuda_device):
     A, P, Am, C, N, K, bs = _problem(cuda_device)
     ws = q4.Workspace(cuda_device)
     outs = [q4.q4_gemm_skinny(A, P, Am, C, N, K, bs, workspace=ws, ctas=5) for _ in range(3)]
     torch.cuda.synchronize()
     for o in outs[1:]:
         assert torch.equal(o.view(torch.int16), outs[0].view(torch.int16))
-    assert ws.buf.numel() > 0 and int(ws.buf.count_nonzero()) == 0
+    off = q4.workspace_counter_offset(cuda_device)
+    assert ws.buf.numel() > off and int(ws.buf[off:].count_nonzero()) == 0
+
+
+@pytest.mark.parametrize("order", [0, 1])
+def test_one_workspace_serves_shapes_in_any_order(cuda_device, order):
+    """Scratch left by a call of one shape must not disturb the next shape."""
+    ws = q4.Workspace(cuda_device)
+    shapes = [(2, 4000, 2560), (3, 300, 1024), (1, 9000, 640)]
+    if order:
+        shapes = shapes[::-1]
+    for M, N, K in shapes:
+        code = inputs.code_normal_quantile()
+        W = inputs.weights(N, K, N + K)
+        packed, absmax = oracle.quantize(W, 64, code)
+        A = inputs.activations(M, K, torch.bfloat16, N)
+        y, S = oracle.gemm(bits_of(A), oracle.BF16, packed, absmax, code, M, N, K, 64)
+        out = q4.q4_gemm_skinny(A.to(cuda_device), torch.from_numpy(packed).to(cuda_device),
+                                torch.from_numpy(absmax).to(cuda_device), torch.from_numpy(code).to(cuda_device),
+                                N, K, 64, workspace=ws)
+        torch.cuda.synchronize()
+        check_gemm(bits_of(out), y, S, "bf16", label=f"M{M} N{N} K{K}")
+
+
+@pytest.mark.parametrize("depth,l2pf,warps", [(1, 1, 16), (1, 256, 16), (2, 128, 16), (1, 128, 8), (2, 1, 8),
+                                              (2, 256, 8), (3, 128, 8), (2, 128, 8)])
+def test_measurement_variants(cuda_device, depth, l2pf, warps):
+    run_case(Case(1, 700, 2048), seed=7000 + depth, device=cuda_device, check_quantizer=False, depth=depth,
+             l2_prefetch=l2pf, warps=warps)
+    run_case(Case(1, 190, 640), seed=7100 + depth, device=cuda_device, check_quantizer=False, depth=depth,
+             l2_prefetch=l2pf, warps=warps, ctas=5)
 
 
 def test_empty_and_degenerate(cuda_device):
