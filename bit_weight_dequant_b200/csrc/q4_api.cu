@@ -140,20 +140,22 @@ const char* q4_status_string(int status) {
 
 int q4_quantize_blockwise(const float* W, int64_t n, int blocksize, const float* code, uint8_t* packed,
                           float* absmax, void* stream) {
-    if (!W || !code || !packed || !absmax || n < 0 || !is_pow2_blocksize(blocksize)) return Q4_ERR_INVALID_ARG;
+    if (n < 0 || !is_pow2_blocksize(blocksize)) return Q4_ERR_INVALID_ARG;
+    if (n == 0) return Q4_OK;  // empty input: pointers may be NULL
+    if (!W || !code || !packed || !absmax) return Q4_ERR_INVALID_ARG;
     if (!aligned(W, 16) || !aligned(code, 4) || !aligned(absmax, 4)) return Q4_ERR_MISALIGNED;
-    if (n == 0) return Q4_OK;
     if (injected_failure()) return Q4_ERR_CUDA;
     return from_cuda(quantize_launch(W, n, blocksize, code, packed, absmax, (cudaStream_t)stream));
 }
 
 int q4_dequantize_blockwise(const uint8_t* packed, const float* absmax, const float* code, int64_t n,
                             int blocksize, int out_dtype, void* out, void* stream) {
-    if (!packed || !absmax || !code || !out || n < 0 || !is_pow2_blocksize(blocksize)) return Q4_ERR_INVALID_ARG;
+    if (n < 0 || !is_pow2_blocksize(blocksize)) return Q4_ERR_INVALID_ARG;
     if (out_dtype != Q4_BF16 && out_dtype != Q4_FP16 && out_dtype != Q4_FP32) return Q4_ERR_INVALID_ARG;
+    if (n == 0) return Q4_OK;  // empty input: pointers may be NULL
+    if (!packed || !absmax || !code || !out) return Q4_ERR_INVALID_ARG;
     if (!aligned(packed, 16) || !aligned(out, 16) || !aligned(absmax, 4) || !aligned(code, 4))
         return Q4_ERR_MISALIGNED;
-    if (n == 0) return Q4_OK;
     if (injected_failure()) return Q4_ERR_CUDA;
     return from_cuda(dequantize_launch(packed, absmax, code, n, blocksize, out_dtype, out, (cudaStream_t)stream));
 }
@@ -192,18 +194,20 @@ int q4_gemm_workspace_size(int M, int N, int K, int blocksize, int act_dtype, si
 int q4_gemm_skinny_ex(const void* A, const uint8_t* Wpacked, const float* absmax, const float* code, int M, int N,
                       int K, int blocksize, int act_dtype, void* out, void* workspace, size_t workspace_bytes,
                       void* stream, const q4_gemm_plan_t* overrides) {
-    if (!A || !Wpacked || !absmax || !code || !out) return Q4_ERR_INVALID_ARG;
+    // Pointers to empty arrays may be NULL; everything else must be given.
+    if (M > 0 && N > 0 && (!out || (K > 0 && (!A || !Wpacked || !absmax || !code)))) return Q4_ERR_INVALID_ARG;
     GemmChoice ch;
     int tiles = 0, sms = 0;
     int64_t units = 0;
     size_t need = 0;
     int rc = gemm_choose(M, N, K, blocksize, act_dtype, 0, overrides, &ch, &tiles, &units, &need, &sms);
     if (rc != Q4_OK) return rc;
-    if (!aligned(A, 16) || !aligned(Wpacked, 16) || !aligned(out, 16) || !aligned(absmax, 4) || !aligned(code, 4))
+    if (M == 0 || N == 0) return Q4_OK;
+    if (!aligned(out, 16) || (K > 0 && (!aligned(A, 16) || !aligned(Wpacked, 16) || !aligned(absmax, 4) ||
+                                         !aligned(code, 4))))
         return Q4_ERR_MISALIGNED;
     if (need > 0 && (!workspace || workspace_bytes < need)) return Q4_ERR_WORKSPACE;
     if (workspace && !aligned(workspace, 16)) return Q4_ERR_MISALIGNED;
-    if (M == 0 || N == 0) return Q4_OK;
     if (injected_failure()) return Q4_ERR_CUDA;
     cudaStream_t st = (cudaStream_t)stream;
     if (K == 0)  // empty contraction: all-zero output (0x0000 is +0 in bf16 and fp16)

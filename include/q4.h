@@ -32,7 +32,7 @@
  * Conventions for every entry point:
  *   - All pointers are caller-owned DEVICE memory unless stated otherwise;
  *     the library allocates nothing and keeps no state besides a per-device
- *     cache of kernel attributes.
+ *     cache of kernel attributes.  Pointers to empty arrays may be NULL.
  *   - `stream` is a cudaStream_t (NULL = legacy default stream); calls are
  *     asynchronous on it.  Argument errors are reported synchronously by
  *     the return value before anything is enqueued.

@@ -41,8 +41,9 @@ def test_quantize_exact_code_points_and_ties(cuda_device):
     """Values exactly on codes and exactly between two codes (ties -> lower index)."""
     code = inputs.code_uniform()
     mids = ((code[:-1].astype(np.float64) + code[1:]) / 2).astype(np.float32)
-    w = np.concatenate([code, mids, -mids, np.zeros(2, np.float32)]).astype(np.float32)
-    w = np.concatenate([w, np.zeros(64 - w.size % 64, np.float32)])
+    w = np.concatenate([code, mids, -mids, np.zeros(2, np.float32)]).astype(np.float32)   # 48 values
+    w = np.concatenate([w[:32], np.zeros(32, np.float32), w[32:], np.zeros(48, np.float32)])
+    assert w.size == 128
     w[63] = 1.0   # each 64-block has absmax 1 -> x = w
     w[127] = 1.0
     p_ref, a_ref = oracle.quantize(w, 64, code)
