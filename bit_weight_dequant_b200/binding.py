@@ -33,7 +33,7 @@ class Q4Error(RuntimeError):
 class q4_gemm_plan_t(ctypes.Structure):
     _fields_ = [("math", ctypes.c_int), ("sub_block", ctypes.c_int), ("m_pad", ctypes.c_int),
                 ("rows_per_tile", ctypes.c_int), ("warps", ctypes.c_int), ("ctas", ctypes.c_int),
-                ("depth", ctypes.c_int), ("l2_prefetch", ctypes.c_int), ("tiles", ctypes.c_int),
+                ("depth", ctypes.c_int), ("l2_prefetch", ctypes.c_int), ("loader", ctypes.c_int), ("tiles", ctypes.c_int),
                 ("units", ctypes.c_int64), ("smem_bytes", ctypes.c_size_t), ("workspace_bytes", ctypes.c_size_t)]
 
 
@@ -150,10 +150,19 @@ _workspaces: dict = {}
 MAX_SLOT_BYTES = 4096     # partial-sum slot of the largest variant (64 rows x 16 columns x fp32)
 
 
+WORKSPACE_HEADER_BYTES = 256   # the first int32 is the error word
+
+
 def workspace_counter_offset(device) -> int:
-    """Byte offset of the per-tile counters inside a GEMM workspace (two
-    partial-sum slots per SM come first; see q4_gemm_skinny in q4.h)."""
-    return torch.cuda.get_device_properties(device).multi_processor_count * 2 * MAX_SLOT_BYTES
+    """Byte offset of the per-tile counters inside a GEMM workspace (a
+    256-byte header and two partial-sum slots per SM come first; see
+    q4_gemm_skinny in q4.h)."""
+    return WORKSPACE_HEADER_BYTES + torch.cuda.get_device_properties(device).multi_processor_count * 2 * MAX_SLOT_BYTES
+
+
+def workspace_error(ws: "Workspace") -> int:
+    """The workspace's error word (0 = no kernel gave up a bounded wait)."""
+    return int(ws.buf[:4].view(torch.int32).item()) if ws.buf.numel() >= 4 else 0
 
 
 
@@ -166,7 +175,7 @@ def _default_workspace(device) -> Workspace:
 
 
 def overrides(**kw) -> q4_gemm_plan_t | None:
-    """Launch-table overrides (math, warps, ctas, depth, l2_prefetch); None if empty."""
+    """Launch-table overrides (math, warps, ctas, depth, l2_prefetch, loader); None if empty."""
     kw = {k: v for k, v in kw.items() if v}
     if not kw:
         return None

@@ -72,11 +72,13 @@ static int from_cuda(cudaError_t e) {
 
 static size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
-// Workspace layout: [partial slots: sms x 2 x kMaxSlotBytes][counters: one int per tile].
-// The counters sit at an offset that depends only on the SM count, so
-// scratch written by a call of one shape never lands on another shape's
-// counters; each call returns the counters it used to zero.
-static size_t ws_counter_offset(int sms) { return (size_t)sms * 2 * kMaxSlotBytes; }
+// Workspace layout: [header: error word, 256 B][partial slots: sms x 2 x
+// kMaxSlotBytes][counters: one int per tile].  The counters sit at an offset
+// that depends only on the SM count, so scratch written by a call of one
+// shape never lands on another shape's counters; each call returns the
+// counters it used to zero.
+static constexpr size_t kWsHeader = 256;
+static size_t ws_counter_offset(int sms) { return kWsHeader + (size_t)sms * 2 * kMaxSlotBytes; }
 
 // Validates a GEMM request.  Returns Q4_OK and fills `ch` with the launch
 // table's choice (with `ov` applied) and the problem's unit counts.
@@ -85,16 +87,29 @@ static int gemm_choose(int M, int N, int K, int blocksize, int act_dtype, int nu
     if (M < 0 || N < 0 || K < 0) return Q4_ERR_INVALID_ARG;
     if (!is_pow2_blocksize(blocksize)) return Q4_ERR_INVALID_ARG;
     if (act_dtype != Q4_BF16 && act_dtype != Q4_FP16 && act_dtype != Q4_FP32) return Q4_ERR_INVALID_ARG;
-    if (ov && (ov->math > 2 || ov->l2_prefetch > 256)) return Q4_ERR_INVALID_ARG;
+    if (ov && (ov->math > 2 || ov->l2_prefetch > 256 || ov->loader > 2)) return Q4_ERR_INVALID_ARG;
     if (M > 16 || act_dtype == Q4_FP32 || K % blocksize != 0) return Q4_ERR_UNSUPPORTED;
     GemmChoice c{};
     c.math = 1;
     c.sub_block = blocksize < 64 ? blocksize : 64;
     c.m_pad = M <= 8 ? 8 : 16;
     c.rows_per_tile = 64;
-    c.warps = c.m_pad == 8 ? 16 : 8;
-    c.depth = 1;
-    c.l2pf = 128;
+    // The TMA stage ring needs 64-k units and absmax rows that are whole
+    // multiples of 16 bytes (a tensor-map stride rule); the pointer itself
+    // must also be 16-byte aligned, which the caller checks at launch.
+    const bool tma_ok = c.sub_block == 64 && (K / blocksize) % 4 == 0 && (int64_t)N * (K / 64) > 1;
+    c.loader = tma_ok ? 2 : 1;
+    if (ov && ov->loader > 0) c.loader = ov->loader;
+    if (c.loader == 2 && !tma_ok) return Q4_ERR_UNSUPPORTED;
+    if (c.loader == 2) {
+        c.warps = 8;
+        c.depth = 2;
+        c.l2pf = 0;
+    } else {
+        c.warps = c.m_pad == 8 ? 16 : 8;
+        c.depth = 1;
+        c.l2pf = 128;
+    }
     if (ov) {
         if (ov->math > 0) c.math = ov->math;
         if (ov->warps > 0) c.warps = ov->warps;
@@ -176,6 +191,7 @@ int q4_gemm_plan(int M, int N, int K, int blocksize, int act_dtype, int num_sms,
     plan->ctas = ch.ctas;
     plan->depth = ch.depth;
     plan->l2_prefetch = ch.l2pf == 0 ? 1 : ch.l2pf;
+    plan->loader = ch.loader;
     plan->tiles = tiles;
     plan->units = units;
     plan->smem_bytes = gemm_smem_bytes(act_dtype == Q4_FP32 ? Q4_BF16 : act_dtype, ch);
@@ -208,6 +224,17 @@ int q4_gemm_skinny_ex(const void* A, const uint8_t* Wpacked, const float* absmax
         return Q4_ERR_MISALIGNED;
     if (need > 0 && (!workspace || workspace_bytes < need)) return Q4_ERR_WORKSPACE;
     if (workspace && !aligned(workspace, 16)) return Q4_ERR_MISALIGNED;
+    if (ch.loader == 2 && !aligned(absmax, 16)) {  // the tensor map needs a 16-byte aligned base
+        if (overrides && overrides->loader == 2) return Q4_ERR_MISALIGNED;
+        GemmChoice fb;
+        q4_gemm_plan_t ov1{};
+        if (overrides) ov1 = *overrides;
+        ov1.loader = 1;
+        ov1.warps = ov1.depth = ov1.l2_prefetch = 0;
+        rc = gemm_choose(M, N, K, blocksize, act_dtype, 0, &ov1, &fb, &tiles, &units, &need, &sms);
+        if (rc != Q4_OK) return rc;
+        ch = fb;
+    }
     if (injected_failure()) return Q4_ERR_CUDA;
     cudaStream_t st = (cudaStream_t)stream;
     if (K == 0)  // empty contraction: all-zero output (0x0000 is +0 in bf16 and fp16)
@@ -218,7 +245,8 @@ int q4_gemm_skinny_ex(const void* A, const uint8_t* Wpacked, const float* absmax
     p.absmax = absmax;
     p.code = code;
     p.out = out;
-    p.partials = static_cast<float*>(workspace);
+    p.error = static_cast<int*>(workspace);
+    p.partials = workspace ? reinterpret_cast<float*>(static_cast<char*>(workspace) + kWsHeader) : nullptr;
     p.counters = workspace ? reinterpret_cast<int*>(static_cast<char*>(workspace) + ws_counter_offset(sms)) : nullptr;
     p.M = M;
     p.N = N;

@@ -32,7 +32,11 @@
 //    (64 rows x 64 k) evenly (see q4_plan.cuh); tiles cut between warps are
 //    combined in shared memory, tiles cut between CTAs through a small
 //    workspace by the last CTA to arrive -- no spinning, deterministic order.
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
+
+#include <mutex>
 
 #include "q4_device.cuh"
 #include "q4_internal.h"
@@ -228,68 +232,15 @@ __device__ __forceinline__ void advance(int& tile, int& kb, int kb_per_tile) {
     }
 }
 
+// Combines the tiles that warps or CTAs share (after a __syncthreads that
+// makes every warp's slots visible): a tile cut only between warps of this
+// CTA is summed in warp order from shared memory and stored; a tile cut
+// between CTAs is published to the workspace, and the last CTA to arrive
+// sums all partials in CTA order and stores the tile.
 template <typename T, class S>
-__global__ void __launch_bounds__(S::NW * 32, 1) q4_gemm_mma_kernel(const GemmParams p) {
-    extern __shared__ __align__(16) uint8_t smem[];
-    const uint32_t sbase = smem_addr(smem);
-    const uint32_t lut = (sbase + 0xFFFFu) & ~0xFFFFu;  // 64 KiB aligned (host reserves the padding)
-    const uint32_t slots = (lut - sbase >= S::SLOT_BYTES) ? sbase : lut + S::LUT_BYTES;
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, tq = lane & 3;
-
-    // Table row b (256 B): 32 copies (one per bank) of the pair (code[b>>4], code[b&15]) as T.
-    for (int e = tid; e < 256 * 8; e += S::NW * 32) {
-        const int b = e >> 3;
-        const uint32_t v = Act<T>::pack(__ldg(p.code + (b >> 4)), __ldg(p.code + (b & 15)));
-        sts_v4(lut + (uint32_t)b * 256u + (uint32_t)(e & 7) * 16u, v, v, v, v);
-    }
-    __syncthreads();
-
-    const int64_t cs = part_start(p.units, p.ctas, blockIdx.x);
-    const int64_t ce = part_start(p.units, p.ctas, blockIdx.x + 1);
+__device__ __forceinline__ void combine_tiles(const GemmParams& p, uint32_t slots, int64_t cs, int64_t ce, int warp,
+                                              int lane, int g, int tq) {
     const int64_t uc = ce - cs;
-    const int64_t ws = cs + part_start(uc, S::NW, warp);
-    const int64_t we = cs + part_start(uc, S::NW, warp + 1);
-    const uint32_t lane4 = lut | ((uint32_t)lane << 2);
-    const int nunits = (int)(we - ws);
-
-    if (nunits > 0) {
-        float acc[S::TW][S::NJ][4];
-        zero_acc<S>(acc);
-        Cursor c;
-        c.tile = (int)(ws / p.kb_per_tile);
-        c.kb = (int)(ws - (int64_t)c.tile * p.kb_per_tile);
-        c.from_start = (c.kb == 0);
-        c.first_tile = true;
-        // Ring of DEPTH + 1 unit buffers: the loads of DEPTH units are in
-        // flight while one unit is computed.
-        constexpr int R = S::DEPTH + 1;
-        int lt = c.tile, lk = c.kb;  // load cursor
-        Unit<S> buf[R];
-#pragma unroll
-        for (int d = 0; d < S::DEPTH; ++d) {
-            if (d < nunits) {
-                load_unit<T, S>(buf[d], p, lt, lk, g, tq);
-                advance(lt, lk, p.kb_per_tile);
-            }
-        }
-        for (int i = 0; i < nunits; i += R) {
-#pragma unroll
-            for (int r = 0; r < R; ++r) {
-                if (i + r < nunits) {
-                    if (i + r + S::DEPTH < nunits) {
-                        load_unit<T, S>(buf[(r + S::DEPTH) % R], p, lt, lk, g, tq);
-                        advance(lt, lk, p.kb_per_tile);
-                    }
-                    mma_unit<T, S>(acc, buf[r], lane4);
-                    finish_unit<T, S>(acc, c, i + r + 1 == nunits, p, slots, warp, lane, g, tq);
-                }
-            }
-        }
-    }
-    __syncthreads();
-    if (uc <= 0) return;
-
-    // Combine the tiles that warps or CTAs share.
     const int ta = (int)(cs / p.kb_per_tile);
     const int tb = (int)((ce - 1) / p.kb_per_tile);
     for (int t = ta + warp; t <= tb; t += S::NW) {
@@ -338,8 +289,360 @@ __global__ void __launch_bounds__(S::NW * 32, 1) q4_gemm_mma_kernel(const GemmPa
                     for (int r = 0; r < 4; ++r) sum[i][j][r] += ldg_cg_f32(src + ((i * S::NJ + j) * 4 + r) * 32 + lane);
         }
         store_tile<T, S>(sum, p, t, g, tq);
-        if (lane == 0) p.counters[t] = 0;  // leave the workspace zero-filled
+        if (lane == 0) p.counters[t] = 0;  // return the counter to zero for the next call
     }
+}
+
+// Table row b (256 B): 32 copies (one per bank) of the pair (code[b>>4], code[b&15]) as T.
+template <typename T>
+__device__ __forceinline__ void build_lut(uint32_t lut, const float* code, int tid, int nthreads) {
+    for (int e = tid; e < 256 * 8; e += nthreads) {
+        const int b = e >> 3;
+        const uint32_t v = Act<T>::pack(__ldg(code + (b >> 4)), __ldg(code + (b & 15)));
+        sts_v4(lut + (uint32_t)b * 256u + (uint32_t)(e & 7) * 16u, v, v, v, v);
+    }
+}
+
+template <typename T, class S>
+__global__ void __launch_bounds__(S::NW * 32, 1) q4_gemm_mma_kernel(const GemmParams p) {
+    extern __shared__ __align__(16) uint8_t smem[];
+    const uint32_t sbase = smem_addr(smem);
+    const uint32_t lut = (sbase + 0xFFFFu) & ~0xFFFFu;  // 64 KiB aligned (host reserves the padding)
+    const uint32_t slots = (lut - sbase >= S::SLOT_BYTES) ? sbase : lut + S::LUT_BYTES;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, tq = lane & 3;
+
+    build_lut<T>(lut, p.code, tid, S::NW * 32);
+    __syncthreads();
+
+    const int64_t cs = part_start(p.units, p.ctas, blockIdx.x);
+    const int64_t ce = part_start(p.units, p.ctas, blockIdx.x + 1);
+    const int64_t uc = ce - cs;
+    const int64_t ws = cs + part_start(uc, S::NW, warp);
+    const int64_t we = cs + part_start(uc, S::NW, warp + 1);
+    const uint32_t lane4 = lut | ((uint32_t)lane << 2);
+    const int nunits = (int)(we - ws);
+
+    if (nunits > 0) {
+        float acc[S::TW][S::NJ][4];
+        zero_acc<S>(acc);
+        Cursor c;
+        c.tile = (int)(ws / p.kb_per_tile);
+        c.kb = (int)(ws - (int64_t)c.tile * p.kb_per_tile);
+        c.from_start = (c.kb == 0);
+        c.first_tile = true;
+        // Ring of DEPTH + 1 unit buffers: the loads of DEPTH units are in
+        // flight while one unit is computed.
+        constexpr int R = S::DEPTH + 1;
+        int lt = c.tile, lk = c.kb;  // load cursor
+        Unit<S> buf[R];
+#pragma unroll
+        for (int d = 0; d < S::DEPTH; ++d) {
+            if (d < nunits) {
+                load_unit<T, S>(buf[d], p, lt, lk, g, tq);
+                advance(lt, lk, p.kb_per_tile);
+            }
+        }
+        for (int i = 0; i < nunits; i += R) {
+#pragma unroll
+            for (int r = 0; r < R; ++r) {
+                if (i + r < nunits) {
+                    if (i + r + S::DEPTH < nunits) {
+                        load_unit<T, S>(buf[(r + S::DEPTH) % R], p, lt, lk, g, tq);
+                        advance(lt, lk, p.kb_per_tile);
+                    }
+                    mma_unit<T, S>(acc, buf[r], lane4);
+                    finish_unit<T, S>(acc, c, i + r + 1 == nunits, p, slots, warp, lane, g, tq);
+                }
+            }
+        }
+    }
+    __syncthreads();
+    if (uc <= 0) return;
+
+    combine_tiles<T, S>(p, slots, cs, ce, warp, lane, g, tq);
+}
+
+// ===========================================================================
+// TMA-staged variant.
+//
+// The direct-load kernel above gives every lane its fragment bytes straight
+// from global memory; each warp-wide load then touches 8 rows (8 lines) and
+// each absmax load 8 lines for 32 useful bytes, and those L1 wavefronts --
+// not DRAM -- limit it.  Here each warp streams its unit range through its
+// own ring of shared-memory stages filled by the Tensor Memory Accelerator:
+//   * weights: a 64-row x 128-byte box (4 units of 64 k) per stage, stored
+//     with the 128-byte swizzle so that ldmatrix reads it conflict-free;
+//   * absmax: the matching 64-row x 4-float box, read with 128-bit LDS.
+// A stage's mbarrier completes when both boxes have landed; the warp's lane
+// 0 issues the copy for stage k + D as soon as stage k has been consumed.
+// Every wait is bounded: on time-out the kernel records an error word in the
+// workspace, stops issuing, drains its copies (also bounded) and returns
+// normally (its outputs are then not valid).
+// ===========================================================================
+static constexpr uint32_t kStageWeightBytes = 64u * 128u;   // 8 KiB, 1024-B aligned
+static constexpr uint32_t kStageAbsmaxBytes = 64u * 4u * 4u; // 1 KiB
+static constexpr uint32_t kStageBytes = kStageWeightBytes + kStageAbsmaxBytes;
+static constexpr int kUnitsPerStage = 4;
+static constexpr uint32_t kWaitLimit = 1u << 20;             // try_wait polls before giving up
+static constexpr int kErrWaitTimeout = 1;
+static constexpr int kErrNoRoom = 2;
+
+struct StageCursor {
+    int tile, kb, left;  // next unit to put in a stage; units of the range still unassigned
+};
+
+// Next stage of a warp's unit range: units [kb, kb + n) of `tile`, all in
+// the same 4-unit window [kb0, kb0 + 4) and the same tile.
+__device__ __forceinline__ void next_stage(StageCursor& c, int kb_per_tile, int& tile, int& kb0, int& kb, int& n) {
+    tile = c.tile;
+    kb = c.kb;
+    kb0 = kb & ~(kUnitsPerStage - 1);
+    int end = kb0 + kUnitsPerStage;
+    if (end > kb_per_tile) end = kb_per_tile;
+    n = end - kb;
+    if (n > c.left) n = c.left;
+    c.left -= n;
+    c.kb += n;
+    if (c.kb == kb_per_tile) {
+        c.kb = 0;
+        ++c.tile;
+    }
+}
+
+__device__ __forceinline__ bool wait_stage(uint32_t bar, uint32_t parity) {
+    for (uint32_t it = 0; it < kWaitLimit; ++it)
+        if (mbar_try_wait(bar, parity)) return true;
+    return false;
+}
+
+// Closes a tile in the TMA kernel.  Partial tiles stay in registers until
+// every warp has left the stage ring (the slots reuse that memory): the
+// warp's first tile goes to `first`, a last partial tile stays in `acc`.
+template <typename T, class S>
+__device__ __forceinline__ void finish_unit_regs(float (&acc)[S::TW][S::NJ][4], float (&first)[S::TW][S::NJ][4],
+                                                 bool& has_first, bool& has_last, Cursor& c, bool range_end,
+                                                 const GemmParams& p, int g, int tq) {
+    const bool tile_end = (c.kb == p.kb_per_tile - 1);
+    if (tile_end || range_end) {
+        if (c.from_start && tile_end) {
+            store_tile<T, S>(acc, p, c.tile, g, tq);  // whole tile computed by this warp alone
+            zero_acc<S>(acc);
+        } else if (c.first_tile) {
+#pragma unroll
+            for (int i = 0; i < S::TW; ++i)
+#pragma unroll
+                for (int j = 0; j < S::NJ; ++j)
+#pragma unroll
+                    for (int r = 0; r < 4; ++r) first[i][j][r] = acc[i][j][r];
+            has_first = true;
+            zero_acc<S>(acc);
+        } else {
+            has_last = true;  // the range ends inside this tile: acc is the slot-1 partial
+        }
+        c.first_tile = false;
+    }
+    if (++c.kb == p.kb_per_tile) {
+        c.kb = 0;
+        ++c.tile;
+        c.from_start = true;
+    }
+}
+
+template <typename T, class S, bool BS64>
+__global__ void __launch_bounds__(S::NW * 32, 1)
+    q4_gemm_tma_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_a,
+                       const GemmParams p) {
+    extern __shared__ __align__(16) uint8_t smem_ring[];
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, tq = lane & 3;
+    constexpr int D = S::DEPTH;  // stages per warp
+
+    // Shared-memory layout (decided at run time from the window base): the
+    // 64 KiB LUT on a 64 KiB boundary; barriers and stages in the space
+    // below and above it.
+    const uint32_t sbase = smem_addr(smem_ring);
+    const uint32_t send = sbase + dynamic_smem_size();
+    const uint32_t lut = (sbase + 0xFFFFu) & ~0xFFFFu;
+    const uint32_t nbar_bytes = (uint32_t)S::NW * D * 8u;
+    uint32_t bars, a0, b0 = lut + S::LUT_BYTES;
+    if (lut - sbase >= nbar_bytes) {
+        bars = sbase;
+        a0 = (sbase + nbar_bytes + 1023u) & ~1023u;
+    } else {
+        bars = b0;
+        b0 = (b0 + nbar_bytes + 1023u) & ~1023u;
+        a0 = lut;
+    }
+    const uint32_t na = a0 < lut ? (lut - a0) / kStageBytes : 0u;
+    const uint32_t nb = b0 < send ? (send - b0) / kStageBytes : 0u;
+    const bool room = (lut + S::LUT_BYTES <= send) && (na + nb >= (uint32_t)(S::NW * D)) &&
+                      ((send > b0 && send - b0 >= S::SLOT_BYTES) || (lut > a0 && lut - a0 >= S::SLOT_BYTES));
+    if (!room) {  // uniform over the CTA: the host sized the launch wrongly
+        if (tid == 0) atomicExch(p.error, kErrNoRoom);
+        return;
+    }
+    const uint32_t slots = (send > b0 && send - b0 >= S::SLOT_BYTES) ? b0 : a0;
+    auto stage_addr = [&](int idx) -> uint32_t {
+        return (uint32_t)idx < na ? a0 + (uint32_t)idx * kStageBytes : b0 + ((uint32_t)idx - na) * kStageBytes;
+    };
+
+    build_lut<T>(lut, p.code, tid, S::NW * 32);
+    if (lane == 0) {
+        for (int d = 0; d < D; ++d) mbar_init(bars + (uint32_t)(warp * D + d) * 8u, 1);
+        mbar_init_fence();
+    }
+    __syncthreads();
+
+    const int64_t cs = part_start(p.units, p.ctas, blockIdx.x);
+    const int64_t ce = part_start(p.units, p.ctas, blockIdx.x + 1);
+    const int64_t uc = ce - cs;
+    const int64_t ws = cs + part_start(uc, S::NW, warp);
+    const int64_t we = cs + part_start(uc, S::NW, warp + 1);
+    const uint32_t lane4 = lut | ((uint32_t)lane << 2);
+    const int nunits = (int)(we - ws);
+
+    float acc[S::TW][S::NJ][4], first[S::TW][S::NJ][4];
+    bool has_first = false, has_last = false;
+    zero_acc<S>(acc);
+    if (nunits > 0) {
+        Cursor c;
+        c.tile = (int)(ws / p.kb_per_tile);
+        c.kb = (int)(ws - (int64_t)c.tile * p.kb_per_tile);
+        c.from_start = (c.kb == 0);
+        c.first_tile = true;
+        StageCursor ld{c.tile, c.kb, nunits}, cm{c.tile, c.kb, nunits};
+
+        // ldmatrix row address pieces: lane l feeds row l%8 of matrix l/8.
+        const int lm_q = lane >> 3, lm_r = lane & 7;
+        const T* Aact = static_cast<const T*>(p.A);
+        bool ok = true;
+        int issued = 0, consumed = 0;
+
+        auto issue = [&](int k) {  // lane 0: stage k into ring slot k % D
+            int tile, kb0, kb, n;
+            next_stage(ld, p.kb_per_tile, tile, kb0, kb, n);
+            const uint32_t st = stage_addr(warp * D + k % D);
+            const uint32_t bar = bars + (uint32_t)(warp * D + k % D) * 8u;
+            if (lane == 0) {
+                mbar_expect_tx(bar, kStageBytes);
+                tma_load_2d(st, &tmap_w, kb0 * 32, tile * S::TR, bar);
+                tma_load_2d(st + kStageWeightBytes, &tmap_a, (kb0 >> p.am_shift) & ~3, tile * S::TR, bar);
+            }
+        };
+        for (; issued < D && ld.left > 0; ++issued) issue(issued);
+
+        while (cm.left > 0) {
+            int tile, kb0, kb, n;
+            next_stage(cm, p.kb_per_tile, tile, kb0, kb, n);
+            const int slot = consumed % D;
+            const uint32_t st = stage_addr(warp * D + slot);
+            const uint32_t bar = bars + (uint32_t)(warp * D + slot) * 8u;
+            if (!wait_stage(bar, (uint32_t)(consumed / D) & 1u)) {
+                ok = false;
+                break;
+            }
+            // absmax of rows g and g+8 of each 16-row tile, 4 columns from x0
+            float am[S::TW][2][4];
+#pragma unroll
+            for (int i = 0; i < S::TW; ++i)
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const uint4 v = lds_v4(st + kStageWeightBytes + (uint32_t)(16 * i + 8 * h + g) * 16u);
+                    am[i][h][0] = __uint_as_float(v.x);
+                    am[i][h][1] = __uint_as_float(v.y);
+                    am[i][h][2] = __uint_as_float(v.z);
+                    am[i][h][3] = __uint_as_float(v.w);
+                }
+            const int x0 = (kb0 >> p.am_shift) & ~3;
+#pragma unroll
+            for (int j = 0; j < kUnitsPerStage; ++j) {
+                if (kb0 + j < kb || kb0 + j >= kb + n) continue;
+                const int kunit = (kb0 + j) * S::SB;
+                // activation runs: row 8jj+g, k = kunit + 32ch + 8tq .. +8
+                uint32_t bw[S::NJ][2][4];
+#pragma unroll
+                for (int jj = 0; jj < S::NJ; ++jj) {
+                    const int m = 8 * jj + g;
+#pragma unroll
+                    for (int ch = 0; ch < 2; ++ch) {
+                        if (m < p.M) {
+                            const uint4 v = ldg_v4(Aact + (size_t)m * p.K + kunit + 32 * ch + 8 * tq);
+                            bw[jj][ch][0] = v.x;
+                            bw[jj][ch][1] = v.y;
+                            bw[jj][ch][2] = v.z;
+                            bw[jj][ch][3] = v.w;
+                        } else {
+                            bw[jj][ch][0] = bw[jj][ch][1] = bw[jj][ch][2] = bw[jj][ch][3] = 0u;
+                        }
+                    }
+                }
+                int col = j;  // absmax column of this unit, relative to x0
+                if constexpr (!BS64) col = ((kb0 + j) >> p.am_shift) - x0;
+                const float zero[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                for (int i = 0; i < S::TW; ++i) {
+                    // rows 16i + 8(q&1) + r, chunk 2j + (q>>1), 128-byte swizzle
+                    const int row = 16 * i + 8 * (lm_q & 1) + lm_r;
+                    const int chunk = 2 * j + (lm_q >> 1);
+                    uint32_t d0, d1, d2, d3;
+                    ldmatrix_x4(st + (uint32_t)row * 128u + (uint32_t)((chunk ^ lm_r) << 4), d0, d1, d2, d3);
+                    float t[S::NJ][4];
+                    // step 0..3: (d0,d1) bytes 0/1, 2/3, then (d2,d3) bytes 0/1, 2/3
+                    uint32_t a0, a1, a2, a3;
+                    a0 = lut_pair<0>(d0, lane4); a2 = lut_pair<1>(d0, lane4);
+                    a1 = lut_pair<0>(d1, lane4); a3 = lut_pair<1>(d1, lane4);
+#pragma unroll
+                    for (int jj = 0; jj < S::NJ; ++jj) mma16816<T>(t[jj], a0, a1, a2, a3, bw[jj][0][0], bw[jj][0][1], zero);
+                    a0 = lut_pair<2>(d0, lane4); a2 = lut_pair<3>(d0, lane4);
+                    a1 = lut_pair<2>(d1, lane4); a3 = lut_pair<3>(d1, lane4);
+#pragma unroll
+                    for (int jj = 0; jj < S::NJ; ++jj) mma16816<T>(t[jj], a0, a1, a2, a3, bw[jj][0][2], bw[jj][0][3], t[jj]);
+                    a0 = lut_pair<0>(d2, lane4); a2 = lut_pair<1>(d2, lane4);
+                    a1 = lut_pair<0>(d3, lane4); a3 = lut_pair<1>(d3, lane4);
+#pragma unroll
+                    for (int jj = 0; jj < S::NJ; ++jj) mma16816<T>(t[jj], a0, a1, a2, a3, bw[jj][1][0], bw[jj][1][1], t[jj]);
+                    a0 = lut_pair<2>(d2, lane4); a2 = lut_pair<3>(d2, lane4);
+                    a1 = lut_pair<2>(d3, lane4); a3 = lut_pair<3>(d3, lane4);
+#pragma unroll
+                    for (int jj = 0; jj < S::NJ; ++jj) mma16816<T>(t[jj], a0, a1, a2, a3, bw[jj][1][2], bw[jj][1][3], t[jj]);
+                    float ag, ag8;
+                    if constexpr (BS64) {
+                        ag = am[i][0][j];
+                        ag8 = am[i][1][j];
+                    } else {
+                        ag = col == 0 ? am[i][0][0] : col == 1 ? am[i][0][1] : col == 2 ? am[i][0][2] : am[i][0][3];
+                        ag8 = col == 0 ? am[i][1][0] : col == 1 ? am[i][1][1] : col == 2 ? am[i][1][2] : am[i][1][3];
+                    }
+#pragma unroll
+                    for (int jj = 0; jj < S::NJ; ++jj) {
+                        acc[i][jj][0] = fmaf(ag, t[jj][0], acc[i][jj][0]);
+                        acc[i][jj][1] = fmaf(ag, t[jj][1], acc[i][jj][1]);
+                        acc[i][jj][2] = fmaf(ag8, t[jj][2], acc[i][jj][2]);
+                        acc[i][jj][3] = fmaf(ag8, t[jj][3], acc[i][jj][3]);
+                    }
+                }
+                finish_unit_regs<T, S>(acc, first, has_first, has_last, c, cm.left == 0 && kb0 + j + 1 == kb + n, p,
+                                       g, tq);
+            }
+            ++consumed;
+            // Hand the slot back to the copy engine: order this warp's reads
+            // of it before the next asynchronous write into it.
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (ld.left > 0) issue(issued++);
+        }
+        if (!ok) {
+            if (lane == 0) atomicExch(p.error, kErrWaitTimeout);
+            // drain the copies still in flight into this warp's stages
+            for (int k = consumed; k < issued; ++k)
+                wait_stage(bars + (uint32_t)(warp * D + k % D) * 8u, (uint32_t)(k / D) & 1u);
+        }
+    }
+    __syncthreads();  // every warp is out of the stage ring: the slots may reuse it
+    if (has_first) store_slot<S>(first, slots, warp * 2, lane);
+    if (has_last) store_slot<S>(acc, slots, warp * 2 + 1, lane);
+    __syncthreads();
+    if (uc <= 0) return;
+    combine_tiles<T, S>(p, slots, cs, ce, warp, lane, g, tq);
 }
 
 // ---------------------------------------------------------------------------
@@ -354,22 +657,98 @@ static cudaError_t launch_mma(const GemmParams& p, cudaStream_t stream) {
     return cudaGetLastError();
 }
 
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no link
+// against libcuda; the driver is already loaded by the runtime).
+static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+        else
+            cudaGetLastError();
+    });
+    return fn;
+}
+
+// Weights: [N rows][K/2 bytes], box 64 x 128 B, 128-byte swizzle.
+// Absmax: [N rows][K/bs floats], box 64 x 4 floats.
+static cudaError_t make_tensor_maps(const GemmParams& p, CUtensorMap* tw, CUtensorMap* ta) {
+    auto enc = tensor_map_encoder();
+    if (!enc) return cudaErrorNotSupported;
+    const cuuint32_t estride[2] = {1, 1};
+    const cuuint64_t wdim[2] = {(cuuint64_t)(p.K / 2), (cuuint64_t)p.N};
+    const cuuint64_t wstride[1] = {(cuuint64_t)(p.K / 2)};
+    const cuuint32_t wbox[2] = {128, 64};
+    if (enc(tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(p.Wp), wdim, wstride, wbox, estride,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return cudaErrorInvalidValue;
+    const cuuint64_t adim[2] = {(cuuint64_t)p.am_per_row, (cuuint64_t)p.N};
+    const cuuint64_t astride[1] = {(cuuint64_t)p.am_per_row * 4};
+    const cuuint32_t abox[2] = {4, 64};
+    if (enc(ta, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(p.absmax), adim, astride, abox, estride,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return cudaErrorInvalidValue;
+    return cudaSuccess;
+}
+
+static int max_dynamic_smem() {
+    int dev = 0, v = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&v, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess) {
+        cudaGetLastError();
+        return 0;
+    }
+    return v;
+}
+
+template <typename T, class S>
+static cudaError_t launch_tma(const GemmParams& p, cudaStream_t stream) {
+    CUtensorMap tw, ta;
+    cudaError_t e = make_tensor_maps(p, &tw, &ta);
+    if (e != cudaSuccess) return e;
+    const int smem = max_dynamic_smem();  // the kernel lays out LUT, barriers and stages itself
+    if (smem <= 0) return cudaErrorInvalidValue;
+    if (p.am_shift == 0) {
+        auto kern = q4_gemm_tma_kernel<T, S, true>;
+        if ((e = ensure_smem_attr((const void*)kern, (size_t)smem)) != cudaSuccess) return e;
+        kern<<<p.ctas, S::NW * 32, smem, stream>>>(tw, ta, p);
+    } else {
+        auto kern = q4_gemm_tma_kernel<T, S, false>;
+        if ((e = ensure_smem_attr((const void*)kern, (size_t)smem)) != cudaSuccess) return e;
+        kern<<<p.ctas, S::NW * 32, smem, stream>>>(tw, ta, p);
+    }
+    return cudaGetLastError();
+}
+
 struct Variant {
-    int act, sub_block, m_pad, warps, depth, l2pf;
+    int act, loader, sub_block, m_pad, warps, depth, l2pf;
     size_t smem;
     cudaError_t (*launch)(const GemmParams&, cudaStream_t);
 };
 
+// Per-lane global loads (loader 1): the depth is the register ring, l2pf the L2 fetch hint.
 #define Q4_VARIANT(ACT, T, SB, MP, NW, D, PF)                                                  \
     Variant {                                                                                 \
-        ACT, SB, MP, NW, D, PF, GemmShape<SB, MP, 4, NW, D, PF>::SMEM_BYTES,                  \
+        ACT, 1, SB, MP, NW, D, PF, GemmShape<SB, MP, 4, NW, D, PF>::SMEM_BYTES,               \
             &launch_mma<T, GemmShape<SB, MP, 4, NW, D, PF>>                                   \
+    }
+// TMA stage ring (loader 2): the depth is the number of stages per warp.
+#define Q4_TMA_VARIANT(ACT, T, MP, NW, D)                                                      \
+    Variant {                                                                                 \
+        ACT, 2, 64, MP, NW, D, 0, 0, &launch_tma<T, GemmShape<64, MP, 4, NW, D, 0>>            \
     }
 
 #define Q4_VARIANTS_FOR(ACT, T)                                                                \
     Q4_VARIANT(ACT, T, 64, 8, 16, 1, 128), Q4_VARIANT(ACT, T, 64, 8, 8, 2, 128),               \
         Q4_VARIANT(ACT, T, 64, 16, 8, 1, 128), Q4_VARIANT(ACT, T, 32, 8, 16, 1, 128),         \
-        Q4_VARIANT(ACT, T, 32, 16, 8, 1, 128)
+        Q4_VARIANT(ACT, T, 32, 16, 8, 1, 128), Q4_TMA_VARIANT(ACT, T, 8, 8, 2),               \
+        Q4_TMA_VARIANT(ACT, T, 16, 8, 2)
 
 static const Variant kVariants[] = {
     Q4_VARIANTS_FOR(0, __nv_bfloat16),
@@ -377,18 +756,17 @@ static const Variant kVariants[] = {
     // measurement-only variants of the main M<=8, blocksize-64, bf16 case
     Q4_VARIANT(0, __nv_bfloat16, 64, 8, 16, 1, 0),
     Q4_VARIANT(0, __nv_bfloat16, 64, 8, 16, 1, 256),
-    Q4_VARIANT(0, __nv_bfloat16, 64, 8, 16, 2, 128),
-    Q4_VARIANT(0, __nv_bfloat16, 64, 8, 8, 1, 128),
     Q4_VARIANT(0, __nv_bfloat16, 64, 8, 8, 2, 0),
-    Q4_VARIANT(0, __nv_bfloat16, 64, 8, 8, 2, 256),
-    Q4_VARIANT(0, __nv_bfloat16, 64, 8, 8, 3, 128),
-    Q4_VARIANT(0, __nv_bfloat16, 64, 16, 8, 2, 128),
+    Q4_TMA_VARIANT(0, __nv_bfloat16, 8, 16, 1),
+    Q4_TMA_VARIANT(0, __nv_bfloat16, 8, 4, 4),
+    Q4_TMA_VARIANT(0, __nv_bfloat16, 8, 12, 1),
+    Q4_TMA_VARIANT(0, __nv_bfloat16, 8, 6, 2),
 };
 
 static const Variant* find_variant(int act, const GemmChoice& ch) {
     for (const Variant& v : kVariants)
-        if (v.act == act && v.sub_block == ch.sub_block && v.m_pad == ch.m_pad && v.warps == ch.warps &&
-            v.depth == ch.depth && v.l2pf == ch.l2pf)
+        if (v.act == act && v.loader == ch.loader && v.sub_block == ch.sub_block && v.m_pad == ch.m_pad &&
+            v.warps == ch.warps && v.depth == ch.depth && (ch.loader == 2 || v.l2pf == ch.l2pf))
             return &v;
     return nullptr;
 }
@@ -397,7 +775,8 @@ bool gemm_variant_exists(int act_dtype, const GemmChoice& ch) { return find_vari
 
 size_t gemm_smem_bytes(int act_dtype, const GemmChoice& ch) {
     const Variant* v = find_variant(act_dtype, ch);
-    return v ? v->smem : 0;
+    if (!v) return 0;
+    return v->loader == 2 ? (size_t)max_dynamic_smem() : v->smem;
 }
 
 cudaError_t gemm_launch(const GemmChoice& ch, int act_dtype, const GemmParams& p, cudaStream_t stream) {

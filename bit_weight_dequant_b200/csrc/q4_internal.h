@@ -18,8 +18,9 @@ struct GemmChoice {
     int warps;      // warps per CTA
     int ctas;       // persistent CTAs
     int rows_per_tile;
-    int depth;      // units in flight ahead of the one being computed
-    int l2pf;       // L2 fetch-size hint on weight loads: 0 (none), 128, 256
+    int depth;      // units (loader 1) or stages (loader 2) in flight per warp
+    int l2pf;       // L2 fetch-size hint on weight loads: 0 (none), 128, 256 (loader 1)
+    int loader;     // 1 = per-lane global loads, 2 = TMA stage ring
 };
 
 // Sets cudaFuncAttributeMaxDynamicSharedMemorySize once per (kernel, device).

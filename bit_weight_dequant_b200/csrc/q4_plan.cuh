@@ -60,6 +60,7 @@ struct GemmParams {
     void* out;
     float* partials;   // [ctas][2][SLOT_FLOATS]
     int* counters;     // [tiles], zero between calls
+    int* error;        // workspace error word (0 = ok); set when a bounded wait gives up
     int M, N, K;
     int kb_per_tile;   // K / SB
     int am_shift;      // log2(blocksize / SB): absmax column of unit column kb = kb >> am_shift

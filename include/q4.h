@@ -123,12 +123,16 @@ int q4_gemm_workspace_size(int M, int N, int K, int blocksize, int act_dtype, si
  *   act_dtype  Q4_BF16 or Q4_FP16 (Q4_FP32 -> Q4_ERR_UNSUPPORTED)
  *   out      [M, N] act_dtype, row-major, 16-byte aligned
  *   workspace  device scratch of at least q4_gemm_workspace_size() bytes,
- *            16-byte aligned, ZERO-FILLED before its first use.  It holds
- *            one counter per weight tile (every call returns the counters
- *            it used to zero) after a fixed-size region of partial sums
- *            (scratch), so one workspace serves every problem size on a
- *            device.  Calls that share a workspace must not overlap on the
- *            GPU (use one per stream).
+ *            16-byte aligned, ZERO-FILLED before its first use.  Layout: a
+ *            256-byte header whose first int32 is an error word, a
+ *            fixed-size region of partial sums (scratch), then one counter
+ *            per weight tile (every call returns the counters it used to
+ *            zero), so one workspace serves every problem size on a device.
+ *            The error word stays 0 unless a kernel gave up a bounded wait
+ *            for its own asynchronous copies (1; outputs of that call are
+ *            not valid) or found too little shared memory (2); the caller
+ *            may read and clear it.  Calls that share a workspace must not
+ *            overlap on the GPU (use one per stream).
  * The result is deterministic: partial sums are combined in a fixed order.
  */
 int q4_gemm_skinny(const void* A, const uint8_t* Wpacked, const float* absmax, const float* code,
@@ -146,6 +150,7 @@ typedef struct {
     int ctas;          /* persistent CTAs (<= SM count, <= number of units)       */
     int depth;         /* work units each warp has in flight ahead of its compute */
     int l2_prefetch;   /* L2 fetch-size hint on weight loads: 1 none, 128, 256 B  */
+    int loader;        /* 1 = per-lane global loads, 2 = TMA shared-memory ring   */
     int tiles;         /* ceil(N / rows_per_tile)                                 */
     int64_t units;     /* tiles * (K / sub_block)                                 */
     size_t smem_bytes; /* dynamic shared memory per CTA                           */
@@ -158,8 +163,8 @@ int q4_gemm_plan(int M, int N, int K, int blocksize, int act_dtype, int num_sms,
 /*
  * Same as q4_gemm_skinny with explicit launch-table overrides, used to
  * measure the choices the table makes.  `overrides` may be NULL; in it,
- * math, warps, ctas, depth and l2_prefetch override the table when > 0 (all
- * other fields are ignored).  A combination that was not compiled returns
+ * math, warps, ctas, depth, l2_prefetch and loader override the table when
+ * > 0 (all other fields are ignored).  A combination that was not compiled returns
  * Q4_ERR_UNSUPPORTED; ctas above the SM count returns Q4_ERR_INVALID_ARG.
  * The workspace size needed does not depend on the overrides.
  */

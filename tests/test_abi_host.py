@@ -95,9 +95,11 @@ def test_launch_table_invariants(wl):
         assert 1 <= p["ctas"] <= min(148, p["units"])
         assert p["smem_bytes"] <= 227 * 1024
         # workspace: 2 slots of 4 KiB per SM, then one int per tile (256-B granules)
-        want_ws = 0 if p["units"] == 1 else 148 * 2 * 4096 + -(-p["tiles"] * 4 // 256) * 256
+        want_ws = 0 if p["units"] == 1 else 256 + 148 * 2 * 4096 + -(-p["tiles"] * 4 // 256) * 256
         assert p["workspace_bytes"] == want_ws
         assert p["depth"] >= 1 and p["l2_prefetch"] in (1, 128, 256)
+        tma_ok = c.blocksize >= 64 and (c.K // c.blocksize) % 4 == 0 and p["units"] > 1
+        assert p["loader"] == (2 if tma_ok else 1)
 
 
 @pytest.mark.parametrize("total,parts", [(1, 1), (1, 16), (7, 3), (40, 148), (4096, 148), (57344, 148),

@@ -97,13 +97,40 @@ def test_one_workspace_serves_shapes_in_any_order(cuda_device, order):
         check_gemm(bits_of(out), y, S, "bf16", label=f"M{M} N{N} K{K}")
 
 
-@pytest.mark.parametrize("depth,l2pf,warps", [(1, 1, 16), (1, 256, 16), (2, 128, 16), (1, 128, 8), (2, 1, 8),
-                                              (2, 256, 8), (3, 128, 8), (2, 128, 8)])
-def test_measurement_variants(cuda_device, depth, l2pf, warps):
+@pytest.mark.parametrize("depth,l2pf,warps", [(1, 1, 16), (1, 256, 16), (1, 128, 16), (2, 128, 8), (2, 1, 8)])
+def test_direct_load_variants(cuda_device, depth, l2pf, warps):
     run_case(Case(1, 700, 2048), seed=7000 + depth, device=cuda_device, check_quantizer=False, depth=depth,
-             l2_prefetch=l2pf, warps=warps)
+             l2_prefetch=l2pf, warps=warps, loader=1)
     run_case(Case(1, 190, 640), seed=7100 + depth, device=cuda_device, check_quantizer=False, depth=depth,
-             l2_prefetch=l2pf, warps=warps, ctas=5)
+             l2_prefetch=l2pf, warps=warps, ctas=5, loader=1)
+
+
+@pytest.mark.parametrize("warps,depth", [(8, 2), (16, 1), (4, 4), (12, 1), (6, 2)])
+def test_tma_ring_variants(cuda_device, warps, depth):
+    run_case(Case(1, 700, 2048), seed=7200 + warps, device=cuda_device, check_quantizer=False, depth=depth,
+             warps=warps, loader=2)
+    run_case(Case(3, 190, 768), seed=7300 + warps, device=cuda_device, check_quantizer=False, depth=depth,
+             warps=warps, ctas=5, loader=2)
+
+
+@pytest.mark.parametrize("M", [1, 7, 8, 9, 16])
+@pytest.mark.parametrize("N,K,bs", [(1, 256, 64), (64, 256, 64), (100, 1280, 64), (513, 1024, 128), (300, 4096, 256),
+                                    (257, 3072, 64), (70, 512, 128)])
+def test_tma_ring_shapes(cuda_device, M, N, K, bs):
+    run_case(Case(M, N, K, blocksize=bs), seed=7400 + M + N, device=cuda_device, check_quantizer=False, loader=2)
+
+
+@pytest.mark.parametrize("ctas", [1, 2, 3, 7, 33, 148])
+def test_tma_ring_partitions(cuda_device, ctas):
+    run_case(Case(2, 257, 1280), seed=7500 + ctas, device=cuda_device, check_quantizer=False, loader=2, ctas=ctas)
+
+
+def test_tma_error_word_stays_zero(cuda_device):
+    ws = q4.Workspace(cuda_device)
+    A, P, Am, C, N, K, bs = _problem(cuda_device)
+    q4.q4_gemm_skinny(A, P, Am, C, N, K, bs, workspace=ws, loader=2)
+    torch.cuda.synchronize()
+    assert q4.workspace_error(ws) == 0
 
 
 def test_empty_and_degenerate(cuda_device):
