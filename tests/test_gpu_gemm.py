@@ -42,19 +42,22 @@ def test_gemm_outliers(cuda_device, M):
     run_case(Case(M, 256, 2048, outliers=True), seed=4000 + M, device=cuda_device)
 
 
-# Launch-table overrides: tiles cut between CTAs (global fix-up) and between
-# warps (shared-memory combine), empty warp ranges, single CTA.
+# Launch-table overrides on the direct-load kernel: tiles cut between CTAs
+# (global fix-up) and between warps (shared-memory combine), empty warp
+# ranges, single CTA.
 @pytest.mark.parametrize("ctas", [1, 2, 3, 7, 64, 148])
 @pytest.mark.parametrize("warps", [8, 16])
 @pytest.mark.parametrize("M", [1, 6])
 def test_gemm_partition_overrides(cuda_device, ctas, warps, M):
-    run_case(Case(M, 257, 1280), seed=5000 + ctas, device=cuda_device, check_quantizer=False, ctas=ctas, warps=warps)
+    run_case(Case(M, 257, 1280), seed=5000 + ctas, device=cuda_device, check_quantizer=False, ctas=ctas, warps=warps,
+             loader=1)
 
 
 @pytest.mark.parametrize("ctas", [1, 5, 33])
 @pytest.mark.parametrize("M", [9, 16])
 def test_gemm_partition_overrides_m16(cuda_device, ctas, M):
-    run_case(Case(M, 190, 960), seed=6000 + ctas, device=cuda_device, check_quantizer=False, ctas=ctas, warps=8)
+    run_case(Case(M, 190, 960), seed=6000 + ctas, device=cuda_device, check_quantizer=False, ctas=ctas, warps=8,
+             loader=1)
 
 
 def _problem(device, M=3, N=300, K=1024, bs=64, seed=7):
@@ -66,15 +69,17 @@ def _problem(device, M=3, N=300, K=1024, bs=64, seed=7):
             torch.from_numpy(code).to(device), N, K, bs)
 
 
-def test_deterministic_and_counters_left_zero(cuda_device):
+@pytest.mark.parametrize("loader", [1, 2])
+def test_deterministic_and_counters_left_zero(cuda_device, loader):
     A, P, Am, C, N, K, bs = _problem(cuda_device)
     ws = q4.Workspace(cuda_device)
-    outs = [q4.q4_gemm_skinny(A, P, Am, C, N, K, bs, workspace=ws, ctas=5) for _ in range(3)]
+    outs = [q4.q4_gemm_skinny(A, P, Am, C, N, K, bs, workspace=ws, ctas=5, loader=loader) for _ in range(3)]
     torch.cuda.synchronize()
     for o in outs[1:]:
         assert torch.equal(o.view(torch.int16), outs[0].view(torch.int16))
     off = q4.workspace_counter_offset(cuda_device)
     assert ws.buf.numel() > off and int(ws.buf[off:].count_nonzero()) == 0
+    assert q4.workspace_error(ws) == 0
 
 
 @pytest.mark.parametrize("order", [0, 1])
