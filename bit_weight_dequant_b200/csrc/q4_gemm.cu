@@ -757,6 +757,7 @@ static const Variant kVariants[] = {
     Q4_VARIANT(0, __nv_bfloat16, 64, 8, 16, 1, 0),
     Q4_VARIANT(0, __nv_bfloat16, 64, 8, 16, 1, 256),
     Q4_VARIANT(0, __nv_bfloat16, 64, 8, 8, 2, 0),
+    Q4_VARIANT(0, __nv_bfloat16, 64, 8, 8, 1, 128),
     Q4_TMA_VARIANT(0, __nv_bfloat16, 8, 16, 1),
     Q4_TMA_VARIANT(0, __nv_bfloat16, 8, 4, 4),
     Q4_TMA_VARIANT(0, __nv_bfloat16, 8, 12, 1),
