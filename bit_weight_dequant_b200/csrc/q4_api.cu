@@ -87,7 +87,7 @@ static int gemm_choose(int M, int N, int K, int blocksize, int act_dtype, int nu
     if (M < 0 || N < 0 || K < 0) return Q4_ERR_INVALID_ARG;
     if (!is_pow2_blocksize(blocksize)) return Q4_ERR_INVALID_ARG;
     if (act_dtype != Q4_BF16 && act_dtype != Q4_FP16 && act_dtype != Q4_FP32) return Q4_ERR_INVALID_ARG;
-    if (ov && (ov->math > 2 || ov->l2_prefetch > 256 || ov->loader > 2)) return Q4_ERR_INVALID_ARG;
+    if (ov && (ov->math > 2 || ov->l2_prefetch > 256 || ov->loader > 3)) return Q4_ERR_INVALID_ARG;
     if (M > 16 || act_dtype == Q4_FP32 || K % blocksize != 0) return Q4_ERR_UNSUPPORTED;
     GemmChoice c{};
     c.math = 1;
@@ -98,12 +98,16 @@ static int gemm_choose(int M, int N, int K, int blocksize, int act_dtype, int nu
     // multiples of 16 bytes (a tensor-map stride rule); the pointer itself
     // must also be 16-byte aligned, which the caller checks at launch.
     const bool tma_ok = c.sub_block == 64 && (K / blocksize) % 4 == 0 && (int64_t)N * (K / 64) > 1;
-    c.loader = tma_ok ? 2 : 1;
+    c.loader = tma_ok ? 3 : 1;
     if (ov && ov->loader > 0) c.loader = ov->loader;
-    if (c.loader == 2 && !tma_ok) return Q4_ERR_UNSUPPORTED;
+    if (c.loader >= 2 && !tma_ok) return Q4_ERR_UNSUPPORTED;
     if (c.loader == 2) {
         c.warps = 8;
         c.depth = 2;
+        c.l2pf = 0;
+    } else if (c.loader == 3) {
+        c.warps = c.m_pad == 8 ? 16 : 8;
+        c.depth = c.m_pad == 8 ? 2 : 4;
         c.l2pf = 0;
     } else {
         c.warps = c.m_pad == 8 ? 16 : 8;
@@ -224,8 +228,8 @@ int q4_gemm_skinny_ex(const void* A, const uint8_t* Wpacked, const float* absmax
         return Q4_ERR_MISALIGNED;
     if (need > 0 && (!workspace || workspace_bytes < need)) return Q4_ERR_WORKSPACE;
     if (workspace && !aligned(workspace, 16)) return Q4_ERR_MISALIGNED;
-    if (ch.loader == 2 && !aligned(absmax, 16)) {  // the tensor map needs a 16-byte aligned base
-        if (overrides && overrides->loader == 2) return Q4_ERR_MISALIGNED;
+    if (ch.loader >= 2 && !aligned(absmax, 16)) {  // the tensor map needs a 16-byte aligned base
+        if (overrides && overrides->loader >= 2) return Q4_ERR_MISALIGNED;
         GemmChoice fb;
         q4_gemm_plan_t ov1{};
         if (overrides) ov1 = *overrides;

@@ -370,20 +370,33 @@ __global__ void __launch_bounds__(S::NW * 32, 1) q4_gemm_mma_kernel(const GemmPa
 // each absmax load 8 lines for 32 useful bytes, and those L1 wavefronts --
 // not DRAM -- limit it.  Here each warp streams its unit range through its
 // own ring of shared-memory stages filled by the Tensor Memory Accelerator:
-//   * weights: a 64-row x 128-byte box (4 units of 64 k) per stage, stored
-//     with the 128-byte swizzle so that ldmatrix reads it conflict-free;
-//   * absmax: the matching 64-row x 4-float box, read with 128-bit LDS.
+//   * weights: a 64-row box of UPS units (UPS x 32 bytes per row) per stage,
+//     stored with the matching 64/128-byte swizzle so ldmatrix reads it
+//     without bank conflicts;
+//   * absmax: the 64-row x 4-float box that covers the stage's blocks.
 // A stage's mbarrier completes when both boxes have landed; the warp's lane
-// 0 issues the copy for stage k + D as soon as stage k has been consumed.
+// 0 issues the copy for stage k + D once stage k has been consumed.  Warps
+// keep little state (the first partial tile is parked in the unused upper
+// half of the LUT rows), so 16 warps fit and hide each other's latency.
 // Every wait is bounded: on time-out the kernel records an error word in the
 // workspace, stops issuing, drains its copies (also bounded) and returns
 // normally (its outputs are then not valid).
 // ===========================================================================
-static constexpr uint32_t kStageWeightBytes = 64u * 128u;   // 8 KiB, 1024-B aligned
-static constexpr uint32_t kStageAbsmaxBytes = 64u * 4u * 4u; // 1 KiB
-static constexpr uint32_t kStageBytes = kStageWeightBytes + kStageAbsmaxBytes;
-static constexpr int kUnitsPerStage = 4;
-static constexpr uint32_t kWaitLimit = 1u << 20;             // try_wait polls before giving up
+template <int UPS>
+struct StageGeom {
+    static constexpr uint32_t ROW_BYTES = 32u * UPS;                   // 64 or 128
+    static constexpr uint32_t WEIGHT_BYTES = 64u * ROW_BYTES;          // 4 or 8 KiB
+    static constexpr uint32_t ABSMAX_BYTES = 64u * 4u * 4u;            // 1 KiB
+    static constexpr uint32_t BYTES = WEIGHT_BYTES + ABSMAX_BYTES;     // multiple of 512
+    // physical address of 16-byte chunk `chunk` of box row `row` (TMA swizzle)
+    __device__ __forceinline__ static uint32_t chunk_addr(uint32_t base, int row, int chunk) {
+        if constexpr (UPS == 4)
+            return base + (uint32_t)row * 128u + (uint32_t)((chunk ^ (row & 7)) << 4);
+        else
+            return base + (uint32_t)row * 64u + (uint32_t)((chunk ^ ((row >> 1) & 3)) << 4);
+    }
+};
+static constexpr uint32_t kWaitLimit = 1u << 20;  // try_wait polls before giving up
 static constexpr int kErrWaitTimeout = 1;
 static constexpr int kErrNoRoom = 2;
 
@@ -392,12 +405,13 @@ struct StageCursor {
 };
 
 // Next stage of a warp's unit range: units [kb, kb + n) of `tile`, all in
-// the same 4-unit window [kb0, kb0 + 4) and the same tile.
+// the same UPS-unit window [kb0, kb0 + UPS) and the same tile.
+template <int UPS>
 __device__ __forceinline__ void next_stage(StageCursor& c, int kb_per_tile, int& tile, int& kb0, int& kb, int& n) {
     tile = c.tile;
     kb = c.kb;
-    kb0 = kb & ~(kUnitsPerStage - 1);
-    int end = kb0 + kUnitsPerStage;
+    kb0 = kb & ~(UPS - 1);
+    int end = kb0 + UPS;
     if (end > kb_per_tile) end = kb_per_tile;
     n = end - kb;
     if (n > c.left) n = c.left;
@@ -415,13 +429,20 @@ __device__ __forceinline__ bool wait_stage(uint32_t bar, uint32_t parity) {
     return false;
 }
 
-// Closes a tile in the TMA kernel.  Partial tiles stay in registers until
-// every warp has left the stage ring (the slots reuse that memory): the
-// warp's first tile goes to `first`, a last partial tile stays in `acc`.
+// The first partial tile of a warp waits for the combine in the upper half
+// of LUT rows warp*SLOT_REGS .. +SLOT_REGS (the lookups only use each row's
+// lower 128 bytes).
+template <class S>
+__device__ __forceinline__ uint32_t parked_addr(uint32_t lut, int warp, int reg, int lane) {
+    return lut + (uint32_t)(warp * S::SLOT_REGS + reg) * 256u + 128u + (uint32_t)lane * 4u;
+}
+
+// Closes a tile in the TMA kernel: a whole tile is stored, the warp's first
+// partial tile is parked, a last partial tile stays in `acc`.
 template <typename T, class S>
-__device__ __forceinline__ void finish_unit_regs(float (&acc)[S::TW][S::NJ][4], float (&first)[S::TW][S::NJ][4],
-                                                 bool& has_first, bool& has_last, Cursor& c, bool range_end,
-                                                 const GemmParams& p, int g, int tq) {
+__device__ __forceinline__ void finish_unit_tma(float (&acc)[S::TW][S::NJ][4], bool& has_first, bool& has_last,
+                                                Cursor& c, bool range_end, const GemmParams& p, uint32_t lut,
+                                                int warp, int lane, int g, int tq) {
     const bool tile_end = (c.kb == p.kb_per_tile - 1);
     if (tile_end || range_end) {
         if (c.from_start && tile_end) {
@@ -433,7 +454,8 @@ __device__ __forceinline__ void finish_unit_regs(float (&acc)[S::TW][S::NJ][4], 
 #pragma unroll
                 for (int j = 0; j < S::NJ; ++j)
 #pragma unroll
-                    for (int r = 0; r < 4; ++r) first[i][j][r] = acc[i][j][r];
+                    for (int r = 0; r < 4; ++r)
+                        sts_f32(parked_addr<S>(lut, warp, (i * S::NJ + j) * 4 + r, lane), acc[i][j][r]);
             has_first = true;
             zero_acc<S>(acc);
         } else {
@@ -448,10 +470,12 @@ __device__ __forceinline__ void finish_unit_regs(float (&acc)[S::TW][S::NJ][4], 
     }
 }
 
-template <typename T, class S, bool BS64>
+template <typename T, class S, int UPS, bool BS64>
 __global__ void __launch_bounds__(S::NW * 32, 1)
     q4_gemm_tma_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_a,
                        const GemmParams p) {
+    using G = StageGeom<UPS>;
+    static_assert(S::NW * S::SLOT_REGS <= 256, "parked partial tiles must fit in the LUT rows");
     extern __shared__ __align__(16) uint8_t smem_ring[];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, tq = lane & 3;
     constexpr int D = S::DEPTH;  // stages per warp
@@ -472,8 +496,8 @@ __global__ void __launch_bounds__(S::NW * 32, 1)
         b0 = (b0 + nbar_bytes + 1023u) & ~1023u;
         a0 = lut;
     }
-    const uint32_t na = a0 < lut ? (lut - a0) / kStageBytes : 0u;
-    const uint32_t nb = b0 < send ? (send - b0) / kStageBytes : 0u;
+    const uint32_t na = a0 < lut ? (lut - a0) / G::BYTES : 0u;
+    const uint32_t nb = b0 < send ? (send - b0) / G::BYTES : 0u;
     const bool room = (lut + S::LUT_BYTES <= send) && (na + nb >= (uint32_t)(S::NW * D)) &&
                       ((send > b0 && send - b0 >= S::SLOT_BYTES) || (lut > a0 && lut - a0 >= S::SLOT_BYTES));
     if (!room) {  // uniform over the CTA: the host sized the launch wrongly
@@ -482,7 +506,7 @@ __global__ void __launch_bounds__(S::NW * 32, 1)
     }
     const uint32_t slots = (send > b0 && send - b0 >= S::SLOT_BYTES) ? b0 : a0;
     auto stage_addr = [&](int idx) -> uint32_t {
-        return (uint32_t)idx < na ? a0 + (uint32_t)idx * kStageBytes : b0 + ((uint32_t)idx - na) * kStageBytes;
+        return (uint32_t)idx < na ? a0 + (uint32_t)idx * G::BYTES : b0 + ((uint32_t)idx - na) * G::BYTES;
     };
 
     build_lut<T>(lut, p.code, tid, S::NW * 32);
@@ -500,7 +524,7 @@ __global__ void __launch_bounds__(S::NW * 32, 1)
     const uint32_t lane4 = lut | ((uint32_t)lane << 2);
     const int nunits = (int)(we - ws);
 
-    float acc[S::TW][S::NJ][4], first[S::TW][S::NJ][4];
+    float acc[S::TW][S::NJ][4];
     bool has_first = false, has_last = false;
     zero_acc<S>(acc);
     if (nunits > 0) {
@@ -519,20 +543,20 @@ __global__ void __launch_bounds__(S::NW * 32, 1)
 
         auto issue = [&](int k) {  // lane 0: stage k into ring slot k % D
             int tile, kb0, kb, n;
-            next_stage(ld, p.kb_per_tile, tile, kb0, kb, n);
+            next_stage<UPS>(ld, p.kb_per_tile, tile, kb0, kb, n);
             const uint32_t st = stage_addr(warp * D + k % D);
             const uint32_t bar = bars + (uint32_t)(warp * D + k % D) * 8u;
             if (lane == 0) {
-                mbar_expect_tx(bar, kStageBytes);
+                mbar_expect_tx(bar, G::BYTES);
                 tma_load_2d(st, &tmap_w, kb0 * 32, tile * S::TR, bar);
-                tma_load_2d(st + kStageWeightBytes, &tmap_a, (kb0 >> p.am_shift) & ~3, tile * S::TR, bar);
+                tma_load_2d(st + G::WEIGHT_BYTES, &tmap_a, (kb0 >> p.am_shift) & ~3, tile * S::TR, bar);
             }
         };
         for (; issued < D && ld.left > 0; ++issued) issue(issued);
 
         while (cm.left > 0) {
             int tile, kb0, kb, n;
-            next_stage(cm, p.kb_per_tile, tile, kb0, kb, n);
+            next_stage<UPS>(cm, p.kb_per_tile, tile, kb0, kb, n);
             const int slot = consumed % D;
             const uint32_t st = stage_addr(warp * D + slot);
             const uint32_t bar = bars + (uint32_t)(warp * D + slot) * 8u;
@@ -540,21 +564,9 @@ __global__ void __launch_bounds__(S::NW * 32, 1)
                 ok = false;
                 break;
             }
-            // absmax of rows g and g+8 of each 16-row tile, 4 columns from x0
-            float am[S::TW][2][4];
-#pragma unroll
-            for (int i = 0; i < S::TW; ++i)
-#pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    const uint4 v = lds_v4(st + kStageWeightBytes + (uint32_t)(16 * i + 8 * h + g) * 16u);
-                    am[i][h][0] = __uint_as_float(v.x);
-                    am[i][h][1] = __uint_as_float(v.y);
-                    am[i][h][2] = __uint_as_float(v.z);
-                    am[i][h][3] = __uint_as_float(v.w);
-                }
             const int x0 = (kb0 >> p.am_shift) & ~3;
 #pragma unroll
-            for (int j = 0; j < kUnitsPerStage; ++j) {
+            for (int j = 0; j < UPS; ++j) {
                 if (kb0 + j < kb || kb0 + j >= kb + n) continue;
                 const int kunit = (kb0 + j) * S::SB;
                 // activation runs: row 8jj+g, k = kunit + 32ch + 8tq .. +8
@@ -575,18 +587,19 @@ __global__ void __launch_bounds__(S::NW * 32, 1)
                         }
                     }
                 }
-                int col = j;  // absmax column of this unit, relative to x0
-                if constexpr (!BS64) col = ((kb0 + j) >> p.am_shift) - x0;
+                // absmax column of this unit inside the stage's 4-float box
+                const int col = BS64 ? (kb0 + j - x0) : (((kb0 + j) >> p.am_shift) - x0);
+                const uint32_t am_base = st + G::WEIGHT_BYTES + (uint32_t)col * 4u;
                 const float zero[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
                 for (int i = 0; i < S::TW; ++i) {
-                    // rows 16i + 8(q&1) + r, chunk 2j + (q>>1), 128-byte swizzle
-                    const int row = 16 * i + 8 * (lm_q & 1) + lm_r;
-                    const int chunk = 2 * j + (lm_q >> 1);
+                    // rows 16i + 8(q&1) + r, chunk 2j + (q>>1)
                     uint32_t d0, d1, d2, d3;
-                    ldmatrix_x4(st + (uint32_t)row * 128u + (uint32_t)((chunk ^ lm_r) << 4), d0, d1, d2, d3);
+                    ldmatrix_x4(G::chunk_addr(st, 16 * i + 8 * (lm_q & 1) + lm_r, 2 * j + (lm_q >> 1)), d0, d1, d2, d3);
+                    const float ag = lds_f32(am_base + (uint32_t)(16 * i + g) * 16u);
+                    const float ag8 = lds_f32(am_base + (uint32_t)(16 * i + 8 + g) * 16u);
                     float t[S::NJ][4];
-                    // step 0..3: (d0,d1) bytes 0/1, 2/3, then (d2,d3) bytes 0/1, 2/3
+                    // steps 0..3: (d0,d1) bytes 0/1, 2/3, then (d2,d3) bytes 0/1, 2/3
                     uint32_t a0, a1, a2, a3;
                     a0 = lut_pair<0>(d0, lane4); a2 = lut_pair<1>(d0, lane4);
                     a1 = lut_pair<0>(d1, lane4); a3 = lut_pair<1>(d1, lane4);
@@ -604,14 +617,6 @@ __global__ void __launch_bounds__(S::NW * 32, 1)
                     a1 = lut_pair<2>(d3, lane4); a3 = lut_pair<3>(d3, lane4);
 #pragma unroll
                     for (int jj = 0; jj < S::NJ; ++jj) mma16816<T>(t[jj], a0, a1, a2, a3, bw[jj][1][2], bw[jj][1][3], t[jj]);
-                    float ag, ag8;
-                    if constexpr (BS64) {
-                        ag = am[i][0][j];
-                        ag8 = am[i][1][j];
-                    } else {
-                        ag = col == 0 ? am[i][0][0] : col == 1 ? am[i][0][1] : col == 2 ? am[i][0][2] : am[i][0][3];
-                        ag8 = col == 0 ? am[i][1][0] : col == 1 ? am[i][1][1] : col == 2 ? am[i][1][2] : am[i][1][3];
-                    }
 #pragma unroll
                     for (int jj = 0; jj < S::NJ; ++jj) {
                         acc[i][jj][0] = fmaf(ag, t[jj][0], acc[i][jj][0]);
@@ -620,8 +625,8 @@ __global__ void __launch_bounds__(S::NW * 32, 1)
                         acc[i][jj][3] = fmaf(ag8, t[jj][3], acc[i][jj][3]);
                     }
                 }
-                finish_unit_regs<T, S>(acc, first, has_first, has_last, c, cm.left == 0 && kb0 + j + 1 == kb + n, p,
-                                       g, tq);
+                finish_unit_tma<T, S>(acc, has_first, has_last, c, cm.left == 0 && kb0 + j + 1 == kb + n, p, lut, warp,
+                                      lane, g, tq);
             }
             ++consumed;
             // Hand the slot back to the copy engine: order this warp's reads
@@ -638,7 +643,16 @@ __global__ void __launch_bounds__(S::NW * 32, 1)
         }
     }
     __syncthreads();  // every warp is out of the stage ring: the slots may reuse it
-    if (has_first) store_slot<S>(first, slots, warp * 2, lane);
+    if (has_first) {
+        float first[S::TW][S::NJ][4];
+#pragma unroll
+        for (int i = 0; i < S::TW; ++i)
+#pragma unroll
+            for (int j = 0; j < S::NJ; ++j)
+#pragma unroll
+                for (int r = 0; r < 4; ++r) first[i][j][r] = lds_f32(parked_addr<S>(lut, warp, (i * S::NJ + j) * 4 + r, lane));
+        store_slot<S>(first, slots, warp * 2, lane);
+    }
     if (has_last) store_slot<S>(acc, slots, warp * 2 + 1, lane);
     __syncthreads();
     if (uc <= 0) return;
@@ -674,18 +688,18 @@ static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
     return fn;
 }
 
-// Weights: [N rows][K/2 bytes], box 64 x 128 B, 128-byte swizzle.
-// Absmax: [N rows][K/bs floats], box 64 x 4 floats.
-static cudaError_t make_tensor_maps(const GemmParams& p, CUtensorMap* tw, CUtensorMap* ta) {
+// Weights: [N rows][K/2 bytes], box 64 rows x (32 * UPS) bytes, 64/128-byte swizzle.
+// Absmax: [N rows][K/bs floats], box 64 rows x 4 floats.
+static cudaError_t make_tensor_maps(const GemmParams& p, int ups, CUtensorMap* tw, CUtensorMap* ta) {
     auto enc = tensor_map_encoder();
     if (!enc) return cudaErrorNotSupported;
     const cuuint32_t estride[2] = {1, 1};
     const cuuint64_t wdim[2] = {(cuuint64_t)(p.K / 2), (cuuint64_t)p.N};
     const cuuint64_t wstride[1] = {(cuuint64_t)(p.K / 2)};
-    const cuuint32_t wbox[2] = {128, 64};
+    const cuuint32_t wbox[2] = {(cuuint32_t)(32 * ups), 64};
     if (enc(tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(p.Wp), wdim, wstride, wbox, estride,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            CU_TENSOR_MAP_INTERLEAVE_NONE, ups == 4 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
         return cudaErrorInvalidValue;
     const cuuint64_t adim[2] = {(cuuint64_t)p.am_per_row, (cuuint64_t)p.N};
     const cuuint64_t astride[1] = {(cuuint64_t)p.am_per_row * 4};
@@ -707,19 +721,19 @@ static int max_dynamic_smem() {
     return v;
 }
 
-template <typename T, class S>
+template <typename T, class S, int UPS>
 static cudaError_t launch_tma(const GemmParams& p, cudaStream_t stream) {
     CUtensorMap tw, ta;
-    cudaError_t e = make_tensor_maps(p, &tw, &ta);
+    cudaError_t e = make_tensor_maps(p, UPS, &tw, &ta);
     if (e != cudaSuccess) return e;
     const int smem = max_dynamic_smem();  // the kernel lays out LUT, barriers and stages itself
     if (smem <= 0) return cudaErrorInvalidValue;
     if (p.am_shift == 0) {
-        auto kern = q4_gemm_tma_kernel<T, S, true>;
+        auto kern = q4_gemm_tma_kernel<T, S, UPS, true>;
         if ((e = ensure_smem_attr((const void*)kern, (size_t)smem)) != cudaSuccess) return e;
         kern<<<p.ctas, S::NW * 32, smem, stream>>>(tw, ta, p);
     } else {
-        auto kern = q4_gemm_tma_kernel<T, S, false>;
+        auto kern = q4_gemm_tma_kernel<T, S, UPS, false>;
         if ((e = ensure_smem_attr((const void*)kern, (size_t)smem)) != cudaSuccess) return e;
         kern<<<p.ctas, S::NW * 32, smem, stream>>>(tw, ta, p);
     }
@@ -738,17 +752,23 @@ struct Variant {
         ACT, 1, SB, MP, NW, D, PF, GemmShape<SB, MP, 4, NW, D, PF>::SMEM_BYTES,               \
             &launch_mma<T, GemmShape<SB, MP, 4, NW, D, PF>>                                   \
     }
-// TMA stage ring (loader 2): the depth is the number of stages per warp.
+// TMA stage rings: loader 2 = 4-unit (128-byte) stages, loader 3 = 2-unit
+// (64-byte) stages; the depth is the number of stages per warp.
 #define Q4_TMA_VARIANT(ACT, T, MP, NW, D)                                                      \
     Variant {                                                                                 \
-        ACT, 2, 64, MP, NW, D, 0, 0, &launch_tma<T, GemmShape<64, MP, 4, NW, D, 0>>            \
+        ACT, 2, 64, MP, NW, D, 0, 0, &launch_tma<T, GemmShape<64, MP, 4, NW, D, 0>, 4>         \
+    }
+#define Q4_TMA2_VARIANT(ACT, T, MP, NW, D)                                                     \
+    Variant {                                                                                 \
+        ACT, 3, 64, MP, NW, D, 0, 0, &launch_tma<T, GemmShape<64, MP, 4, NW, D, 0>, 2>         \
     }
 
 #define Q4_VARIANTS_FOR(ACT, T)                                                                \
     Q4_VARIANT(ACT, T, 64, 8, 16, 1, 128), Q4_VARIANT(ACT, T, 64, 8, 8, 2, 128),               \
         Q4_VARIANT(ACT, T, 64, 16, 8, 1, 128), Q4_VARIANT(ACT, T, 32, 8, 16, 1, 128),         \
         Q4_VARIANT(ACT, T, 32, 16, 8, 1, 128), Q4_TMA_VARIANT(ACT, T, 8, 8, 2),               \
-        Q4_TMA_VARIANT(ACT, T, 16, 8, 2)
+        Q4_TMA_VARIANT(ACT, T, 16, 8, 2), Q4_TMA2_VARIANT(ACT, T, 8, 16, 2),                  \
+        Q4_TMA2_VARIANT(ACT, T, 16, 8, 4)
 
 static const Variant kVariants[] = {
     Q4_VARIANTS_FOR(0, __nv_bfloat16),
@@ -759,15 +779,16 @@ static const Variant kVariants[] = {
     Q4_VARIANT(0, __nv_bfloat16, 64, 8, 8, 2, 0),
     Q4_VARIANT(0, __nv_bfloat16, 64, 8, 8, 1, 128),
     Q4_TMA_VARIANT(0, __nv_bfloat16, 8, 16, 1),
-    Q4_TMA_VARIANT(0, __nv_bfloat16, 8, 4, 4),
     Q4_TMA_VARIANT(0, __nv_bfloat16, 8, 12, 1),
-    Q4_TMA_VARIANT(0, __nv_bfloat16, 8, 6, 2),
+    Q4_TMA2_VARIANT(0, __nv_bfloat16, 8, 8, 4),
+    Q4_TMA2_VARIANT(0, __nv_bfloat16, 8, 12, 2),
+    Q4_TMA2_VARIANT(0, __nv_bfloat16, 8, 16, 1),
 };
 
 static const Variant* find_variant(int act, const GemmChoice& ch) {
     for (const Variant& v : kVariants)
         if (v.act == act && v.loader == ch.loader && v.sub_block == ch.sub_block && v.m_pad == ch.m_pad &&
-            v.warps == ch.warps && v.depth == ch.depth && (ch.loader == 2 || v.l2pf == ch.l2pf))
+            v.warps == ch.warps && v.depth == ch.depth && (ch.loader >= 2 || v.l2pf == ch.l2pf))
             return &v;
     return nullptr;
 }
@@ -777,7 +798,7 @@ bool gemm_variant_exists(int act_dtype, const GemmChoice& ch) { return find_vari
 size_t gemm_smem_bytes(int act_dtype, const GemmChoice& ch) {
     const Variant* v = find_variant(act_dtype, ch);
     if (!v) return 0;
-    return v->loader == 2 ? (size_t)max_dynamic_smem() : v->smem;
+    return v->loader >= 2 ? (size_t)max_dynamic_smem() : v->smem;
 }
 
 cudaError_t gemm_launch(const GemmChoice& ch, int act_dtype, const GemmParams& p, cudaStream_t stream) {

@@ -150,7 +150,8 @@ typedef struct {
     int ctas;          /* persistent CTAs (<= SM count, <= number of units)       */
     int depth;         /* work units each warp has in flight ahead of its compute */
     int l2_prefetch;   /* L2 fetch-size hint on weight loads: 1 none, 128, 256 B  */
-    int loader;        /* 1 = per-lane global loads, 2 = TMA shared-memory ring   */
+    int loader;        /* 1 = per-lane global loads; TMA shared-memory ring with  */
+                       /* 2 = 4-unit (128-byte) or 3 = 2-unit (64-byte) stages   */
     int tiles;         /* ceil(N / rows_per_tile)                                 */
     int64_t units;     /* tiles * (K / sub_block)                                 */
     size_t smem_bytes; /* dynamic shared memory per CTA                           */

@@ -69,7 +69,7 @@ def _problem(device, M=3, N=300, K=1024, bs=64, seed=7):
             torch.from_numpy(code).to(device), N, K, bs)
 
 
-@pytest.mark.parametrize("loader", [1, 2])
+@pytest.mark.parametrize("loader", [1, 2, 3])
 def test_deterministic_and_counters_left_zero(cuda_device, loader):
     A, P, Am, C, N, K, bs = _problem(cuda_device)
     ws = q4.Workspace(cuda_device)
@@ -110,30 +110,34 @@ def test_direct_load_variants(cuda_device, depth, l2pf, warps):
              l2_prefetch=l2pf, warps=warps, ctas=5, loader=1)
 
 
-@pytest.mark.parametrize("warps,depth", [(8, 2), (16, 1), (4, 4), (12, 1), (6, 2)])
-def test_tma_ring_variants(cuda_device, warps, depth):
+@pytest.mark.parametrize("loader,warps,depth", [(2, 8, 2), (2, 16, 1), (2, 12, 1), (3, 16, 2), (3, 8, 4), (3, 12, 2),
+                                                (3, 16, 1)])
+def test_tma_ring_variants(cuda_device, loader, warps, depth):
     run_case(Case(1, 700, 2048), seed=7200 + warps, device=cuda_device, check_quantizer=False, depth=depth,
-             warps=warps, loader=2)
+             warps=warps, loader=loader)
     run_case(Case(3, 190, 768), seed=7300 + warps, device=cuda_device, check_quantizer=False, depth=depth,
-             warps=warps, ctas=5, loader=2)
+             warps=warps, ctas=5, loader=loader)
 
 
 @pytest.mark.parametrize("M", [1, 7, 8, 9, 16])
 @pytest.mark.parametrize("N,K,bs", [(1, 256, 64), (64, 256, 64), (100, 1280, 64), (513, 1024, 128), (300, 4096, 256),
                                     (257, 3072, 64), (70, 512, 128)])
-def test_tma_ring_shapes(cuda_device, M, N, K, bs):
-    run_case(Case(M, N, K, blocksize=bs), seed=7400 + M + N, device=cuda_device, check_quantizer=False, loader=2)
+@pytest.mark.parametrize("loader", [2, 3])
+def test_tma_ring_shapes(cuda_device, M, N, K, bs, loader):
+    run_case(Case(M, N, K, blocksize=bs), seed=7400 + M + N, device=cuda_device, check_quantizer=False, loader=loader)
 
 
 @pytest.mark.parametrize("ctas", [1, 2, 3, 7, 33, 148])
-def test_tma_ring_partitions(cuda_device, ctas):
-    run_case(Case(2, 257, 1280), seed=7500 + ctas, device=cuda_device, check_quantizer=False, loader=2, ctas=ctas)
+@pytest.mark.parametrize("loader", [2, 3])
+def test_tma_ring_partitions(cuda_device, ctas, loader):
+    run_case(Case(2, 257, 1280), seed=7500 + ctas, device=cuda_device, check_quantizer=False, loader=loader, ctas=ctas)
 
 
 def test_tma_error_word_stays_zero(cuda_device):
     ws = q4.Workspace(cuda_device)
     A, P, Am, C, N, K, bs = _problem(cuda_device)
-    q4.q4_gemm_skinny(A, P, Am, C, N, K, bs, workspace=ws, loader=2)
+    for loader in (2, 3):
+        q4.q4_gemm_skinny(A, P, Am, C, N, K, bs, workspace=ws, loader=loader)
     torch.cuda.synchronize()
     assert q4.workspace_error(ws) == 0
 
