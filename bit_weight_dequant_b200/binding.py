@@ -33,7 +33,8 @@ class Q4Error(RuntimeError):
 class q4_gemm_plan_t(ctypes.Structure):
     _fields_ = [("math", ctypes.c_int), ("sub_block", ctypes.c_int), ("m_pad", ctypes.c_int),
                 ("rows_per_tile", ctypes.c_int), ("warps", ctypes.c_int), ("ctas", ctypes.c_int),
-                ("depth", ctypes.c_int), ("l2_prefetch", ctypes.c_int), ("loader", ctypes.c_int), ("tiles", ctypes.c_int),
+                ("depth", ctypes.c_int), ("l2_prefetch", ctypes.c_int), ("loader", ctypes.c_int), ("pdl", ctypes.c_int),
+                ("tiles", ctypes.c_int),
                 ("units", ctypes.c_int64), ("smem_bytes", ctypes.c_size_t), ("workspace_bytes", ctypes.c_size_t)]
 
 
@@ -175,7 +176,7 @@ def _default_workspace(device) -> Workspace:
 
 
 def overrides(**kw) -> q4_gemm_plan_t | None:
-    """Launch-table overrides (math, warps, ctas, depth, l2_prefetch, loader); None if empty."""
+    """Launch-table overrides (math, warps, ctas, depth, l2_prefetch, loader, pdl); None if empty."""
     kw = {k: v for k, v in kw.items() if v}
     if not kw:
         return None
@@ -191,7 +192,8 @@ def q4_gemm_skinny(A: torch.Tensor, Wpacked: torch.Tensor, absmax: torch.Tensor,
     """out[M, N] = A[M, K] . dequant(W)[N, K]^T on the GPU (fused kernel).
 
     ``launch`` may hold launch-table overrides (math, warps, ctas, depth,
-    l2_prefetch) for measurements; by default the table decides."""
+    l2_prefetch, loader) for measurements, and ``pdl`` to opt into
+    programmatic dependent launch (see q4.h); by default the table decides."""
     M = A.shape[0] if A.dim() == 2 else 1
     if out is None:
         out = torch.empty((M, N), dtype=A.dtype, device=A.device)

@@ -87,7 +87,7 @@ static int gemm_choose(int M, int N, int K, int blocksize, int act_dtype, int nu
     if (M < 0 || N < 0 || K < 0) return Q4_ERR_INVALID_ARG;
     if (!is_pow2_blocksize(blocksize)) return Q4_ERR_INVALID_ARG;
     if (act_dtype != Q4_BF16 && act_dtype != Q4_FP16 && act_dtype != Q4_FP32) return Q4_ERR_INVALID_ARG;
-    if (ov && (ov->math > 2 || ov->l2_prefetch > 256 || ov->loader > 3)) return Q4_ERR_INVALID_ARG;
+    if (ov && (ov->math > 2 || ov->l2_prefetch > 256 || ov->loader > 3 || ov->pdl > 2)) return Q4_ERR_INVALID_ARG;
     if (M > 16 || act_dtype == Q4_FP32 || K % blocksize != 0) return Q4_ERR_UNSUPPORTED;
     GemmChoice c{};
     c.math = 1;
@@ -114,8 +114,10 @@ static int gemm_choose(int M, int N, int K, int blocksize, int act_dtype, int nu
         c.depth = 1;
         c.l2pf = 128;
     }
+    c.pdl = 0;
     if (ov) {
         if (ov->math > 0) c.math = ov->math;
+        if (ov->pdl > 0) c.pdl = c.loader == 1 ? 1 : ov->pdl;  // the direct kernel reads nothing early
         if (ov->warps > 0) c.warps = ov->warps;
         if (ov->depth > 0) c.depth = ov->depth;
         if (ov->l2_prefetch > 0) c.l2pf = ov->l2_prefetch == 1 ? 0 : ov->l2_prefetch;
@@ -196,6 +198,7 @@ int q4_gemm_plan(int M, int N, int K, int blocksize, int act_dtype, int num_sms,
     plan->depth = ch.depth;
     plan->l2_prefetch = ch.l2pf == 0 ? 1 : ch.l2pf;
     plan->loader = ch.loader;
+    plan->pdl = ch.pdl;
     plan->tiles = tiles;
     plan->units = units;
     plan->smem_bytes = gemm_smem_bytes(act_dtype == Q4_FP32 ? Q4_BF16 : act_dtype, ch);
@@ -234,7 +237,7 @@ int q4_gemm_skinny_ex(const void* A, const uint8_t* Wpacked, const float* absmax
         q4_gemm_plan_t ov1{};
         if (overrides) ov1 = *overrides;
         ov1.loader = 1;
-        ov1.warps = ov1.depth = ov1.l2_prefetch = 0;
+        ov1.warps = ov1.depth = ov1.l2_prefetch = 0;  // keep ctas and pdl
         rc = gemm_choose(M, N, K, blocksize, act_dtype, 0, &ov1, &fb, &tiles, &units, &need, &sms);
         if (rc != Q4_OK) return rc;
         ch = fb;
@@ -260,6 +263,7 @@ int q4_gemm_skinny_ex(const void* A, const uint8_t* Wpacked, const float* absmax
     while ((ch.sub_block << sh) < blocksize) ++sh;
     p.am_shift = sh;
     p.am_per_row = K / blocksize;
+    p.pdl = ch.pdl;
     p.tiles = tiles;
     p.ctas = ch.ctas;
     p.units = units;

@@ -175,6 +175,12 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const void* tmap, int 
         : "memory");
 }
 
+// Programmatic dependent launch: block until the grids this one depends on
+// have completed and their writes are visible (a no-op without the launch
+// attribute); allow the next dependent grid to begin launching.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 __device__ __forceinline__ uint32_t dynamic_smem_size() {
     uint32_t v;
     asm("mov.u32 %0, %%dynamic_smem_size;" : "=r"(v));

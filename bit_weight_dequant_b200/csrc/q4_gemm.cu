@@ -305,6 +305,7 @@ __device__ __forceinline__ void build_lut(uint32_t lut, const float* code, int t
 
 template <typename T, class S>
 __global__ void __launch_bounds__(S::NW * 32, 1) q4_gemm_mma_kernel(const GemmParams p) {
+    griddep_wait();  // no overlap with a preceding grid in this kernel
     extern __shared__ __align__(16) uint8_t smem[];
     const uint32_t sbase = smem_addr(smem);
     const uint32_t lut = (sbase + 0xFFFFu) & ~0xFFFFu;  // 64 KiB aligned (host reserves the padding)
@@ -509,6 +510,7 @@ __global__ void __launch_bounds__(S::NW * 32, 1)
         return (uint32_t)idx < na ? a0 + (uint32_t)idx * G::BYTES : b0 + ((uint32_t)idx - na) * G::BYTES;
     };
 
+    if (p.pdl != 2) griddep_wait();
     build_lut<T>(lut, p.code, tid, S::NW * 32);
     if (lane == 0) {
         for (int d = 0; d < D; ++d) mbar_init(bars + (uint32_t)(warp * D + d) * 8u, 1);
@@ -527,6 +529,7 @@ __global__ void __launch_bounds__(S::NW * 32, 1)
     float acc[S::TW][S::NJ][4];
     bool has_first = false, has_last = false;
     zero_acc<S>(acc);
+    if (nunits <= 0 && p.pdl == 2) griddep_wait();
     if (nunits > 0) {
         Cursor c;
         c.tile = (int)(ws / p.kb_per_tile);
@@ -553,6 +556,32 @@ __global__ void __launch_bounds__(S::NW * 32, 1)
             }
         };
         for (; issued < D && ld.left > 0; ++issued) issue(issued);
+        // Activations, outputs and the workspace may belong to the preceding
+        // grid: touch them only after the dependency wait.
+        if (p.pdl == 2) griddep_wait();
+        griddep_launch_dependents();
+
+        // activations of the unit being computed (bw) and of the next one (bwn)
+        uint32_t bw[S::NJ][2][4], bwn[S::NJ][2][4];
+        auto load_act = [&](int kunit, uint32_t(&dst)[S::NJ][2][4]) {
+#pragma unroll
+            for (int jj = 0; jj < S::NJ; ++jj) {
+                const int m = 8 * jj + g;
+#pragma unroll
+                for (int ch = 0; ch < 2; ++ch) {
+                    if (m < p.M) {
+                        const uint4 v = ldg_v4(Aact + (size_t)m * p.K + kunit + 32 * ch + 8 * tq);
+                        dst[jj][ch][0] = v.x;
+                        dst[jj][ch][1] = v.y;
+                        dst[jj][ch][2] = v.z;
+                        dst[jj][ch][3] = v.w;
+                    } else {
+                        dst[jj][ch][0] = dst[jj][ch][1] = dst[jj][ch][2] = dst[jj][ch][3] = 0u;
+                    }
+                }
+            }
+        };
+        load_act(c.kb * S::SB, bw);
 
         while (cm.left > 0) {
             int tile, kb0, kb, n;
@@ -568,25 +597,12 @@ __global__ void __launch_bounds__(S::NW * 32, 1)
 #pragma unroll
             for (int j = 0; j < UPS; ++j) {
                 if (kb0 + j < kb || kb0 + j >= kb + n) continue;
-                const int kunit = (kb0 + j) * S::SB;
-                // activation runs: row 8jj+g, k = kunit + 32ch + 8tq .. +8
-                uint32_t bw[S::NJ][2][4];
-#pragma unroll
-                for (int jj = 0; jj < S::NJ; ++jj) {
-                    const int m = 8 * jj + g;
-#pragma unroll
-                    for (int ch = 0; ch < 2; ++ch) {
-                        if (m < p.M) {
-                            const uint4 v = ldg_v4(Aact + (size_t)m * p.K + kunit + 32 * ch + 8 * tq);
-                            bw[jj][ch][0] = v.x;
-                            bw[jj][ch][1] = v.y;
-                            bw[jj][ch][2] = v.z;
-                            bw[jj][ch][3] = v.w;
-                        } else {
-                            bw[jj][ch][0] = bw[jj][ch][1] = bw[jj][ch][2] = bw[jj][ch][3] = 0u;
-                        }
-                    }
-                }
+                // prefetch the activations of the next unit of the range
+                // (activation runs: row 8jj+g, k = kunit + 32ch + 8tq .. +8)
+                if (kb0 + j + 1 < kb + n)
+                    load_act((kb0 + j + 1) * S::SB, bwn);
+                else if (cm.left > 0)
+                    load_act(cm.kb * S::SB, bwn);
                 // absmax column of this unit inside the stage's 4-float box
                 const int col = BS64 ? (kb0 + j - x0) : (((kb0 + j) >> p.am_shift) - x0);
                 const uint32_t am_base = st + G::WEIGHT_BYTES + (uint32_t)col * 4u;
@@ -627,6 +643,12 @@ __global__ void __launch_bounds__(S::NW * 32, 1)
                 }
                 finish_unit_tma<T, S>(acc, has_first, has_last, c, cm.left == 0 && kb0 + j + 1 == kb + n, p, lut, warp,
                                       lane, g, tq);
+#pragma unroll
+                for (int jj = 0; jj < S::NJ; ++jj)
+#pragma unroll
+                    for (int ch = 0; ch < 2; ++ch)
+#pragma unroll
+                        for (int w = 0; w < 4; ++w) bw[jj][ch][w] = bwn[jj][ch][w];
             }
             ++consumed;
             // Hand the slot back to the copy engine: order this warp's reads
@@ -667,7 +689,18 @@ static cudaError_t launch_mma(const GemmParams& p, cudaStream_t stream) {
     auto kern = q4_gemm_mma_kernel<T, S>;
     cudaError_t e = ensure_smem_attr((const void*)kern, S::SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    kern<<<p.ctas, S::NW * 32, S::SMEM_BYTES, stream>>>(p);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)p.ctas);
+    cfg.blockDim = dim3(S::NW * 32);
+    cfg.dynamicSmemBytes = S::SMEM_BYTES;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = p.pdl ? 1 : 0;
+    e = cudaLaunchKernelEx(&cfg, kern, p);
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 
@@ -728,15 +761,20 @@ static cudaError_t launch_tma(const GemmParams& p, cudaStream_t stream) {
     if (e != cudaSuccess) return e;
     const int smem = max_dynamic_smem();  // the kernel lays out LUT, barriers and stages itself
     if (smem <= 0) return cudaErrorInvalidValue;
-    if (p.am_shift == 0) {
-        auto kern = q4_gemm_tma_kernel<T, S, UPS, true>;
-        if ((e = ensure_smem_attr((const void*)kern, (size_t)smem)) != cudaSuccess) return e;
-        kern<<<p.ctas, S::NW * 32, smem, stream>>>(tw, ta, p);
-    } else {
-        auto kern = q4_gemm_tma_kernel<T, S, UPS, false>;
-        if ((e = ensure_smem_attr((const void*)kern, (size_t)smem)) != cudaSuccess) return e;
-        kern<<<p.ctas, S::NW * 32, smem, stream>>>(tw, ta, p);
-    }
+    auto kern = p.am_shift == 0 ? q4_gemm_tma_kernel<T, S, UPS, true> : q4_gemm_tma_kernel<T, S, UPS, false>;
+    if ((e = ensure_smem_attr((const void*)kern, (size_t)smem)) != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)p.ctas);
+    cfg.blockDim = dim3(S::NW * 32);
+    cfg.dynamicSmemBytes = (size_t)smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = p.pdl ? 1 : 0;
+    e = cudaLaunchKernelEx(&cfg, kern, tw, ta, p);
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 

@@ -21,6 +21,7 @@ struct GemmChoice {
     int depth;      // units (loader 1) or stages (loader 2) in flight per warp
     int l2pf;       // L2 fetch-size hint on weight loads: 0 (none), 128, 256 (loader 1)
     int loader;     // 1 = per-lane global loads, 2/3 = TMA stage ring of 4/2-unit stages
+    int pdl;        // programmatic dependent launch mode (0, 1, 2)
 };
 
 // Sets cudaFuncAttributeMaxDynamicSharedMemorySize once per (kernel, device).

@@ -61,6 +61,8 @@ struct GemmParams {
     float* partials;   // [ctas][2][SLOT_FLOATS]
     int* counters;     // [tiles], zero between calls
     int* error;        // workspace error word (0 = ok); set when a bounded wait gives up
+    int pdl;           // 0: plain launch; 1: dependent launch, every global access after the
+                       // dependency wait; 2: code/weights/absmax read before that wait
     int M, N, K;
     int kb_per_tile;   // K / SB
     int am_shift;      // log2(blocksize / SB): absmax column of unit column kb = kb >> am_shift

@@ -152,6 +152,11 @@ typedef struct {
     int l2_prefetch;   /* L2 fetch-size hint on weight loads: 1 none, 128, 256 B  */
     int loader;        /* 1 = per-lane global loads; TMA shared-memory ring with  */
                        /* 2 = 4-unit (128-byte) or 3 = 2-unit (64-byte) stages   */
+    int pdl;           /* programmatic dependent launch: 0 off; 1 on, the kernel  */
+                       /* touches global memory only after the preceding grid    */
+                       /* completed; 2 on, and code/Wpacked/absmax may be read   */
+                       /* before that (they must not be written by the grid that */
+                       /* precedes the call on the stream, e.g. static weights)  */
     int tiles;         /* ceil(N / rows_per_tile)                                 */
     int64_t units;     /* tiles * (K / sub_block)                                 */
     size_t smem_bytes; /* dynamic shared memory per CTA                           */
@@ -163,9 +168,10 @@ int q4_gemm_plan(int M, int N, int K, int blocksize, int act_dtype, int num_sms,
 
 /*
  * Same as q4_gemm_skinny with explicit launch-table overrides, used to
- * measure the choices the table makes.  `overrides` may be NULL; in it,
- * math, warps, ctas, depth, l2_prefetch and loader override the table when
- * > 0 (all other fields are ignored).  A combination that was not compiled returns
+ * measure the choices the table makes and to opt into programmatic
+ * dependent launch.  `overrides` may be NULL; in it, math, warps, ctas,
+ * depth, l2_prefetch, loader and pdl override the table when > 0 (all
+ * other fields are ignored).  A combination that was not compiled returns
  * Q4_ERR_UNSUPPORTED; ctas above the SM count returns Q4_ERR_INVALID_ARG.
  * The workspace size needed does not depend on the overrides.
  */

@@ -196,3 +196,34 @@ def test_one_hot_activation_selects_dequantized_column(cuda_device):
         want = want_all[:, k]
         got = out[0].to(torch.float64).cpu().numpy()
         assert np.all(np.abs(got - want) <= oracle.ulp(want, oracle.BF16)), k
+
+
+@pytest.mark.parametrize("pdl", [1, 2])
+@pytest.mark.parametrize("loader", [1, 3])
+def test_dependent_launch_chain(cuda_device, pdl, loader):
+    """A chain where each GEMM reads the previous GEMM's output as its
+    activations: with programmatic dependent launch the second kernel may
+    start early, but must read its activations only after the first one
+    finished.  The result must equal the chain run without it, bit for bit."""
+    dims = [2048, 1536, 2560, 1024]                  # K of step i = N of step i-1
+    code = inputs.code_normal_quantile()
+    C = torch.from_numpy(code).to(cuda_device)
+    layers = []
+    for i in range(len(dims) - 1):
+        K, N = dims[i], dims[i + 1]
+        packed, absmax = oracle.quantize(inputs.weights(N, K, 900 + i), 64, code)
+        layers.append((torch.from_numpy(packed).to(cuda_device), torch.from_numpy(absmax).to(cuda_device), N, K))
+    A0 = inputs.activations(4, dims[0], torch.bfloat16, 901).to(cuda_device)
+
+    def chain(**launch):
+        x = A0
+        for (P, Am, N, K) in layers:
+            x = q4.q4_gemm_skinny(x, P, Am, C, N, K, 64, loader=loader, **launch)
+        return x
+
+    ref = chain()
+    torch.cuda.synchronize()
+    for _ in range(3):
+        got = chain(pdl=pdl)
+        torch.cuda.synchronize()
+        assert torch.equal(got.view(torch.int16), ref.view(torch.int16))
