@@ -57,11 +57,13 @@ def lib() -> ctypes.CDLL:
         L.q4_gemm_skinny.argtypes = [P, P, P, P, ci, ci, ci, ci, ci, P, P, sz, P]
         L.q4_gemm_skinny_ex.argtypes = [P, P, P, P, ci, ci, ci, ci, ci, P, P, sz, P, ctypes.POINTER(q4_gemm_plan_t)]
         L.q4_gemm_plan.argtypes = [ci, ci, ci, ci, ci, ci, ctypes.POINTER(q4_gemm_plan_t)]
+        L.q4_gemm_skinny_noalloc.argtypes = [P, P, P, P, ci, ci, ci, ci, ci, P, P]
         L.q4_partition_start.argtypes = [i64, ci, ci]
         L.q4_partition_start.restype = i64
         L.q4_partition_owner.argtypes = [i64, ci, i64]
         for f in ("q4_quantize_blockwise", "q4_dequantize_blockwise", "q4_gemm_workspace_size",
-                  "q4_gemm_skinny", "q4_gemm_skinny_ex", "q4_gemm_plan", "q4_partition_owner"):
+                  "q4_gemm_skinny", "q4_gemm_skinny_ex", "q4_gemm_plan", "q4_partition_owner",
+                  "q4_gemm_skinny_noalloc"):
             getattr(L, f).restype = ci
         _lib = L
     return _lib
@@ -207,4 +209,17 @@ def q4_gemm_skinny(A: torch.Tensor, Wpacked: torch.Tensor, absmax: torch.Tensor,
                                  _ptr(out), _ptr(ws), ws.numel() if ws is not None else 0, _stream(A.device),
                                  ctypes.byref(ov) if ov is not None else None)
     _check(rc, "q4_gemm_skinny")
+    return out
+
+
+def q4_gemm_skinny_noalloc(A: torch.Tensor, Wpacked: torch.Tensor, absmax: torch.Tensor, code: torch.Tensor, N: int,
+                           K: int, blocksize: int, out: torch.Tensor | None = None) -> torch.Tensor:
+    """q4_gemm_skinny on the library's built-in scratch array: no workspace
+    is allocated, by this call or by the library (see q4.h)."""
+    M = A.shape[0] if A.dim() == 2 else 1
+    if out is None:
+        out = torch.empty((M, N), dtype=A.dtype, device=A.device)
+    rc = lib().q4_gemm_skinny_noalloc(_ptr(A), _ptr(Wpacked), _ptr(absmax), _ptr(code), M, N, K, blocksize,
+                                      _TORCH_TO_Q4[A.dtype], _ptr(out), _stream(A.device))
+    _check(rc, "q4_gemm_skinny_noalloc")
     return out

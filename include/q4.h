@@ -139,6 +139,32 @@ int q4_gemm_skinny(const void* A, const uint8_t* Wpacked, const float* absmax, c
                    int M, int N, int K, int blocksize, int act_dtype, void* out, void* workspace,
                    size_t workspace_bytes, void* stream);
 
+/*
+ * q4_gemm_skinny for callers that cannot allocate device memory (code that
+ * runs while a stream is captured into a CUDA graph, runtimes that forbid
+ * device allocations after start-up, plugin hosts that hand out no memory).
+ * The paper has no counterpart: it exists for such callers only.
+ *
+ * Same arguments and results as q4_gemm_skinny, without the workspace: the
+ * scratch is a fixed array of Q4_NOALLOC_WORKSPACE_BYTES compiled into the
+ * library, which every GPU that loads the library holds until the process
+ * exits.  No call allocates or frees memory (no cudaMalloc, no cudaFree,
+ * no allocating library routine).
+ *   - A problem whose workspace (q4_gemm_workspace_size) exceeds that size
+ *     returns Q4_ERR_WORKSPACE and enqueues nothing.
+ *   - The first call on a device looks the array's device address up once,
+ *     with that device current (cudaGetSymbolAddress); make that first call
+ *     before capturing a stream into a CUDA graph.
+ *   - Every call shares the one array and clears its error word and tile
+ *     counters with cudaMemsetAsync on `stream` before the kernel; calls that
+ *     overlap on the GPU (other streams, other threads) race on it.
+ */
+#define Q4_NOALLOC_WORKSPACE_BYTES (2u << 20) /* 2 MiB */
+
+int q4_gemm_skinny_noalloc(const void* A, const uint8_t* Wpacked, const float* absmax,
+                           const float* code, int M, int N, int K, int blocksize, int act_dtype,
+                           void* out, void* stream);
+
 /* Launch-table entry chosen for a GEMM problem (host-only, for reporting and
  * tests).  `num_sms` <= 0 means "the current device's SM count". */
 typedef struct {
