@@ -92,6 +92,15 @@ __device__ __forceinline__ uint4 ldg_v4(const void* p) {
     return v;
 }
 
+// gpu-scope atomic add with acquire-release semantics: publishes this
+// thread's (and, by cumulativity, its warp's synchronised) earlier writes and
+// observes the writes published by earlier adds to the same counter.
+__device__ __forceinline__ int atom_add_acq_rel_gpu(int* p, int v) {
+    int old;
+    asm volatile("atom.add.acq_rel.gpu.s32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+    return old;
+}
+
 // L2-coherent load (bypasses L1): for data other CTAs wrote in this launch.
 __device__ __forceinline__ float ldg_cg_f32(const float* p) {
     float v;

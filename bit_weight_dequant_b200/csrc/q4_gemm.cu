@@ -269,14 +269,14 @@ __device__ __forceinline__ void combine_tiles(const GemmParams& p, uint32_t slot
             for (int j = 0; j < S::NJ; ++j)
 #pragma unroll
                 for (int r = 0; r < 4; ++r) mine[((i * S::NJ + j) * 4 + r) * 32 + lane] = sum[i][j][r];
-        __threadfence();
+        // Release the warp's partial and count it in; the add also acquires
+        // the partials the other CTAs released before it.
         __syncwarp();
         int prev = 0;
-        if (lane == 0) prev = atomicAdd(p.counters + t, 1);
+        if (lane == 0) prev = atom_add_acq_rel_gpu(p.counters + t, 1);
         prev = __shfl_sync(0xffffffffu, prev, 0);
         const int cf = part_owner(p.units, p.ctas, t0), cl = part_owner(p.units, p.ctas, t1 - 1);
         if (prev != cl - cf) continue;
-        __threadfence();
         zero_acc<S>(sum);
         for (int cta = cf; cta <= cl; ++cta) {
             const int which = (part_start(p.units, p.ctas, cta) / p.kb_per_tile == t) ? 0 : 1;
@@ -511,12 +511,11 @@ __global__ void __launch_bounds__(S::NW * 32, 1)
     };
 
     if (p.pdl != 2) griddep_wait();
-    build_lut<T>(lut, p.code, tid, S::NW * 32);
-    if (lane == 0) {
+    if (lane == 0) {  // each warp's own stage barriers; only this warp uses them
         for (int d = 0; d < D; ++d) mbar_init(bars + (uint32_t)(warp * D + d) * 8u, 1);
         mbar_init_fence();
     }
-    __syncthreads();
+    __syncwarp();
 
     const int64_t cs = part_start(p.units, p.ctas, blockIdx.x);
     const int64_t ce = part_start(p.units, p.ctas, blockIdx.x + 1);
@@ -529,37 +528,39 @@ __global__ void __launch_bounds__(S::NW * 32, 1)
     float acc[S::TW][S::NJ][4];
     bool has_first = false, has_last = false;
     zero_acc<S>(acc);
-    if (nunits <= 0 && p.pdl == 2) griddep_wait();
-    if (nunits > 0) {
-        Cursor c;
-        c.tile = (int)(ws / p.kb_per_tile);
-        c.kb = (int)(ws - (int64_t)c.tile * p.kb_per_tile);
-        c.from_start = (c.kb == 0);
-        c.first_tile = true;
-        StageCursor ld{c.tile, c.kb, nunits}, cm{c.tile, c.kb, nunits};
+    Cursor c;
+    c.tile = nunits > 0 ? (int)(ws / p.kb_per_tile) : 0;
+    c.kb = nunits > 0 ? (int)(ws - (int64_t)c.tile * p.kb_per_tile) : 0;
+    c.from_start = (c.kb == 0);
+    c.first_tile = true;
+    StageCursor ld{c.tile, c.kb, nunits}, cm{c.tile, c.kb, nunits};
+    int issued = 0, consumed = 0;
+    auto issue = [&](int k) {  // lane 0: stage k into ring slot k % D
+        int tile, kb0, kb, n;
+        next_stage<UPS>(ld, p.kb_per_tile, tile, kb0, kb, n);
+        const uint32_t st = stage_addr(warp * D + k % D);
+        const uint32_t bar = bars + (uint32_t)(warp * D + k % D) * 8u;
+        if (lane == 0) {
+            mbar_expect_tx(bar, G::BYTES);
+            tma_load_2d(st, &tmap_w, kb0 * 32, tile * S::TR, bar);
+            tma_load_2d(st + G::WEIGHT_BYTES, &tmap_a, (kb0 >> p.am_shift) & ~3, tile * S::TR, bar);
+        }
+    };
+    // Start the first copies before anything else; the table is built while
+    // they are in flight.
+    for (; issued < D && ld.left > 0; ++issued) issue(issued);
+    build_lut<T>(lut, p.code, tid, S::NW * 32);
+    __syncthreads();
+    // Activations, outputs and the workspace may belong to the preceding
+    // grid: touch them only after the dependency wait.
+    if (p.pdl == 2) griddep_wait();
+    griddep_launch_dependents();
 
+    if (nunits > 0) {
         // ldmatrix row address pieces: lane l feeds row l%8 of matrix l/8.
         const int lm_q = lane >> 3, lm_r = lane & 7;
         const T* Aact = static_cast<const T*>(p.A);
         bool ok = true;
-        int issued = 0, consumed = 0;
-
-        auto issue = [&](int k) {  // lane 0: stage k into ring slot k % D
-            int tile, kb0, kb, n;
-            next_stage<UPS>(ld, p.kb_per_tile, tile, kb0, kb, n);
-            const uint32_t st = stage_addr(warp * D + k % D);
-            const uint32_t bar = bars + (uint32_t)(warp * D + k % D) * 8u;
-            if (lane == 0) {
-                mbar_expect_tx(bar, G::BYTES);
-                tma_load_2d(st, &tmap_w, kb0 * 32, tile * S::TR, bar);
-                tma_load_2d(st + G::WEIGHT_BYTES, &tmap_a, (kb0 >> p.am_shift) & ~3, tile * S::TR, bar);
-            }
-        };
-        for (; issued < D && ld.left > 0; ++issued) issue(issued);
-        // Activations, outputs and the workspace may belong to the preceding
-        // grid: touch them only after the dependency wait.
-        if (p.pdl == 2) griddep_wait();
-        griddep_launch_dependents();
 
         // activations of the unit being computed (bw) and of the next one (bwn)
         uint32_t bw[S::NJ][2][4], bwn[S::NJ][2][4];
