@@ -87,7 +87,7 @@ static int gemm_choose(int M, int N, int K, int blocksize, int act_dtype, int nu
     if (M < 0 || N < 0 || K < 0) return Q4_ERR_INVALID_ARG;
     if (!is_pow2_blocksize(blocksize)) return Q4_ERR_INVALID_ARG;
     if (act_dtype != Q4_BF16 && act_dtype != Q4_FP16 && act_dtype != Q4_FP32) return Q4_ERR_INVALID_ARG;
-    if (ov && (ov->math > 2 || ov->l2_prefetch > 256 || ov->loader > 3 || ov->pdl > 2)) return Q4_ERR_INVALID_ARG;
+    if (ov && (ov->math > 2 || ov->l2_prefetch > 256 || ov->loader > 5 || ov->pdl > 2)) return Q4_ERR_INVALID_ARG;
     if (M > 16 || act_dtype == Q4_FP32 || K % blocksize != 0) return Q4_ERR_UNSUPPORTED;
     GemmChoice c{};
     c.math = 1;
@@ -109,6 +109,14 @@ static int gemm_choose(int M, int N, int K, int blocksize, int act_dtype, int nu
         c.warps = c.m_pad == 8 ? 16 : 8;
         c.depth = c.m_pad == 8 ? 2 : 4;
         c.l2pf = 0;
+    } else if (c.loader == 4) {
+        c.warps = 8;
+        c.depth = 2;
+        c.l2pf = 0;
+    } else if (c.loader == 5) {
+        c.warps = 16;
+        c.depth = 2;
+        c.l2pf = 0;
     } else {
         c.warps = c.m_pad == 8 ? 16 : 8;
         c.depth = 1;
@@ -123,6 +131,8 @@ static int gemm_choose(int M, int N, int K, int blocksize, int act_dtype, int nu
         if (ov->l2_prefetch > 0) c.l2pf = ov->l2_prefetch == 1 ? 0 : ov->l2_prefetch;
     }
     if (c.math != 1 || !gemm_variant_exists(act_dtype, c)) return Q4_ERR_UNSUPPORTED;
+    if ((int64_t)(N > 0 ? (N + c.rows_per_tile - 1) / c.rows_per_tile : 0) * (K / c.sub_block) >= (int64_t)kMaxUnits)
+        return Q4_ERR_UNSUPPORTED;  // more than 2^23 work units (> 2^35 weights)
     int sms = num_sms;
     if (sms <= 0 && device_sm_count(&sms) != 0) return Q4_ERR_CUDA;
     if (ov && ov->ctas > sms) return Q4_ERR_INVALID_ARG;
@@ -266,7 +276,7 @@ int q4_gemm_skinny_ex(const void* A, const uint8_t* Wpacked, const float* absmax
     p.pdl = ch.pdl;
     p.tiles = tiles;
     p.ctas = ch.ctas;
-    p.units = units;
+    p.units = (uint32_t)units;
     return from_cuda(gemm_launch(ch, act_dtype, p, st));
 }
 
@@ -277,14 +287,19 @@ int q4_gemm_skinny(const void* A, const uint8_t* Wpacked, const float* absmax, c
                              workspace_bytes, stream, nullptr);
 }
 
+// The exported partition functions compute with 64-bit integers; the kernels
+// use the 32-bit forms of the same formulas, which agree whenever
+// total * parts < 2^32 (the launcher enforces units < 2^23, parts <= 512).
 int64_t q4_partition_start(int64_t total, int parts, int part) {
     if (total < 0 || parts <= 0 || part < 0 || part > parts) return -1;
-    return part_start(total, parts, part);
+    if (total < (int64_t)kMaxUnits && parts <= 512) return part_start((uint32_t)total, (uint32_t)parts, (uint32_t)part);
+    return part_start64(total, parts, part);
 }
 
 int q4_partition_owner(int64_t total, int parts, int64_t u) {
     if (total <= 0 || parts <= 0 || u < 0 || u >= total) return -1;
-    return part_owner(total, parts, u);
+    if (total < (int64_t)kMaxUnits && parts <= 512) return (int)part_owner((uint32_t)total, (uint32_t)parts, (uint32_t)u);
+    return part_owner64(total, parts, u);
 }
 
 }  // extern "C"

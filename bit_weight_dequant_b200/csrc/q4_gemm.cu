@@ -238,23 +238,23 @@ __device__ __forceinline__ void advance(int& tile, int& kb, int kb_per_tile) {
 // between CTAs is published to the workspace, and the last CTA to arrive
 // sums all partials in CTA order and stores the tile.
 template <typename T, class S>
-__device__ __forceinline__ void combine_tiles(const GemmParams& p, uint32_t slots, int64_t cs, int64_t ce, int warp,
+__device__ __forceinline__ void combine_tiles(const GemmParams& p, uint32_t slots, uint32_t cs, uint32_t ce, int warp,
                                               int lane, int g, int tq) {
-    const int64_t uc = ce - cs;
-    const int ta = (int)(cs / p.kb_per_tile);
-    const int tb = (int)((ce - 1) / p.kb_per_tile);
+    const uint32_t uc = ce - cs, kbt = (uint32_t)p.kb_per_tile;
+    const int ta = (int)(cs / kbt);
+    const int tb = (int)((ce - 1) / kbt);
     for (int t = ta + warp; t <= tb; t += S::NW) {
-        const int64_t t0 = (int64_t)t * p.kb_per_tile, t1 = t0 + p.kb_per_tile;
-        const int64_t lo = t0 > cs ? t0 : cs, hi = t1 < ce ? t1 : ce;
-        const int wlo = part_owner(uc, S::NW, lo - cs), whi = part_owner(uc, S::NW, hi - 1 - cs);
+        const uint32_t t0 = (uint32_t)t * kbt, t1 = t0 + kbt;
+        const uint32_t lo = t0 > cs ? t0 : cs, hi = t1 < ce ? t1 : ce;
+        const int wlo = (int)part_owner(uc, S::NW, lo - cs), whi = (int)part_owner(uc, S::NW, hi - 1 - cs);
         const bool inside = (lo == t0) && (hi == t1);
         if (inside && wlo == whi) continue;  // already stored by its only warp
         float sum[S::TW][S::NJ][4];
         zero_acc<S>(sum);
         for (int w = wlo; w <= whi; ++w) {
-            const int64_t w0 = cs + part_start(uc, S::NW, w), w1 = cs + part_start(uc, S::NW, w + 1);
+            const uint32_t w0 = cs + part_start(uc, S::NW, w), w1 = cs + part_start(uc, S::NW, w + 1);
             if (w1 == w0) continue;  // empty warp range
-            add_slot<S>(sum, slots, w * 2 + ((w0 / p.kb_per_tile == t) ? 0 : 1), lane);
+            add_slot<S>(sum, slots, w * 2 + ((w0 >= t0) ? 0 : 1), lane);  // w0 >= t0: tile t is w's first
         }
         if (inside) {
             store_tile<T, S>(sum, p, t, g, tq);
@@ -275,11 +275,11 @@ __device__ __forceinline__ void combine_tiles(const GemmParams& p, uint32_t slot
         int prev = 0;
         if (lane == 0) prev = atom_add_acq_rel_gpu(p.counters + t, 1);
         prev = __shfl_sync(0xffffffffu, prev, 0);
-        const int cf = part_owner(p.units, p.ctas, t0), cl = part_owner(p.units, p.ctas, t1 - 1);
+        const int cf = (int)part_owner(p.units, p.ctas, t0), cl = (int)part_owner(p.units, p.ctas, t1 - 1);
         if (prev != cl - cf) continue;
         zero_acc<S>(sum);
         for (int cta = cf; cta <= cl; ++cta) {
-            const int which = (part_start(p.units, p.ctas, cta) / p.kb_per_tile == t) ? 0 : 1;
+            const int which = (part_start(p.units, p.ctas, cta) >= t0) ? 0 : 1;  // tile t is the CTA's first
             const float* src = p.partials + ((size_t)cta * 2 + which) * S::SLOT_FLOATS;
 #pragma unroll
             for (int i = 0; i < S::TW; ++i)
@@ -315,11 +315,11 @@ __global__ void __launch_bounds__(S::NW * 32, 1) q4_gemm_mma_kernel(const GemmPa
     build_lut<T>(lut, p.code, tid, S::NW * 32);
     __syncthreads();
 
-    const int64_t cs = part_start(p.units, p.ctas, blockIdx.x);
-    const int64_t ce = part_start(p.units, p.ctas, blockIdx.x + 1);
-    const int64_t uc = ce - cs;
-    const int64_t ws = cs + part_start(uc, S::NW, warp);
-    const int64_t we = cs + part_start(uc, S::NW, warp + 1);
+    const uint32_t cs = part_start(p.units, p.ctas, blockIdx.x);
+    const uint32_t ce = part_start(p.units, p.ctas, blockIdx.x + 1);
+    const uint32_t uc = ce - cs;
+    const uint32_t ws = cs + part_start(uc, S::NW, warp);
+    const uint32_t we = cs + part_start(uc, S::NW, warp + 1);
     const uint32_t lane4 = lut | ((uint32_t)lane << 2);
     const int nunits = (int)(we - ws);
 
@@ -327,8 +327,8 @@ __global__ void __launch_bounds__(S::NW * 32, 1) q4_gemm_mma_kernel(const GemmPa
         float acc[S::TW][S::NJ][4];
         zero_acc<S>(acc);
         Cursor c;
-        c.tile = (int)(ws / p.kb_per_tile);
-        c.kb = (int)(ws - (int64_t)c.tile * p.kb_per_tile);
+        c.tile = (int)(ws / (uint32_t)p.kb_per_tile);
+        c.kb = (int)(ws - (uint32_t)c.tile * (uint32_t)p.kb_per_tile);
         c.from_start = (c.kb == 0);
         c.first_tile = true;
         // Ring of DEPTH + 1 unit buffers: the loads of DEPTH units are in
@@ -517,11 +517,11 @@ __global__ void __launch_bounds__(S::NW * 32, 1)
     }
     __syncwarp();
 
-    const int64_t cs = part_start(p.units, p.ctas, blockIdx.x);
-    const int64_t ce = part_start(p.units, p.ctas, blockIdx.x + 1);
-    const int64_t uc = ce - cs;
-    const int64_t ws = cs + part_start(uc, S::NW, warp);
-    const int64_t we = cs + part_start(uc, S::NW, warp + 1);
+    const uint32_t cs = part_start(p.units, p.ctas, blockIdx.x);
+    const uint32_t ce = part_start(p.units, p.ctas, blockIdx.x + 1);
+    const uint32_t uc = ce - cs;
+    const uint32_t ws = cs + part_start(uc, S::NW, warp);
+    const uint32_t we = cs + part_start(uc, S::NW, warp + 1);
     const uint32_t lane4 = lut | ((uint32_t)lane << 2);
     const int nunits = (int)(we - ws);
 
@@ -529,8 +529,8 @@ __global__ void __launch_bounds__(S::NW * 32, 1)
     bool has_first = false, has_last = false;
     zero_acc<S>(acc);
     Cursor c;
-    c.tile = nunits > 0 ? (int)(ws / p.kb_per_tile) : 0;
-    c.kb = nunits > 0 ? (int)(ws - (int64_t)c.tile * p.kb_per_tile) : 0;
+    c.tile = nunits > 0 ? (int)(ws / (uint32_t)p.kb_per_tile) : 0;
+    c.kb = nunits > 0 ? (int)(ws - (uint32_t)c.tile * (uint32_t)p.kb_per_tile) : 0;
     c.from_start = (c.kb == 0);
     c.first_tile = true;
     StageCursor ld{c.tile, c.kb, nunits}, cm{c.tile, c.kb, nunits};
@@ -682,6 +682,234 @@ __global__ void __launch_bounds__(S::NW * 32, 1)
     combine_tiles<T, S>(p, slots, cs, ce, warp, lane, g, tq);
 }
 
+
+// ===========================================================================
+// Warp-specialised variant.
+//
+// Issuing a TMA copy can block the issuing thread while the SM's copy engine
+// works through earlier boxes (it walks them row by row), so in the kernel
+// above every consumer warp stalls behind its own lane 0 during the initial
+// burst.  Here one producer warp issues all copies -- its lane w feeds
+// consumer warp w's ring -- and consumers hand each stage back through an
+// "empty" mbarrier.  Stages are 64 rows x 128 bytes (4 units), halving the
+// copy engine's row requests per byte compared with 64-byte rows.
+// ===========================================================================
+template <typename T, class S, int UPS, bool BS64>
+__global__ void __launch_bounds__((S::NW + 1) * 32, 1)
+    q4_gemm_ws_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_a,
+                      const GemmParams p) {
+    using G = StageGeom<UPS>;
+    static_assert(S::NW * S::SLOT_REGS <= 256, "parked partial tiles must fit in the LUT rows");
+    static_assert(S::NW <= 32, "one producer lane per consumer warp");
+    constexpr int NC = S::NW;     // consumer warps
+    constexpr int D = S::DEPTH;   // stages per consumer
+    extern __shared__ __align__(16) uint8_t smem_ws[];
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, tq = lane & 3;
+    const bool producer = (warp == NC);
+
+    // Layout: 64 KiB LUT on a 64 KiB boundary; full/empty barriers and the
+    // stages below and above it.
+    const uint32_t sbase = smem_addr(smem_ws);
+    const uint32_t send = sbase + dynamic_smem_size();
+    const uint32_t lut = (sbase + 0xFFFFu) & ~0xFFFFu;
+    const uint32_t nbar_bytes = (uint32_t)NC * D * 16u;
+    uint32_t bars, a0, b0 = lut + S::LUT_BYTES;
+    if (lut - sbase >= nbar_bytes) {
+        bars = sbase;
+        a0 = (sbase + nbar_bytes + 1023u) & ~1023u;
+    } else {
+        bars = b0;
+        b0 = (b0 + nbar_bytes + 1023u) & ~1023u;
+        a0 = lut;
+    }
+    const uint32_t na = a0 < lut ? (lut - a0) / G::BYTES : 0u;
+    const uint32_t nb = b0 < send ? (send - b0) / G::BYTES : 0u;
+    const bool room = (lut + S::LUT_BYTES <= send) && (na + nb >= (uint32_t)(NC * D)) &&
+                      ((send > b0 && send - b0 >= S::SLOT_BYTES) || (lut > a0 && lut - a0 >= S::SLOT_BYTES));
+    if (!room) {
+        if (tid == 0) atomicExch(p.error, kErrNoRoom);
+        return;
+    }
+    const uint32_t slots = (send > b0 && send - b0 >= S::SLOT_BYTES) ? b0 : a0;
+    auto stage_addr = [&](int idx) -> uint32_t {
+        return (uint32_t)idx < na ? a0 + (uint32_t)idx * G::BYTES : b0 + ((uint32_t)idx - na) * G::BYTES;
+    };
+    auto full_bar = [&](int w, int d) -> uint32_t { return bars + (uint32_t)(w * D + d) * 8u; };
+    auto empty_bar = [&](int w, int d) -> uint32_t { return bars + (uint32_t)(NC * D + w * D + d) * 8u; };
+
+    if (p.pdl != 2) griddep_wait();
+    if (producer && lane < NC) {
+        for (int d = 0; d < D; ++d) {
+            mbar_init(full_bar(lane, d), 1);
+            mbar_init(empty_bar(lane, d), 1);
+        }
+        mbar_init_fence();
+    }
+    __syncthreads();
+
+    const uint32_t cs = part_start(p.units, p.ctas, blockIdx.x);
+    const uint32_t ce = part_start(p.units, p.ctas, blockIdx.x + 1);
+    const uint32_t uc = ce - cs;
+    float acc[S::TW][S::NJ][4];
+    bool has_first = false, has_last = false;
+    zero_acc<S>(acc);
+
+    if (producer) {
+        // Lane w streams consumer w's unit range into its ring.
+        if (lane < NC) {
+            const uint32_t ws = cs + part_start(uc, NC, lane), we = cs + part_start(uc, NC, lane + 1);
+            const int nunits = (int)(we - ws);
+            const int tile0 = nunits > 0 ? (int)(ws / (uint32_t)p.kb_per_tile) : 0;
+            StageCursor ld{tile0, nunits > 0 ? (int)(ws - (uint32_t)tile0 * (uint32_t)p.kb_per_tile) : 0, nunits};
+            for (int k = 0; ld.left > 0; ++k) {
+                const int slot = k % D;
+                if (k >= D && !wait_stage(empty_bar(lane, slot), (uint32_t)(k / D - 1) & 1u)) {
+                    if (p.pdl == 2) griddep_wait();
+                    atomicExch(p.error, kErrWaitTimeout);
+                    break;
+                }
+                int tile, kb0, kb, n;
+                next_stage<UPS>(ld, p.kb_per_tile, tile, kb0, kb, n);
+                const uint32_t st = stage_addr(lane * D + slot);
+                mbar_expect_tx(full_bar(lane, slot), G::BYTES);
+                tma_load_2d(st, &tmap_w, kb0 * 32, tile * S::TR, full_bar(lane, slot));
+                tma_load_2d(st + G::WEIGHT_BYTES, &tmap_a, (kb0 >> p.am_shift) & ~3, tile * S::TR, full_bar(lane, slot));
+            }
+        }
+    } else {
+        build_lut<T>(lut, p.code, tid, NC * 32);
+        named_bar_sync(1, NC * 32);
+        if (p.pdl == 2) griddep_wait();
+        griddep_launch_dependents();
+        const uint32_t ws = cs + part_start(uc, NC, warp), we = cs + part_start(uc, NC, warp + 1);
+        const int nunits = (int)(we - ws);
+        const uint32_t lane4 = lut | ((uint32_t)lane << 2);
+        if (nunits > 0) {
+            Cursor c;
+            c.tile = (int)(ws / (uint32_t)p.kb_per_tile);
+            c.kb = (int)(ws - (uint32_t)c.tile * (uint32_t)p.kb_per_tile);
+            c.from_start = (c.kb == 0);
+            c.first_tile = true;
+            StageCursor cm{c.tile, c.kb, nunits};
+            const int lm_q = lane >> 3, lm_r = lane & 7;
+            const T* Aact = static_cast<const T*>(p.A);
+            bool ok = true;
+            int consumed = 0;
+            uint32_t bw[S::NJ][2][4], bwn[S::NJ][2][4];
+            auto load_act = [&](int kunit, uint32_t(&dst)[S::NJ][2][4]) {
+#pragma unroll
+                for (int jj = 0; jj < S::NJ; ++jj) {
+                    const int m = 8 * jj + g;
+#pragma unroll
+                    for (int ch = 0; ch < 2; ++ch) {
+                        if (m < p.M) {
+                            const uint4 v = ldg_v4(Aact + (size_t)m * p.K + kunit + 32 * ch + 8 * tq);
+                            dst[jj][ch][0] = v.x;
+                            dst[jj][ch][1] = v.y;
+                            dst[jj][ch][2] = v.z;
+                            dst[jj][ch][3] = v.w;
+                        } else {
+                            dst[jj][ch][0] = dst[jj][ch][1] = dst[jj][ch][2] = dst[jj][ch][3] = 0u;
+                        }
+                    }
+                }
+            };
+            load_act(c.kb * S::SB, bw);
+            while (cm.left > 0) {
+                int tile, kb0, kb, n;
+                next_stage<UPS>(cm, p.kb_per_tile, tile, kb0, kb, n);
+                const int slot = consumed % D;
+                const uint32_t st = stage_addr(warp * D + slot);
+                if (!wait_stage(full_bar(warp, slot), (uint32_t)(consumed / D) & 1u)) {
+                    ok = false;
+                    break;
+                }
+                const int x0 = (kb0 >> p.am_shift) & ~3;
+#pragma unroll
+                for (int j = 0; j < UPS; ++j) {
+                    if (kb0 + j < kb || kb0 + j >= kb + n) continue;
+                    if (kb0 + j + 1 < kb + n)
+                        load_act((kb0 + j + 1) * S::SB, bwn);
+                    else if (cm.left > 0)
+                        load_act(cm.kb * S::SB, bwn);
+                    const int col = BS64 ? (kb0 + j - x0) : (((kb0 + j) >> p.am_shift) - x0);
+                    const uint32_t am_base = st + G::WEIGHT_BYTES + (uint32_t)col * 4u;
+                    const float zero[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                    for (int i = 0; i < S::TW; ++i) {
+                        uint32_t d0, d1, d2, d3;
+                        ldmatrix_x4(G::chunk_addr(st, 16 * i + 8 * (lm_q & 1) + lm_r, 2 * j + (lm_q >> 1)), d0, d1, d2,
+                                    d3);
+                        const float ag = lds_f32(am_base + (uint32_t)(16 * i + g) * 16u);
+                        const float ag8 = lds_f32(am_base + (uint32_t)(16 * i + 8 + g) * 16u);
+                        float t[S::NJ][4];
+                        uint32_t a0, a1, a2, a3;
+                        a0 = lut_pair<0>(d0, lane4); a2 = lut_pair<1>(d0, lane4);
+                        a1 = lut_pair<0>(d1, lane4); a3 = lut_pair<1>(d1, lane4);
+#pragma unroll
+                        for (int jj = 0; jj < S::NJ; ++jj) mma16816<T>(t[jj], a0, a1, a2, a3, bw[jj][0][0], bw[jj][0][1], zero);
+                        a0 = lut_pair<2>(d0, lane4); a2 = lut_pair<3>(d0, lane4);
+                        a1 = lut_pair<2>(d1, lane4); a3 = lut_pair<3>(d1, lane4);
+#pragma unroll
+                        for (int jj = 0; jj < S::NJ; ++jj) mma16816<T>(t[jj], a0, a1, a2, a3, bw[jj][0][2], bw[jj][0][3], t[jj]);
+                        a0 = lut_pair<0>(d2, lane4); a2 = lut_pair<1>(d2, lane4);
+                        a1 = lut_pair<0>(d3, lane4); a3 = lut_pair<1>(d3, lane4);
+#pragma unroll
+                        for (int jj = 0; jj < S::NJ; ++jj) mma16816<T>(t[jj], a0, a1, a2, a3, bw[jj][1][0], bw[jj][1][1], t[jj]);
+                        a0 = lut_pair<2>(d2, lane4); a2 = lut_pair<3>(d2, lane4);
+                        a1 = lut_pair<2>(d3, lane4); a3 = lut_pair<3>(d3, lane4);
+#pragma unroll
+                        for (int jj = 0; jj < S::NJ; ++jj) mma16816<T>(t[jj], a0, a1, a2, a3, bw[jj][1][2], bw[jj][1][3], t[jj]);
+#pragma unroll
+                        for (int jj = 0; jj < S::NJ; ++jj) {
+                            acc[i][jj][0] = fmaf(ag, t[jj][0], acc[i][jj][0]);
+                            acc[i][jj][1] = fmaf(ag, t[jj][1], acc[i][jj][1]);
+                            acc[i][jj][2] = fmaf(ag8, t[jj][2], acc[i][jj][2]);
+                            acc[i][jj][3] = fmaf(ag8, t[jj][3], acc[i][jj][3]);
+                        }
+                    }
+                    finish_unit_tma<T, S>(acc, has_first, has_last, c, cm.left == 0 && kb0 + j + 1 == kb + n, p, lut,
+                                          warp, lane, g, tq);
+#pragma unroll
+                    for (int jj = 0; jj < S::NJ; ++jj)
+#pragma unroll
+                        for (int ch = 0; ch < 2; ++ch)
+#pragma unroll
+                            for (int w = 0; w < 4; ++w) bw[jj][ch][w] = bwn[jj][ch][w];
+                }
+                // hand the stage back to the producer
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(empty_bar(warp, slot));
+                ++consumed;
+            }
+            if (!ok) {
+                if (lane == 0) atomicExch(p.error, kErrWaitTimeout);
+                for (int k = 0; k < D; ++k)  // drain whatever the producer may still have in flight
+                    wait_stage(full_bar(warp, (consumed + k) % D), (uint32_t)((consumed + k) / D) & 1u);
+            }
+        }
+    }
+    __syncthreads();  // every warp is out of the stage ring: the slots may reuse it
+    if (!producer) {
+        if (has_first) {
+            float first[S::TW][S::NJ][4];
+#pragma unroll
+            for (int i = 0; i < S::TW; ++i)
+#pragma unroll
+                for (int j = 0; j < S::NJ; ++j)
+#pragma unroll
+                    for (int r = 0; r < 4; ++r)
+                        first[i][j][r] = lds_f32(parked_addr<S>(lut, warp, (i * S::NJ + j) * 4 + r, lane));
+            store_slot<S>(first, slots, warp * 2, lane);
+        }
+        if (has_last) store_slot<S>(acc, slots, warp * 2 + 1, lane);
+    }
+    __syncthreads();
+    if (uc <= 0 || producer) return;
+    combine_tiles<T, S>(p, slots, cs, ce, warp, lane, g, tq);
+}
+
 // ---------------------------------------------------------------------------
 // Host launchers: the table of compiled variants.
 // ---------------------------------------------------------------------------
@@ -779,6 +1007,30 @@ static cudaError_t launch_tma(const GemmParams& p, cudaStream_t stream) {
     return cudaGetLastError();
 }
 
+template <typename T, class S, int UPS>
+static cudaError_t launch_ws(const GemmParams& p, cudaStream_t stream) {
+    CUtensorMap tw, ta;
+    cudaError_t e = make_tensor_maps(p, UPS, &tw, &ta);
+    if (e != cudaSuccess) return e;
+    const int smem = max_dynamic_smem();
+    if (smem <= 0) return cudaErrorInvalidValue;
+    auto kern = p.am_shift == 0 ? q4_gemm_ws_kernel<T, S, UPS, true> : q4_gemm_ws_kernel<T, S, UPS, false>;
+    if ((e = ensure_smem_attr((const void*)kern, (size_t)smem)) != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)p.ctas);
+    cfg.blockDim = dim3((S::NW + 1) * 32);
+    cfg.dynamicSmemBytes = (size_t)smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = p.pdl ? 1 : 0;
+    e = cudaLaunchKernelEx(&cfg, kern, tw, ta, p);
+    if (e != cudaSuccess) return e;
+    return cudaGetLastError();
+}
+
 struct Variant {
     int act, loader, sub_block, m_pad, warps, depth, l2pf;
     size_t smem;
@@ -802,12 +1054,23 @@ struct Variant {
         ACT, 3, 64, MP, NW, D, 0, 0, &launch_tma<T, GemmShape<64, MP, 4, NW, D, 0>, 2>         \
     }
 
+// Warp-specialised rings: loader 4 = 4-unit stages, loader 5 = 2-unit stages;
+// `warps` counts the consumer warps (plus one producer warp).
+#define Q4_WS_VARIANT(ACT, T, MP, NW, D)                                                       \
+    Variant {                                                                                 \
+        ACT, 4, 64, MP, NW, D, 0, 0, &launch_ws<T, GemmShape<64, MP, 4, NW, D, 0>, 4>          \
+    }
+#define Q4_WS2_VARIANT(ACT, T, MP, NW, D)                                                      \
+    Variant {                                                                                 \
+        ACT, 5, 64, MP, NW, D, 0, 0, &launch_ws<T, GemmShape<64, MP, 4, NW, D, 0>, 2>          \
+    }
+
 #define Q4_VARIANTS_FOR(ACT, T)                                                                \
     Q4_VARIANT(ACT, T, 64, 8, 16, 1, 128), Q4_VARIANT(ACT, T, 64, 8, 8, 2, 128),               \
         Q4_VARIANT(ACT, T, 64, 16, 8, 1, 128), Q4_VARIANT(ACT, T, 32, 8, 16, 1, 128),         \
         Q4_VARIANT(ACT, T, 32, 16, 8, 1, 128), Q4_TMA_VARIANT(ACT, T, 8, 8, 2),               \
         Q4_TMA_VARIANT(ACT, T, 16, 8, 2), Q4_TMA2_VARIANT(ACT, T, 8, 16, 2),                  \
-        Q4_TMA2_VARIANT(ACT, T, 16, 8, 4)
+        Q4_TMA2_VARIANT(ACT, T, 16, 8, 4), Q4_WS_VARIANT(ACT, T, 8, 8, 2), Q4_WS_VARIANT(ACT, T, 16, 8, 2)
 
 static const Variant kVariants[] = {
     Q4_VARIANTS_FOR(0, __nv_bfloat16),
@@ -822,6 +1085,10 @@ static const Variant kVariants[] = {
     Q4_TMA2_VARIANT(0, __nv_bfloat16, 8, 8, 4),
     Q4_TMA2_VARIANT(0, __nv_bfloat16, 8, 12, 2),
     Q4_TMA2_VARIANT(0, __nv_bfloat16, 8, 16, 1),
+    Q4_WS_VARIANT(0, __nv_bfloat16, 8, 16, 1),
+    Q4_WS_VARIANT(0, __nv_bfloat16, 8, 12, 1),
+    Q4_WS2_VARIANT(0, __nv_bfloat16, 8, 16, 2),
+    Q4_WS2_VARIANT(0, __nv_bfloat16, 8, 8, 4),
 };
 
 static const Variant* find_variant(int act, const GemmChoice& ch) {

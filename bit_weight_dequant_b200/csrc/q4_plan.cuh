@@ -16,15 +16,25 @@
 namespace q4 {
 
 // First unit of part p when `total` units are split into `parts` ranges.
-__host__ __device__ __forceinline__ int64_t part_start(int64_t total, int parts, int p) {
-    return (total * (int64_t)p) / parts;
+// 32-bit arithmetic (the kernels' hot path): the launcher guarantees
+// total * parts < 2^32.
+__host__ __device__ __forceinline__ uint32_t part_start(uint32_t total, uint32_t parts, uint32_t p) {
+    return (total * p) / parts;
 }
 
 // The unique part p with part_start(p) <= u < part_start(p + 1).
 // part_start(p) <= u  <=>  total*p < (u+1)*parts  <=>  p <= ((u+1)*parts - 1) / total.
-__host__ __device__ __forceinline__ int part_owner(int64_t total, int parts, int64_t u) {
-    return (int)(((u + 1) * (int64_t)parts - 1) / total);
+__host__ __device__ __forceinline__ uint32_t part_owner(uint32_t total, uint32_t parts, uint32_t u) {
+    return ((u + 1) * parts - 1) / total;
 }
+
+// The same two functions without the range limit (host-side reference).
+inline int64_t part_start64(int64_t total, int parts, int p) { return (total * (int64_t)p) / parts; }
+inline int part_owner64(int64_t total, int parts, int64_t u) { return (int)(((u + 1) * (int64_t)parts - 1) / total); }
+
+// Largest unit count the kernels accept (keeps total * parts below 2^32 for
+// up to 512 parts).
+static constexpr uint32_t kMaxUnits = (1u << 23);
 
 // Compile-time shape of one GEMM kernel variant.
 template <int SB_, int MPAD_, int TW_, int NW_, int DEPTH_, int L2PF_>
@@ -69,7 +79,7 @@ struct GemmParams {
     int am_per_row;    // K / blocksize
     int tiles;
     int ctas;
-    int64_t units;
+    uint32_t units;    // < kMaxUnits
 };
 
 }  // namespace q4

@@ -69,7 +69,7 @@ def _problem(device, M=3, N=300, K=1024, bs=64, seed=7):
             torch.from_numpy(code).to(device), N, K, bs)
 
 
-@pytest.mark.parametrize("loader", [1, 2, 3])
+@pytest.mark.parametrize("loader", [1, 2, 3, 4, 5])
 def test_deterministic_and_counters_left_zero(cuda_device, loader):
     A, P, Am, C, N, K, bs = _problem(cuda_device)
     ws = q4.Workspace(cuda_device)
@@ -111,7 +111,7 @@ def test_direct_load_variants(cuda_device, depth, l2pf, warps):
 
 
 @pytest.mark.parametrize("loader,warps,depth", [(2, 8, 2), (2, 16, 1), (2, 12, 1), (3, 16, 2), (3, 8, 4), (3, 12, 2),
-                                                (3, 16, 1)])
+                                                (3, 16, 1), (4, 8, 2), (4, 16, 1), (4, 12, 1), (5, 16, 2), (5, 8, 4)])
 def test_tma_ring_variants(cuda_device, loader, warps, depth):
     run_case(Case(1, 700, 2048), seed=7200 + warps, device=cuda_device, check_quantizer=False, depth=depth,
              warps=warps, loader=loader)
@@ -122,13 +122,13 @@ def test_tma_ring_variants(cuda_device, loader, warps, depth):
 @pytest.mark.parametrize("M", [1, 7, 8, 9, 16])
 @pytest.mark.parametrize("N,K,bs", [(1, 256, 64), (64, 256, 64), (100, 1280, 64), (513, 1024, 128), (300, 4096, 256),
                                     (257, 3072, 64), (70, 512, 128)])
-@pytest.mark.parametrize("loader", [2, 3])
+@pytest.mark.parametrize("loader", [2, 3, 4])
 def test_tma_ring_shapes(cuda_device, M, N, K, bs, loader):
     run_case(Case(M, N, K, blocksize=bs), seed=7400 + M + N, device=cuda_device, check_quantizer=False, loader=loader)
 
 
 @pytest.mark.parametrize("ctas", [1, 2, 3, 7, 33, 148])
-@pytest.mark.parametrize("loader", [2, 3])
+@pytest.mark.parametrize("loader", [2, 3, 4, 5])
 def test_tma_ring_partitions(cuda_device, ctas, loader):
     run_case(Case(2, 257, 1280), seed=7500 + ctas, device=cuda_device, check_quantizer=False, loader=loader, ctas=ctas)
 
@@ -136,7 +136,7 @@ def test_tma_ring_partitions(cuda_device, ctas, loader):
 def test_tma_error_word_stays_zero(cuda_device):
     ws = q4.Workspace(cuda_device)
     A, P, Am, C, N, K, bs = _problem(cuda_device)
-    for loader in (2, 3):
+    for loader in (2, 3, 4, 5):
         q4.q4_gemm_skinny(A, P, Am, C, N, K, bs, workspace=ws, loader=loader)
     torch.cuda.synchronize()
     assert q4.workspace_error(ws) == 0
@@ -199,7 +199,7 @@ def test_one_hot_activation_selects_dequantized_column(cuda_device):
 
 
 @pytest.mark.parametrize("pdl", [1, 2])
-@pytest.mark.parametrize("loader", [1, 3])
+@pytest.mark.parametrize("loader", [1, 3, 4])
 def test_dependent_launch_chain(cuda_device, pdl, loader):
     """A chain where each GEMM reads the previous GEMM's output as its
     activations: with programmatic dependent launch the second kernel may
