@@ -98,7 +98,7 @@ static int gemm_choose(int M, int N, int K, int blocksize, int act_dtype, int nu
     // multiples of 16 bytes (a tensor-map stride rule); the pointer itself
     // must also be 16-byte aligned, which the caller checks at launch.
     const bool tma_ok = c.sub_block == 64 && (K / blocksize) % 4 == 0 && (int64_t)N * (K / 64) > 1;
-    c.loader = tma_ok ? 3 : 1;
+    c.loader = tma_ok ? 2 : 1;
     if (ov && ov->loader > 0) c.loader = ov->loader;
     if (c.loader >= 2 && !tma_ok) return Q4_ERR_UNSUPPORTED;
     if (c.loader == 2) {

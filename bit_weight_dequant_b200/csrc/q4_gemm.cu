@@ -562,31 +562,75 @@ __global__ void __launch_bounds__(S::NW * 32, 1)
         const T* Aact = static_cast<const T*>(p.A);
         bool ok = true;
 
-        // activations of the unit being computed (bw) and of the next one (bwn)
-        uint32_t bw[S::NJ][2][4], bwn[S::NJ][2][4];
-        auto load_act = [&](int kunit, uint32_t(&dst)[S::NJ][2][4]) {
+        // Activations of the current stage's UPS-unit window (aw) and of the
+        // next stage's window (awn), loaded a whole stage ahead of use.
+        // Windows are UPS-aligned and tiles hold a multiple of UPS units, so
+        // a window never reaches past K.
+        uint32_t aw[UPS][S::NJ][2][4], awn[UPS][S::NJ][2][4];
+        auto load_window = [&](int kbw, uint32_t(&dst)[UPS][S::NJ][2][4]) {
 #pragma unroll
-            for (int jj = 0; jj < S::NJ; ++jj) {
-                const int m = 8 * jj + g;
+            for (int j = 0; j < UPS; ++j)
 #pragma unroll
-                for (int ch = 0; ch < 2; ++ch) {
-                    if (m < p.M) {
-                        const uint4 v = ldg_v4(Aact + (size_t)m * p.K + kunit + 32 * ch + 8 * tq);
-                        dst[jj][ch][0] = v.x;
-                        dst[jj][ch][1] = v.y;
-                        dst[jj][ch][2] = v.z;
-                        dst[jj][ch][3] = v.w;
-                    } else {
-                        dst[jj][ch][0] = dst[jj][ch][1] = dst[jj][ch][2] = dst[jj][ch][3] = 0u;
+                for (int jj = 0; jj < S::NJ; ++jj) {
+                    const int m = 8 * jj + g;
+#pragma unroll
+                    for (int ch = 0; ch < 2; ++ch) {
+                        if (m < p.M) {
+                            const uint4 v = ldg_v4(Aact + (size_t)m * p.K + (kbw + j) * S::SB + 32 * ch + 8 * tq);
+                            dst[j][jj][ch][0] = v.x;
+                            dst[j][jj][ch][1] = v.y;
+                            dst[j][jj][ch][2] = v.z;
+                            dst[j][jj][ch][3] = v.w;
+                        } else {
+                            dst[j][jj][ch][0] = dst[j][jj][ch][1] = dst[j][jj][ch][2] = dst[j][jj][ch][3] = 0u;
+                        }
                     }
                 }
+        };
+        load_window(c.kb & ~(UPS - 1), aw);
+
+        // One 64-row x 64-k unit (window position j) of the stage at `st`,
+        // scaled by the per-row absmax (ag: rows 16i+g, ag8: rows 16i+8+g).
+        auto unit_rows = [&](uint32_t st, int j, int i, float ag, float ag8) {
+            const float zero[4] = {0.f, 0.f, 0.f, 0.f};
+            // rows 16i + 8(q&1) + r, chunk 2j + (q>>1)
+            uint32_t d0, d1, d2, d3;
+            ldmatrix_x4(G::chunk_addr(st, 16 * i + 8 * (lm_q & 1) + lm_r, 2 * j + (lm_q >> 1)), d0, d1, d2, d3);
+            float t[S::NJ][4];
+            // steps 0..3: (d0,d1) bytes 0/1, 2/3, then (d2,d3) bytes 0/1, 2/3
+            uint32_t a0, a1, a2, a3;
+            a0 = lut_pair<0>(d0, lane4); a2 = lut_pair<1>(d0, lane4);
+            a1 = lut_pair<0>(d1, lane4); a3 = lut_pair<1>(d1, lane4);
+#pragma unroll
+            for (int jj = 0; jj < S::NJ; ++jj) mma16816<T>(t[jj], a0, a1, a2, a3, aw[j][jj][0][0], aw[j][jj][0][1], zero);
+            a0 = lut_pair<2>(d0, lane4); a2 = lut_pair<3>(d0, lane4);
+            a1 = lut_pair<2>(d1, lane4); a3 = lut_pair<3>(d1, lane4);
+#pragma unroll
+            for (int jj = 0; jj < S::NJ; ++jj) mma16816<T>(t[jj], a0, a1, a2, a3, aw[j][jj][0][2], aw[j][jj][0][3], t[jj]);
+            a0 = lut_pair<0>(d2, lane4); a2 = lut_pair<1>(d2, lane4);
+            a1 = lut_pair<0>(d3, lane4); a3 = lut_pair<1>(d3, lane4);
+#pragma unroll
+            for (int jj = 0; jj < S::NJ; ++jj) mma16816<T>(t[jj], a0, a1, a2, a3, aw[j][jj][1][0], aw[j][jj][1][1], t[jj]);
+            a0 = lut_pair<2>(d2, lane4); a2 = lut_pair<3>(d2, lane4);
+            a1 = lut_pair<2>(d3, lane4); a3 = lut_pair<3>(d3, lane4);
+#pragma unroll
+            for (int jj = 0; jj < S::NJ; ++jj) mma16816<T>(t[jj], a0, a1, a2, a3, aw[j][jj][1][2], aw[j][jj][1][3], t[jj]);
+#pragma unroll
+            for (int jj = 0; jj < S::NJ; ++jj) {
+                acc[i][jj][0] = fmaf(ag, t[jj][0], acc[i][jj][0]);
+                acc[i][jj][1] = fmaf(ag, t[jj][1], acc[i][jj][1]);
+                acc[i][jj][2] = fmaf(ag8, t[jj][2], acc[i][jj][2]);
+                acc[i][jj][3] = fmaf(ag8, t[jj][3], acc[i][jj][3]);
             }
         };
-        load_act(c.kb * S::SB, bw);
+        // With 4-unit stages and one absmax per unit, a row's 4-float absmax
+        // box is exactly the stage's 4 units: one 16-byte read per row.
+        constexpr bool kAmRow = (UPS == 4) && BS64;
 
         while (cm.left > 0) {
             int tile, kb0, kb, n;
             next_stage<UPS>(cm, p.kb_per_tile, tile, kb0, kb, n);
+            if (cm.left > 0) load_window(cm.kb & ~(UPS - 1), awn);
             const int slot = consumed % D;
             const uint32_t st = stage_addr(warp * D + slot);
             const uint32_t bar = bars + (uint32_t)(warp * D + slot) * 8u;
@@ -595,61 +639,58 @@ __global__ void __launch_bounds__(S::NW * 32, 1)
                 break;
             }
             const int x0 = (kb0 >> p.am_shift) & ~3;
+            const uint32_t am_stage = st + G::WEIGHT_BYTES;
+            float am[S::TW][2][4];
+            if constexpr (kAmRow) {
 #pragma unroll
-            for (int j = 0; j < UPS; ++j) {
-                if (kb0 + j < kb || kb0 + j >= kb + n) continue;
-                // prefetch the activations of the next unit of the range
-                // (activation runs: row 8jj+g, k = kunit + 32ch + 8tq .. +8)
-                if (kb0 + j + 1 < kb + n)
-                    load_act((kb0 + j + 1) * S::SB, bwn);
-                else if (cm.left > 0)
-                    load_act(cm.kb * S::SB, bwn);
+                for (int i = 0; i < S::TW; ++i)
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        const uint4 v = lds_v4(am_stage + (uint32_t)(16 * i + 8 * h + g) * 16u);
+                        am[i][h][0] = __uint_as_float(v.x);
+                        am[i][h][1] = __uint_as_float(v.y);
+                        am[i][h][2] = __uint_as_float(v.z);
+                        am[i][h][3] = __uint_as_float(v.w);
+                    }
+            }
+            auto unit_all_rows = [&](int j) {
                 // absmax column of this unit inside the stage's 4-float box
                 const int col = BS64 ? (kb0 + j - x0) : (((kb0 + j) >> p.am_shift) - x0);
-                const uint32_t am_base = st + G::WEIGHT_BYTES + (uint32_t)col * 4u;
-                const float zero[4] = {0.f, 0.f, 0.f, 0.f};
+                const uint32_t am_base = am_stage + (uint32_t)col * 4u;
 #pragma unroll
                 for (int i = 0; i < S::TW; ++i) {
-                    // rows 16i + 8(q&1) + r, chunk 2j + (q>>1)
-                    uint32_t d0, d1, d2, d3;
-                    ldmatrix_x4(G::chunk_addr(st, 16 * i + 8 * (lm_q & 1) + lm_r, 2 * j + (lm_q >> 1)), d0, d1, d2, d3);
-                    const float ag = lds_f32(am_base + (uint32_t)(16 * i + g) * 16u);
-                    const float ag8 = lds_f32(am_base + (uint32_t)(16 * i + 8 + g) * 16u);
-                    float t[S::NJ][4];
-                    // steps 0..3: (d0,d1) bytes 0/1, 2/3, then (d2,d3) bytes 0/1, 2/3
-                    uint32_t a0, a1, a2, a3;
-                    a0 = lut_pair<0>(d0, lane4); a2 = lut_pair<1>(d0, lane4);
-                    a1 = lut_pair<0>(d1, lane4); a3 = lut_pair<1>(d1, lane4);
-#pragma unroll
-                    for (int jj = 0; jj < S::NJ; ++jj) mma16816<T>(t[jj], a0, a1, a2, a3, bw[jj][0][0], bw[jj][0][1], zero);
-                    a0 = lut_pair<2>(d0, lane4); a2 = lut_pair<3>(d0, lane4);
-                    a1 = lut_pair<2>(d1, lane4); a3 = lut_pair<3>(d1, lane4);
-#pragma unroll
-                    for (int jj = 0; jj < S::NJ; ++jj) mma16816<T>(t[jj], a0, a1, a2, a3, bw[jj][0][2], bw[jj][0][3], t[jj]);
-                    a0 = lut_pair<0>(d2, lane4); a2 = lut_pair<1>(d2, lane4);
-                    a1 = lut_pair<0>(d3, lane4); a3 = lut_pair<1>(d3, lane4);
-#pragma unroll
-                    for (int jj = 0; jj < S::NJ; ++jj) mma16816<T>(t[jj], a0, a1, a2, a3, bw[jj][1][0], bw[jj][1][1], t[jj]);
-                    a0 = lut_pair<2>(d2, lane4); a2 = lut_pair<3>(d2, lane4);
-                    a1 = lut_pair<2>(d3, lane4); a3 = lut_pair<3>(d3, lane4);
-#pragma unroll
-                    for (int jj = 0; jj < S::NJ; ++jj) mma16816<T>(t[jj], a0, a1, a2, a3, bw[jj][1][2], bw[jj][1][3], t[jj]);
-#pragma unroll
-                    for (int jj = 0; jj < S::NJ; ++jj) {
-                        acc[i][jj][0] = fmaf(ag, t[jj][0], acc[i][jj][0]);
-                        acc[i][jj][1] = fmaf(ag, t[jj][1], acc[i][jj][1]);
-                        acc[i][jj][2] = fmaf(ag8, t[jj][2], acc[i][jj][2]);
-                        acc[i][jj][3] = fmaf(ag8, t[jj][3], acc[i][jj][3]);
-                    }
+                    if constexpr (kAmRow)
+                        unit_rows(st, j, i, am[i][0][j], am[i][1][j]);
+                    else
+                        unit_rows(st, j, i, lds_f32(am_base + (uint32_t)(16 * i + g) * 16u),
+                                  lds_f32(am_base + (uint32_t)(16 * i + 8 + g) * 16u));
                 }
-                finish_unit_tma<T, S>(acc, has_first, has_last, c, cm.left == 0 && kb0 + j + 1 == kb + n, p, lut, warp,
-                                      lane, g, tq);
+            };
+            if (n == UPS) {
+                // Whole stage inside one tile and the range: no tile can end
+                // before its last unit, so the units run back to back.
 #pragma unroll
-                for (int jj = 0; jj < S::NJ; ++jj)
+                for (int j = 0; j < UPS; ++j) unit_all_rows(j);
+                c.kb += UPS - 1;
+                finish_unit_tma<T, S>(acc, has_first, has_last, c, cm.left == 0, p, lut, warp, lane, g, tq);
+            } else {
 #pragma unroll
-                    for (int ch = 0; ch < 2; ++ch)
+                for (int j = 0; j < UPS; ++j) {
+                    if (kb0 + j < kb || kb0 + j >= kb + n) continue;
+                    unit_all_rows(j);
+                    finish_unit_tma<T, S>(acc, has_first, has_last, c, cm.left == 0 && kb0 + j + 1 == kb + n, p, lut,
+                                          warp, lane, g, tq);
+                }
+            }
+            if (cm.left > 0) {
 #pragma unroll
-                        for (int w = 0; w < 4; ++w) bw[jj][ch][w] = bwn[jj][ch][w];
+                for (int j = 0; j < UPS; ++j)
+#pragma unroll
+                    for (int jj = 0; jj < S::NJ; ++jj)
+#pragma unroll
+                        for (int ch = 0; ch < 2; ++ch)
+#pragma unroll
+                            for (int w = 0; w < 4; ++w) aw[j][jj][ch][w] = awn[j][jj][ch][w];
             }
             ++consumed;
             // Hand the slot back to the copy engine: order this warp's reads

@@ -99,7 +99,7 @@ def test_launch_table_invariants(wl):
         assert p["workspace_bytes"] == want_ws
         assert p["depth"] >= 1 and p["l2_prefetch"] in (1, 128, 256)
         tma_ok = c.blocksize >= 64 and (c.K // c.blocksize) % 4 == 0 and p["units"] > 1
-        assert p["loader"] == (3 if tma_ok else 1)
+        assert p["loader"] == (2 if tma_ok else 1)
 
 
 @pytest.mark.parametrize("total,parts", [(1, 1), (1, 16), (7, 3), (40, 148), (4096, 148), (57344, 148),
