@@ -294,11 +294,16 @@ __device__ __forceinline__ void combine_tiles(const GemmParams& p, uint32_t slot
 }
 
 // Table row b (256 B): 32 copies (one per bank) of the pair (code[b>>4], code[b&15]) as T.
+// `cv` is code[lane & 15] in every lane; the pair is gathered by shuffles, so
+// the table costs one global load per thread.  nthreads is a multiple of 32
+// that divides the 2048 row pieces evenly per warp (the shuffles need whole warps).
 template <typename T>
-__device__ __forceinline__ void build_lut(uint32_t lut, const float* code, int tid, int nthreads) {
+__device__ __forceinline__ void build_lut(uint32_t lut, float cv, int tid, int nthreads) {
     for (int e = tid; e < 256 * 8; e += nthreads) {
         const int b = e >> 3;
-        const uint32_t v = Act<T>::pack(__ldg(code + (b >> 4)), __ldg(code + (b & 15)));
+        const float hi = __shfl_sync(0xffffffffu, cv, b >> 4);
+        const float lo = __shfl_sync(0xffffffffu, cv, b & 15);
+        const uint32_t v = Act<T>::pack(hi, lo);
         sts_v4(lut + (uint32_t)b * 256u + (uint32_t)(e & 7) * 16u, v, v, v, v);
     }
 }
@@ -312,7 +317,7 @@ __global__ void __launch_bounds__(S::NW * 32, 1) q4_gemm_mma_kernel(const GemmPa
     const uint32_t slots = (lut - sbase >= S::SLOT_BYTES) ? sbase : lut + S::LUT_BYTES;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, tq = lane & 3;
 
-    build_lut<T>(lut, p.code, tid, S::NW * 32);
+    build_lut<T>(lut, __ldg(p.code + (lane & 15)), tid, S::NW * 32);
     __syncthreads();
 
     const uint32_t cs = part_start(p.units, p.ctas, blockIdx.x);
@@ -398,6 +403,7 @@ struct StageGeom {
     }
 };
 static constexpr uint32_t kWaitLimit = 1u << 20;  // try_wait polls before giving up
+
 static constexpr int kErrWaitTimeout = 1;
 static constexpr int kErrNoRoom = 2;
 
@@ -511,6 +517,7 @@ __global__ void __launch_bounds__(S::NW * 32, 1)
     };
 
     if (p.pdl != 2) griddep_wait();
+    const float cv = __ldg(p.code + (lane & 15));  // the table build's one global load, issued early
     if (lane == 0) {  // each warp's own stage barriers; only this warp uses them
         for (int d = 0; d < D; ++d) mbar_init(bars + (uint32_t)(warp * D + d) * 8u, 1);
         mbar_init_fence();
@@ -535,6 +542,7 @@ __global__ void __launch_bounds__(S::NW * 32, 1)
     c.first_tile = true;
     StageCursor ld{c.tile, c.kb, nunits}, cm{c.tile, c.kb, nunits};
     int issued = 0, consumed = 0;
+    const uint64_t stream_once = l2_evict_first();  // weights are read once; absmax lines are reused
     auto issue = [&](int k) {  // lane 0: stage k into ring slot k % D
         int tile, kb0, kb, n;
         next_stage<UPS>(ld, p.kb_per_tile, tile, kb0, kb, n);
@@ -542,14 +550,14 @@ __global__ void __launch_bounds__(S::NW * 32, 1)
         const uint32_t bar = bars + (uint32_t)(warp * D + k % D) * 8u;
         if (lane == 0) {
             mbar_expect_tx(bar, G::BYTES);
-            tma_load_2d(st, &tmap_w, kb0 * 32, tile * S::TR, bar);
+            tma_load_2d_hint(st, &tmap_w, kb0 * 32, tile * S::TR, bar, stream_once);
             tma_load_2d(st + G::WEIGHT_BYTES, &tmap_a, (kb0 >> p.am_shift) & ~3, tile * S::TR, bar);
         }
     };
     // Start the first copies before anything else; the table is built while
     // they are in flight.
     for (; issued < D && ld.left > 0; ++issued) issue(issued);
-    build_lut<T>(lut, p.code, tid, S::NW * 32);
+    build_lut<T>(lut, cv, tid, S::NW * 32);
     __syncthreads();
     // Activations, outputs and the workspace may belong to the preceding
     // grid: touch them only after the dependency wait.
@@ -562,59 +570,66 @@ __global__ void __launch_bounds__(S::NW * 32, 1)
         const T* Aact = static_cast<const T*>(p.A);
         bool ok = true;
 
-        // Activations of the current stage's UPS-unit window (aw) and of the
-        // next stage's window (awn), loaded a whole stage ahead of use.
-        // Windows are UPS-aligned and tiles hold a multiple of UPS units, so
-        // a window never reaches past K.
-        uint32_t aw[UPS][S::NJ][2][4], awn[UPS][S::NJ][2][4];
-        auto load_window = [&](int kbw, uint32_t(&dst)[UPS][S::NJ][2][4]) {
+        // Activations of the current stage's UPS-unit window.  Windows are
+        // UPS-aligned and tiles hold a multiple of UPS units, so a window
+        // never reaches past K.  As soon as a unit is computed its registers
+        // are refilled with the same unit of the next stage's window, so the
+        // loads have most of a stage to land.
+        uint32_t aw[UPS][S::NJ][2][4];
+        auto load_unit = [&](int kbu, uint32_t(&dst)[S::NJ][2][4]) {
 #pragma unroll
-            for (int j = 0; j < UPS; ++j)
+            for (int jj = 0; jj < S::NJ; ++jj) {
+                const int m = 8 * jj + g;
 #pragma unroll
-                for (int jj = 0; jj < S::NJ; ++jj) {
-                    const int m = 8 * jj + g;
-#pragma unroll
-                    for (int ch = 0; ch < 2; ++ch) {
-                        if (m < p.M) {
-                            const uint4 v = ldg_v4(Aact + (size_t)m * p.K + (kbw + j) * S::SB + 32 * ch + 8 * tq);
-                            dst[j][jj][ch][0] = v.x;
-                            dst[j][jj][ch][1] = v.y;
-                            dst[j][jj][ch][2] = v.z;
-                            dst[j][jj][ch][3] = v.w;
-                        } else {
-                            dst[j][jj][ch][0] = dst[j][jj][ch][1] = dst[j][jj][ch][2] = dst[j][jj][ch][3] = 0u;
-                        }
+                for (int ch = 0; ch < 2; ++ch) {
+                    if (m < p.M) {
+                        const uint4 v = ldg_v4(Aact + (size_t)m * p.K + kbu * S::SB + 32 * ch + 8 * tq);
+                        dst[jj][ch][0] = v.x;
+                        dst[jj][ch][1] = v.y;
+                        dst[jj][ch][2] = v.z;
+                        dst[jj][ch][3] = v.w;
+                    } else {
+                        dst[jj][ch][0] = dst[jj][ch][1] = dst[jj][ch][2] = dst[jj][ch][3] = 0u;
                     }
                 }
+            }
         };
-        load_window(c.kb & ~(UPS - 1), aw);
+        auto load_window = [&](int kbw) {
+#pragma unroll
+            for (int j = 0; j < UPS; ++j) load_unit(kbw + j, aw[j]);
+        };
+        load_window(c.kb & ~(UPS - 1));
 
         // One 64-row x 64-k unit (window position j) of the stage at `st`,
         // scaled by the per-row absmax (ag: rows 16i+g, ag8: rows 16i+8+g).
         auto unit_rows = [&](uint32_t st, int j, int i, float ag, float ag8) {
             const float zero[4] = {0.f, 0.f, 0.f, 0.f};
             // rows 16i + 8(q&1) + r, chunk 2j + (q>>1)
-            uint32_t d0, d1, d2, d3;
-            ldmatrix_x4(G::chunk_addr(st, 16 * i + 8 * (lm_q & 1) + lm_r, 2 * j + (lm_q >> 1)), d0, d1, d2, d3);
+            uint32_t d[4];
+            ldmatrix_x4(G::chunk_addr(st, 16 * i + 8 * (lm_q & 1) + lm_r, 2 * j + (lm_q >> 1)), d[0], d[1], d[2], d[3]);
+            // q[x][b]: table pair of byte b of word d[x]
+            uint32_t q[4][4];
+#pragma unroll
+            for (int x = 0; x < 4; ++x) {
+                q[x][0] = lut_pair<0>(d[x], lane4);
+                q[x][1] = lut_pair<1>(d[x], lane4);
+                q[x][2] = lut_pair<2>(d[x], lane4);
+                q[x][3] = lut_pair<3>(d[x], lane4);
+            }
             float t[S::NJ][4];
             // steps 0..3: (d0,d1) bytes 0/1, 2/3, then (d2,d3) bytes 0/1, 2/3
-            uint32_t a0, a1, a2, a3;
-            a0 = lut_pair<0>(d0, lane4); a2 = lut_pair<1>(d0, lane4);
-            a1 = lut_pair<0>(d1, lane4); a3 = lut_pair<1>(d1, lane4);
 #pragma unroll
-            for (int jj = 0; jj < S::NJ; ++jj) mma16816<T>(t[jj], a0, a1, a2, a3, aw[j][jj][0][0], aw[j][jj][0][1], zero);
-            a0 = lut_pair<2>(d0, lane4); a2 = lut_pair<3>(d0, lane4);
-            a1 = lut_pair<2>(d1, lane4); a3 = lut_pair<3>(d1, lane4);
+            for (int jj = 0; jj < S::NJ; ++jj)
+                mma16816<T>(t[jj], q[0][0], q[1][0], q[0][1], q[1][1], aw[j][jj][0][0], aw[j][jj][0][1], zero);
 #pragma unroll
-            for (int jj = 0; jj < S::NJ; ++jj) mma16816<T>(t[jj], a0, a1, a2, a3, aw[j][jj][0][2], aw[j][jj][0][3], t[jj]);
-            a0 = lut_pair<0>(d2, lane4); a2 = lut_pair<1>(d2, lane4);
-            a1 = lut_pair<0>(d3, lane4); a3 = lut_pair<1>(d3, lane4);
+            for (int jj = 0; jj < S::NJ; ++jj)
+                mma16816<T>(t[jj], q[0][2], q[1][2], q[0][3], q[1][3], aw[j][jj][0][2], aw[j][jj][0][3], t[jj]);
 #pragma unroll
-            for (int jj = 0; jj < S::NJ; ++jj) mma16816<T>(t[jj], a0, a1, a2, a3, aw[j][jj][1][0], aw[j][jj][1][1], t[jj]);
-            a0 = lut_pair<2>(d2, lane4); a2 = lut_pair<3>(d2, lane4);
-            a1 = lut_pair<2>(d3, lane4); a3 = lut_pair<3>(d3, lane4);
+            for (int jj = 0; jj < S::NJ; ++jj)
+                mma16816<T>(t[jj], q[2][0], q[3][0], q[2][1], q[3][1], aw[j][jj][1][0], aw[j][jj][1][1], t[jj]);
 #pragma unroll
-            for (int jj = 0; jj < S::NJ; ++jj) mma16816<T>(t[jj], a0, a1, a2, a3, aw[j][jj][1][2], aw[j][jj][1][3], t[jj]);
+            for (int jj = 0; jj < S::NJ; ++jj)
+                mma16816<T>(t[jj], q[2][2], q[3][2], q[2][3], q[3][3], aw[j][jj][1][2], aw[j][jj][1][3], t[jj]);
 #pragma unroll
             for (int jj = 0; jj < S::NJ; ++jj) {
                 acc[i][jj][0] = fmaf(ag, t[jj][0], acc[i][jj][0]);
@@ -630,7 +645,7 @@ __global__ void __launch_bounds__(S::NW * 32, 1)
         while (cm.left > 0) {
             int tile, kb0, kb, n;
             next_stage<UPS>(cm, p.kb_per_tile, tile, kb0, kb, n);
-            if (cm.left > 0) load_window(cm.kb & ~(UPS - 1), awn);
+            const int kbn = cm.kb & ~(UPS - 1);  // next stage's window (when cm.left > 0)
             const int slot = consumed % D;
             const uint32_t st = stage_addr(warp * D + slot);
             const uint32_t bar = bars + (uint32_t)(warp * D + slot) * 8u;
@@ -670,7 +685,10 @@ __global__ void __launch_bounds__(S::NW * 32, 1)
                 // Whole stage inside one tile and the range: no tile can end
                 // before its last unit, so the units run back to back.
 #pragma unroll
-                for (int j = 0; j < UPS; ++j) unit_all_rows(j);
+                for (int j = 0; j < UPS; ++j) {
+                    unit_all_rows(j);
+                    if (cm.left > 0) load_unit(kbn + j, aw[j]);
+                }
                 c.kb += UPS - 1;
                 finish_unit_tma<T, S>(acc, has_first, has_last, c, cm.left == 0, p, lut, warp, lane, g, tq);
             } else {
@@ -681,16 +699,7 @@ __global__ void __launch_bounds__(S::NW * 32, 1)
                     finish_unit_tma<T, S>(acc, has_first, has_last, c, cm.left == 0 && kb0 + j + 1 == kb + n, p, lut,
                                           warp, lane, g, tq);
                 }
-            }
-            if (cm.left > 0) {
-#pragma unroll
-                for (int j = 0; j < UPS; ++j)
-#pragma unroll
-                    for (int jj = 0; jj < S::NJ; ++jj)
-#pragma unroll
-                        for (int ch = 0; ch < 2; ++ch)
-#pragma unroll
-                            for (int w = 0; w < 4; ++w) aw[j][jj][ch][w] = awn[j][jj][ch][w];
+                if (cm.left > 0) load_window(kbn);  // first or last stage of a range only
             }
             ++consumed;
             // Hand the slot back to the copy engine: order this warp's reads
@@ -798,6 +807,7 @@ __global__ void __launch_bounds__((S::NW + 1) * 32, 1)
     if (producer) {
         // Lane w streams consumer w's unit range into its ring.
         if (lane < NC) {
+            const uint64_t stream_once = l2_evict_first();
             const uint32_t ws = cs + part_start(uc, NC, lane), we = cs + part_start(uc, NC, lane + 1);
             const int nunits = (int)(we - ws);
             const int tile0 = nunits > 0 ? (int)(ws / (uint32_t)p.kb_per_tile) : 0;
@@ -813,12 +823,12 @@ __global__ void __launch_bounds__((S::NW + 1) * 32, 1)
                 next_stage<UPS>(ld, p.kb_per_tile, tile, kb0, kb, n);
                 const uint32_t st = stage_addr(lane * D + slot);
                 mbar_expect_tx(full_bar(lane, slot), G::BYTES);
-                tma_load_2d(st, &tmap_w, kb0 * 32, tile * S::TR, full_bar(lane, slot));
+                tma_load_2d_hint(st, &tmap_w, kb0 * 32, tile * S::TR, full_bar(lane, slot), stream_once);
                 tma_load_2d(st + G::WEIGHT_BYTES, &tmap_a, (kb0 >> p.am_shift) & ~3, tile * S::TR, full_bar(lane, slot));
             }
         }
     } else {
-        build_lut<T>(lut, p.code, tid, NC * 32);
+        build_lut<T>(lut, __ldg(p.code + (lane & 15)), tid, NC * 32);
         named_bar_sync(1, NC * 32);
         if (p.pdl == 2) griddep_wait();
         griddep_launch_dependents();
@@ -1002,7 +1012,10 @@ static cudaError_t make_tensor_maps(const GemmParams& p, int ups, CUtensorMap* t
     const cuuint32_t wbox[2] = {(cuuint32_t)(32 * ups), 64};
     if (enc(tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(p.Wp), wdim, wstride, wbox, estride,
             CU_TENSOR_MAP_INTERLEAVE_NONE, ups == 4 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            // no promotion past the box: a wider L2 fill would take the next
+            // stage's bytes, which at a warp boundary belong to another warp
+            // that reads them much later (by then evicted, so read twice)
+            CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
         return cudaErrorInvalidValue;
     const cuuint64_t adim[2] = {(cuuint64_t)p.am_per_row, (cuuint64_t)p.N};
     const cuuint64_t astride[1] = {(cuuint64_t)p.am_per_row * 4};
