@@ -201,6 +201,85 @@ class Layer:
                                  self.case.blocksize, out=self.out, pdl=self.pdl)
 
 
+def split_time_est_us(case: inputs.Case, peak_gbs: float) -> float:
+    """Time at the HBM peak of the split path: read the packed weights and
+    absmax, write the bf16 weights, read them back in a dense GEMM, plus A
+    and C once."""
+    nk = case.N * case.K
+    b = nk * (0.5 + 4.0 / case.blocksize) + 2 * nk + 2 * nk + 2 * case.M * case.K + 2 * case.M * case.N
+    return b / (peak_gbs * 1e3)
+
+
+def crossover_estimates(layers, per_shape, peak_gbs: float) -> list:
+    """Per weight shape measured at several M: the smallest M at which the
+    split path's HBM-peak time undercuts the measured fused time, taken
+    from the measured points or, past them, from a line through the last two."""
+    by_shape = {}
+    for L, ps in zip(layers, per_shape):
+        c = L.case
+        by_shape.setdefault((c.N, c.K, c.blocksize), []).append((c.M, ps["us_serialized"], c))
+    res = []
+    for (N, K, bs), pts in by_shape.items():
+        pts.sort(key=lambda x: x[0])
+        if len(pts) < 2:
+            continue
+        est = None
+        for M, t, c in pts:
+            if t > split_time_est_us(c, peak_gbs):
+                est = {"M": M, "how": "measured point"}
+                break
+        if est is None:
+            (m1, t1, c1), (m2, t2, c2) = pts[-2], pts[-1]
+            s_fused = (t2 - t1) / (m2 - m1)
+            a2, b2 = split_time_est_us(c2, peak_gbs), 2 * (K + N) / (peak_gbs * 1e3)
+            if s_fused > b2:
+                m_star = m2 + (a2 - t2) / (s_fused - b2)
+                est = {"M": round(m_star, 1), "how": "extrapolated (line through the last two measured M)"}
+            else:
+                est = {"M": None, "how": "fused time grows no faster than the split estimate: no crossover"}
+        res.append({"shape": f"K{K} N{N} bs{bs}", "M_measured": [p[0] for p in pts], **est})
+    return res
+
+
+def measure_split_path(layers, device, stream, reps: int = 20) -> list:
+    """Device time of dequantize (this library) + cuBLAS bf16 GEMM per layer:
+    each half captured as a CUDA graph of `reps` launches, timed by events
+    around its replay."""
+    out = []
+    for L in layers:
+        c = L.case
+        dt = L.A.dtype
+        W = torch.empty((c.N, c.K), dtype=dt, device=device)
+        Y = torch.empty((c.M, c.N), dtype=dt, device=device)
+        deq = lambda: q4.q4_dequantize_blockwise(L.packed, L.absmax, L.code, c.N * c.K, c.blocksize, out=W.view(-1))
+        mm = lambda: torch.matmul(L.A, W.t(), out=Y)
+        times = []
+        for fn in (deq, mm):
+            with torch.cuda.stream(stream):
+                for _ in range(3):
+                    fn()
+            stream.synchronize()
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                for _ in range(reps):
+                    fn()
+            best = float("inf")
+            for _ in range(3):
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                with torch.cuda.stream(stream):
+                    e0.record(stream)
+                    g.replay()
+                    e1.record(stream)
+                stream.synchronize()
+                best = min(best, e0.elapsed_time(e1) * 1e3 / reps)
+            times.append(best)
+            del g
+        del W, Y
+        out.append({"tag": c.tag, "dequant_us": round(times[0], 2), "gemm_us": round(times[1], 2),
+                    "us": round(times[0] + times[1], 2), "timing": f"CUDA graph of {reps} launches per half, best of 3"})
+    return out
+
+
 def run_ours(args, world, rank, local):
     device = torch.device("cuda", local)
     torch.cuda.set_device(device)
@@ -294,7 +373,12 @@ def run_ours(args, world, rank, local):
         per_shape.append({"shape": f"M{L.case.M} K{L.case.K} N{L.case.N} bs{L.case.blocksize}", "tag": L.case.tag,
                           "us_serialized": round(us, 3), "GB/s": round(gbs, 1), "frac_of_peak": round(gbs / peak, 4),
                           "bytes": L.bytes, "bf16_weight_roofline_us": round(bf16_roof_us, 3),
+                          "t_split_est_us": round(split_time_est_us(L.case, peak), 3),
                           "plan": {k: L.plan[k] for k in ("ctas", "warps", "depth", "loader", "m_pad", "units")}})
+
+    # The split path the fused kernel competes with (opt-in): the library's
+    # dequantize kernel into a bf16 weight matrix, then a cuBLAS bf16 GEMM.
+    split_path = measure_split_path(layers, device, stream) if args.split_path else None
 
     # End to end through the public Python API: per step, H2D of the
     # activations from pinned memory, the four calls, D2H of the outputs.
@@ -334,6 +418,8 @@ def run_ours(args, world, rank, local):
                      "per_unit": "0.5 B per weight (codes) + 4/bs B (absmax) + A and C once",
                      "duration": "average launch = timed-region device time / launches (all launches are this kernel)"},
         "per_shape": per_shape,
+        "crossover": crossover_estimates(layers, per_shape, peak),
+        "split_path": split_path if args.split_path else None,
         "e2e": {"value": round(e2e_value, 2) if e2e_value else None, "unit": "GB/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "steps": e2e_steps,
                 "api": "bit_weight_dequant_b200.q4_gemm_skinny (ctypes -> libq4 C ABI), wall clock"},
@@ -436,6 +522,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end leg (profiling runs)")
     ap.add_argument("--only", default="", help="comma-separated case tags of the workload to run (profiling)")
+    ap.add_argument("--split-path", action="store_true",
+                    help="also time the split path (dequantize kernel + cuBLAS bf16 GEMM) per layer")
     ap.add_argument("--pdl", type=int, default=2, choices=[0, 1, 2],
                     help="programmatic dependent launch mode for the GEMMs (2: static weights read early)")
     args = ap.parse_args()

@@ -8,6 +8,7 @@ there is no fallback of any kind, a missing library raises.
 from __future__ import annotations
 
 import ctypes
+import functools
 import os
 import re
 
@@ -86,11 +87,12 @@ def _check(rc: int, what: str):
 
 
 def _ptr(t):
-    return ctypes.c_void_p(t.data_ptr()) if t is not None else None
+    """Device address of a tensor as a plain int (ctypes converts it), or None."""
+    return t.data_ptr() if t is not None else None
 
 
-def _stream(device) -> ctypes.c_void_p:
-    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+def _stream(device) -> int:
+    return torch.cuda.current_stream(device).cuda_stream
 
 
 def q4_quantize_blockwise(W: torch.Tensor, blocksize: int, code: torch.Tensor):
@@ -118,9 +120,13 @@ def q4_dequantize_blockwise(packed: torch.Tensor, absmax: torch.Tensor, code: to
 
 
 def q4_gemm_workspace_size(M: int, N: int, K: int, blocksize: int, act_dtype: torch.dtype) -> int:
+    return _workspace_bytes(M, N, K, blocksize, _TORCH_TO_Q4[act_dtype])
+
+
+@functools.lru_cache(maxsize=4096)
+def _workspace_bytes(M: int, N: int, K: int, blocksize: int, act: int) -> int:
     v = ctypes.c_size_t(0)
-    _check(lib().q4_gemm_workspace_size(M, N, K, blocksize, _TORCH_TO_Q4[act_dtype], ctypes.byref(v)),
-           "q4_gemm_workspace_size")
+    _check(lib().q4_gemm_workspace_size(M, N, K, blocksize, act, ctypes.byref(v)), "q4_gemm_workspace_size")
     return v.value
 
 
@@ -169,8 +175,8 @@ def workspace_error(ws: "Workspace") -> int:
 
 
 
-def _default_workspace(device) -> Workspace:
-    key = (torch.device(device), torch.cuda.current_stream(device).cuda_stream)
+def _default_workspace(device, stream: int) -> Workspace:
+    key = (device, stream)
     ws = _workspaces.get(key)
     if ws is None:
         ws = _workspaces[key] = Workspace(device)
@@ -188,6 +194,13 @@ def overrides(**kw) -> q4_gemm_plan_t | None:
     return ov
 
 
+@functools.lru_cache(maxsize=256)
+def _overrides_ref(items: tuple):
+    """byref() of a cached, never-modified overrides struct (None if empty)."""
+    ov = overrides(**dict(items))
+    return (ov, ctypes.byref(ov)) if ov is not None else (None, None)
+
+
 def q4_gemm_skinny(A: torch.Tensor, Wpacked: torch.Tensor, absmax: torch.Tensor, code: torch.Tensor, N: int,
                    K: int, blocksize: int, out: torch.Tensor | None = None, workspace: Workspace | None = None,
                    **launch) -> torch.Tensor:
@@ -195,19 +208,20 @@ def q4_gemm_skinny(A: torch.Tensor, Wpacked: torch.Tensor, absmax: torch.Tensor,
 
     ``launch`` may hold launch-table overrides (math, warps, ctas, depth,
     l2_prefetch, loader) for measurements, and ``pdl`` to opt into
-    programmatic dependent launch (see q4.h); by default the table decides."""
+    programmatic dependent launch (see q4.h); by default the table decides.
+    Argument marshalling only: the per-call work on the host is a few
+    dictionary lookups and one C call."""
     M = A.shape[0] if A.dim() == 2 else 1
     if out is None:
         out = torch.empty((M, N), dtype=A.dtype, device=A.device)
     act = _TORCH_TO_Q4[A.dtype]
-    need = ctypes.c_size_t(0)
-    _check(lib().q4_gemm_workspace_size(M, N, K, blocksize, act, ctypes.byref(need)), "q4_gemm_workspace_size")
-    nbytes = need.value
-    ws = (workspace or _default_workspace(A.device)).get(nbytes) if nbytes else None
-    ov = overrides(**launch)
-    rc = lib().q4_gemm_skinny_ex(_ptr(A), _ptr(Wpacked), _ptr(absmax), _ptr(code), M, N, K, blocksize, act,
-                                 _ptr(out), _ptr(ws), ws.numel() if ws is not None else 0, _stream(A.device),
-                                 ctypes.byref(ov) if ov is not None else None)
+    nbytes = _workspace_bytes(M, N, K, blocksize, act)
+    stream = torch.cuda.current_stream(A.device).cuda_stream
+    ws = (workspace or _default_workspace(A.device, stream)).get(nbytes) if nbytes else None
+    ov_ref = _overrides_ref(tuple(sorted(launch.items())))[1] if launch else None
+    rc = lib().q4_gemm_skinny_ex(A.data_ptr(), Wpacked.data_ptr(), absmax.data_ptr(), code.data_ptr(), M, N, K,
+                                 blocksize, act, out.data_ptr(), ws.data_ptr() if ws is not None else None,
+                                 ws.numel() if ws is not None else 0, stream, ov_ref)
     _check(rc, "q4_gemm_skinny")
     return out
 

@@ -94,20 +94,63 @@ struct DequantOut<1> {  // fp16
     }
 };
 
-// One thread per 32 elements (16 packed bytes -> one 128-bit load); a chunk
+// Writes dominate (2 or 4 output bytes per 0.5 input byte), so every store
+// is a contiguous 16-byte piece of a warp-wide run: a warp takes 1024-element
+// chunks, and in quarter w lane t dequantizes elements 256w + 8t .. +8 from
+// the 4 packed bytes at 128w + 4t (one 128-byte load per quarter, 512 or
+// 1024 contiguous output bytes per store instruction).  An 8-element run
 // never straddles an absmax block because blocksize is a multiple of 32.
+// Elements past the last whole chunk go 32 per thread, then one per thread.
 template <int OUT>
 __global__ void __launch_bounds__(256) q4_dequant_kernel(const uint8_t* __restrict__ packed,
                                                          const float* __restrict__ absmax,
                                                          const float* __restrict__ code, int64_t n, int bs_shift,
                                                          void* __restrict__ out) {
-    __shared__ float sc[16];
+    __shared__ float sc[16];  // 16 entries in 16 banks: lookups never conflict
     if (threadIdx.x < 16) sc[threadIdx.x] = code[threadIdx.x];
     __syncthreads();
-    const int64_t nchunks = n >> 5;
-    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-    const int64_t t0 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    for (int64_t q = t0; q < nchunks; q += stride) {
+    const int lane = threadIdx.x & 31;
+    const int64_t tid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const int64_t nthreads = (int64_t)gridDim.x * blockDim.x;
+    const int64_t nwchunks = n >> 10;
+    for (int64_t q = tid >> 5; q < nwchunks; q += nthreads >> 5) {
+        uint32_t words[4];
+        float am[4];
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+            words[w] = ldg_stream_u32(packed + (q << 9) + 128 * w + 4 * lane);
+            am[w] = __ldg(absmax + (((q << 10) + 256 * w + 8 * lane) >> bs_shift));
+        }
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+            const int64_t e0 = (q << 10) + 256 * w + 8 * lane;  // first of this lane's 8 elements
+            if constexpr (OUT == 2) {
+                float f[8];
+#pragma unroll
+                for (int by = 0; by < 4; ++by) {
+                    const uint32_t b = (words[w] >> (8 * by)) & 0xFFu;
+                    f[2 * by] = __fmul_rn(sc[b >> 4], am[w]);
+                    f[2 * by + 1] = __fmul_rn(sc[b & 15u], am[w]);
+                }
+                float4* o = reinterpret_cast<float4*>(static_cast<float*>(out) + e0);
+                o[0] = make_float4(f[0], f[1], f[2], f[3]);
+                o[1] = make_float4(f[4], f[5], f[6], f[7]);
+            } else {
+                uint32_t r[4];
+#pragma unroll
+                for (int by = 0; by < 4; ++by) {
+                    const uint32_t b = (words[w] >> (8 * by)) & 0xFFu;
+                    r[by] = DequantOut<OUT>::pair(__fmul_rn(sc[b >> 4], am[w]), __fmul_rn(sc[b & 15u], am[w]));
+                }
+                *reinterpret_cast<uint4*>(static_cast<uint16_t*>(out) + e0) = make_uint4(r[0], r[1], r[2], r[3]);
+            }
+        }
+    }
+    // Whole 32-element chunks after the last 1024-element chunk.
+    const int64_t c0 = nwchunks << 5, nchunks = n >> 5;
+    const int64_t t0 = tid;
+    const int64_t stride = nthreads;
+    for (int64_t q = c0 + t0; q < nchunks; q += stride) {
         const uint4 v = ldg_stream_v4(packed + 16 * q);
         const float am = __ldg(absmax + ((q << 5) >> bs_shift));
         const uint32_t words[4] = {v.x, v.y, v.z, v.w};

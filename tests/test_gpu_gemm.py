@@ -70,16 +70,21 @@ def _problem(device, M=3, N=300, K=1024, bs=64, seed=7):
 
 
 @pytest.mark.parametrize("loader", [1, 2, 3, 4, 5])
-def test_deterministic_and_counters_left_zero(cuda_device, loader):
-    A, P, Am, C, N, K, bs = _problem(cuda_device)
+@pytest.mark.parametrize("N,K,ctas", [(300, 1024, 5), (64, 4096, 20), (200, 2048, 7)])
+def test_deterministic_and_counters_left_zero(cuda_device, loader, N, K, ctas):
+    """Repeated calls agree bit for bit, match the oracle and leave every tile
+    counter at zero: tiles cut between 2, 3 or 20 CTAs."""
+    A, P, Am, C, N, K, bs = _problem(cuda_device, N=N, K=K)
     ws = q4.Workspace(cuda_device)
-    outs = [q4.q4_gemm_skinny(A, P, Am, C, N, K, bs, workspace=ws, ctas=5, loader=loader) for _ in range(3)]
+    outs = [q4.q4_gemm_skinny(A, P, Am, C, N, K, bs, workspace=ws, ctas=ctas, loader=loader) for _ in range(3)]
     torch.cuda.synchronize()
     for o in outs[1:]:
         assert torch.equal(o.view(torch.int16), outs[0].view(torch.int16))
+    assert q4.workspace_error(ws) == 0
     off = q4.workspace_counter_offset(cuda_device)
     assert ws.buf.numel() > off and int(ws.buf[off:].count_nonzero()) == 0
-    assert q4.workspace_error(ws) == 0
+    y, S = oracle.gemm(bits_of(A.cpu()), oracle.BF16, P.cpu().numpy(), Am.cpu().numpy(), C.cpu().numpy(), A.shape[0], N, K, bs)
+    check_gemm(bits_of(outs[0].cpu()), y, S, "bf16", f"loader {loader} ctas {ctas}")
 
 
 @pytest.mark.parametrize("order", [0, 1])
