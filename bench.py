@@ -169,6 +169,7 @@ class Layer:
         W = inputs.weights_device(case.N, case.K, seed, device, case.outliers)
         self.packed, self.absmax = q4.q4_quantize_blockwise(W.reshape(-1), case.blocksize, self.code)
         del W
+        torch.cuda.empty_cache()  # the fp32 weights were transient: hand their memory back
         self.A_host = inputs.activations(case.M, case.K, dt, seed).pin_memory()
         self.A = self.A_host.to(device)
         self.out = torch.empty((case.M, case.N), dtype=dt, device=device)

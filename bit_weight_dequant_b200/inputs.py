@@ -154,7 +154,7 @@ class Workload:
 
 
 def workloads() -> dict:
-    """The five configurations, each a list of Cases."""
+    """The five configurations, each a list of Cases, and one profiling shape."""
     w = {}
     # 0: small square check case.
     w["square4096"] = Workload("M=1 K=4096 N=4096 bs64 bf16 normal-table", 0,
@@ -188,4 +188,8 @@ def workloads() -> dict:
             ext.append(Case(M, N, K, tag=f"K{K}N{N}M{M}"))
     w["aspect"] = Workload("extreme aspect ratios at M=1..8: K2560/N248320, K320/N10240, K10240/N320, "
                            "K2560/N12", 4, ext)
+    # Not one of the five: one long-K layer whose launch is almost all main
+    # loop (start-up and tail are a few percent), for profiling the loop.
+    w["longk"] = Workload("M=1 K=131072 N=8192 bs64 bf16 normal-table (main-loop profiling shape)", 5,
+                          [Case(1, 8192, 131072, tag="longk")])
     return w
