@@ -53,7 +53,24 @@ def code_normal_quantile(eps: float = 1.0 / 32.0) -> np.ndarray:
     return np.array(vals, dtype=np.float64).astype(np.float32)
 
 
-CODE_TABLES = {"normal": code_normal_quantile, "uniform": code_uniform}
+def code_fp4_e2m1() -> np.ndarray:
+    """The 16 values of a 4-bit float (1 sign, 2 exponent, 1 mantissa bit,
+    exponent bias 1), indexed by their bit pattern and divided by the
+    largest magnitude, 6, so that the table spans [-1, 1].
+
+    Code i has sign = bit 3, exponent e = bits 2..1, mantissa m = bit 0.
+    Its magnitude is m/2 for e = 0 (zero and the one subnormal, 1/2) and
+    2^(e-1) * (1 + m/2) otherwise, i.e. 0, 1/2, 1, 3/2, 2, 3, 4, 6.  The
+    table is in bit order, not sorted, and code 8 is -0."""
+    vals = []
+    for i in range(16):
+        s, e, m = i >> 3, (i >> 1) & 3, i & 1
+        mag = m / 2.0 if e == 0 else 2.0 ** (e - 1) * (1.0 + m / 2.0)
+        vals.append((-mag if s else mag) / 6.0)
+    return np.array(vals, dtype=np.float64).astype(np.float32)
+
+
+CODE_TABLES = {"normal": code_normal_quantile, "uniform": code_uniform, "fp4": code_fp4_e2m1}
 
 # ---------------------------------------------------------------------------
 # Random inputs.

@@ -50,10 +50,11 @@ def _load():
         lib.oracle_quantize.argtypes = [P, i64, ci, P, P, P]
         lib.oracle_dequantize.argtypes = [P, P, P, i64, ci, ci, P]
         lib.oracle_gemm.argtypes = [P, ci, P, P, P, ci, ci, ci, ci, P, P]
+        lib.oracle_gemm_bias.argtypes = [P, ci, P, P, P, P, ci, ci, ci, ci, P, P]
         lib.oracle_round.argtypes = [P, i64, ci, P]
         lib.oracle_decode.argtypes = [P, i64, ci, P]
         lib.oracle_ulp.argtypes = [P, i64, ci, P]
-        for f in ("oracle_quantize", "oracle_dequantize", "oracle_gemm", "oracle_round",
+        for f in ("oracle_quantize", "oracle_dequantize", "oracle_gemm", "oracle_gemm_bias", "oracle_round",
                   "oracle_decode", "oracle_ulp"):
             getattr(lib, f).restype = ci
         _lib = lib
@@ -96,8 +97,9 @@ def dequantize(packed: np.ndarray, absmax: np.ndarray, code: np.ndarray, n: int,
 
 
 def gemm(a_bits: np.ndarray, act_dtype: int, packed: np.ndarray, absmax: np.ndarray, code: np.ndarray,
-         M: int, N: int, K: int, blocksize: int, want_s: bool = True):
-    """fp64 reference ``y[M,N]`` (unrounded) and ``S[M,N] = sum |a*w|``."""
+         M: int, N: int, K: int, blocksize: int, want_s: bool = True, bias_bits: np.ndarray | None = None):
+    """fp64 reference ``y[M,N]`` (unrounded) and ``S[M,N] = sum |a*w|``;
+    with ``bias_bits`` (N bf16/fp16 patterns) the bias is added to y."""
     a_bits = np.ascontiguousarray(a_bits, dtype=np.uint16).reshape(-1)
     assert a_bits.size == M * K
     packed = np.ascontiguousarray(packed, dtype=np.uint8)
@@ -105,8 +107,15 @@ def gemm(a_bits: np.ndarray, act_dtype: int, packed: np.ndarray, absmax: np.ndar
     code = np.ascontiguousarray(code, dtype=np.float32)
     y = np.zeros((M, N), dtype=np.float64)
     S = np.zeros((M, N), dtype=np.float64) if want_s else None
-    _check(_load().oracle_gemm(_ptr(a_bits), act_dtype, _ptr(packed), _ptr(absmax), _ptr(code), M, N, K,
-                               blocksize, _ptr(y), _ptr(S) if want_s else None), "gemm")
+    if bias_bits is None:
+        _check(_load().oracle_gemm(_ptr(a_bits), act_dtype, _ptr(packed), _ptr(absmax), _ptr(code), M, N, K,
+                                   blocksize, _ptr(y), _ptr(S) if want_s else None), "gemm")
+    else:
+        bias_bits = np.ascontiguousarray(bias_bits, dtype=np.uint16).reshape(-1)
+        assert bias_bits.size == N
+        _check(_load().oracle_gemm_bias(_ptr(a_bits), act_dtype, _ptr(packed), _ptr(absmax), _ptr(code),
+                                        _ptr(bias_bits), M, N, K, blocksize, _ptr(y),
+                                        _ptr(S) if want_s else None), "gemm_bias")
     return (y, S) if want_s else y
 
 

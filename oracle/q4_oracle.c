@@ -313,3 +313,24 @@ int oracle_gemm(const uint16_t* A, int act_dtype, const uint8_t* packed, const f
     }
     return OR_OK;
 }
+
+/*
+ * The same layer with a bias, the epilogue of the planned gemm_4bit op
+ * (bitsandbytes PR #1920, "Technical details"):
+ *     y[m,n] = bias[n] + sum_k double(a[m,k]) * double(w[n,k])
+ * with bias given as N bf16/fp16 bit patterns of the activation type.  The
+ * bias enters the fp64 value once, after the k sum; S is the same as without
+ * a bias (the bias is exact, it adds no rounding of its own).
+ */
+int oracle_gemm_bias(const uint16_t* A, int act_dtype, const uint8_t* packed, const float* absmax,
+                     const float* code, const uint16_t* bias, int M, int N, int K, int bs, double* y, double* S) {
+    if (!bias) return OR_BAD;
+    int rc = oracle_gemm(A, act_dtype, packed, absmax, code, M, N, K, bs, y, S);
+    if (rc != OR_OK || !y) return rc;
+    for (int m = 0; m < M; ++m)
+        for (int n = 0; n < N; ++n) {
+            float b = act_dtype == OR_BF16 ? or_bf16_to_float(bias[n]) : or_fp16_to_float(bias[n]);
+            y[(int64_t)m * N + n] += (double)b;
+        }
+    return OR_OK;
+}

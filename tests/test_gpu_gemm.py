@@ -32,7 +32,8 @@ def test_gemm_blocksizes(cuda_device, M, bs):
 
 
 @pytest.mark.parametrize("M", [1, 5, 16])
-@pytest.mark.parametrize("act,table", [("fp16", "normal"), ("bf16", "uniform"), ("fp16", "uniform")])
+@pytest.mark.parametrize("act,table", [("fp16", "normal"), ("bf16", "uniform"), ("fp16", "uniform"), ("bf16", "fp4"),
+                                       ("fp16", "fp4")])
 def test_gemm_dtypes_tables(cuda_device, M, act, table):
     run_case(Case(M, 300, 1536, act=act, table=table), seed=3000 + M, device=cuda_device)
 

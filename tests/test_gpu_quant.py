@@ -25,7 +25,7 @@ def _weights(n, bs, seed, outliers):
     return w
 
 
-@pytest.mark.parametrize("table", ["normal", "uniform"])
+@pytest.mark.parametrize("table", ["normal", "uniform", "fp4"])
 @pytest.mark.parametrize("n,bs", SIZES)
 @pytest.mark.parametrize("outliers", [False, True])
 def test_quantize_bit_exact(cuda_device, table, n, bs, outliers):

@@ -19,7 +19,7 @@ import oracle
 from bit_weight_dequant_b200 import inputs
 from conftest import read_golden
 
-TABLES = {"uniform": inputs.code_uniform(), "normal": inputs.code_normal_quantile()}
+TABLES = {"uniform": inputs.code_uniform(), "normal": inputs.code_normal_quantile(), "fp4": inputs.code_fp4_e2m1()}
 
 
 # ---------------------------------------------------------------------------
@@ -107,11 +107,30 @@ def test_normal_table_against_scipy():
     assert (c > 0).sum() == 8 and (c < 0).sum() == 7
 
 
+def test_fp4_table_is_the_e2m1_format():
+    """Rebuild the table from binary16 bit patterns (a different route: the
+    E2M1 fields moved into an IEEE half and decoded by numpy)."""
+    c = inputs.code_fp4_e2m1()
+    for i in range(16):
+        s, e, m = i >> 3, (i >> 1) & 3, i & 1
+        if e == 0 and m == 0:
+            bits = s << 15                                   # +-0
+        elif e == 0:
+            bits = (s << 15) | ((15 - 1) << 10)              # subnormal 0.5 = 2^-1
+        else:
+            bits = (s << 15) | ((e - 1 + 15) << 10) | (m << 9)
+        half = np.array([bits], dtype=np.uint16).view(np.float16)[0]
+        want = np.float32(np.float64(half) / 6.0)
+        assert c[i] == want and np.signbit(c[i]) == bool(s), i
+    assert sorted(set(np.round(np.abs(c).astype(np.float64) * 6, 6))) == [0, 0.5, 1, 1.5, 2, 3, 4, 6]
+    assert c[7] == 1 and c[15] == -1
+
+
 # ---------------------------------------------------------------------------
 # quantize: brute force and invariants
 # ---------------------------------------------------------------------------
 
-@pytest.mark.parametrize("table", ["uniform", "normal"])
+@pytest.mark.parametrize("table", ["uniform", "normal", "fp4"])
 @pytest.mark.parametrize("n,bs", [(1, 32), (31, 32), (64, 64), (1001, 64), (777, 128), (2049, 256),
                                   (300, 4096)])
 def test_quantize_brute_force(table, n, bs):
@@ -135,7 +154,7 @@ def test_quantize_brute_force(table, n, bs):
     assert np.all(idx == first), "ties must go to the lowest index"
 
 
-@pytest.mark.parametrize("table", ["uniform", "normal"])
+@pytest.mark.parametrize("table", ["uniform", "normal", "fp4"])
 def test_quantize_error_bound_and_extremes(table):
     code = TABLES[table]
     bs = 64
@@ -145,7 +164,7 @@ def test_quantize_error_bound_and_extremes(table):
     w[64 * 7 + 5] *= 20                          # an outlier
     packed, absmax = oracle.quantize(w, bs, code)
     wq = np_weights(packed, absmax, code, w.size, bs).astype(np.float64)
-    gap = float(np.max(np.diff(code.astype(np.float64))))
+    gap = float(np.max(np.diff(np.sort(code.astype(np.float64)))))   # largest gap between adjacent levels
     am = absmax[np.arange(w.size) // bs].astype(np.float64)
     err = np.abs(wq - w.astype(np.float64))
     assert np.all(err <= am * gap / 2 * (1 + 1e-6) + 1e-30)
@@ -190,7 +209,7 @@ def test_quantize_rejects_nonfinite():
 # dequantize vs library conversions
 # ---------------------------------------------------------------------------
 
-@pytest.mark.parametrize("table", ["uniform", "normal"])
+@pytest.mark.parametrize("table", ["uniform", "normal", "fp4"])
 @pytest.mark.parametrize("bs", [32, 64, 256])
 def test_dequantize_matches_library_rounding(table, bs):
     code = TABLES[table]
@@ -291,6 +310,31 @@ def test_gemm_brute_force(act, M, N, K, bs):
     assert y.shape == (M, N)
     np.testing.assert_allclose(y, yref, rtol=0, atol=1e-12 * (Sref.max() + 1))
     np.testing.assert_allclose(S, Sref, rtol=1e-12)
+
+
+@pytest.mark.parametrize("act", [oracle.BF16, oracle.FP16])
+def test_gemm_bias_against_numpy_and_zero_weights(act):
+    """The bias epilogue: numpy fp64 matmul plus the decoded bias; with every
+    absmax 0 the layer is the bias itself, exactly."""
+    code = TABLES["normal"]
+    M, N, K, bs = 3, 40, 128, 64
+    rng = np.random.default_rng(77)
+    w = (rng.standard_normal(N * K) * 0.02).astype(np.float32)
+    packed, absmax = oracle.quantize(w, bs, code)
+    a32 = rng.standard_normal((M, K)).astype(np.float32)
+    b32 = rng.standard_normal(N).astype(np.float32)
+    if act == oracle.BF16:
+        abits, bbits = torch_bf16_bits(a32).reshape(M, K), torch_bf16_bits(b32)
+        a64, b64 = torch_bf16_values(abits.reshape(-1)).reshape(M, K), torch_bf16_values(bbits)
+    else:
+        abits, bbits = np_fp16_bits(a32).reshape(M, K), np_fp16_bits(b32)
+        a64, b64 = abits.view(np.float16).astype(np.float64), bbits.view(np.float16).astype(np.float64)
+    W64 = np_weights(packed, absmax, code, N * K, bs).astype(np.float64).reshape(N, K)
+    y, S = oracle.gemm(abits, act, packed, absmax, code, M, N, K, bs, bias_bits=bbits)
+    np.testing.assert_allclose(y, a64 @ W64.T + b64[None, :], rtol=0, atol=1e-12 * (S.max() + 1))
+    np.testing.assert_allclose(S, np.abs(a64) @ np.abs(W64).T, rtol=1e-12)
+    y0, S0 = oracle.gemm(abits, act, packed, np.zeros_like(absmax), code, M, N, K, bs, bias_bits=bbits)
+    assert np.array_equal(y0, np.broadcast_to(b64, (M, N))) and np.all(S0 == 0)
 
 
 def test_gemm_all_codes_one_closed_form():
