@@ -59,12 +59,14 @@ def lib() -> ctypes.CDLL:
         L.q4_gemm_skinny_ex.argtypes = [P, P, P, P, ci, ci, ci, ci, ci, P, P, sz, P, ctypes.POINTER(q4_gemm_plan_t)]
         L.q4_gemm_plan.argtypes = [ci, ci, ci, ci, ci, ci, ctypes.POINTER(q4_gemm_plan_t)]
         L.q4_gemm_skinny_noalloc.argtypes = [P, P, P, P, ci, ci, ci, ci, ci, P, P]
+        L.q4_gemm_skinny_bias.argtypes = [P, P, P, P, P, ci, ci, ci, ci, ci, P, P, sz, P,
+                                          ctypes.POINTER(q4_gemm_plan_t)]
         L.q4_partition_start.argtypes = [i64, ci, ci]
         L.q4_partition_start.restype = i64
         L.q4_partition_owner.argtypes = [i64, ci, i64]
         for f in ("q4_quantize_blockwise", "q4_dequantize_blockwise", "q4_gemm_workspace_size",
                   "q4_gemm_skinny", "q4_gemm_skinny_ex", "q4_gemm_plan", "q4_partition_owner",
-                  "q4_gemm_skinny_noalloc"):
+                  "q4_gemm_skinny_noalloc", "q4_gemm_skinny_bias"):
             getattr(L, f).restype = ci
         _lib = L
     return _lib
@@ -203,14 +205,15 @@ def _overrides_ref(items: tuple):
 
 def q4_gemm_skinny(A: torch.Tensor, Wpacked: torch.Tensor, absmax: torch.Tensor, code: torch.Tensor, N: int,
                    K: int, blocksize: int, out: torch.Tensor | None = None, workspace: Workspace | None = None,
-                   **launch) -> torch.Tensor:
-    """out[M, N] = A[M, K] . dequant(W)[N, K]^T on the GPU (fused kernel).
+                   bias: torch.Tensor | None = None, **launch) -> torch.Tensor:
+    """out[M, N] = A[M, K] . dequant(W)[N, K]^T (+ bias[N]) on the GPU (fused kernel).
 
-    ``launch`` may hold launch-table overrides (math, warps, ctas, depth,
-    l2_prefetch, loader) for measurements, and ``pdl`` to opt into
-    programmatic dependent launch (see q4.h); by default the table decides.
-    Argument marshalling only: the per-call work on the host is a few
-    dictionary lookups and one C call."""
+    ``bias`` (N values of A's dtype) is added in the epilogue before the
+    rounding (q4_gemm_skinny_bias).  ``launch`` may hold launch-table
+    overrides (math, warps, ctas, depth, l2_prefetch, loader) for
+    measurements, and ``pdl`` to opt into programmatic dependent launch (see
+    q4.h); by default the table decides.  Argument marshalling only: the
+    per-call work on the host is a few dictionary lookups and one C call."""
     M = A.shape[0] if A.dim() == 2 else 1
     if out is None:
         out = torch.empty((M, N), dtype=A.dtype, device=A.device)
@@ -219,9 +222,16 @@ def q4_gemm_skinny(A: torch.Tensor, Wpacked: torch.Tensor, absmax: torch.Tensor,
     stream = torch.cuda.current_stream(A.device).cuda_stream
     ws = (workspace or _default_workspace(A.device, stream)).get(nbytes) if nbytes else None
     ov_ref = _overrides_ref(tuple(sorted(launch.items())))[1] if launch else None
-    rc = lib().q4_gemm_skinny_ex(A.data_ptr(), Wpacked.data_ptr(), absmax.data_ptr(), code.data_ptr(), M, N, K,
-                                 blocksize, act, out.data_ptr(), ws.data_ptr() if ws is not None else None,
-                                 ws.numel() if ws is not None else 0, stream, ov_ref)
+    if bias is None:
+        rc = lib().q4_gemm_skinny_ex(A.data_ptr(), Wpacked.data_ptr(), absmax.data_ptr(), code.data_ptr(), M, N, K,
+                                     blocksize, act, out.data_ptr(), ws.data_ptr() if ws is not None else None,
+                                     ws.numel() if ws is not None else 0, stream, ov_ref)
+    else:
+        assert bias.dtype == A.dtype and bias.numel() == N and bias.is_contiguous()
+        rc = lib().q4_gemm_skinny_bias(A.data_ptr(), Wpacked.data_ptr(), absmax.data_ptr(), code.data_ptr(),
+                                       bias.data_ptr(), M, N, K, blocksize, act, out.data_ptr(),
+                                       ws.data_ptr() if ws is not None else None,
+                                       ws.numel() if ws is not None else 0, stream, ov_ref)
     _check(rc, "q4_gemm_skinny")
     return out
 

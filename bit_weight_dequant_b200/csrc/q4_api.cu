@@ -224,9 +224,10 @@ int q4_gemm_workspace_size(int M, int N, int K, int blocksize, int act_dtype, si
     return gemm_choose(M, N, K, blocksize, act_dtype, 0, nullptr, &ch, &tiles, &units, bytes, &sms);
 }
 
-int q4_gemm_skinny_ex(const void* A, const uint8_t* Wpacked, const float* absmax, const float* code, int M, int N,
-                      int K, int blocksize, int act_dtype, void* out, void* workspace, size_t workspace_bytes,
-                      void* stream, const q4_gemm_plan_t* overrides) {
+// The fused GEMM behind every entry point; `bias` may be nullptr.
+static int gemm_entry(const void* A, const uint8_t* Wpacked, const float* absmax, const float* code, const void* bias,
+                      int M, int N, int K, int blocksize, int act_dtype, void* out, void* workspace,
+                      size_t workspace_bytes, void* stream, const q4_gemm_plan_t* overrides) {
     // Pointers to empty arrays may be NULL; everything else must be given.
     if (M > 0 && N > 0 && (!out || (K > 0 && (!A || !Wpacked || !absmax || !code)))) return Q4_ERR_INVALID_ARG;
     GemmChoice ch;
@@ -237,7 +238,8 @@ int q4_gemm_skinny_ex(const void* A, const uint8_t* Wpacked, const float* absmax
     if (rc != Q4_OK) return rc;
     if (M == 0 || N == 0) return Q4_OK;
     if (!aligned(out, 16) || (K > 0 && (!aligned(A, 16) || !aligned(Wpacked, 16) || !aligned(absmax, 4) ||
-                                         !aligned(code, 4))))
+                                         !aligned(code, 4))) ||
+        (bias && !aligned(bias, 2)))
         return Q4_ERR_MISALIGNED;
     if (need > 0 && (!workspace || workspace_bytes < need)) return Q4_ERR_WORKSPACE;
     if (workspace && !aligned(workspace, 16)) return Q4_ERR_MISALIGNED;
@@ -254,14 +256,22 @@ int q4_gemm_skinny_ex(const void* A, const uint8_t* Wpacked, const float* absmax
     }
     if (injected_failure()) return Q4_ERR_CUDA;
     cudaStream_t st = (cudaStream_t)stream;
-    if (K == 0)  // empty contraction: all-zero output (0x0000 is +0 in bf16 and fp16)
-        return from_cuda(cudaMemsetAsync(out, 0, (size_t)M * N * 2, st));
+    if (K == 0) {  // empty contraction: every row is the bias, or +0 (0x0000 in bf16 and fp16)
+        if (!bias) return from_cuda(cudaMemsetAsync(out, 0, (size_t)M * N * 2, st));
+        for (int m = 0; m < M; ++m) {
+            cudaError_t e = cudaMemcpyAsync(static_cast<char*>(out) + (size_t)m * N * 2, bias, (size_t)N * 2,
+                                            cudaMemcpyDeviceToDevice, st);
+            if (e != cudaSuccess) return from_cuda(e);
+        }
+        return Q4_OK;
+    }
     GemmParams p{};
     p.A = A;
     p.Wp = Wpacked;
     p.absmax = absmax;
     p.code = code;
     p.out = out;
+    p.bias = bias;
     p.error = static_cast<int*>(workspace);
     p.partials = workspace ? reinterpret_cast<float*>(static_cast<char*>(workspace) + kWsHeader) : nullptr;
     p.counters = workspace ? reinterpret_cast<int*>(static_cast<char*>(workspace) + ws_counter_offset(sms)) : nullptr;
@@ -280,11 +290,26 @@ int q4_gemm_skinny_ex(const void* A, const uint8_t* Wpacked, const float* absmax
     return from_cuda(gemm_launch(ch, act_dtype, p, st));
 }
 
+int q4_gemm_skinny_ex(const void* A, const uint8_t* Wpacked, const float* absmax, const float* code, int M, int N,
+                      int K, int blocksize, int act_dtype, void* out, void* workspace, size_t workspace_bytes,
+                      void* stream, const q4_gemm_plan_t* overrides) {
+    return gemm_entry(A, Wpacked, absmax, code, nullptr, M, N, K, blocksize, act_dtype, out, workspace,
+                      workspace_bytes, stream, overrides);
+}
+
 int q4_gemm_skinny(const void* A, const uint8_t* Wpacked, const float* absmax, const float* code, int M, int N,
                    int K, int blocksize, int act_dtype, void* out, void* workspace, size_t workspace_bytes,
                    void* stream) {
-    return q4_gemm_skinny_ex(A, Wpacked, absmax, code, M, N, K, blocksize, act_dtype, out, workspace,
-                             workspace_bytes, stream, nullptr);
+    return gemm_entry(A, Wpacked, absmax, code, nullptr, M, N, K, blocksize, act_dtype, out, workspace,
+                      workspace_bytes, stream, nullptr);
+}
+
+int q4_gemm_skinny_bias(const void* A, const uint8_t* Wpacked, const float* absmax, const float* code,
+                        const void* bias, int M, int N, int K, int blocksize, int act_dtype, void* out,
+                        void* workspace, size_t workspace_bytes, void* stream, const q4_gemm_plan_t* overrides) {
+    if (M > 0 && N > 0 && !bias) return Q4_ERR_INVALID_ARG;
+    return gemm_entry(A, Wpacked, absmax, code, bias, M, N, K, blocksize, act_dtype, out, workspace,
+                      workspace_bytes, stream, overrides);
 }
 
 // The exported partition functions compute with 64-bit integers; the kernels

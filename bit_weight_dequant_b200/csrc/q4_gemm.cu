@@ -148,6 +148,7 @@ template <typename T, class S>
 __device__ __forceinline__ void store_tile(const float (&v)[S::TW][S::NJ][4], const GemmParams& p, int tile, int g,
                                            int tq) {
     T* out = static_cast<T*>(p.out);
+    const T* bias = static_cast<const T*>(p.bias);
 #pragma unroll
     for (int i = 0; i < S::TW; ++i)
 #pragma unroll
@@ -156,7 +157,10 @@ __device__ __forceinline__ void store_tile(const float (&v)[S::TW][S::NJ][4], co
             for (int r = 0; r < 4; ++r) {
                 const int n = tile * S::TR + 16 * i + g + ((r & 2) ? 8 : 0);
                 const int m = 8 * j + 2 * tq + (r & 1);
-                if (n < p.N && m < p.M) out[(size_t)m * p.N + n] = Act<T>::from_float(v[i][j][r]);
+                if (n < p.N && m < p.M) {
+                    const float b = bias ? static_cast<float>(bias[n]) : 0.f;  // exact widening
+                    out[(size_t)m * p.N + n] = Act<T>::from_float(v[i][j][r] + b);
+                }
             }
 }
 

@@ -68,6 +68,7 @@ struct GemmParams {
     const float* absmax;
     const float* code;
     void* out;
+    const void* bias;  // [N] activation type, or nullptr: added in fp32 before the rounding
     float* partials;   // [ctas][2][SLOT_FLOATS]
     int* counters;     // [tiles], zero between calls
     int* error;        // workspace error word (0 = ok); set when a bounded wait gives up

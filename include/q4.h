@@ -207,6 +207,21 @@ int q4_gemm_skinny_ex(const void* A, const uint8_t* Wpacked, const float* absmax
                       const q4_gemm_plan_t* overrides);
 
 /*
+ * The layer with a bias, fused into the epilogue (the planned gemm_4bit op of
+ * bitsandbytes PR #1920, "Technical details", takes an optional bias):
+ *     out[m, n] = round_rn_act( bias[n] + sum_k A[m,k] * dequant(W)[n,k] )
+ * the bias added in fp32 to the fp32 sum before the single rounding.
+ *   bias       [N] act_dtype, 2-byte aligned, not NULL when M, N > 0 (use
+ *              q4_gemm_skinny for no bias); with K = 0 every output row is
+ *              the bias.
+ *   overrides  as for q4_gemm_skinny_ex (NULL: the launch table decides).
+ * Every other argument, result and error as q4_gemm_skinny.
+ */
+int q4_gemm_skinny_bias(const void* A, const uint8_t* Wpacked, const float* absmax, const float* code,
+                        const void* bias, int M, int N, int K, int blocksize, int act_dtype, void* out,
+                        void* workspace, size_t workspace_bytes, void* stream, const q4_gemm_plan_t* overrides);
+
+/*
  * Work partition used by the GEMM (host-callable so it can be checked
  * without a GPU): `total` units split into `parts` contiguous ranges,
  * part p owning [q4_partition_start(total, parts, p),

@@ -76,6 +76,9 @@ def test_gemm_validation_before_cuda():
     for (M, N, K, bs, dt), want in cases.items():
         assert g(*args, M, N, K, bs, dt, ALIGNED, None, 0, None) == want, (M, N, K, bs, dt)
     assert g(None, *args[1:], 1, 64, 4096, 64, 0, ALIGNED, None, 0, None) == b.Q4_ERR_INVALID_ARG
+    bias = b.lib().q4_gemm_skinny_bias
+    assert bias(*args, None, 1, 64, 4096, 64, 0, ALIGNED, None, 0, None, None) == b.Q4_ERR_INVALID_ARG  # no bias
+    assert bias(*args, ALIGNED, 17, 64, 4096, 64, 0, ALIGNED, None, 0, None, None) == b.Q4_ERR_UNSUPPORTED
     ex = b.lib().q4_gemm_skinny_ex
     assert ex(*args, 1, 64, 4096, 64, 0, ALIGNED, None, 0, None, b.overrides(math=3)) == b.Q4_ERR_INVALID_ARG
     assert ex(*args, 12, 64, 4096, 64, 0, ALIGNED, None, 0, None, b.overrides(warps=16)) == b.Q4_ERR_UNSUPPORTED
