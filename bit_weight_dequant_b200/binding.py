@@ -53,6 +53,7 @@ def lib() -> ctypes.CDLL:
         L.q4_status_string.argtypes = [ci]
         L.q4_status_string.restype = ctypes.c_char_p
         L.q4_quantize_blockwise.argtypes = [P, i64, ci, P, P, P, P]
+        L.q4_quantize_blockwise_ex.argtypes = [P, ci, i64, ci, P, P, P, P]
         L.q4_dequantize_blockwise.argtypes = [P, P, P, i64, ci, ci, P, P]
         L.q4_gemm_workspace_size.argtypes = [ci, ci, ci, ci, ci, ctypes.POINTER(sz)]
         L.q4_gemm_skinny.argtypes = [P, P, P, P, ci, ci, ci, ci, ci, P, P, sz, P]
@@ -64,7 +65,7 @@ def lib() -> ctypes.CDLL:
         L.q4_partition_start.argtypes = [i64, ci, ci]
         L.q4_partition_start.restype = i64
         L.q4_partition_owner.argtypes = [i64, ci, i64]
-        for f in ("q4_quantize_blockwise", "q4_dequantize_blockwise", "q4_gemm_workspace_size",
+        for f in ("q4_quantize_blockwise", "q4_quantize_blockwise_ex", "q4_dequantize_blockwise", "q4_gemm_workspace_size",
                   "q4_gemm_skinny", "q4_gemm_skinny_ex", "q4_gemm_plan", "q4_partition_owner",
                   "q4_gemm_skinny_noalloc", "q4_gemm_skinny_bias"):
             getattr(L, f).restype = ci
@@ -98,13 +99,13 @@ def _stream(device) -> int:
 
 
 def q4_quantize_blockwise(W: torch.Tensor, blocksize: int, code: torch.Tensor):
-    """Quantize a CUDA fp32 tensor blockwise; returns (packed uint8, absmax fp32)."""
-    assert W.is_cuda and W.dtype == torch.float32 and W.is_contiguous()
+    """Quantize a CUDA fp32, bf16 or fp16 tensor blockwise; returns (packed uint8, absmax fp32)."""
+    assert W.is_cuda and W.dtype in _TORCH_TO_Q4 and W.is_contiguous()
     n = W.numel()
     packed = torch.empty((n + 1) // 2, dtype=torch.uint8, device=W.device)
     absmax = torch.empty((n + blocksize - 1) // blocksize, dtype=torch.float32, device=W.device)
-    rc = lib().q4_quantize_blockwise(_ptr(W), n, blocksize, _ptr(code), _ptr(packed), _ptr(absmax),
-                                     _stream(W.device))
+    rc = lib().q4_quantize_blockwise_ex(_ptr(W), _TORCH_TO_Q4[W.dtype], n, blocksize, _ptr(code), _ptr(packed),
+                                        _ptr(absmax), _stream(W.device))
     _check(rc, "q4_quantize_blockwise")
     return packed, absmax
 

@@ -169,14 +169,20 @@ const char* q4_status_string(int status) {
     }
 }
 
-int q4_quantize_blockwise(const float* W, int64_t n, int blocksize, const float* code, uint8_t* packed,
-                          float* absmax, void* stream) {
+int q4_quantize_blockwise_ex(const void* W, int w_dtype, int64_t n, int blocksize, const float* code,
+                             uint8_t* packed, float* absmax, void* stream) {
     if (n < 0 || !is_pow2_blocksize(blocksize)) return Q4_ERR_INVALID_ARG;
+    if (w_dtype != Q4_BF16 && w_dtype != Q4_FP16 && w_dtype != Q4_FP32) return Q4_ERR_INVALID_ARG;
     if (n == 0) return Q4_OK;  // empty input: pointers may be NULL
     if (!W || !code || !packed || !absmax) return Q4_ERR_INVALID_ARG;
     if (!aligned(W, 16) || !aligned(code, 4) || !aligned(absmax, 4)) return Q4_ERR_MISALIGNED;
     if (injected_failure()) return Q4_ERR_CUDA;
-    return from_cuda(quantize_launch(W, n, blocksize, code, packed, absmax, (cudaStream_t)stream));
+    return from_cuda(quantize_launch(W, w_dtype, n, blocksize, code, packed, absmax, (cudaStream_t)stream));
+}
+
+int q4_quantize_blockwise(const float* W, int64_t n, int blocksize, const float* code, uint8_t* packed,
+                          float* absmax, void* stream) {
+    return q4_quantize_blockwise_ex(W, Q4_FP32, n, blocksize, code, packed, absmax, stream);
 }
 
 int q4_dequantize_blockwise(const uint8_t* packed, const float* absmax, const float* code, int64_t n,

@@ -32,8 +32,8 @@ bool gemm_variant_exists(int act_dtype, const GemmChoice& ch);
 size_t gemm_smem_bytes(int act_dtype, const GemmChoice& ch);
 size_t gemm_slot_floats(int m_pad);
 
-cudaError_t quantize_launch(const float* W, int64_t n, int blocksize, const float* code, uint8_t* packed,
-                            float* absmax, cudaStream_t stream);
+cudaError_t quantize_launch(const void* W, int w_dtype, int64_t n, int blocksize, const float* code,
+                            uint8_t* packed, float* absmax, cudaStream_t stream);
 cudaError_t dequantize_launch(const uint8_t* packed, const float* absmax, const float* code, int64_t n,
                               int blocksize, int out_dtype, void* out, cudaStream_t stream);
 

@@ -6,6 +6,8 @@
 // kernel reads.  Both are memory-bound streams; both must match the
 // definition exactly (codes and absmax equal, dequantized values bit-equal),
 // so every floating-point step is an explicitly rounded intrinsic.
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
 #include "q4_device.cuh"
@@ -29,50 +31,132 @@ __device__ __forceinline__ int nearest_code(float x, const float (&c)[16]) {
     return best;
 }
 
-// One warp per block of `bs` elements (grid-stride over blocks).  Pairs of
-// elements map to one output byte (even element -> high nibble); blocks
-// start at even indices because bs is even, so pairs never straddle blocks.
-__global__ void __launch_bounds__(256) q4_quantize_kernel(const float* __restrict__ W, int64_t n, int bs_shift,
+// Weights arrive as fp32, bf16 or fp16; every element is widened to fp32
+// exactly, so the quantizer's arithmetic (and result) does not depend on the
+// input type.
+template <typename TW>
+struct WeightIn;
+template <>
+struct WeightIn<float> {
+    __device__ __forceinline__ static float get(const float* p, int64_t i) { return __ldg(p + i); }
+    // 16 consecutive elements from a 16-byte aligned address
+    __device__ __forceinline__ static void get16(const float* p, float (&f)[16]) {
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+            const uint4 u = ldg_stream_v4(p + 4 * v);
+            f[4 * v] = __uint_as_float(u.x);
+            f[4 * v + 1] = __uint_as_float(u.y);
+            f[4 * v + 2] = __uint_as_float(u.z);
+            f[4 * v + 3] = __uint_as_float(u.w);
+        }
+    }
+};
+template <typename H, float (*TO_F)(H)>
+struct WeightIn16 {
+    __device__ __forceinline__ static float get(const H* p, int64_t i) {
+        const unsigned short b = __ldg(reinterpret_cast<const unsigned short*>(p) + i);
+        return TO_F(*reinterpret_cast<const H*>(&b));
+    }
+    __device__ __forceinline__ static void get16(const H* p, float (&f)[16]) {
+#pragma unroll
+        for (int v = 0; v < 2; ++v) {
+            const uint4 u = ldg_stream_v4(p + 8 * v);
+            const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const unsigned short lo = (unsigned short)(w[k] & 0xFFFFu), hi = (unsigned short)(w[k] >> 16);
+                f[8 * v + 2 * k] = TO_F(*reinterpret_cast<const H*>(&lo));
+                f[8 * v + 2 * k + 1] = TO_F(*reinterpret_cast<const H*>(&hi));
+            }
+        }
+    }
+};
+__device__ __forceinline__ float bf16_to_f(__nv_bfloat16 v) { return __bfloat162float(v); }
+__device__ __forceinline__ float f16_to_f(__half v) { return __half2float(v); }
+template <>
+struct WeightIn<__nv_bfloat16> : WeightIn16<__nv_bfloat16, bf16_to_f> {};
+template <>
+struct WeightIn<__half> : WeightIn16<__half, f16_to_f> {};
+
+// One warp per block of `bs` elements (grid-stride over the blocks from
+// `b0`).  Pairs of elements map to one output byte (even element -> high
+// nibble); blocks start at even indices because bs is even, so pairs never
+// straddle blocks.  Serves any blocksize and the ragged end of the input.
+template <typename TW>
+__device__ __forceinline__ void quantize_blocks_per_warp(const TW* __restrict__ W, int64_t n, int bs_shift,
+                                                         const float (&c)[16], uint8_t* __restrict__ packed,
+                                                         float* __restrict__ absmax, int64_t b0, int64_t nblocks) {
+    const int lane = threadIdx.x & 31;
+    const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+    for (int64_t b = b0 + (((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5); b < nblocks; b += nwarps) {
+        const int64_t lo = b << bs_shift;
+        const int64_t rem = n - lo;
+        const int cnt = rem < ((int64_t)1 << bs_shift) ? (int)rem : (1 << bs_shift);
+        const TW* wb = W + lo;
+        float amax = 0.f;
+        for (int i = lane; i < cnt; i += 32) amax = fmaxf(amax, fabsf(WeightIn<TW>::get(wb, i)));
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+        if (lane == 0) absmax[b] = amax;
+        for (int p = lane; 2 * p < cnt; p += 32) {
+            const bool has1 = 2 * p + 1 < cnt;
+            const float w0 = WeightIn<TW>::get(wb, 2 * p);
+            const float w1 = has1 ? WeightIn<TW>::get(wb, 2 * p + 1) : 0.f;
+            const int i0 = nearest_code(amax > 0.f ? __fdiv_rn(w0, amax) : 0.f, c);
+            const int i1 = has1 ? nearest_code(amax > 0.f ? __fdiv_rn(w1, amax) : 0.f, c) : 0;
+            packed[(lo >> 1) + p] = (uint8_t)((i0 << 4) | i1);
+        }
+    }
+}
+
+template <typename TW>
+__global__ void __launch_bounds__(256) q4_quantize_kernel(const TW* __restrict__ W, int64_t n, int bs_shift,
                                                           const float* __restrict__ code,
                                                           uint8_t* __restrict__ packed,
                                                           float* __restrict__ absmax, int64_t nblocks) {
     float c[16];
 #pragma unroll
     for (int j = 0; j < 16; ++j) c[j] = __ldg(code + j);
-    const int lane = threadIdx.x & 31;
-    const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
-    for (int64_t b = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; b < nblocks; b += nwarps) {
-        const int64_t lo = b << bs_shift;
-        const int64_t rem = n - lo;
-        const int cnt = rem < ((int64_t)1 << bs_shift) ? (int)rem : (1 << bs_shift);
-        const float* wb = W + lo;
-        float amax = 0.f;
-        for (int p = lane; 2 * p < cnt; p += 32) {
-            if (2 * p + 1 < cnt) {
-                const float2 v = __ldg(reinterpret_cast<const float2*>(wb) + p);
-                amax = fmaxf(amax, fmaxf(fabsf(v.x), fabsf(v.y)));
-            } else {
-                amax = fmaxf(amax, fabsf(__ldg(wb + 2 * p)));
-            }
-        }
+    quantize_blocks_per_warp<TW>(W, n, bs_shift, c, packed, absmax, 0, nblocks);
+}
+
+// Blocksizes 32..512: a warp takes 512-element chunks, each lane 16
+// consecutive elements (vector loads, one 8-byte packed store; a warp writes
+// 256 contiguous bytes).  The bs/16 lanes of a block reduce its absmax with
+// shuffles; 16 independent elements per lane keep the division and the
+// 16-way search in flight.  Elements after the last whole chunk (whole blocks,
+// since 512 is a multiple of bs) go through the per-warp form.
+template <typename TW>
+__global__ void __launch_bounds__(256) q4_quantize_lanes_kernel(const TW* __restrict__ W, int64_t n, int bs_shift,
+                                                                const float* __restrict__ code,
+                                                                uint8_t* __restrict__ packed,
+                                                                float* __restrict__ absmax, int64_t nblocks) {
+    float c[16];
 #pragma unroll
-        for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
-        if (lane == 0) absmax[b] = amax;
-        for (int p = lane; 2 * p < cnt; p += 32) {
-            float w0, w1 = 0.f;
-            const bool has1 = 2 * p + 1 < cnt;
-            if (has1) {
-                const float2 v = __ldg(reinterpret_cast<const float2*>(wb) + p);
-                w0 = v.x;
-                w1 = v.y;
-            } else {
-                w0 = __ldg(wb + 2 * p);
-            }
-            const int i0 = nearest_code(amax > 0.f ? __fdiv_rn(w0, amax) : 0.f, c);
-            const int i1 = has1 ? nearest_code(amax > 0.f ? __fdiv_rn(w1, amax) : 0.f, c) : 0;
-            packed[(lo >> 1) + p] = (uint8_t)((i0 << 4) | i1);
+    for (int j = 0; j < 16; ++j) c[j] = __ldg(code + j);
+    const int lane = threadIdx.x & 31;
+    const int group = 1 << (bs_shift - 4);  // lanes per block: 2 .. 32
+    const int64_t nchunks = n >> 9;
+    const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+    for (int64_t q = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; q < nchunks; q += nwarps) {
+        const int64_t e0 = (q << 9) + 16 * lane;
+        float f[16];
+        WeightIn<TW>::get16(W + e0, f);
+        float amax = 0.f;
+#pragma unroll
+        for (int e = 0; e < 16; ++e) amax = fmaxf(amax, fabsf(f[e]));
+        for (int off = 1; off < group; off <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+        if ((lane & (group - 1)) == 0) absmax[e0 >> bs_shift] = amax;
+        uint32_t word[2] = {0u, 0u};
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+            const uint32_t idx = (uint32_t)nearest_code(amax > 0.f ? __fdiv_rn(f[e], amax) : 0.f, c);
+            // byte e/2 of the lane's 8 output bytes; even element in the high nibble
+            word[e >> 3] |= idx << (8 * ((e >> 1) & 3) + ((e & 1) ? 0 : 4));
         }
+        *reinterpret_cast<uint2*>(packed + (e0 >> 1)) = make_uint2(word[0], word[1]);
     }
+    quantize_blocks_per_warp<TW>(W, n, bs_shift, c, packed, absmax, (nchunks << 9) >> bs_shift, nblocks);
 }
 
 template <int OUT>
@@ -210,12 +294,33 @@ static int grid_for(int64_t work_items, int threads, int per_sm) {
     return (int)blocks;
 }
 
-cudaError_t quantize_launch(const float* W, int64_t n, int blocksize, const float* code, uint8_t* packed,
-                            float* absmax, cudaStream_t stream) {
+cudaError_t quantize_launch(const void* W, int w_dtype, int64_t n, int blocksize, const float* code,
+                            uint8_t* packed, float* absmax, cudaStream_t stream) {
     const int64_t nblocks = (n + blocksize - 1) / blocksize;
     const int threads = 256;
-    const int grid = grid_for(nblocks * 32, threads, 8);
-    q4_quantize_kernel<<<grid, threads, 0, stream>>>(W, n, log2_exact(blocksize), code, packed, absmax, nblocks);
+    const int sh = log2_exact(blocksize);
+    // The lane-per-16-elements form needs bs <= 512 and an 8-byte aligned
+    // packed array (its stores are 8 bytes wide).
+    const bool lanes = blocksize <= 512 && (reinterpret_cast<uintptr_t>(packed) & 7u) == 0;
+    // one warp per 512-element chunk (plus the tail's blocks), or per block
+    const int64_t warps = lanes ? (n >> 9) + (512 >> sh) : nblocks;
+    const int grid = grid_for(warps * 32, threads, 8);
+#define Q4_QUANT(TW)                                                                                              \
+    do {                                                                                                          \
+        if (lanes)                                                                                                \
+            q4_quantize_lanes_kernel<TW><<<grid, threads, 0, stream>>>(static_cast<const TW*>(W), n, sh, code,  \
+                                                                       packed, absmax, nblocks);                 \
+        else                                                                                                      \
+            q4_quantize_kernel<TW><<<grid, threads, 0, stream>>>(static_cast<const TW*>(W), n, sh, code, packed, \
+                                                                 absmax, nblocks);                               \
+    } while (0)
+    if (w_dtype == 0)
+        Q4_QUANT(__nv_bfloat16);
+    else if (w_dtype == 1)
+        Q4_QUANT(__half);
+    else
+        Q4_QUANT(float);
+#undef Q4_QUANT
     return cudaGetLastError();
 }
 

@@ -85,6 +85,16 @@ int q4_quantize_blockwise(const float* W, int64_t n, int blocksize, const float*
                           uint8_t* packed, float* absmax, void* stream);
 
 /*
+ * The same quantization with the weights given as bf16, fp16 or fp32
+ * (w_dtype: Q4_BF16, Q4_FP16, Q4_FP32; anything else -> Q4_ERR_INVALID_ARG).
+ * Each element is widened to fp32 exactly, so the result equals
+ * q4_quantize_blockwise on the widened values.  W is 16-byte aligned; every
+ * other argument as above.
+ */
+int q4_quantize_blockwise_ex(const void* W, int w_dtype, int64_t n, int blocksize, const float* code,
+                             uint8_t* packed, float* absmax, void* stream);
+
+/*
  * Blockwise 4-bit dequantization (the building block of the split path of
  * PR #1920, "split dequantize + GEMM").
  *   packed  uint8 [ceil(n/2)], 16-byte aligned

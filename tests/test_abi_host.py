@@ -42,6 +42,10 @@ def test_quantize_validation():
         assert q(ALIGNED, 16, bs, ALIGNED, ALIGNED, ALIGNED, None) == b.Q4_ERR_INVALID_ARG
     assert q(MISALIGNED, 16, 64, ALIGNED, ALIGNED, ALIGNED, None) == b.Q4_ERR_MISALIGNED
     assert q(ALIGNED, 0, 64, ALIGNED, ALIGNED, ALIGNED, None) == b.Q4_OK   # empty input: no-op
+    qx = L.q4_quantize_blockwise_ex
+    assert qx(ALIGNED, 7, 16, 64, ALIGNED, ALIGNED, ALIGNED, None) == b.Q4_ERR_INVALID_ARG   # unknown weight type
+    assert qx(MISALIGNED, b.Q4_BF16, 16, 64, ALIGNED, ALIGNED, ALIGNED, None) == b.Q4_ERR_MISALIGNED
+    assert qx(ALIGNED, b.Q4_FP16, 0, 64, ALIGNED, ALIGNED, ALIGNED, None) == b.Q4_OK
 
 
 def test_dequantize_validation():

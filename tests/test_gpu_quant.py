@@ -98,3 +98,34 @@ def test_misaligned_pointer_rejected(cuda_device):
     with pytest.raises(q4.Q4Error) as e:
         q4.q4_quantize_blockwise(w, 64, cd)
     assert e.value.status == q4.Q4_ERR_MISALIGNED
+
+
+@pytest.mark.parametrize("wdt", [torch.bfloat16, torch.float16])
+@pytest.mark.parametrize("n,bs", [(4097, 64), (100003, 128), (65536 * 3 + 5, 512), (12345, 4096), (1 << 20, 32)])
+def test_quantize_16bit_weights_bit_exact(cuda_device, wdt, n, bs):
+    """bf16 / fp16 weights: the result equals the oracle on the exactly widened fp32 values."""
+    code = inputs.code_normal_quantile()
+    w16 = torch.from_numpy(_weights(n, bs, n + bs, True)).to(wdt)
+    p_ref, a_ref = oracle.quantize(w16.float().numpy(), bs, code)
+    p, a = q4.q4_quantize_blockwise(w16.to(cuda_device), bs, torch.from_numpy(code).to(cuda_device))
+    assert np.array_equal(p.cpu().numpy(), p_ref)
+    assert np.array_equal(a.cpu().numpy().view(np.uint32), a_ref.view(np.uint32))
+
+
+@pytest.mark.parametrize("bs", [64, 256])
+def test_quantize_unaligned_packed_output(cuda_device, bs):
+    """A packed array that is not 8-byte aligned takes the per-warp form; same bytes."""
+    n = 3 * 4096 + 96
+    code = inputs.code_uniform()
+    w = _weights(n, bs, 5, False)
+    p_ref, a_ref = oracle.quantize(w, bs, code)
+    raw = torch.zeros((n + 1) // 2 + 16, dtype=torch.uint8, device=cuda_device)
+    packed = raw[3:3 + (n + 1) // 2]
+    absmax = torch.zeros((n + bs - 1) // bs, dtype=torch.float32, device=cuda_device)
+    wd, cd = torch.from_numpy(w).to(cuda_device), torch.from_numpy(code).to(cuda_device)
+    rc = q4.lib().q4_quantize_blockwise(wd.data_ptr(), n, bs, cd.data_ptr(), packed.data_ptr(), absmax.data_ptr(),
+                                        torch.cuda.current_stream().cuda_stream)
+    assert rc == q4.Q4_OK
+    assert np.array_equal(packed.cpu().numpy(), p_ref)
+    assert np.array_equal(absmax.cpu().numpy(), a_ref)
+    assert int(raw[:3].count_nonzero()) == 0 and int(raw[3 + (n + 1) // 2:].count_nonzero()) == 0
