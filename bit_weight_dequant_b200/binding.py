@@ -144,12 +144,18 @@ def q4_gemm_plan(M: int, N: int, K: int, blocksize: int, act_dtype: torch.dtype 
 class Workspace:
     """Zero-filled device scratch for q4_gemm_skinny, grown on demand.
 
-    Every call returns the workspace's tile counters to zero, so it is
-    zero-filled once, at allocation; one per stream."""
+    Every successful call returns the workspace's tile counters (and the
+    tensor-memory kernel's partial slots) to zero, so it is zero-filled once,
+    at allocation, and again by ``reset()`` after a call that set the error
+    word; one per stream."""
 
     def __init__(self, device):
         self.device = torch.device(device)
         self.buf = torch.zeros(0, dtype=torch.uint8, device=self.device)
+
+    def reset(self):
+        """Zero the whole workspace (needed after a call that set the error word)."""
+        self.buf.zero_()
 
     def get(self, nbytes: int) -> torch.Tensor:
         if self.buf.numel() < nbytes:

@@ -87,9 +87,43 @@ static int gemm_choose(int M, int N, int K, int blocksize, int act_dtype, int nu
     if (M < 0 || N < 0 || K < 0) return Q4_ERR_INVALID_ARG;
     if (!is_pow2_blocksize(blocksize)) return Q4_ERR_INVALID_ARG;
     if (act_dtype != Q4_BF16 && act_dtype != Q4_FP16 && act_dtype != Q4_FP32) return Q4_ERR_INVALID_ARG;
-    if (ov && (ov->math > 2 || ov->l2_prefetch > 256 || ov->loader > 5 || ov->pdl > 2)) return Q4_ERR_INVALID_ARG;
-    if (M > 16 || act_dtype == Q4_FP32 || K % blocksize != 0) return Q4_ERR_UNSUPPORTED;
+    if (ov && (ov->math > 3 || ov->l2_prefetch > 256 || ov->loader > 6 || ov->pdl > 2)) return Q4_ERR_INVALID_ARG;
+    if (M > 128 || act_dtype == Q4_FP32 || K % blocksize != 0) return Q4_ERR_UNSUPPORTED;
     GemmChoice c{};
+    if (M > 16 || (ov && (ov->math == 3 || ov->loader == 6))) {
+        // Tensor-memory kernel (tcgen05): 128-row tiles, 64-k units, 4-unit
+        // stages whose absmax box is 4 floats per row.
+        if (blocksize < 64 || K % 256 != 0 || (K / blocksize) % 4 != 0) return Q4_ERR_UNSUPPORTED;
+        c.math = 3;
+        c.sub_block = 64;
+        c.m_pad = M <= 32 ? 32 : M <= 64 ? 64 : 128;
+        c.rows_per_tile = 128;
+        c.loader = 6;
+        c.warps = 6;
+        c.depth = 0;  // stages: as many as shared memory holds (set at launch)
+        c.l2pf = 0;
+        c.pdl = (ov && ov->pdl > 0) ? 1 : 0;  // activations and weights are read after the dependency wait
+        const int64_t t64 = N > 0 ? ((int64_t)N + 127) / 128 : 0;
+        if (t64 * (K / 64) >= (int64_t)kMaxUnits) return Q4_ERR_UNSUPPORTED;
+        int sms = num_sms;
+        if (sms <= 0 && device_sm_count(&sms) != 0) return Q4_ERR_CUDA;
+        if (ov && ov->ctas > sms) return Q4_ERR_INVALID_ARG;
+        const int t = (int)t64;
+        const int64_t u = t64 * (K / 64);
+        int64_t g = (ov && ov->ctas > 0) ? ov->ctas : sms;
+        if (g > u) g = u;
+        if (g < 1) g = 1;
+        c.ctas = (int)g;
+        *ch = c;
+        *tiles = t;
+        *units = u;
+        *sms_out = sms;
+        // counters at the fixed offset, then two partial slots (m_pad x 128 fp32) per CTA
+        *ws_bytes = u > 1 ? ws_counter_offset(sms) + align_up((size_t)t * sizeof(int), 256) +
+                                (size_t)c.ctas * 2 * umma_slot_bytes(c.m_pad)
+                          : 0;
+        return Q4_OK;
+    }
     c.math = 1;
     c.sub_block = blocksize < 64 ? blocksize : 64;
     c.m_pad = M <= 8 ? 8 : 16;
@@ -249,7 +283,8 @@ static int gemm_entry(const void* A, const uint8_t* Wpacked, const float* absmax
         return Q4_ERR_MISALIGNED;
     if (need > 0 && (!workspace || workspace_bytes < need)) return Q4_ERR_WORKSPACE;
     if (workspace && !aligned(workspace, 16)) return Q4_ERR_MISALIGNED;
-    if (ch.loader >= 2 && !aligned(absmax, 16)) {  // the tensor map needs a 16-byte aligned base
+    if (ch.math == 3 && !aligned(absmax, 16)) return Q4_ERR_MISALIGNED;  // tensor-map base
+    if (ch.math != 3 && ch.loader >= 2 && !aligned(absmax, 16)) {  // the tensor map needs a 16-byte aligned base
         if (overrides && overrides->loader >= 2) return Q4_ERR_MISALIGNED;
         GemmChoice fb;
         q4_gemm_plan_t ov1{};
@@ -293,6 +328,16 @@ static int gemm_entry(const void* A, const uint8_t* Wpacked, const float* absmax
     p.tiles = tiles;
     p.ctas = ch.ctas;
     p.units = (uint32_t)units;
+    if (ch.math == 3) {
+        if (workspace)
+            p.partials = reinterpret_cast<float*>(static_cast<char*>(workspace) + ws_counter_offset(sms) +
+                                                  align_up((size_t)tiles * sizeof(int), 256));
+        int smem = 0, dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
+            return from_cuda(cudaGetLastError());
+        return from_cuda(umma_launch(act_dtype, ch.m_pad, p, smem, st));
+    }
     return from_cuda(gemm_launch(ch, act_dtype, p, st));
 }
 

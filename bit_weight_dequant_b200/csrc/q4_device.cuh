@@ -135,6 +135,10 @@ __device__ __forceinline__ void sts_v4(uint32_t addr, uint32_t a, uint32_t b, ui
     asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d));
 }
 
+__device__ __forceinline__ void sts_u32(uint32_t addr, uint32_t v) {
+    asm volatile("st.shared.b32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+
 __device__ __forceinline__ uint4 lds_v4(uint32_t addr) {
     uint4 v;
     asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
@@ -248,6 +252,18 @@ struct Act<__nv_bfloat16> {
         return *reinterpret_cast<uint32_t*>(&h);
     }
     __device__ __forceinline__ static __nv_bfloat16 from_float(float v) { return __float2bfloat16_rn(v); }
+};
+
+// Operand format code of a 16-bit type in a tcgen05 instruction descriptor.
+template <typename T>
+struct Act16Format;
+template <>
+struct Act16Format<__nv_bfloat16> {
+    static constexpr uint32_t value = 1;
+};
+template <>
+struct Act16Format<__half> {
+    static constexpr uint32_t value = 0;
 };
 
 template <>

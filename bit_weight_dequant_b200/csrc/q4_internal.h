@@ -12,7 +12,7 @@ namespace q4 {
 
 // One launch-table decision for the GEMM.
 struct GemmChoice {
-    int math;       // 1 = tensor-core MMA, 2 = CUDA-core FMA
+    int math;       // 1 = tensor-core mma.sync, 2 = CUDA-core FMA, 3 = tcgen05 with tensor memory
     int sub_block;  // 32 or 64
     int m_pad;      // 8 or 16
     int warps;      // warps per CTA
@@ -20,7 +20,7 @@ struct GemmChoice {
     int rows_per_tile;
     int depth;      // units (loader 1) or stages (loader 2) in flight per warp
     int l2pf;       // L2 fetch-size hint on weight loads: 0 (none), 128, 256 (loader 1)
-    int loader;     // 1 = per-lane global loads, 2/3 = TMA stage ring of 4/2-unit stages
+    int loader;     // 1 = per-lane global loads, 2/3 = TMA stage ring of 4/2-unit stages, 6 = tcgen05 kernel
     int pdl;        // programmatic dependent launch mode (0, 1, 2)
 };
 
@@ -31,6 +31,11 @@ cudaError_t gemm_launch(const GemmChoice& ch, int act_dtype, const GemmParams& p
 bool gemm_variant_exists(int act_dtype, const GemmChoice& ch);
 size_t gemm_smem_bytes(int act_dtype, const GemmChoice& ch);
 size_t gemm_slot_floats(int m_pad);
+
+// Tensor-memory (tcgen05) GEMM for 17 <= M <= 128 (q4_umma.cu).
+cudaError_t umma_launch(int act_dtype, int m_pad, const GemmParams& p, int smem_bytes, cudaStream_t stream);
+int umma_stages(int m_pad, int smem_bytes);
+size_t umma_slot_bytes(int m_pad);
 
 cudaError_t quantize_launch(const void* W, int w_dtype, int64_t n, int blocksize, const float* code,
                             uint8_t* packed, float* absmax, cudaStream_t stream);

@@ -205,6 +205,13 @@ def workloads() -> dict:
             ext.append(Case(M, N, K, tag=f"K{K}N{N}M{M}"))
     w["aspect"] = Workload("extreme aspect ratios at M=1..8: K2560/N248320, K320/N10240, K10240/N320, "
                            "K2560/N12", 4, ext)
+    # Beyond the five: the M sweep's shapes at 17 <= M <= 128 (the
+    # tensor-memory kernel), for parity and for the fused-vs-split crossover.
+    big = []
+    for (K, N) in ((5120, 5120), (5120, 8192), (17408, 5120)):
+        for M in (17, 32, 64, 128):
+            big.append(Case(M, N, K, tag=f"K{K}N{N}M{M}"))
+    w["mlarge"] = Workload("M 17,32,64,128 on K5120/N5120, K5120/N8192, K17408/N5120 (tcgen05 kernel)", 6, big)
     # Not one of the five: one long-K layer whose launch is almost all main
     # loop (start-up and tail are a few percent), for profiling the loop.
     w["longk"] = Workload("M=1 K=131072 N=8192 bs64 bf16 normal-table (main-loop profiling shape)", 5,

@@ -70,7 +70,7 @@ def test_gemm_validation_before_cuda():
     g = b.lib().q4_gemm_skinny
     args = [ALIGNED] * 4
     # (M, N, K, bs, dtype) -> status; all decided before the device is queried
-    cases = {(17, 64, 4096, 64, 0): b.Q4_ERR_UNSUPPORTED,
+    cases = {(129, 64, 4096, 64, 0): b.Q4_ERR_UNSUPPORTED,
              (1, 64, 4000, 64, 0): b.Q4_ERR_UNSUPPORTED,
              (1, 64, 4096, 64, 2): b.Q4_ERR_UNSUPPORTED,
              (-1, 64, 4096, 64, 0): b.Q4_ERR_INVALID_ARG,
@@ -82,17 +82,34 @@ def test_gemm_validation_before_cuda():
     assert g(None, *args[1:], 1, 64, 4096, 64, 0, ALIGNED, None, 0, None) == b.Q4_ERR_INVALID_ARG
     bias = b.lib().q4_gemm_skinny_bias
     assert bias(*args, None, 1, 64, 4096, 64, 0, ALIGNED, None, 0, None, None) == b.Q4_ERR_INVALID_ARG  # no bias
-    assert bias(*args, ALIGNED, 17, 64, 4096, 64, 0, ALIGNED, None, 0, None, None) == b.Q4_ERR_UNSUPPORTED
+    assert bias(*args, ALIGNED, 129, 64, 4096, 64, 0, ALIGNED, None, 0, None, None) == b.Q4_ERR_UNSUPPORTED
     ex = b.lib().q4_gemm_skinny_ex
-    assert ex(*args, 1, 64, 4096, 64, 0, ALIGNED, None, 0, None, b.overrides(math=3)) == b.Q4_ERR_INVALID_ARG
+    assert ex(*args, 1, 64, 4096, 64, 0, ALIGNED, None, 0, None, b.overrides(math=4)) == b.Q4_ERR_INVALID_ARG
+    # the tensor-memory kernel (M > 16) needs blocksize >= 64 and K % 256 == 0
+    assert ex(*args, 32, 64, 4096, 32, 0, ALIGNED, None, 0, None, None) == b.Q4_ERR_UNSUPPORTED
+    assert ex(*args, 32, 64, 4160, 64, 0, ALIGNED, None, 0, None, None) == b.Q4_ERR_UNSUPPORTED
     assert ex(*args, 12, 64, 4096, 64, 0, ALIGNED, None, 0, None, b.overrides(warps=16)) == b.Q4_ERR_UNSUPPORTED
     assert ex(*args, 1, 64, 4096, 64, 0, ALIGNED, None, 0, None, b.overrides(depth=7)) == b.Q4_ERR_UNSUPPORTED
     assert ex(*args, 1, 64, 4096, 64, 0, ALIGNED, None, 0, None, b.overrides(math=2)) == b.Q4_ERR_UNSUPPORTED
 
 
+@pytest.mark.parametrize("M,N,K", [(17, 4096, 4096), (32, 300, 1024), (64, 28672, 8192), (128, 8192, 28672)])
+def test_launch_table_tcgen05(M, N, K):
+    p = b.q4_gemm_plan(M, N, K, 64, num_sms=148)
+    assert p["math"] == 3 and p["loader"] == 6 and p["rows_per_tile"] == 128 and p["sub_block"] == 64
+    assert p["m_pad"] == (32 if M <= 32 else 64 if M <= 64 else 128)
+    tiles = -(-N // 128)
+    assert p["tiles"] == tiles and p["units"] == tiles * (K // 64)
+    assert 1 <= p["ctas"] <= min(148, p["units"])
+    slots = p["ctas"] * 2 * p["m_pad"] * 128 * 4
+    assert p["workspace_bytes"] == 256 + 148 * 2 * 4096 + -(-tiles * 4 // 256) * 256 + slots
+
+
 @pytest.mark.parametrize("wl", list(inputs.workloads()))
 def test_launch_table_invariants(wl):
     for c in inputs.workloads()[wl].cases:
+        if c.M > 16:
+            continue  # the tensor-memory kernel's table: test_launch_table_tcgen05
         p = b.q4_gemm_plan(c.M, c.N, c.K, c.blocksize, num_sms=148)
         assert p["math"] == 1
         assert p["sub_block"] == min(c.blocksize, 64)

@@ -1,0 +1,121 @@
+"""GPU parity of the tensor-memory (tcgen05) kernel that serves 17 <= M <= 128
+(and M <= 16 on request, math=3): every output element within
+1e-2 * sum_k |a w| + ulp(y) of the oracle.  The weights enter the MMA as
+bf16_rn(code * absmax) (fp16 for fp16 activations), i.e. exactly the values
+the standalone dequantizer writes; the fp32 accumulation follows.  The
+operation is the fused path of bitsandbytes PR #1920 ("Fused path support
+for M > 1") at larger M."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from bit_weight_dequant_b200 import binding as q4
+from bit_weight_dequant_b200 import inputs
+from bit_weight_dequant_b200.inputs import Case
+from parity import ORACLE_ACT, TORCH_ACT, bits_of, check_gemm, run_case
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.mark.parametrize("M", [17, 24, 32, 33, 48, 64, 65, 96, 127, 128])
+@pytest.mark.parametrize("N,K", [(128, 256), (300, 1024), (513, 2048), (1000, 512)])
+def test_tcgen05_bf16(cuda_device, M, N, K):
+    run_case(Case(M, N, K), seed=7000 + M * 3 + N + K, device=cuda_device, check_quantizer=False)
+
+
+@pytest.mark.parametrize("M", [20, 64, 128])
+@pytest.mark.parametrize("act,table", [("fp16", "normal"), ("bf16", "uniform"), ("bf16", "fp4"), ("fp16", "fp4")])
+def test_tcgen05_dtypes_tables(cuda_device, M, act, table):
+    run_case(Case(M, 384, 1536, act=act, table=table), seed=7100 + M, device=cuda_device, check_quantizer=False)
+
+
+@pytest.mark.parametrize("M", [40, 128])
+@pytest.mark.parametrize("bs", [128, 256, 1024])
+def test_tcgen05_blocksizes(cuda_device, M, bs):
+    run_case(Case(M, 256, 4096, blocksize=bs), seed=7200 + bs + M, device=cuda_device, check_quantizer=False)
+
+
+@pytest.mark.parametrize("ctas", [1, 2, 3, 7, 33, 148])
+@pytest.mark.parametrize("M", [18, 100])
+def test_tcgen05_partitions(cuda_device, ctas, M):
+    """Tiles cut between CTAs (workspace fix-up) at every CTA count."""
+    run_case(Case(M, 640, 2048), seed=7300 + ctas, device=cuda_device, check_quantizer=False, ctas=ctas)
+
+
+@pytest.mark.parametrize("M", [1, 5, 16])
+def test_tcgen05_small_m_on_request(cuda_device, M):
+    run_case(Case(M, 512, 1024), seed=7400 + M, device=cuda_device, check_quantizer=False, math=3)
+
+
+def test_tcgen05_outliers(cuda_device):
+    run_case(Case(64, 256, 2048, outliers=True), seed=7500, device=cuda_device, check_quantizer=False)
+
+
+@pytest.mark.parametrize("ctas", [5, 37])
+def test_tcgen05_deterministic_and_counters_left_zero(cuda_device, ctas):
+    M, N, K = 48, 700, 2048
+    code = inputs.code_normal_quantile()
+    W = inputs.weights(N, K, 9)
+    packed, absmax = oracle.quantize(W, 64, code)
+    A = inputs.activations(M, K, torch.bfloat16, 9).to(cuda_device)
+    P, Am, C = (torch.from_numpy(x).to(cuda_device) for x in (packed, absmax, code))
+    ws = q4.Workspace(cuda_device)
+    outs = [q4.q4_gemm_skinny(A, P, Am, C, N, K, 64, workspace=ws, ctas=ctas) for _ in range(3)]
+    torch.cuda.synchronize()
+    for o in outs[1:]:
+        assert torch.equal(o.view(torch.int16), outs[0].view(torch.int16))
+    assert q4.workspace_error(ws) == 0
+    off = q4.workspace_counter_offset(cuda_device)
+    assert int(ws.buf[off:].count_nonzero()) == 0, "counters and partial slots must return to zero"
+    y, S = oracle.gemm(bits_of(A.cpu()), oracle.BF16, packed, absmax, code, M, N, K, 64)
+    check_gemm(bits_of(outs[0].cpu()), y, S, "bf16", "tcgen05 determinism")
+
+
+@pytest.mark.parametrize("act", ["bf16", "fp16"])
+@pytest.mark.parametrize("launch", [{}, {"ctas": 9}])
+def test_tcgen05_bias(cuda_device, act, launch):
+    M, N, K = 50, 300, 1024
+    code = inputs.code_normal_quantile()
+    W = inputs.weights(N, K, 21)
+    packed, absmax = oracle.quantize(W, 64, code)
+    A = inputs.activations(M, K, TORCH_ACT[act], 21)
+    bias = inputs.activations(1, N, TORCH_ACT[act], 22).reshape(N)
+    y, S = oracle.gemm(bits_of(A), ORACLE_ACT[act], packed, absmax, code, M, N, K, 64, bias_bits=bits_of(bias))
+    dev = cuda_device
+    out = q4.q4_gemm_skinny(A.to(dev), torch.from_numpy(packed).to(dev), torch.from_numpy(absmax).to(dev),
+                            torch.from_numpy(code).to(dev), N, K, 64, bias=bias.to(dev), **launch)
+    check_gemm(bits_of(out), y, S, act, f"tcgen05 bias {act} {launch}")
+
+
+def test_tcgen05_requirements(cuda_device):
+    """M > 16 outside the kernel's layout rules is reported, not run."""
+    dev = cuda_device
+    A = torch.zeros((32, 4160), dtype=torch.bfloat16, device=dev)
+    P = torch.zeros(64 * 4160 // 2, dtype=torch.uint8, device=dev)
+    Am = torch.zeros(64 * 4160 // 64, dtype=torch.float32, device=dev)
+    C = torch.from_numpy(inputs.code_normal_quantile()).to(dev)
+    with pytest.raises(q4.Q4Error) as e:
+        q4.q4_gemm_skinny(A, P, Am, C, 64, 4160, 64)        # K % 256 != 0
+    assert e.value.status == q4.Q4_ERR_UNSUPPORTED
+    A2 = torch.zeros((129, 256), dtype=torch.bfloat16, device=dev)
+    with pytest.raises(q4.Q4Error) as e:
+        q4.q4_gemm_skinny(A2, P[:64 * 128], Am[:256], C, 64, 256, 64)
+    assert e.value.status == q4.Q4_ERR_UNSUPPORTED
+
+
+def test_tcgen05_then_small_m_share_a_workspace(cuda_device):
+    """A tensor-memory call leaves nothing behind that a later call of another
+    shape (whose counters may lie where the first call's slots were) could
+    misread."""
+    ws = q4.Workspace(cuda_device)
+    for M, N, K in [(48, 300, 1024), (1, 10240, 1024), (64, 1000, 2048), (3, 20000, 512)]:
+        code = inputs.code_normal_quantile()
+        W = inputs.weights(N, K, N + M)
+        packed, absmax = oracle.quantize(W, 64, code)
+        A = inputs.activations(M, K, torch.bfloat16, N)
+        y, S = oracle.gemm(bits_of(A), oracle.BF16, packed, absmax, code, M, N, K, 64)
+        out = q4.q4_gemm_skinny(A.to(cuda_device), torch.from_numpy(packed).to(cuda_device),
+                                torch.from_numpy(absmax).to(cuda_device), torch.from_numpy(code).to(cuda_device),
+                                N, K, 64, workspace=ws, ctas=17)
+        check_gemm(bits_of(out.cpu()), y, S, "bf16", f"shared workspace M{M} N{N}")
