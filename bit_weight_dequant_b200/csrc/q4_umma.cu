@@ -330,10 +330,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tc_fence_after();
                     const uint32_t dcol = (seg & 1) ? kColD1 : kColD0;
                     const uint32_t acol = kColA + 32u * (uint32_t)b;
-                    const uint32_t xs = st + G::X0 + (uint32_t)j * G::XBYTES;
+                    // B descriptor of this unit's activations; each 16-k step
+                    // advances the start address by 32 bytes (2 in its units)
+                    const uint64_t xd = smem_desc_sw128(st + G::X0 + (uint32_t)j * G::XBYTES);
 #pragma unroll
                     for (int k4 = 0; k4 < 4; ++k4)
-                        mma_ts(tbase + dcol, tbase + acol + 8u * k4, smem_desc_sw128(xs + 32u * k4), idesc,
+                        mma_ts(tbase + dcol, tbase + acol + 8u * k4, xd + 2u * (uint32_t)k4, idesc,
                                !(seg_start && k4 == 0));
                     tc_commit(afree + 8u * b);
                     const bool seg_end = (kb0 + j + 1 == kbt) || (q.left == 0 && j == kb - kb0 + n - 1);
