@@ -53,7 +53,10 @@ constexpr uint32_t kAmBytes = kRows * 16;   // absmax of a stage (128 rows x 4 f
 constexpr uint32_t kTmemCols = 512;         // the whole tensor memory (one CTA per SM)
 constexpr uint32_t kColD0 = 0, kColD1 = 128, kColA = 256;  // A buffer b at kColA + 32 b
 constexpr int kNA = 8;                                       // A buffers (64-k units in flight)
-constexpr uint32_t kWaitLimit = 1u << 22;
+// Bounded waits: each try may sleep up to kWaitSleepNs; at most kWaitTries
+// tries (about two seconds) before the wait gives up.
+constexpr uint32_t kWaitSleepNs = 50000;
+constexpr uint32_t kWaitTries = 40000;
 constexpr int kErrWaitTimeout = 1;
 constexpr int kThreads = 320;  // producer, MMA issuer, two dequantizing warpgroups
 
@@ -141,8 +144,8 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr) {
 }
 
 __device__ __forceinline__ bool wait_parity(uint32_t bar, uint32_t parity) {
-    for (uint32_t it = 0; it < kWaitLimit; ++it)
-        if (mbar_try_wait(bar, parity)) return true;
+    for (uint32_t it = 0; it < kWaitTries; ++it)
+        if (mbar_try_wait_sleep(bar, parity, kWaitSleepNs)) return true;
     return false;
 }
 
