@@ -51,10 +51,12 @@ def _load():
         lib.oracle_dequantize.argtypes = [P, P, P, i64, ci, ci, P]
         lib.oracle_gemm.argtypes = [P, ci, P, P, P, ci, ci, ci, ci, P, P]
         lib.oracle_gemm_bias.argtypes = [P, ci, P, P, P, P, ci, ci, ci, ci, P, P]
+        lib.oracle_gemm_f32.argtypes = [P, P, P, P, P, ci, ci, ci, ci, P, P]
         lib.oracle_round.argtypes = [P, i64, ci, P]
         lib.oracle_decode.argtypes = [P, i64, ci, P]
         lib.oracle_ulp.argtypes = [P, i64, ci, P]
-        for f in ("oracle_quantize", "oracle_dequantize", "oracle_gemm", "oracle_gemm_bias", "oracle_round",
+        for f in ("oracle_quantize", "oracle_dequantize", "oracle_gemm", "oracle_gemm_bias", "oracle_gemm_f32",
+                  "oracle_round",
                   "oracle_decode", "oracle_ulp"):
             getattr(lib, f).restype = ci
         _lib = lib
@@ -119,6 +121,26 @@ def gemm(a_bits: np.ndarray, act_dtype: int, packed: np.ndarray, absmax: np.ndar
     return (y, S) if want_s else y
 
 
+def gemm_f32(a: np.ndarray, packed: np.ndarray, absmax: np.ndarray, code: np.ndarray, M: int, N: int, K: int,
+             blocksize: int, want_s: bool = True, bias: np.ndarray | None = None):
+    """fp64 reference ``y[M,N]`` and ``S[M,N] = sum |a*w|`` for fp32
+    activations ``a[M,K]``; ``bias`` (N fp32 values) is added to y."""
+    a = np.ascontiguousarray(a, dtype=np.float32).reshape(-1)
+    assert a.size == M * K
+    packed = np.ascontiguousarray(packed, dtype=np.uint8)
+    absmax = np.ascontiguousarray(absmax, dtype=np.float32)
+    code = np.ascontiguousarray(code, dtype=np.float32)
+    if bias is not None:
+        bias = np.ascontiguousarray(bias, dtype=np.float32).reshape(-1)
+        assert bias.size == N
+    y = np.zeros((M, N), dtype=np.float64)
+    S = np.zeros((M, N), dtype=np.float64) if want_s else None
+    _check(_load().oracle_gemm_f32(_ptr(a), _ptr(packed), _ptr(absmax), _ptr(code),
+                                   _ptr(bias) if bias is not None else None, M, N, K, blocksize, _ptr(y),
+                                   _ptr(S) if want_s else None), "gemm_f32")
+    return (y, S) if want_s else y
+
+
 def round_to(x: np.ndarray, dtype: int) -> np.ndarray:
     """Round doubles once (nearest-even) to bf16/fp16; returns uint16 bits."""
     x = np.ascontiguousarray(x, dtype=np.float64).reshape(-1)
@@ -136,7 +158,7 @@ def decode(bits: np.ndarray, dtype: int) -> np.ndarray:
 
 
 def ulp(y: np.ndarray, dtype: int) -> np.ndarray:
-    """Spacing of the bf16/fp16 format at |y| (subnormal spacing at 0)."""
+    """Spacing of the bf16/fp16/fp32 format at |y| (subnormal spacing at 0)."""
     y = np.ascontiguousarray(y, dtype=np.float64).reshape(-1)
     out = np.zeros(y.size, dtype=np.float64)
     _check(_load().oracle_ulp(_ptr(y), y.size, dtype, _ptr(out)), "ulp")

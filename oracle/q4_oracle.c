@@ -32,7 +32,10 @@
  *     fp32 multiply, then one round-to-nearest-even into the output format;
  *   - GEMM: y = sum_k double(a) * double(w) in k order, w the fp32 product
  *     code[idx] * absmax (not rounded to 16 bits), then one RNE rounding of
- *     the fp64 sum into the activation dtype.
+ *     the fp64 sum into the activation dtype;
+ *   - fp32 activations (the reply: the SIMT kernel takes fp32, fp16 and
+ *     bf16 inputs, all with fp32 accumulation): the same sum with a taken as
+ *     given, and an fp32 bias.
  *
  * Parity pins: every function here is pinned by the CPU tests (hand-worked
  * examples, brute force on tiny inputs, closed forms, invariants, library
@@ -68,6 +71,7 @@ typedef struct {
 
 static const or_format OR_FMT_BF16 = {8, -126, 127};
 static const or_format OR_FMT_FP16 = {11, -14, 15};
+static const or_format OR_FMT_FP32 = {24, -126, 127};
 
 /* Largest finite value of the format: (2 - 2^(1-p)) * 2^emax. */
 static double or_max_finite(or_format f) {
@@ -184,10 +188,10 @@ int oracle_decode(const uint16_t* bits, int64_t count, int dtype, double* out) {
     return OR_OK;
 }
 
-/* Spacing (ulp) of the output dtype at each y[i]. */
+/* Spacing (ulp) of the output dtype (bf16, fp16 or fp32) at each y[i]. */
 int oracle_ulp(const double* y, int64_t count, int dtype, double* out) {
-    if (dtype != OR_BF16 && dtype != OR_FP16) return OR_BAD;
-    or_format f = dtype == OR_BF16 ? OR_FMT_BF16 : OR_FMT_FP16;
+    if (dtype != OR_BF16 && dtype != OR_FP16 && dtype != OR_FP32) return OR_BAD;
+    or_format f = dtype == OR_BF16 ? OR_FMT_BF16 : dtype == OR_FP16 ? OR_FMT_FP16 : OR_FMT_FP32;
     for (int64_t i = 0; i < count; ++i) out[i] = or_ulp(y[i], f);
     return OR_OK;
 }
@@ -332,5 +336,36 @@ int oracle_gemm_bias(const uint16_t* A, int act_dtype, const uint8_t* packed, co
             float b = act_dtype == OR_BF16 ? or_bf16_to_float(bias[n]) : or_fp16_to_float(bias[n]);
             y[(int64_t)m * N + n] += (double)b;
         }
+    return OR_OK;
+}
+
+/*
+ * The skinny matmul with fp32 activations (the maintainer's reply in PR
+ * #1920: the replacement SIMT kernel accepts fp32 as well as fp16/bf16
+ * inputs):
+ *     y[m,n] = [bias[n]] + sum_{k=0}^{K-1} double(a[m,k]) * double(w[n,k])
+ *     S[m,n] = sum_k |double(a[m,k]) * double(w[n,k])|
+ * in k order in fp64, w[n,k] = code[idx(n*K+k)] *_fp32 absmax[(n*K+k)/bs]
+ * as in oracle_gemm, A given as binary32 values, row-major [M, K], and bias
+ * (N binary32 values) optional (NULL: none).  Either output may be NULL.
+ */
+int oracle_gemm_f32(const float* A, const uint8_t* packed, const float* absmax, const float* code,
+                    const float* bias, int M, int N, int K, int bs, double* y, double* S) {
+    if (M < 0 || N < 0 || K < 0 || bs <= 0) return OR_BAD;
+    for (int m = 0; m < M; ++m) {
+        for (int n = 0; n < N; ++n) {
+            double acc = 0.0, accabs = 0.0;
+            for (int k = 0; k < K; ++k) {
+                float a = A[(int64_t)m * K + k];
+                float w = or_weight_at(packed, absmax, code, (int64_t)n * K + k, bs);
+                double prod = (double)a * (double)w;
+                acc += prod;
+                accabs += fabs(prod);
+            }
+            if (bias) acc += (double)bias[n];
+            if (y) y[(int64_t)m * N + n] = acc;
+            if (S) S[(int64_t)m * N + n] = accabs;
+        }
+    }
     return OR_OK;
 }

@@ -380,3 +380,73 @@ def test_tolerance_formula():
     S = np.array([10.0, 3.0, 0.0])
     tol = oracle.gemm_tolerance(y, S, oracle.BF16)
     assert tol.tolist() == [0.1 + 2.0 ** -7, 0.03 + 2.0 ** -6, 2.0 ** -133]
+
+
+# ---------------------------------------------------------------------------
+# fp32 activations (the reply's SIMT kernel: fp32, fp16 and bf16 inputs)
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("M,N,K,bs", [(1, 1, 64, 64), (3, 7, 64, 32), (4, 9, 128, 64), (2, 5, 96, 32),
+                                      (5, 3, 40, 8)])
+def test_gemm_f32_brute_force(M, N, K, bs):
+    """Full-mantissa fp32 activations: numpy fp64 matmul over the explicitly
+    dequantized weights."""
+    code = TABLES["normal"]
+    rng = np.random.default_rng(9000 + M * 100 + N * 10 + K)
+    w = (rng.standard_normal(N * K) * 0.02).astype(np.float32)
+    packed, absmax = oracle.quantize(w, bs, code)
+    a32 = rng.standard_normal((M, K)).astype(np.float32)
+    a64 = a32.astype(np.float64)
+    W64 = np_weights(packed, absmax, code, N * K, bs).astype(np.float64).reshape(N, K)
+    y, S = oracle.gemm_f32(a32, packed, absmax, code, M, N, K, bs)
+    np.testing.assert_allclose(y, a64 @ W64.T, rtol=0, atol=1e-12 * ((np.abs(a64) @ np.abs(W64).T).max() + 1))
+    np.testing.assert_allclose(S, np.abs(a64) @ np.abs(W64).T, rtol=1e-12)
+
+
+def test_gemm_f32_agrees_with_bf16_path_on_bf16_values():
+    """Activations that bf16 holds exactly give the same fp64 sums through
+    the fp32 entry as through the (separately pinned) bf16 entry."""
+    code = TABLES["fp4"]
+    M, N, K, bs = 3, 11, 256, 64
+    rng = np.random.default_rng(31)
+    w = (rng.standard_normal(N * K) * 0.02).astype(np.float32)
+    packed, absmax = oracle.quantize(w, bs, code)
+    abits = torch_bf16_bits(rng.standard_normal((M, K)).astype(np.float32)).reshape(M, K)
+    a32 = torch_bf16_values(abits.reshape(-1)).astype(np.float32).reshape(M, K)
+    y16, S16 = oracle.gemm(abits, oracle.BF16, packed, absmax, code, M, N, K, bs)
+    y32, S32 = oracle.gemm_f32(a32, packed, absmax, code, M, N, K, bs)
+    assert np.array_equal(y16, y32) and np.array_equal(S16, S32)
+
+
+def test_gemm_f32_one_hot_and_bias():
+    """One-hot rows select a dequantized weight exactly; the fp32 bias is
+    added once, exactly, and with every absmax 0 the layer is the bias."""
+    code = TABLES["normal"]
+    N, K, bs = 6, 128, 32
+    rng = np.random.default_rng(5)
+    w = (rng.standard_normal(N * K) * 0.02).astype(np.float32)
+    packed, absmax = oracle.quantize(w, bs, code)
+    wq = np_weights(packed, absmax, code, N * K, bs).reshape(N, K)
+    a = np.zeros((4, K), dtype=np.float32)
+    ks = (0, 31, 32, 127)
+    for m, k in enumerate(ks):
+        a[m, k] = 1.0
+    y, _ = oracle.gemm_f32(a, packed, absmax, code, 4, N, K, bs)
+    for m, k in enumerate(ks):
+        assert np.array_equal(y[m], wq[:, k].astype(np.float64))
+    b = rng.standard_normal(N).astype(np.float32)
+    yb, _ = oracle.gemm_f32(a, packed, absmax, code, 4, N, K, bs, bias=b)
+    assert np.array_equal(yb, y + b.astype(np.float64)[None, :])
+    y0, S0 = oracle.gemm_f32(a, packed, np.zeros_like(absmax), code, 4, N, K, bs, bias=b)
+    assert np.array_equal(y0, np.broadcast_to(b.astype(np.float64), (4, N))) and np.all(S0 == 0)
+
+
+def test_ulp_fp32_against_numpy_spacing():
+    """The fp32 spacing is numpy's own ``spacing`` of the binary32 value
+    (normal, subnormal and zero)."""
+    rng = np.random.default_rng(2)
+    y = np.concatenate([rng.standard_normal(200) * 10.0 ** rng.integers(-30, 30, 200),
+                        [0.0, 1.0, -1.0, 2.0 ** -126, 2.0 ** -140, 3.0e38]]).astype(np.float32)
+    want = np.abs(np.spacing(np.abs(y))).astype(np.float64)
+    got = oracle.ulp(y.astype(np.float64), oracle.FP32)
+    assert np.array_equal(got, want)
