@@ -62,6 +62,16 @@ def gemm_kernel_hash() -> str:
     return h.hexdigest()[:16]
 
 
+def kernel_name(plan: dict) -> str:
+    """The GEMM kernel a launch-table entry runs."""
+    if plan["math"] == 2:
+        return "q4_gemm_f32_kernel"
+    if plan["math"] == 3:
+        return "q4_gemm_umma_kernel"
+    return {1: "q4_gemm_mma_kernel", 2: "q4_gemm_tma_kernel", 3: "q4_gemm_tma_kernel"}.get(plan["loader"],
+                                                                                            "q4_gemm_ws_kernel")
+
+
 def ncu_traffic(workload: str):
     """DRAM bytes per launch of the GEMM kernel from the committed ncu
     summary, if it was taken on the current kernel source; else None."""
@@ -157,13 +167,16 @@ def barrier(world: int):
 # Our arm
 # ---------------------------------------------------------------------------
 
+TORCH_ACT = {"bf16": torch.bfloat16, "fp16": torch.float16, "fp32": torch.float32}
+
+
 class Layer:
     """One 4-bit linear layer resident on the device, with its C-ABI call
     arguments prepared once (the timed loop only makes the call)."""
 
     def __init__(self, case: inputs.Case, seed: int, device, pdl: int = 2):
         self.case = case
-        dt = torch.bfloat16 if case.act == "bf16" else torch.float16
+        dt = TORCH_ACT[case.act]
         code = inputs.CODE_TABLES[case.table]()
         self.code = torch.from_numpy(code).to(device)
         W = inputs.weights_device(case.N, case.K, seed, device, case.outliers)
@@ -176,7 +189,7 @@ class Layer:
         self.out_host = torch.empty((case.M, case.N), dtype=dt).pin_memory()
         self.ws_bytes = q4.q4_gemm_workspace_size(case.M, case.N, case.K, case.blocksize, dt)
         self.ws = torch.zeros(max(self.ws_bytes, 16), dtype=torch.uint8, device=device)
-        self.act = q4.Q4_BF16 if case.act == "bf16" else q4.Q4_FP16
+        self.act = {"bf16": q4.Q4_BF16, "fp16": q4.Q4_FP16, "fp32": q4.Q4_FP32}[case.act]
         self.plan = q4.q4_gemm_plan(case.M, case.N, case.K, case.blocksize, dt)
         self.rebind(self.A, self.out)
         # Decode-time weights are static model parameters: let each GEMM's
@@ -441,12 +454,13 @@ def run_ours(args, world, rank, local):
         return None
     cpu = cpu_baseline(wl, args.cpu_seconds) if (world == 1 and not args.no_cpu_baseline) else None
     total_weight_bytes = sum(L.packed.numel() + 4 * L.absmax.numel() for L in layers)
+    act_dtype = "+".join(sorted({ {"bf16": "bf16", "fp16": "f16", "fp32": "f32"}[L.case.act] for L in layers}))
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms_step, 5), "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "vs_baseline": None, "dtype": act_dtype, "data": "synthetic",
         "config": {"workload": wl.name + (f" [only {args.only}]" if args.only else ""), "M": sorted({c.M for c in wl.cases}), "blocksize": 64,
-                   "code_table": "normal-quantile", "activations": "bf16 ~N(0,1)", "weights": "N(0,0.02^2) fp32 -> 4-bit",
+                   "code_table": "normal-quantile", "activations": f"{act_dtype} ~N(0,1)", "weights": "N(0,0.02^2) fp32 -> 4-bit",
                    "l2": f"inputs larger than L2: {total_weight_bytes / 1e6:.0f} MB of packed weights per step "
                          f"vs {L2_BYTES / 2**20:.0f} MiB L2, no flush",
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
@@ -454,7 +468,7 @@ def run_ours(args, world, rank, local):
                    "dependent_launch": args.pdl},
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "traffic": ncu_traffic(args.workload),
-                     "peak_source": peak_src, "kernel": "q4_gemm_tma_kernel",
+                     "peak_source": peak_src, "kernel": "+".join(sorted({kernel_name(L.plan) for L in layers})),
                      "per_unit": "0.5 B per weight (codes) + 4/bs B (absmax) + A and C once",
                      "duration": "average launch = timed-region device time / launches (all launches are this kernel)"},
         "per_shape": per_shape,
@@ -484,16 +498,22 @@ def _oracle_sample(case: inputs.Case, rows: int, seed: int):
     code = inputs.CODE_TABLES[case.table]()
     W = inputs.weight_rows(case.K, seed, 0, rows, case.outliers)
     packed, absmax = oracle.quantize(W, case.blocksize, code)
-    A = inputs.activations(case.M, case.K, torch.bfloat16, seed)
+    if case.act == "fp32":
+        return (inputs.activations_fp32(case.M, case.K, seed), packed, absmax, code)
+    A = inputs.activations(case.M, case.K, TORCH_ACT[case.act], seed)
     abits = A.view(torch.int16).numpy().view(np.uint16)
     return (abits, packed, absmax, code)
 
 
 def _oracle_time(case, rows, prepared):
     import oracle
-    abits, packed, absmax, code = prepared
+    a, packed, absmax, code = prepared
     t0 = time.perf_counter()
-    oracle.gemm(abits, oracle.BF16, packed, absmax, code, case.M, rows, case.K, case.blocksize, want_s=False)
+    if case.act == "fp32":
+        oracle.gemm_f32(a, packed, absmax, code, case.M, rows, case.K, case.blocksize, want_s=False)
+    else:
+        oracle.gemm(a, oracle.BF16 if case.act == "bf16" else oracle.FP16, packed, absmax, code, case.M, rows,
+                    case.K, case.blocksize, want_s=False)
     return time.perf_counter() - t0
 
 
@@ -510,7 +530,7 @@ def cpu_baseline(wl, seconds: float) -> dict:
             spent += _oracle_time(c, rows, prep)
             reps += 1
         tot_s += spent
-        tot_bytes += reps * inputs.Case(c.M, rows, c.K, c.blocksize).algorithmic_bytes()
+        tot_bytes += reps * inputs.Case(c.M, rows, c.K, c.blocksize, act=c.act).algorithmic_bytes()
         desc.append(f"{reps}x {rows}/{c.N} rows of K{c.K}N{c.N}")
     return {"value": round(tot_bytes / tot_s / 1e9, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
             "sample": "; ".join(desc) + f" (M={wl.cases[0].M}; {tot_s:.1f} s single-threaded)"}
@@ -538,7 +558,8 @@ def run_reference(args, world, rank):
     for _ in range(args.steps):
         for c, r, p in zip(wl.cases, rows, preps):
             tot_s += _oracle_time(c, r, p)
-    step_bytes = sum(inputs.Case(c.M, r, c.K, c.blocksize).algorithmic_bytes() for c, r in zip(wl.cases, rows))
+    step_bytes = sum(inputs.Case(c.M, r, c.K, c.blocksize, act=c.act).algorithmic_bytes()
+                     for c, r in zip(wl.cases, rows))
     value = step_bytes * args.steps / tot_s / 1e9
     sample = "; ".join(f"{r}/{c.N} rows of K{c.K}N{c.N}" for c, r in zip(wl.cases, rows))
     return {"impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus": world,

@@ -88,8 +88,45 @@ static int gemm_choose(int M, int N, int K, int blocksize, int act_dtype, int nu
     if (!is_pow2_blocksize(blocksize)) return Q4_ERR_INVALID_ARG;
     if (act_dtype != Q4_BF16 && act_dtype != Q4_FP16 && act_dtype != Q4_FP32) return Q4_ERR_INVALID_ARG;
     if (ov && (ov->math > 3 || ov->l2_prefetch > 256 || ov->loader > 6 || ov->pdl > 2)) return Q4_ERR_INVALID_ARG;
-    if (M > 128 || act_dtype == Q4_FP32 || K % blocksize != 0) return Q4_ERR_UNSUPPORTED;
+    if (M > 128 || K % blocksize != 0) return Q4_ERR_UNSUPPORTED;
     GemmChoice c{};
+    if (act_dtype == Q4_FP32) {
+        // fp32 activations: the CUDA-core kernel (M <= 16), units of R rows x
+        // 512 k split over every warp of the grid.
+        if (M > 16) return Q4_ERR_UNSUPPORTED;
+        if (ov && ((ov->math > 0 && ov->math != 2) || ov->loader > 1)) return Q4_ERR_UNSUPPORTED;
+        const SimtShape sh = simt_shape(M);
+        if (ov && ov->warps > 0 && ov->warps != sh.warps) return Q4_ERR_UNSUPPORTED;
+        c.math = 2;
+        c.sub_block = 512;
+        c.m_pad = sh.m_pad;
+        c.rows_per_tile = sh.rows;
+        c.warps = sh.warps;
+        c.loader = 1;
+        c.depth = 2;  // units in flight per warp
+        c.l2pf = 0;
+        c.pdl = (ov && ov->pdl > 0) ? ov->pdl : 0;
+        const int64_t t64 = N > 0 ? ((int64_t)N + sh.rows - 1) / sh.rows : 0;
+        const int64_t u = t64 * (((int64_t)K + 511) / 512);
+        if (u >= ((int64_t)1 << 31) || K >= (1 << 29)) return Q4_ERR_UNSUPPORTED;  // 32-bit row offsets
+        int sms = num_sms;
+        if (sms <= 0 && device_sm_count(&sms) != 0) return Q4_ERR_CUDA;
+        if (ov && ov->ctas > sms) return Q4_ERR_INVALID_ARG;
+        int64_t g = (ov && ov->ctas > 0) ? ov->ctas : sms;
+        const int64_t need_ctas = (u + sh.warps - 1) / sh.warps;  // at least one unit per warp where possible
+        if (g > need_ctas) g = need_ctas;
+        if (g < 1) g = 1;
+        c.ctas = (int)g;
+        *ch = c;
+        *tiles = (int)t64;
+        *units = u;
+        *sms_out = sms;
+        // Pieces of row groups go to the fixed partial region (at most
+        // 2 x 128 floats per warp-slot pair and 8 KiB per SM); one counter
+        // per row group sits at the fixed counter offset.
+        *ws_bytes = u > 1 ? ws_counter_offset(sms) + align_up((size_t)t64 * sizeof(int), 256) : 0;
+        return Q4_OK;
+    }
     if (M > 16 || (ov && (ov->math == 3 || ov->loader == 6))) {
         // Tensor-memory kernel (tcgen05): 128-row tiles, 64-k units, 4-unit
         // stages whose absmax box is 4 floats per row.
@@ -251,7 +288,7 @@ int q4_gemm_plan(int M, int N, int K, int blocksize, int act_dtype, int num_sms,
     plan->pdl = ch.pdl;
     plan->tiles = tiles;
     plan->units = units;
-    plan->smem_bytes = gemm_smem_bytes(act_dtype == Q4_FP32 ? Q4_BF16 : act_dtype, ch);
+    plan->smem_bytes = ch.math == 2 ? simt_smem_bytes() : gemm_smem_bytes(act_dtype, ch);
     plan->workspace_bytes = ws;
     return Q4_OK;
 }
@@ -279,7 +316,7 @@ static int gemm_entry(const void* A, const uint8_t* Wpacked, const float* absmax
     if (M == 0 || N == 0) return Q4_OK;
     if (!aligned(out, 16) || (K > 0 && (!aligned(A, 16) || !aligned(Wpacked, 16) || !aligned(absmax, 4) ||
                                          !aligned(code, 4))) ||
-        (bias && !aligned(bias, 2)))
+        (bias && !aligned(bias, act_dtype == Q4_FP32 ? 4 : 2)))
         return Q4_ERR_MISALIGNED;
     if (need > 0 && (!workspace || workspace_bytes < need)) return Q4_ERR_WORKSPACE;
     if (workspace && !aligned(workspace, 16)) return Q4_ERR_MISALIGNED;
@@ -297,10 +334,11 @@ static int gemm_entry(const void* A, const uint8_t* Wpacked, const float* absmax
     }
     if (injected_failure()) return Q4_ERR_CUDA;
     cudaStream_t st = (cudaStream_t)stream;
-    if (K == 0) {  // empty contraction: every row is the bias, or +0 (0x0000 in bf16 and fp16)
-        if (!bias) return from_cuda(cudaMemsetAsync(out, 0, (size_t)M * N * 2, st));
+    if (K == 0) {  // empty contraction: every row is the bias, or +0 (all-zero bits in every dtype)
+        const size_t esize = act_dtype == Q4_FP32 ? 4 : 2;
+        if (!bias) return from_cuda(cudaMemsetAsync(out, 0, (size_t)M * N * esize, st));
         for (int m = 0; m < M; ++m) {
-            cudaError_t e = cudaMemcpyAsync(static_cast<char*>(out) + (size_t)m * N * 2, bias, (size_t)N * 2,
+            cudaError_t e = cudaMemcpyAsync(static_cast<char*>(out) + (size_t)m * N * esize, bias, (size_t)N * esize,
                                             cudaMemcpyDeviceToDevice, st);
             if (e != cudaSuccess) return from_cuda(e);
         }
@@ -328,6 +366,11 @@ static int gemm_entry(const void* A, const uint8_t* Wpacked, const float* absmax
     p.tiles = tiles;
     p.ctas = ch.ctas;
     p.units = (uint32_t)units;
+    if (ch.math == 2) {
+        int lbs = 0;
+        while ((1 << lbs) < blocksize) ++lbs;
+        return from_cuda(simt_launch(simt_shape(M), ch.ctas, p, lbs, st));
+    }
     if (ch.math == 3) {
         if (workspace)
             p.partials = reinterpret_cast<float*>(static_cast<char*>(workspace) + ws_counter_offset(sms) +

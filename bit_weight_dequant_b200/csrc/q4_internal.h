@@ -37,6 +37,15 @@ cudaError_t umma_launch(int act_dtype, int m_pad, const GemmParams& p, int smem_
 int umma_stages(int m_pad, int smem_bytes);
 size_t umma_slot_bytes(int m_pad);
 
+// fp32-activation GEMM on the CUDA cores, M <= 16 (q4_simt.cu): padded M,
+// rows per work unit (units are 512 k wide) and warps per CTA.
+struct SimtShape {
+    int m_pad, rows, warps;
+};
+SimtShape simt_shape(int M);
+size_t simt_smem_bytes();
+cudaError_t simt_launch(const SimtShape& sh, int ctas, const GemmParams& p, int log2_bs, cudaStream_t stream);
+
 cudaError_t quantize_launch(const void* W, int w_dtype, int64_t n, int blocksize, const float* code,
                             uint8_t* packed, float* absmax, cudaStream_t stream);
 cudaError_t dequantize_launch(const uint8_t* packed, const float* absmax, const float* code, int64_t n,

@@ -1,0 +1,461 @@
+// q4_simt.cu -- fused blockwise 4-bit dequantize + skinny GEMM with fp32
+// activations, on the CUDA cores, for sm_100a:
+//
+//     out[m, n] = [bias[n]] + sum_k A[m, k] * code[idx(n, k)] * absmax(n, k)
+//     M <= 16, A / out / bias fp32.
+//
+// The maintainer's reply in bitsandbytes PR #1920 ("[ROCm] Optimize
+// kgemm_4bit_inference_naive ...") describes the replacement kernels: the
+// tensor-core versions take fp16/bf16, the SIMT kernel also takes fp32, and
+// all accumulate in fp32.  This is that fp32 case.  Every product is an fp32
+// FMA of the activation with the exact fp32 code value; nothing is rounded
+// to 16 bits.
+//
+// Design for B200:
+//  * HBM-bound at M = 1 (0.5625 B per weight at blocksize 64), so the code
+//    bytes stream through registers with coalesced 4-byte loads per lane and
+//    row (128 B per warp instruction), the next unit in flight while one is
+//    computed.  (Deeper register rings with fewer warps measured slower: the
+//    loop is bound by instruction latency, which more warps hide better.)
+//  * Dequantization is one shared-memory lookup per packed BYTE: a 256-row
+//    table maps a byte to the float2 (code[hi], code[lo]).  Each 256-B row
+//    holds 16 copies of the pair, one per bank pair, so a half-warp's 64-bit
+//    lookups never conflict; the table sits on a 64 KiB boundary of the
+//    shared window, so one byte-permute turns a packed word into the lookup
+//    address (table base | byte << 8 | copy << 3).
+//  * A lane covers 8 consecutive k of a row in each 256-k group: the 8
+//    weights lie in one absmax block (blocksize >= 32), so the block scale is
+//    applied once per 8 products (acc += absmax * t).
+//  * Work units of R rows x 512 k are split evenly over all warps of the grid
+//    (stream-K at warp granularity): every warp streams the same number of
+//    weight bytes to within one unit.  A row group cut by a warp boundary is
+//    combined deterministically through the GEMM workspace: each piece is
+//    published with a release add on the group's counter, and the last
+//    arriver sums the pieces in warp order.  No thread ever waits on another.
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "q4_device.cuh"
+#include "q4_internal.h"
+#include "q4_plan.cuh"
+
+namespace q4 {
+namespace simt {
+
+static constexpr int kUnitK = 512;                    // k-width of a work unit (two 256-k groups)
+static constexpr uint32_t kTableBytes = 256u * 256u;  // 256 rows of 256 B (lower 128 B used)
+static constexpr size_t kSmemBytes = 65536u + kTableBytes;  // + padding to a 64 KiB boundary
+
+struct Params {
+    const float* A;        // [M, K]
+    const uint8_t* Wp;     // [N, K/2]
+    const float* absmax;   // [N * K / blocksize]
+    const float* code;     // [16]
+    float* out;            // [M, N]
+    const float* bias;     // [N] or nullptr
+    float* partials;       // [warps][2][R * MP]
+    int* counters;         // [row groups], zero between calls
+    int M, N, K;
+    int lbs;               // log2(blocksize)
+    int ku;                // units per row group: ceil(K / 512)
+    int row_groups;
+    int pdl;               // 0, 1: wait before any global access; 2: code/weights/absmax first
+    uint32_t units;        // row_groups * ku
+    uint32_t warps;        // grid warps
+    int narrow;            // units * warps < 2^32: the partition in 32-bit arithmetic
+    int a32;               // A is 32-byte aligned: 256-bit activation loads
+};
+
+// First unit of part `p` when `total` units are split into `parts` ranges,
+// and the part owning unit `u` (the formulas of q4_partition_start/_owner).
+// `narrow`: total * parts < 2^32, so 32-bit arithmetic is exact.
+__host__ __device__ __forceinline__ uint32_t wpart_start(uint32_t total, uint32_t parts, uint32_t p, bool narrow) {
+    return narrow ? (total * p) / parts : (uint32_t)(((uint64_t)total * p) / parts);
+}
+__host__ __device__ __forceinline__ uint32_t wpart_owner(uint32_t total, uint32_t parts, uint32_t u, bool narrow) {
+    return narrow ? ((u + 1) * parts - 1) / total : (uint32_t)((((uint64_t)u + 1) * parts - 1) / total);
+}
+
+// The loads below read data that no thread writes while the kernel runs (the
+// table is complete before the first lookup), so they are plain asm the
+// compiler may schedule freely.  Float pairs travel as 64-bit registers
+// (first value in the low half), the operand form of fma.rn.f32x2.
+__device__ __forceinline__ uint64_t lds_pair(uint32_t addr) {
+    uint64_t v;
+    asm("ld.shared.b64 %0, [%1];" : "=l"(v) : "r"(addr));
+    return v;
+}
+
+// Four consecutive floats as two pairs (16-byte aligned).
+__device__ __forceinline__ void ldg_pairs(const float* p, uint64_t& lo, uint64_t& hi) {
+    asm("ld.global.nc.v2.b64 {%0, %1}, [%2];" : "=l"(lo), "=l"(hi) : "l"(p));
+}
+
+// Eight consecutive floats as four pairs in one 256-bit load (32-byte aligned).
+__device__ __forceinline__ void ldg_pairs8(const float* p, uint64_t (&v)[4]) {
+    asm("ld.global.nc.v4.b64 {%0, %1, %2, %3}, [%4];" : "=l"(v[0]), "=l"(v[1]), "=l"(v[2]), "=l"(v[3]) : "l"(p));
+}
+
+__device__ __forceinline__ uint32_t ldg_code_word(const uint8_t* p) {
+    uint32_t v;
+    asm("ld.global.nc.L1::no_allocate.b32 %0, [%1];" : "=r"(v) : "l"(p));
+    return v;
+}
+
+__device__ __forceinline__ float ldg_scale(const float* p) {
+    float v;
+    asm("ld.global.nc.L1::no_allocate.f32 %0, [%1];" : "=f"(v) : "l"(p));
+    return v;
+}
+
+// An opaque copy of `v`: values derived from it cannot be computed before
+// this point of the program (an ordering fence for the plain-asm loads).
+template <typename V>
+__device__ __forceinline__ void launder(V& v) {
+    static_assert(sizeof(V) == 4 || sizeof(V) == 8, "32- or 64-bit values");
+    if constexpr (sizeof(V) == 8)
+        asm volatile("" : "+l"(v)::"memory");
+    else
+        asm volatile("" : "+r"(v)::"memory");
+}
+
+// d = a * b on both halves, each rounded once.
+__device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+
+// d = a * b + c on both halves, each an fp32 FMA rounded once.
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+__device__ __forceinline__ float lo_f32(uint64_t v) { return __uint_as_float((uint32_t)v); }
+__device__ __forceinline__ float hi_f32(uint64_t v) { return __uint_as_float((uint32_t)(v >> 32)); }
+
+// Byte BYTE of `word` -> the table pair (code[hi nibble], code[lo nibble]) of
+// that byte, from this lane's copy.
+template <int BYTE>
+__device__ __forceinline__ uint64_t pair_of(uint32_t word, uint32_t lane8) {
+    // result bytes: [0] = lane8.b0 (copy * 8), [1] = word.b<BYTE>, [2..3] = table base >> 16
+    return lds_pair(prmt<0x7604u | (BYTE << 4)>(word, lane8));
+}
+
+// One unit's streamed operands for one lane: the packed word of each row for
+// both 256-k groups, and the absmax of the block each word lies in.
+template <int R>
+struct UnitRegs {
+    uint32_t w[R][2];
+    float am[R][2];
+};
+
+template <int MP, int R, int NW, int D>
+__global__ void __launch_bounds__(NW * 32, 1) q4_gemm_f32_kernel(const Params p) {
+    extern __shared__ __align__(16) uint8_t smem[];
+    const uint32_t sbase = smem_addr(smem);
+    const uint32_t table = (sbase + 0xFFFFu) & ~0xFFFFu;  // 64 KiB aligned (the host reserves the padding)
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    uint32_t lane8 = table | ((uint32_t)(lane & 15) << 3);
+    const uint8_t* Wp = p.Wp;
+    const float* absmax = p.absmax;
+    const float* Aact = p.A;
+
+    if (p.pdl != 2) griddep_wait();
+    // The loads are plain asm the compiler may move: each one takes its
+    // address from a value laundered after the point it must follow.
+    launder(Wp);
+    launder(absmax);
+    // Table: row b = 16 copies of (code[b >> 4], code[b & 15]); the pair is
+    // gathered by shuffles from one global load per thread.
+    {
+        const float cv = __ldg(p.code + (lane & 15));
+        for (int e = tid; e < 256 * 8; e += NW * 32) {
+            const int b = e >> 3;
+            const float hi = __shfl_sync(0xffffffffu, cv, b >> 4);
+            const float lo = __shfl_sync(0xffffffffu, cv, b & 15);
+            sts_v4(table + (uint32_t)b * 256u + (uint32_t)(e & 7) * 16u, __float_as_uint(hi), __float_as_uint(lo),
+                   __float_as_uint(hi), __float_as_uint(lo));
+        }
+    }
+
+    const uint32_t gw = blockIdx.x * NW + warp;
+    const bool narrow = p.narrow != 0;
+    auto start_of = [&](uint32_t w) { return wpart_start(p.units, p.warps, w, narrow); };
+    const uint32_t ws = start_of(gw), we = start_of(gw + 1);
+    const size_t row_bytes = (size_t)p.K >> 1;
+    const int am_row = p.K >> p.lbs;
+
+    // Position of a unit: row group and unit column inside it.
+    struct Cursor {
+        uint32_t rg;
+        int kc;
+    };
+    auto advance = [&](Cursor& c) {
+        if (++c.kc == p.ku) {
+            c.kc = 0;
+            ++c.rg;
+        }
+    };
+    Cursor lc{0u, 0}, cc{0u, 0};
+    if (ws < we) {
+        lc.rg = cc.rg = ws / (uint32_t)p.ku;
+        lc.kc = cc.kc = (int)(ws - lc.rg * (uint32_t)p.ku);
+    }
+
+    // Streams the packed words and absmax of the unit at `c` into `x` (rows
+    // past N and groups past K read nothing).
+    auto load = [&](const Cursor& c, UnitRegs<R>& x) {
+        const int n0 = (int)c.rg * R;
+        const int kq = c.kc * kUnitK + 8 * lane;  // this lane's first k in the unit (group q adds 256 q)
+        const int a0 = kq >> p.lbs, a1 = (kq + 256) >> p.lbs;
+        const uint8_t* wb = Wp + (size_t)n0 * row_bytes + (kq >> 1);
+        const float* ab = absmax + (size_t)n0 * am_row + a0;
+        const int da = a1 - a0;
+        const bool k0ok = kq < p.K, k1ok = kq + 256 < p.K;
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+            const bool nok = n0 + r < p.N;
+            // R rows of K/2 bytes stay below 2^32 bytes (K < 2^29): 32-bit row offsets
+            const uint8_t* wr = wb + (uint32_t)r * (uint32_t)row_bytes;
+            const float* ar = ab + (uint32_t)r * (uint32_t)am_row;
+            x.w[r][0] = (nok && k0ok) ? ldg_code_word(wr) : 0u;
+            x.am[r][0] = (nok && k0ok) ? ldg_scale(ar) : 0.f;
+            x.w[r][1] = (nok && k1ok) ? ldg_code_word(wr + 128) : 0u;
+            x.am[r][1] = (nok && k1ok) ? ldg_scale(ar + da) : 0.f;
+        }
+    };
+
+    // A ring of D register buffers: D - 1 units in flight while one is computed.
+    UnitRegs<R> xb[D];
+#pragma unroll
+    for (int i = 0; i < D - 1; ++i)
+        if (ws + i < we) {
+            load(lc, xb[i]);
+            advance(lc);
+        }
+    __syncthreads();  // the table is complete
+    launder(lane8);   // every lookup address derives from lane8: none moves above the barrier
+    // Activations, outputs and the workspace may belong to the preceding
+    // grid: touch them only after the dependency wait.
+    if (p.pdl == 2) griddep_wait();
+    launder(Aact);  // activations only after the dependency wait
+    griddep_launch_dependents();
+    if (ws >= we) return;
+
+    float acc[R][MP];
+#pragma unroll
+    for (int r = 0; r < R; ++r)
+#pragma unroll
+        for (int m = 0; m < MP; ++m) acc[r][m] = 0.f;
+
+    // acc += this lane's share of the unit at `c`: per 256-k group, 8
+    // consecutive k of every row, scaled once by that block's absmax.
+    auto compute = [&](const Cursor& c, const UnitRegs<R>& x) {
+        const int k0 = c.kc * kUnitK;
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+            const int kq = k0 + 256 * q + 8 * lane;
+            if (kq >= p.K) continue;  // only in the last unit of a row, K % 512 != 0
+            // The 8 activations of every row m: pairs (k, k+1), (k+2, k+3), ...
+            uint64_t a[MP][4];
+#pragma unroll
+            for (int m = 0; m < MP; ++m) {
+                if (m < p.M) {
+                    const float* src = Aact + (size_t)m * p.K + kq;
+                    if (p.a32) {
+                        ldg_pairs8(src, a[m]);
+                    } else {
+                        ldg_pairs(src, a[m][0], a[m][1]);
+                        ldg_pairs(src + 4, a[m][2], a[m][3]);
+                    }
+                } else {
+                    a[m][0] = a[m][1] = a[m][2] = a[m][3] = 0ull;
+                }
+            }
+            // Two running sums per (row, m): even and odd k of the pairs.
+            uint64_t t[R][MP];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {  // byte j of the word: k = kq + 2j, kq + 2j + 1
+#pragma unroll
+                for (int r = 0; r < R; ++r) {
+                    const uint64_t cp = j == 0   ? pair_of<0>(x.w[r][q], lane8)
+                                        : j == 1 ? pair_of<1>(x.w[r][q], lane8)
+                                        : j == 2 ? pair_of<2>(x.w[r][q], lane8)
+                                                 : pair_of<3>(x.w[r][q], lane8);
+#pragma unroll
+                    for (int m = 0; m < MP; ++m) t[r][m] = j == 0 ? mul2(a[m][0], cp) : fma2(a[m][j], cp, t[r][m]);
+                }
+            }
+#pragma unroll
+            for (int r = 0; r < R; ++r)
+#pragma unroll
+                for (int m = 0; m < MP; ++m) {
+                    acc[r][m] = fmaf(x.am[r][q], lo_f32(t[r][m]), acc[r][m]);
+                    acc[r][m] = fmaf(x.am[r][q], hi_f32(t[r][m]), acc[r][m]);
+                }
+        }
+    };
+
+    // Output element e = m * R + r of row group rg (lane e % 32 writes it).
+    auto store = [&](uint32_t rg, int e, float v) {
+        const int r = e % R, m = e / R;
+        const int n = (int)rg * R + r;
+        if (n < p.N && m < p.M) p.out[(size_t)m * p.N + n] = p.bias ? v + p.bias[n] : v;
+    };
+    constexpr int RM = R * MP;
+
+    // Closes row group `rg` after this warp's last unit of it.
+    auto finish = [&](uint32_t rg) {
+        // Sum over lanes; the butterfly leaves the same total in every lane
+        // (each step adds the same two values, in either order).
+#pragma unroll
+        for (int r = 0; r < R; ++r)
+#pragma unroll
+            for (int m = 0; m < MP; ++m) {
+                float v = acc[r][m];
+#pragma unroll
+                for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+                acc[r][m] = v;
+            }
+        const uint32_t g0 = rg * (uint32_t)p.ku, g1 = g0 + (uint32_t)p.ku;
+        if (ws <= g0 && we >= g1) {  // the whole group is this warp's
+#pragma unroll
+            for (int e = 0; e < RM; ++e)
+                if ((e & 31) == lane) store(rg, e, acc[e % R][e / R]);
+        } else {
+            // Publish this warp's piece (slot 0: the group is the range's
+            // first; 1: its last) and count it in.
+            const uint32_t slot = ws >= g0 ? 0u : 1u;
+            float* mine = p.partials + ((size_t)gw * 2 + slot) * RM;
+#pragma unroll
+            for (int e = 0; e < RM; ++e)
+                if ((e & 31) == lane) mine[e] = acc[e % R][e / R];
+            __syncwarp();
+            int prev = 0;
+            if (lane == 0) prev = atom_add_acq_rel_gpu(p.counters + rg, 1);
+            prev = __shfl_sync(0xffffffffu, prev, 0);
+            __syncwarp();
+            // Contributors: the warps whose ranges meet the group.  With more
+            // warps than units some ranges are empty; they own no unit and
+            // publish nothing.
+            const uint32_t cf = wpart_owner(p.units, p.warps, g0, narrow);
+            const uint32_t cl = wpart_owner(p.units, p.warps, g1 - 1, narrow);
+            uint32_t pieces = 0;
+            for (uint32_t c = cf, c0 = start_of(cf); c <= cl; ++c) {
+                const uint32_t c1 = start_of(c + 1);
+                pieces += c0 != c1 ? 1u : 0u;
+                c0 = c1;
+            }
+            if ((uint32_t)prev + 1u == pieces) {  // last to arrive: sum the pieces in warp order
+                // lane e (and e + 32) sums output element e over the pieces
+                float v0 = 0.f, v1 = 0.f;
+                for (uint32_t c = cf, c0 = start_of(cf); c <= cl; ++c) {
+                    const uint32_t c1 = start_of(c + 1);
+                    if (c0 != c1) {
+                        const float* src = p.partials + ((size_t)c * 2 + (c0 >= g0 ? 0u : 1u)) * RM;
+                        if (lane < RM) v0 += ldg_cg_f32(src + lane);
+                        if (RM > 32 && lane + 32 < RM) v1 += ldg_cg_f32(src + lane + 32);
+                    }
+                    c0 = c1;
+                }
+                if (lane < RM) store(rg, lane, v0);
+                if (RM > 32 && lane + 32 < RM) store(rg, lane + 32, v1);
+                if (lane == 0) p.counters[rg] = 0;  // back to zero for the next call
+            }
+        }
+#pragma unroll
+        for (int r = 0; r < R; ++r)
+#pragma unroll
+            for (int m = 0; m < MP; ++m) acc[r][m] = 0.f;
+    };
+    auto step = [&](const UnitRegs<R>& x, bool last_of_range) {
+        compute(cc, x);
+        if (cc.kc == p.ku - 1 || last_of_range) finish(cc.rg);
+        advance(cc);
+    };
+
+    // Unit u sits in buffer (u - ws) % D; before it is computed the loads of
+    // unit u + D - 1 go into the buffer computed last.  The loop is unrolled
+    // D times so that every buffer index is a compile-time constant.
+    for (uint32_t u = ws; u < we; u += D) {
+#pragma unroll
+        for (int i = 0; i < D; ++i) {
+            if (u + i >= we) break;
+            if (u + i + D - 1 < we) {
+                load(lc, xb[(i + D - 1) % D]);
+                advance(lc);
+            }
+            step(xb[i], u + i + 1 == we);
+        }
+    }
+}
+
+// Compiled variants: MP = padded M, R = rows per unit, NW = warps per CTA,
+// D = register buffers per warp.
+template <int MP, int R, int NW, int D>
+static cudaError_t launch_variant(const Params& p, int ctas, cudaStream_t stream) {
+    auto kern = q4_gemm_f32_kernel<MP, R, NW, D>;
+    cudaError_t e = ensure_smem_attr((const void*)kern, kSmemBytes);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)ctas);
+    cfg.blockDim = dim3(NW * 32);
+    cfg.dynamicSmemBytes = kSmemBytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = p.pdl ? 1 : 0;
+    e = cudaLaunchKernelEx(&cfg, kern, p);
+    if (e != cudaSuccess) return e;
+    return cudaGetLastError();
+}
+
+}  // namespace simt
+
+// Launch-table shape of the fp32 kernel for a padded M.
+SimtShape simt_shape(int M) {
+    if (M <= 1) return {1, 8, 16};
+    if (M <= 2) return {2, 8, 8};
+    if (M <= 4) return {4, 8, 8};
+    if (M <= 8) return {8, 4, 8};
+    return {16, 2, 8};
+}
+
+size_t simt_smem_bytes() { return simt::kSmemBytes; }
+
+cudaError_t simt_launch(const SimtShape& sh, int ctas, const GemmParams& g, int log2_bs, cudaStream_t stream) {
+    simt::Params p{};
+    p.A = static_cast<const float*>(g.A);
+    p.Wp = g.Wp;
+    p.absmax = g.absmax;
+    p.code = g.code;
+    p.out = static_cast<float*>(g.out);
+    p.bias = static_cast<const float*>(g.bias);
+    p.partials = g.partials;
+    p.counters = g.counters;
+    p.M = g.M;
+    p.N = g.N;
+    p.K = g.K;
+    p.lbs = log2_bs;
+    p.ku = (g.K + simt::kUnitK - 1) / simt::kUnitK;
+    p.row_groups = (g.N + sh.rows - 1) / sh.rows;
+    p.pdl = g.pdl;
+    p.units = (uint32_t)((uint64_t)p.row_groups * (uint64_t)p.ku);
+    p.warps = (uint32_t)ctas * (uint32_t)sh.warps;
+    p.narrow = (uint64_t)p.units * p.warps < ((uint64_t)1 << 32) ? 1 : 0;
+    p.a32 = (reinterpret_cast<uintptr_t>(g.A) & 31u) == 0 ? 1 : 0;
+    switch (sh.m_pad) {
+        case 1: return simt::launch_variant<1, 8, 16, 2>(p, ctas, stream);
+        case 2: return simt::launch_variant<2, 8, 8, 2>(p, ctas, stream);
+        case 4: return simt::launch_variant<4, 8, 8, 2>(p, ctas, stream);
+        case 8: return simt::launch_variant<8, 4, 8, 2>(p, ctas, stream);
+        case 16: return simt::launch_variant<16, 2, 8, 2>(p, ctas, stream);
+        default: return cudaErrorInvalidConfiguration;
+    }
+}
+
+}  // namespace q4

@@ -93,7 +93,7 @@ def activations_fp32(M: int, K: int, seed: int) -> np.ndarray:
 
 def activations(M: int, K: int, dtype: torch.dtype, seed: int) -> torch.Tensor:
     """A ~ N(0, 1) drawn in fp32 and rounded (RNE, torch's conversion) to
-    ``dtype`` (bf16 or fp16); a CPU tensor of shape [M, K]."""
+    ``dtype`` (bf16 or fp16; fp32 keeps the draws); a CPU tensor of shape [M, K]."""
     return torch.from_numpy(activations_fp32(M, K, seed)).to(dtype)
 
 
@@ -151,16 +151,18 @@ class Case:
     N: int
     K: int
     blocksize: int = 64
-    act: str = "bf16"          # "bf16" | "fp16"
+    act: str = "bf16"          # "bf16" | "fp16" | "fp32"
     table: str = "normal"      # "normal" | "uniform"
     outliers: bool = False
     tag: str = ""
 
     def algorithmic_bytes(self) -> int:
-        """M*K*2 + N*K/2 + 4*N*K/bs + M*N*2 (activations, codes, absmax, out)."""
+        """M*K*e + N*K/2 + 4*N*K/bs + M*N*e (activations, codes, absmax, out;
+        e = 2 bytes for bf16/fp16 activations, 4 for fp32)."""
         nk = self.N * self.K
-        return self.M * self.K * 2 + nk // 2 + 4 * ((nk + self.blocksize - 1) // self.blocksize) \
-            + self.M * self.N * 2
+        e = 4 if self.act == "fp32" else 2
+        return self.M * self.K * e + nk // 2 + 4 * ((nk + self.blocksize - 1) // self.blocksize) \
+            + self.M * self.N * e
 
 
 @dataclass
@@ -212,6 +214,18 @@ def workloads() -> dict:
         for M in (17, 32, 64, 128):
             big.append(Case(M, N, K, tag=f"K{K}N{N}M{M}"))
     w["mlarge"] = Workload("M 17,32,64,128 on K5120/N5120, K5120/N8192, K17408/N5120 (tcgen05 kernel)", 6, big)
+    # Beyond the five: fp32 activations (the CUDA-core kernel) on the decode
+    # shapes at M=1 and on the M sweep's shapes.
+    w["decode70b_f32"] = Workload(
+        "M=1 decode shapes of a 70B-class layer (K8192/N10240, K8192/N28672, K28672/N8192, K8192/N8192), "
+        "bs64 fp32 activations, normal-table", 7,
+        [Case(1, 10240, 8192, act="fp32", tag="qkv"), Case(1, 28672, 8192, act="fp32", tag="gate_up"),
+         Case(1, 8192, 28672, act="fp32", tag="down"), Case(1, 8192, 8192, act="fp32", tag="o_proj")])
+    f32 = []
+    for (K, N) in ((5120, 5120), (17408, 5120)):
+        for M in (1, 2, 4, 8, 16):
+            f32.append(Case(M, N, K, act="fp32", tag=f"K{K}N{N}M{M}"))
+    w["msweep_f32"] = Workload("fp32 activations, M 1,2,4,8,16 on K5120/N5120, K17408/N5120", 8, f32)
     # Not one of the five: one long-K layer whose launch is almost all main
     # loop (start-up and tail are a few percent), for profiling the loop.
     w["longk"] = Workload("M=1 K=131072 N=8192 bs64 bf16 normal-table (main-loop profiling shape)", 5,

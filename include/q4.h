@@ -120,17 +120,24 @@ int q4_gemm_workspace_size(int M, int N, int K, int blocksize, int act_dtype, si
  * Fused dequantize + skinny matmul (PR #1920's kgemm_4bit_inference_naive
  * generalised to M > 1, "Fused path support for M > 1"):
  *     out[m, n] = round_rn_act( sum_k A[m,k] * code[idx(n,k)] * absmax(n,k) )
- * accumulated in fp32 (codes enter the tensor-core contraction rounded to
- * the activation dtype; the per-block absmax scale is applied in fp32).
+ * accumulated in fp32.  bf16/fp16: codes enter the tensor-core contraction
+ * rounded to the activation dtype and the per-block absmax scale is applied
+ * in fp32.  fp32 (the reply's SIMT kernel, which also takes fp32 inputs):
+ * every product is an fp32 FMA with the exact fp32 code, scaled in fp32.
  *   A        [M, K] act_dtype, row-major contiguous, 16-byte aligned
  *   Wpacked  uint8 [N*K/2] (rows of K/2 bytes), 16-byte aligned
  *   absmax   fp32 [N*K/blocksize], 4-byte aligned
  *   code     fp32 [16], 4-byte aligned
- *   M        0..16 (0 is a no-op; > 16 -> Q4_ERR_UNSUPPORTED)
+ *   M        0 is a no-op.  bf16/fp16: 1..16 on the mma.sync kernels;
+ *            17..128 on the tcgen05 (tensor-memory) kernel, which also
+ *            needs blocksize >= 64, K % 256 == 0, (K / blocksize) % 4 == 0
+ *            (else Q4_ERR_UNSUPPORTED) and a 16-byte aligned absmax (else
+ *            Q4_ERR_MISALIGNED).  fp32: 1..16.  Larger M ->
+ *            Q4_ERR_UNSUPPORTED (the caller's cue for dequantize + GEMM).
  *   N, K     >= 0; K % blocksize == 0 (else Q4_ERR_UNSUPPORTED); N = 0 is
  *            a no-op; K = 0 writes zeros
  *   blocksize  power of two in [32, 4096]
- *   act_dtype  Q4_BF16 or Q4_FP16 (Q4_FP32 -> Q4_ERR_UNSUPPORTED)
+ *   act_dtype  Q4_BF16, Q4_FP16 or Q4_FP32
  *   out      [M, N] act_dtype, row-major, 16-byte aligned
  *   workspace  device scratch of at least q4_gemm_workspace_size() bytes,
  *            16-byte aligned, ZERO-FILLED before its first use.  Layout: a
@@ -179,8 +186,11 @@ int q4_gemm_skinny_noalloc(const void* A, const uint8_t* Wpacked, const float* a
  * tests).  `num_sms` <= 0 means "the current device's SM count". */
 typedef struct {
     int math;          /* 1 = tensor-core (mma.sync m16n8k16), 2 = CUDA-core FMA  */
-    int sub_block;     /* k-width of one work unit: min(blocksize, 64)            */
-    int m_pad;         /* M padded to the MMA column count: 8 or 16               */
+                       /* (fp32 activations), 3 = tcgen05 with tensor memory     */
+    int sub_block;     /* k-width of one work unit: min(blocksize, 64); 512 for  */
+                       /* math 2                                                 */
+    int m_pad;         /* M padded to the MMA column count: 8 or 16 (math 1),   */
+                       /* 32/64/128 (math 3), 1/2/4/8/16 (math 2)                */
     int rows_per_tile; /* weight rows per work unit                               */
     int warps;         /* warps per CTA                                           */
     int ctas;          /* persistent CTAs (<= SM count, <= number of units)       */
@@ -221,7 +231,8 @@ int q4_gemm_skinny_ex(const void* A, const uint8_t* Wpacked, const float* absmax
  * bitsandbytes PR #1920, "Technical details", takes an optional bias):
  *     out[m, n] = round_rn_act( bias[n] + sum_k A[m,k] * dequant(W)[n,k] )
  * the bias added in fp32 to the fp32 sum before the single rounding.
- *   bias       [N] act_dtype, 2-byte aligned, not NULL when M, N > 0 (use
+ *   bias       [N] act_dtype, aligned to its element size (2 or 4 bytes),
+ *              not NULL when M, N > 0 (use
  *              q4_gemm_skinny for no bias); with K = 0 every output row is
  *              the bias.
  *   overrides  as for q4_gemm_skinny_ex (NULL: the launch table decides).

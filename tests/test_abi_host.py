@@ -72,7 +72,7 @@ def test_gemm_validation_before_cuda():
     # (M, N, K, bs, dtype) -> status; all decided before the device is queried
     cases = {(129, 64, 4096, 64, 0): b.Q4_ERR_UNSUPPORTED,
              (1, 64, 4000, 64, 0): b.Q4_ERR_UNSUPPORTED,
-             (1, 64, 4096, 64, 2): b.Q4_ERR_UNSUPPORTED,
+             (17, 64, 4096, 64, 2): b.Q4_ERR_UNSUPPORTED,   # fp32 activations: M <= 16
              (-1, 64, 4096, 64, 0): b.Q4_ERR_INVALID_ARG,
              (1, -5, 4096, 64, 0): b.Q4_ERR_INVALID_ARG,
              (1, 64, 4096, 96, 0): b.Q4_ERR_INVALID_ARG,
@@ -105,11 +105,61 @@ def test_launch_table_tcgen05(M, N, K):
     assert p["workspace_bytes"] == 256 + 148 * 2 * 4096 + -(-tiles * 4 // 256) * 256 + slots
 
 
+@pytest.mark.parametrize("M,N,K,bs", [(1, 8192, 28672, 64), (2, 300, 1024, 32), (3, 61, 1088, 64),
+                                      (5, 10240, 8192, 64), (12, 1, 32, 32), (16, 5120, 16384, 4096)])
+def test_launch_table_f32(M, N, K, bs):
+    """fp32 activations: the CUDA-core kernel, units of R rows x 512 k."""
+    import torch
+    p = b.q4_gemm_plan(M, N, K, bs, act_dtype=torch.float32, num_sms=148)
+    mp = 1 if M == 1 else 2 if M == 2 else 4 if M <= 4 else 8 if M <= 8 else 16
+    assert p["math"] == 2 and p["sub_block"] == 512 and p["m_pad"] == mp and p["loader"] == 1
+    R = p["rows_per_tile"]
+    assert p["tiles"] == -(-N // R) and p["units"] == p["tiles"] * -(-K // 512)
+    assert 1 <= p["ctas"] <= 148 and (p["ctas"] - 1) * p["warps"] < p["units"]
+    # the pieces of every warp fit the fixed partial region: 2 slots of R x MP floats
+    assert p["ctas"] * p["warps"] * 2 * R * mp * 4 <= 148 * 2 * 4096
+    want_ws = 0 if p["units"] == 1 else 256 + 148 * 2 * 4096 + -(-p["tiles"] * 4 // 256) * 256
+    assert p["workspace_bytes"] == want_ws
+
+
+@pytest.mark.parametrize("M,N,K,ctas", [(1, 64, 16384, 0), (4, 24, 32768, 0), (2, 1000, 4096, 3), (1, 8, 512, 0),
+                                        (16, 130, 8192, 5), (8, 9, 65536, 0), (1, 8192, 28672, 0)])
+def test_f32_piece_bookkeeping(M, N, K, ctas):
+    """The fp32 kernel's row-group pieces, replayed on the host with the
+    exported partition: each (warp, slot) holds at most one group's piece,
+    and the warps the finaliser sums (the non-empty ranges meeting the group,
+    slot 0 where the group is the range's first) are exactly the writers."""
+    import torch
+    L = b.lib()
+    p = b.q4_gemm_plan(M, N, K, 64, act_dtype=torch.float32, num_sms=148)
+    ku, U = -(-K // 512), p["units"]
+    W = (min(ctas, p["ctas"]) if ctas else p["ctas"]) * p["warps"]
+    start = [L.q4_partition_start(U, W, w) for w in range(W + 1)]
+    used = {}
+    for w in range(W):
+        ws, we = start[w], start[w + 1]
+        for g in range(ws // ku, (we - 1) // ku + 1) if ws < we else ():
+            g0, g1 = g * ku, g * ku + ku
+            if ws <= g0 and we >= g1:
+                continue
+            key = (w, 0 if ws >= g0 else 1)
+            assert key not in used
+            used[key] = g
+    by_group = {}
+    for key, g in used.items():
+        by_group.setdefault(g, []).append(key)
+    for g in range(p["tiles"]):
+        g0, g1 = g * ku, g * ku + ku
+        cf, cl = L.q4_partition_owner(U, W, g0), L.q4_partition_owner(U, W, g1 - 1)
+        summed = [(c, 0 if start[c] >= g0 else 1) for c in range(cf, cl + 1) if start[c] != start[c + 1]]
+        assert sorted(by_group.get(g, [])) == (summed if len(summed) > 1 else [])
+
+
 @pytest.mark.parametrize("wl", list(inputs.workloads()))
 def test_launch_table_invariants(wl):
     for c in inputs.workloads()[wl].cases:
-        if c.M > 16:
-            continue  # the tensor-memory kernel's table: test_launch_table_tcgen05
+        if c.M > 16 or c.act == "fp32":
+            continue  # tensor-memory and fp32 tables: test_launch_table_tcgen05, test_launch_table_f32
         p = b.q4_gemm_plan(c.M, c.N, c.K, c.blocksize, num_sms=148)
         assert p["math"] == 1
         assert p["sub_block"] == min(c.blocksize, 64)
