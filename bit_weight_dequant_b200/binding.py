@@ -20,6 +20,7 @@ HEADER = os.path.join(os.path.dirname(_HERE), "include", "q4.h")
 
 Q4_OK, Q4_ERR_INVALID_ARG, Q4_ERR_UNSUPPORTED, Q4_ERR_MISALIGNED, Q4_ERR_CUDA, Q4_ERR_WORKSPACE = range(6)
 Q4_BF16, Q4_FP16, Q4_FP32 = 0, 1, 2
+Q4_ROUTE_FUSED, Q4_ROUTE_SPLIT = 0, 1
 
 _TORCH_TO_Q4 = {torch.bfloat16: Q4_BF16, torch.float16: Q4_FP16, torch.float32: Q4_FP32}
 _Q4_TO_TORCH = {v: k for k, v in _TORCH_TO_Q4.items()}
@@ -62,12 +63,13 @@ def lib() -> ctypes.CDLL:
         L.q4_gemm_skinny_noalloc.argtypes = [P, P, P, P, ci, ci, ci, ci, ci, P, P]
         L.q4_gemm_skinny_bias.argtypes = [P, P, P, P, P, ci, ci, ci, ci, ci, P, P, sz, P,
                                           ctypes.POINTER(q4_gemm_plan_t)]
+        L.q4_gemm_route.argtypes = [ci, ci, ci, ci, ci, ctypes.POINTER(ci)]
         L.q4_partition_start.argtypes = [i64, ci, ci]
         L.q4_partition_start.restype = i64
         L.q4_partition_owner.argtypes = [i64, ci, i64]
         for f in ("q4_quantize_blockwise", "q4_quantize_blockwise_ex", "q4_dequantize_blockwise", "q4_gemm_workspace_size",
                   "q4_gemm_skinny", "q4_gemm_skinny_ex", "q4_gemm_plan", "q4_partition_owner",
-                  "q4_gemm_skinny_noalloc", "q4_gemm_skinny_bias"):
+                  "q4_gemm_skinny_noalloc", "q4_gemm_skinny_bias", "q4_gemm_route"):
             getattr(L, f).restype = ci
         _lib = L
     return _lib
@@ -254,3 +256,33 @@ def q4_gemm_skinny_noalloc(A: torch.Tensor, Wpacked: torch.Tensor, absmax: torch
                                       _TORCH_TO_Q4[A.dtype], _ptr(out), _stream(A.device))
     _check(rc, "q4_gemm_skinny_noalloc")
     return out
+
+
+@functools.lru_cache(maxsize=1024)
+def _route(M: int, N: int, K: int, blocksize: int, act: int) -> int:
+    r = ctypes.c_int(-1)
+    _check(lib().q4_gemm_route(M, N, K, blocksize, act, ctypes.byref(r)), "q4_gemm_route")
+    return r.value
+
+
+def q4_gemm_route(M: int, N: int, K: int, blocksize: int, act_dtype: torch.dtype = torch.bfloat16) -> int:
+    """Q4_ROUTE_FUSED or Q4_ROUTE_SPLIT: the library's fused-vs-split choice (see q4.h)."""
+    return _route(M, N, K, blocksize, _TORCH_TO_Q4[act_dtype])
+
+
+def q4_linear(A: torch.Tensor, Wpacked: torch.Tensor, absmax: torch.Tensor, code: torch.Tensor, N: int, K: int,
+              blocksize: int, bias: torch.Tensor | None = None, out: torch.Tensor | None = None,
+              workspace: Workspace | None = None) -> torch.Tensor:
+    """out = A . dequant(W)^T (+ bias) on the path q4_gemm_route picks: the
+    fused kernel, or this library's dequantize into a temporary dense matrix
+    followed by a cuBLAS GEMM (torch.matmul / torch.addmm)."""
+    M = A.shape[0] if A.dim() == 2 else 1
+    if q4_gemm_route(M, N, K, blocksize, A.dtype) == Q4_ROUTE_FUSED:
+        return q4_gemm_skinny(A, Wpacked, absmax, code, N, K, blocksize, out=out, workspace=workspace, bias=bias)
+    W = q4_dequantize_blockwise(Wpacked, absmax, code, N * K, blocksize, out_dtype=A.dtype).view(N, K)
+    A2 = A.view(M, K)
+    if out is None:
+        out = torch.empty((M, N), dtype=A.dtype, device=A.device)
+    if bias is None:
+        return torch.matmul(A2, W.t(), out=out)
+    return torch.addmm(bias, A2, W.t(), out=out)

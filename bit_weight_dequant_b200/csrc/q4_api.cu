@@ -406,6 +406,28 @@ int q4_gemm_skinny_bias(const void* A, const uint8_t* Wpacked, const float* absm
                       workspace_bytes, stream, overrides);
 }
 
+int q4_gemm_route(int M, int N, int K, int blocksize, int act_dtype, int* route) {
+    if (!route) return Q4_ERR_INVALID_ARG;
+    GemmChoice ch;
+    int tiles = 0, sms = 0;
+    int64_t units = 0;
+    size_t ws = 0;
+    // Any positive SM count: the choice of path does not depend on it, and a
+    // host-only query must not touch the device.
+    const int rc = gemm_choose(M, N, K, blocksize, act_dtype, 148, nullptr, &ch, &tiles, &units, &ws, &sms);
+    if (rc == Q4_ERR_UNSUPPORTED) {
+        *route = Q4_ROUTE_SPLIT;
+        return Q4_OK;
+    }
+    if (rc != Q4_OK) return rc;
+    if (M <= 16) {
+        *route = Q4_ROUTE_FUSED;
+        return Q4_OK;
+    }
+    *route = (M <= 64 && (int64_t)N * K >= ((int64_t)1 << 26)) ? Q4_ROUTE_FUSED : Q4_ROUTE_SPLIT;
+    return Q4_OK;
+}
+
 // The exported partition functions compute with 64-bit integers; the kernels
 // use the 32-bit forms of the same formulas, which agree whenever
 // total * parts < 2^32 (the launcher enforces units < 2^23, parts <= 512).

@@ -58,7 +58,8 @@ constexpr int kNA = 8;                                       // A buffers (64-k 
 constexpr uint32_t kWaitSleepNs = 50000;
 constexpr uint32_t kWaitTries = 40000;
 constexpr int kErrWaitTimeout = 1;
-constexpr int kThreads = 320;  // producer, MMA issuer, two dequantizing warpgroups
+constexpr int kNWG = 2;                      // dequantizing warpgroups (unit u goes to u % kNWG)
+constexpr int kThreads = 64 + 128 * kNWG;    // producer, MMA issuer, the dequantizing warpgroups
 
 template <int MP>
 struct Geo {
@@ -224,7 +225,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t drain = dfree + 16u;                                                // MMA drain on error
     const uint32_t tslot = drain + 8u;                                                 // tensor-memory base
     // Cross-CTA epilogue handshakes: a CTA has at most two tiles it shares
-    // with other CTAs (its first and its last), and the two warpgroups may
+    // with other CTAs (its first and its last), and two warpgroups may
     // run those epilogues at the same time, so each gets its own pair of
     // barriers and its own broadcast word, each used once per launch.
     const uint32_t ctl = tslot + 8u;      // [2] words
@@ -361,7 +362,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ---------------- dequantize + epilogue (one thread per weight row) ----------------
         const int row = 32 * (warp & 3) + lane;             // this warp's tensor-memory lane quarter
         const uint32_t lane_bits = (uint32_t)(32 * (warp & 3)) << 16;
-        const int wg = (warp - 2) >> 2;                      // warpgroup: takes the units u with u % 2 == wg
+        const int wg = (warp - 2) >> 2;                      // warpgroup: takes the units u with u % kNWG == wg
         const int ew = (warp - 2) & 3;                       // warp within the warpgroup
         float c[16];
 #pragma unroll
@@ -380,7 +381,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // (a one-unit stage at a range edge may belong to the other
                 // one); a wait on a stage it never reads could alias a later
                 // fill of the same slot.
-                const bool mine = n >= 2 || (u & 1) == wg;
+                const bool mine = n >= kNWG || (wg - u % kNWG + kNWG) % kNWG < n;
                 if (mine && !wait_parity(full(slot), (uint32_t)(stage / S) & 1u)) {
                     ok = false;
                     break;
@@ -393,8 +394,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int x0 = (kb0 >> p.am_shift) & ~3;
                 for (int j = kb - kb0; j < kb - kb0 + n; ++j, ++u) {
                     const bool seg_end = (kb0 + j + 1 == kbt) || (q.left == 0 && j == kb - kb0 + n - 1);
-                    if ((u & 1) != wg) {
-                        // the other warpgroup's unit: only keep the segment bookkeeping
+                    if (u % kNWG != wg) {
+                        // another warpgroup's unit: only keep the segment bookkeeping
                         if (seg_end) {
                             const uint32_t t0s = (uint32_t)tile * (uint32_t)kbt;
                             if (!((t0s >= cs) && (t0s + (uint32_t)kbt <= ce))) ++xsegs;

@@ -226,6 +226,8 @@ def workloads() -> dict:
         for M in (1, 2, 4, 8, 16):
             f32.append(Case(M, N, K, act="fp32", tag=f"K{K}N{N}M{M}"))
     w["msweep_f32"] = Workload("fp32 activations, M 1,2,4,8,16 on K5120/N5120, K17408/N5120", 8, f32)
+    w["longk_f32"] = Workload("M=1 K=131072 N=2048 bs64 fp32 activations (main-loop profiling shape)", 9,
+                              [Case(1, 2048, 131072, act="fp32", tag="longk")])
     # Not one of the five: one long-K layer whose launch is almost all main
     # loop (start-up and tail are a few percent), for profiling the loop.
     w["longk"] = Workload("M=1 K=131072 N=8192 bs64 bf16 normal-table (main-loop profiling shape)", 5,

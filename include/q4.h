@@ -243,6 +243,29 @@ int q4_gemm_skinny_bias(const void* A, const uint8_t* Wpacked, const float* absm
                         void* workspace, size_t workspace_bytes, void* stream, const q4_gemm_plan_t* overrides);
 
 /*
+ * Fused-vs-split routing (host-only; no GPU work, no device query).  The
+ * maintainer's reply in PR #1920 describes heuristics that route each layer
+ * to dequantize + matmul or to one of the fused kernels by problem size.
+ * This is that choice for this library on B200:
+ *   *route = Q4_ROUTE_FUSED  call q4_gemm_skinny (measured faster), or
+ *          = Q4_ROUTE_SPLIT  dequantize (q4_dequantize_blockwise) and run a
+ *                            dense GEMM: the fused kernels do not take the
+ *                            problem, or are measured slower on it.
+ * The rule, fitted to measurements on B200:
+ *   - M <= 16 (bf16, fp16, fp32): fused (2.5-4.9x faster than the split
+ *     path for bf16, 1.4-7.7x for fp32);
+ *   - 17 <= M <= 64, bf16/fp16, with at least 2^26 weights (N*K): fused (the
+ *     tcgen05 kernel beats the split path there; below it, its fixed
+ *     start-up and cross-CTA combine cost more than the split path saves);
+ *   - everything else the fused entry rejects (M > 128, fp32 with M > 16,
+ *     the tcgen05 kernel's shape rules) or loses on: split.
+ * Argument errors as q4_gemm_skinny (Q4_ERR_INVALID_ARG); route NULL ->
+ * Q4_ERR_INVALID_ARG.
+ */
+typedef enum { Q4_ROUTE_FUSED = 0, Q4_ROUTE_SPLIT = 1 } q4_route;
+int q4_gemm_route(int M, int N, int K, int blocksize, int act_dtype, int* route);
+
+/*
  * Work partition used by the GEMM (host-callable so it can be checked
  * without a GPU): `total` units split into `parts` contiguous ranges,
  * part p owning [q4_partition_start(total, parts, p),

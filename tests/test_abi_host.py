@@ -190,3 +190,27 @@ def test_partition_invariants(total, parts):
         p = L.q4_partition_owner(total, parts, u)
         assert starts[p] <= u < starts[p + 1], (u, p)
     assert L.q4_partition_owner(total, parts, total) == -1
+
+
+def test_route_table():
+    """Fused-vs-split advice: fused at M <= 16 (any dtype) and for the
+    tcgen05 kernel's M <= 64 on layers of >= 2^26 weights; split for the rest
+    and for everything the fused entry rejects."""
+    import torch
+    F, S = b.Q4_ROUTE_FUSED, b.Q4_ROUTE_SPLIT
+    cases = {(1, 8192, 8192, 64, torch.bfloat16): F, (16, 5120, 5120, 64, torch.float16): F,
+             (8, 5120, 17408, 32, torch.float32): F, (16, 5120, 5120, 64, torch.float32): F,
+             (17, 5120, 5120, 64, torch.float32): S,                       # fp32 stops at M = 16
+             (32, 5120, 17408, 64, torch.bfloat16): F, (64, 5120, 17408, 64, torch.bfloat16): F,
+             (65, 5120, 17408, 64, torch.bfloat16): S, (128, 5120, 17408, 64, torch.bfloat16): S,
+             (32, 5120, 5120, 64, torch.bfloat16): S, (32, 8192, 5120, 64, torch.bfloat16): S,
+             (32, 8192, 8192, 64, torch.bfloat16): F,                      # exactly 2^26 weights
+             (32, 5120, 17408, 32, torch.bfloat16): S,                     # tcgen05 needs blocksize >= 64
+             (129, 8192, 8192, 64, torch.bfloat16): S, (4, 64, 4000, 64, torch.bfloat16): S}
+    for (M, N, K, bs, dt), want in cases.items():
+        assert b.q4_gemm_route(M, N, K, bs, dt) == want, (M, N, K, bs, dt)
+    r = ctypes.c_int(-1)
+    L = b.lib()
+    assert L.q4_gemm_route(1, 64, 4096, 96, 0, ctypes.byref(r)) == b.Q4_ERR_INVALID_ARG
+    assert L.q4_gemm_route(1, 64, 4096, 64, 0, None) == b.Q4_ERR_INVALID_ARG
+    assert L.q4_gemm_route(-1, 64, 4096, 64, 0, ctypes.byref(r)) == b.Q4_ERR_INVALID_ARG
