@@ -286,3 +286,46 @@ def q4_linear(A: torch.Tensor, Wpacked: torch.Tensor, absmax: torch.Tensor, code
     if bias is None:
         return torch.matmul(A2, W.t(), out=out)
     return torch.addmm(bias, A2, W.t(), out=out)
+
+
+class Q4Layer:
+    """A 4-bit linear layer bound once for repeated calls (a decode loop).
+
+    Weights, code table, the activation buffer ``A`` [M, K], the output buffer,
+    optional bias, workspace, stream and launch options are marshalled at
+    construction.  Each call is then a single C call
+    (``q4_gemm_skinny_ex`` / ``q4_gemm_skinny_bias``) with the prepared
+    arguments.  It computes ``out = A . dequant(W)^T (+ bias)`` from whatever
+    ``A`` holds at the time: write the next activations into ``A`` in place
+    between calls."""
+
+    def __init__(self, Wpacked: torch.Tensor, absmax: torch.Tensor, code: torch.Tensor, N: int, K: int,
+                 blocksize: int, A: torch.Tensor, out: torch.Tensor | None = None, bias: torch.Tensor | None = None,
+                 workspace: Workspace | None = None, stream: torch.cuda.Stream | None = None, **launch):
+        M = A.shape[0] if A.dim() == 2 else 1
+        act = _TORCH_TO_Q4[A.dtype]
+        assert A.is_cuda and A.is_contiguous() and A.numel() == M * K
+        self.A, self.Wpacked, self.absmax, self.code, self.bias = A, Wpacked, absmax, code, bias
+        self.out = out if out is not None else torch.empty((M, N), dtype=A.dtype, device=A.device)
+        assert self.out.dtype == A.dtype and self.out.numel() == M * N and self.out.is_contiguous()
+        nbytes = _workspace_bytes(M, N, K, blocksize, act)
+        self.workspace = workspace if workspace is not None else Workspace(A.device)
+        ws = self.workspace.get(nbytes) if nbytes else None
+        self.stream = stream if stream is not None else torch.cuda.current_stream(A.device)
+        self._ov = overrides(**launch)
+        P = ctypes.c_void_p
+        head = (P(A.data_ptr()), P(Wpacked.data_ptr()), P(absmax.data_ptr()), P(code.data_ptr()))
+        tail = (M, N, K, blocksize, act, P(self.out.data_ptr()), P(ws.data_ptr()) if ws is not None else None,
+                ws.numel() if ws is not None else 0, P(self.stream.cuda_stream),
+                ctypes.byref(self._ov) if self._ov is not None else None)
+        if bias is None:
+            self._fn, self._args = lib().q4_gemm_skinny_ex, head + tail
+        else:
+            assert bias.dtype == A.dtype and bias.numel() == N and bias.is_contiguous()
+            self._fn, self._args = lib().q4_gemm_skinny_bias, head + (P(bias.data_ptr()),) + tail
+
+    def __call__(self) -> torch.Tensor:
+        rc = self._fn(*self._args)
+        if rc != Q4_OK:
+            raise Q4Error(rc, "q4_gemm_skinny")
+        return self.out

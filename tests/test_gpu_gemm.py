@@ -233,3 +233,25 @@ def test_dependent_launch_chain(cuda_device, pdl, loader):
         got = chain(pdl=pdl)
         torch.cuda.synchronize()
         assert torch.equal(got.view(torch.int16), ref.view(torch.int16))
+
+
+def test_q4layer_matches_gemm_and_follows_in_place_activations(cuda_device):
+    """Q4Layer (the bound, one-C-call form of q4_gemm_skinny) gives the same
+    bits as q4_gemm_skinny and reads whatever its activation buffer holds."""
+    dev = cuda_device
+    M, N, K = 3, 300, 2048
+    code = torch.from_numpy(inputs.code_normal_quantile()).to(dev)
+    W = inputs.weights_device(N, K, 55, dev)
+    packed, absmax = q4.q4_quantize_blockwise(W.reshape(-1), 64, code)
+    A = torch.empty((M, K), dtype=torch.bfloat16, device=dev)
+    bias = inputs.activations(1, N, torch.bfloat16, 57).reshape(N).to(dev)
+    layer = q4.Q4Layer(packed, absmax, code, N, K, 64, A)
+    layer_b = q4.Q4Layer(packed, absmax, code, N, K, 64, A, bias=bias, pdl=2)
+    for seed in (1, 2):
+        A.copy_(inputs.activations(M, K, torch.bfloat16, seed).to(dev))
+        want = q4.q4_gemm_skinny(A, packed, absmax, code, N, K, 64)
+        want_b = q4.q4_gemm_skinny(A, packed, absmax, code, N, K, 64, bias=bias)
+        got, got_b = layer().clone(), layer_b().clone()
+        torch.cuda.synchronize(dev)
+        assert torch.equal(got.view(torch.int16), want.view(torch.int16)), seed
+        assert torch.equal(got_b.view(torch.int16), want_b.view(torch.int16)), seed
