@@ -10,7 +10,7 @@ import oracle
 from bit_weight_dequant_b200 import binding as q4
 from bit_weight_dequant_b200 import inputs
 
-TORCH_ACT = {"bf16": torch.bfloat16, "fp16": torch.float16}
+TORCH_ACT = {"bf16": torch.bfloat16, "fp16": torch.float16, "fp32": torch.float32}
 ORACLE_ACT = {"bf16": oracle.BF16, "fp16": oracle.FP16}
 
 
@@ -33,6 +33,48 @@ def check_gemm(out_bits: np.ndarray, y: np.ndarray, S: np.ndarray, act: str, lab
     return float((err / np.maximum(tol, 1e-300)).max()) if err.size else 0.0
 
 
+def check_f32(out: torch.Tensor, y: np.ndarray, S: np.ndarray, K: int, label: str = "") -> float:
+    """fp32 outputs: within the contract bound 1e-2 * S + ulp_fp32(y) and
+    within the fp32-arithmetic bound (32 + K/128) * 2^-24 * S + ulp(y) (the
+    fp32 kernel rounds each term at most 8 times in its block piece, K/256
+    times along a lane's running sum, 5 times across lanes and once per warp
+    piece it is combined with; the oracle's fp32 weight adds one)."""
+    got = out.detach().cpu().numpy().astype(np.float64).reshape(y.shape)
+    u = oracle.ulp(y, oracle.FP32).reshape(y.shape)
+    err = np.abs(got - y)
+    worst = 0.0
+    for name, tol in (("contract", 1e-2 * S + u), ("fp32", (32 + K / 128) * 2.0 ** -24 * S + u)):
+        bad = ~(err <= tol)
+        if bad.any():
+            i = tuple(np.argwhere(bad)[0])
+            raise AssertionError(f"{label}: {int(bad.sum())}/{bad.size} outputs outside the {name} bound; first "
+                                 f"at {i}: gpu={got[i]!r} oracle={y[i]!r} tol={tol[i]!r}")
+        if name == "contract" and err.size:
+            worst = float((err / np.maximum(tol, 1e-300)).max())
+    return worst
+
+
+def _activations(case: inputs.Case, seed: int):
+    """(A as a CPU tensor, the oracle's expected values and S) for a case."""
+    if case.act == "fp32":
+        a = inputs.activations_fp32(case.M, case.K, seed)
+        return torch.from_numpy(a), a
+    A = inputs.activations(case.M, case.K, TORCH_ACT[case.act], seed)
+    return A, bits_of(A)
+
+
+def _oracle_gemm(case: inputs.Case, a, packed, absmax, code, n_rows: int):
+    if case.act == "fp32":
+        return oracle.gemm_f32(a, packed, absmax, code, case.M, n_rows, case.K, case.blocksize)
+    return oracle.gemm(a, ORACLE_ACT[case.act], packed, absmax, code, case.M, n_rows, case.K, case.blocksize)
+
+
+def _check(case: inputs.Case, out: torch.Tensor, y, S, label: str) -> float:
+    if case.act == "fp32":
+        return check_f32(out, y, S, case.K, label)
+    return check_gemm(bits_of(out), y, S, case.act, label=label)
+
+
 def run_case(case: inputs.Case, seed: int, device, check_quantizer: bool = True, **launch) -> float:
     """Quantize with the oracle, run the GPU GEMM on the oracle's packed
     weights, compare every output against the oracle.  Returns the worst
@@ -45,14 +87,13 @@ def run_case(case: inputs.Case, seed: int, device, check_quantizer: bool = True,
         gp, ga = q4.q4_quantize_blockwise(torch.from_numpy(W).to(device).reshape(-1), case.blocksize, code_d)
         assert np.array_equal(gp.cpu().numpy(), packed), "GPU codes differ from the oracle's"
         assert np.array_equal(ga.cpu().numpy().view(np.uint32), absmax.view(np.uint32)), "absmax differs"
-    A = inputs.activations(case.M, case.K, TORCH_ACT[case.act], seed)
-    y, S = oracle.gemm(bits_of(A), ORACLE_ACT[case.act], packed, absmax, code, case.M, case.N, case.K,
-                       case.blocksize)
+    A, a_ref = _activations(case, seed)
+    y, S = _oracle_gemm(case, a_ref, packed, absmax, code, case.N)
     out = q4.q4_gemm_skinny(A.to(device), torch.from_numpy(packed).to(device), torch.from_numpy(absmax).to(device),
                             code_d, case.N, case.K, case.blocksize, **launch)
     torch.cuda.synchronize(device)
     assert tuple(out.shape) == (case.M, case.N) and out.dtype == TORCH_ACT[case.act]
-    return check_gemm(bits_of(out), y, S, case.act, label=str(case))
+    return _check(case, out, y, S, str(case))
 
 
 def sample_rows(N: int, extra: int = 40, seed: int = 0) -> np.ndarray:
@@ -75,16 +116,14 @@ def run_case_sampled(case: inputs.Case, seed: int, device, rows: np.ndarray | No
     packed, absmax = q4.q4_quantize_blockwise(W.reshape(-1), case.blocksize, code_d)
     Wr = W[torch.from_numpy(rows).to(device)].cpu().numpy()
     del W
-    A = inputs.activations(case.M, case.K, TORCH_ACT[case.act], seed)
+    A, a_ref = _activations(case, seed)
     out = q4.q4_gemm_skinny(A.to(device), packed, absmax, code_d, case.N, case.K, case.blocksize)
     torch.cuda.synchronize(device)
-    p_ref, a_ref = oracle.quantize(Wr, case.blocksize, code)
+    p_ref, ab_ref = oracle.quantize(Wr, case.blocksize, code)
     rows_d = torch.from_numpy(rows).to(device)
     gp = packed.view(case.N, case.K // 2)[rows_d].cpu().numpy().reshape(-1)
     ga = absmax.view(case.N, case.K // case.blocksize)[rows_d].cpu().numpy().reshape(-1)
     assert np.array_equal(gp, p_ref), "GPU codes differ from the oracle's on sampled rows"
-    assert np.array_equal(ga.view(np.uint32), a_ref.view(np.uint32)), "absmax differs on sampled rows"
-    y, S = oracle.gemm(bits_of(A), ORACLE_ACT[case.act], p_ref, a_ref, code, case.M, rows.size, case.K,
-                       case.blocksize)
-    got = bits_of(out[:, rows_d])
-    return check_gemm(got, y, S, case.act, label=f"{case} rows={rows.size}")
+    assert np.array_equal(ga.view(np.uint32), ab_ref.view(np.uint32)), "absmax differs on sampled rows"
+    y, S = _oracle_gemm(case, a_ref, p_ref, ab_ref, code, rows.size)
+    return _check(case, out[:, rows_d], y, S, f"{case} rows={rows.size}")

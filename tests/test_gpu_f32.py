@@ -19,24 +19,9 @@ import torch
 import oracle
 from bit_weight_dequant_b200 import binding as q4
 from bit_weight_dequant_b200 import inputs
-from parity import sample_rows
+from parity import check_f32, sample_rows
 
 pytestmark = pytest.mark.gpu
-
-U32 = 2.0 ** -24
-
-
-def check_f32(out: torch.Tensor, y: np.ndarray, S: np.ndarray, K: int, label: str):
-    got = out.detach().cpu().numpy().astype(np.float64).reshape(y.shape)
-    ulp = oracle.ulp(y, oracle.FP32).reshape(y.shape)
-    err = np.abs(got - y)
-    for name, tol in (("contract", 1e-2 * S + ulp), ("fp32", (32 + K / 128) * U32 * S + ulp)):
-        bad = ~(err <= tol)
-        if bad.any():
-            i = tuple(np.argwhere(bad)[0])
-            raise AssertionError(f"{label}: {int(bad.sum())}/{bad.size} outputs outside the {name} bound; first "
-                                 f"at {i}: gpu={got[i]!r} oracle={y[i]!r} tol={tol[i]!r}")
-
 
 def _problem(M, N, K, bs, seed, table="normal", outliers=False):
     code = inputs.CODE_TABLES[table]()
