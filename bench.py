@@ -219,10 +219,11 @@ class Layer:
 
 def split_time_est_us(case: inputs.Case, peak_gbs: float) -> float:
     """Time at the HBM peak of the split path: read the packed weights and
-    absmax, write the bf16 weights, read them back in a dense GEMM, plus A
-    and C once."""
+    absmax, write the dequantized weights in the activation type (2 or 4
+    bytes), read them back in a dense GEMM, plus A and C once."""
     nk = case.N * case.K
-    b = nk * (0.5 + 4.0 / case.blocksize) + 2 * nk + 2 * nk + 2 * case.M * case.K + 2 * case.M * case.N
+    e = 4 if case.act == "fp32" else 2
+    b = nk * (0.5 + 4.0 / case.blocksize) + e * nk + e * nk + e * case.M * case.K + e * case.M * case.N
     return b / (peak_gbs * 1e3)
 
 
