@@ -44,7 +44,17 @@ namespace simt {
 
 static constexpr int kUnitK = 512;                    // k-width of a work unit (two 256-k groups)
 static constexpr uint32_t kTableBytes = 256u * 256u;  // 256 rows of 256 B (lower 128 B used)
-static constexpr size_t kSmemBytes = 65536u + kTableBytes;  // + padding to a 64 KiB boundary
+// Dynamic shared memory: the device's opt-in maximum (the table on a 64 KiB
+// boundary, the warps' copy rings below and above it).
+static int max_smem() {
+    int dev = 0, v = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&v, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess) {
+        cudaGetLastError();
+        return 0;
+    }
+    return v;
+}
 
 struct Params {
     const float* A;        // [M, K]
@@ -64,6 +74,7 @@ struct Params {
     uint32_t warps;        // grid warps
     int narrow;            // units * warps < 2^32: the partition in 32-bit arithmetic
     int a32;               // A is 32-byte aligned: 256-bit activation loads
+    int* error;            // workspace error word (set to 2 when shared memory is short), or nullptr
 };
 
 // First unit of part `p` when `total` units are split into `parts` ranges,
@@ -143,13 +154,28 @@ __device__ __forceinline__ uint64_t pair_of(uint32_t word, uint32_t lane8) {
     return lds_pair(prmt<0x7604u | (BYTE << 4)>(word, lane8));
 }
 
-// One unit's streamed operands for one lane: the packed word of each row for
-// both 256-k groups, and the absmax of the block each word lies in.
+// Asynchronous copies into the warp's shared-memory ring (the copy bytes
+// beyond src_size are zero-filled, so rows past N and k past K read nothing).
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_size) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_size) : "memory");
+}
+__device__ __forceinline__ void cp_async4(uint32_t dst, const void* src, uint32_t src_size) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(dst), "l"(src), "r"(src_size) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+// Ring slot of one unit: R rows x 256 B of packed codes (row r, group q at
+// r * 256 + q * 128), then R rows x 16 floats of absmax (the unit's blocks,
+// 512 / blocksize of them, at least 1).
 template <int R>
-struct UnitRegs {
-    uint32_t w[R][2];
-    float am[R][2];
+struct Slot {
+    static constexpr uint32_t CODES = (uint32_t)R * 256u;
+    static constexpr uint32_t BYTES = CODES + (uint32_t)R * 64u;
 };
+
+static constexpr int kErrNoRoom = 2;
 
 template <int MP, int R, int NW, int D>
 __global__ void __launch_bounds__(NW * 32, 1) q4_gemm_f32_kernel(const Params p) {
@@ -180,6 +206,20 @@ __global__ void __launch_bounds__(NW * 32, 1) q4_gemm_f32_kernel(const Params p)
         }
     }
 
+    // Ring slots: NW * D of them, below and above the table.
+    using SL = Slot<R>;
+    const uint32_t send = sbase + dynamic_smem_size();
+    const uint32_t a0s = sbase, b0s = table + kTableBytes;
+    const uint32_t na = (table - a0s) / SL::BYTES;
+    const uint32_t nb = send > b0s ? (send - b0s) / SL::BYTES : 0u;
+    if (na + nb < (uint32_t)(NW * D)) {  // uniform over the CTA: the host sized the launch wrongly
+        if (tid == 0 && p.error) atomicExch(p.error, kErrNoRoom);
+        return;
+    }
+    auto slot_addr = [&](int idx) -> uint32_t {
+        return (uint32_t)idx < na ? a0s + (uint32_t)idx * SL::BYTES : b0s + ((uint32_t)idx - na) * SL::BYTES;
+    };
+
     const uint32_t gw = blockIdx.x * NW + warp;
     const bool narrow = p.narrow != 0;
     auto start_of = [&](uint32_t w) { return wpart_start(p.units, p.warps, w, narrow); };
@@ -204,37 +244,43 @@ __global__ void __launch_bounds__(NW * 32, 1) q4_gemm_f32_kernel(const Params p)
         lc.kc = cc.kc = (int)(ws - lc.rg * (uint32_t)p.ku);
     }
 
-    // Streams the packed words and absmax of the unit at `c` into `x` (rows
-    // past N and groups past K read nothing).
-    auto load = [&](const Cursor& c, UnitRegs<R>& x) {
-        const int n0 = (int)c.rg * R;
-        const int kq = c.kc * kUnitK + 8 * lane;  // this lane's first k in the unit (group q adds 256 q)
-        const int a0 = kq >> p.lbs, a1 = (kq + 256) >> p.lbs;
-        const uint8_t* wb = Wp + (size_t)n0 * row_bytes + (kq >> 1);
-        const float* ab = absmax + (size_t)n0 * am_row + a0;
-        const int da = a1 - a0;
-        const bool k0ok = kq < p.K, k1ok = kq + 256 < p.K;
+    // Copies the packed words and absmax of the unit at `c` into ring slot
+    // `st` and commits them as one group (an empty group past the range).
+    const int nab = (kUnitK >> p.lbs) > 0 ? (kUnitK >> p.lbs) : 1;  // absmax values per row and unit
+    auto issue = [&](bool valid, const Cursor& c, uint32_t st) {
+        if (valid) {
+            const int n0 = (int)c.rg * R;
+            const int k0 = c.kc * kUnitK;
+            // codes: R x 256 B = R x 16 chunks of 16 B; lane l copies chunks l, l + 32, ...
 #pragma unroll
-        for (int r = 0; r < R; ++r) {
-            const bool nok = n0 + r < p.N;
-            // R rows of K/2 bytes stay below 2^32 bytes (K < 2^29): 32-bit row offsets
-            const uint8_t* wr = wb + (uint32_t)r * (uint32_t)row_bytes;
-            const float* ar = ab + (uint32_t)r * (uint32_t)am_row;
-            x.w[r][0] = (nok && k0ok) ? ldg_code_word(wr) : 0u;
-            x.am[r][0] = (nok && k0ok) ? ldg_scale(ar) : 0.f;
-            x.w[r][1] = (nok && k1ok) ? ldg_code_word(wr + 128) : 0u;
-            x.am[r][1] = (nok && k1ok) ? ldg_scale(ar + da) : 0.f;
+            for (int i = 0; i < R / 2; ++i) {
+                const int ch = lane + 32 * i;           // chunk: row ch / 16, bytes 16 (ch % 16)
+                const int r = ch >> 4, cb = (ch & 15) * 16;
+                const int kc0 = k0 + 2 * cb;            // first k of the chunk (32 k per 16 B)
+                const bool ok = (n0 + r < p.N) && (kc0 < p.K);
+                const uint8_t* src = ok ? Wp + (size_t)(n0 + r) * row_bytes + (kc0 >> 1) : Wp;
+                cp_async16(st + (uint32_t)(r * 256 + cb), src, ok ? 16u : 0u);
+            }
+            // absmax: R rows x nab values; lane l copies values l, l + 32, ...
+            for (int v = lane; v < R * nab; v += 32) {
+                const int r = v / nab, j = v - r * nab;
+                const int kb = k0 + (j << p.lbs);       // first k of block j of the unit
+                const bool ok = (n0 + r < p.N) && (kb < p.K);
+                const float* src = ok ? absmax + (size_t)(n0 + r) * am_row + (kb >> p.lbs) : absmax;
+                cp_async4(st + SL::CODES + (uint32_t)(r * 64 + 4 * j), src, ok ? 4u : 0u);
+            }
         }
+        cp_async_commit();
     };
 
-    // A ring of D register buffers: D - 1 units in flight while one is computed.
-    UnitRegs<R> xb[D];
+    // Units ws .. we-1 go through slots warp * D + (u - ws) % D; D - 1 are
+    // copied ahead of the one being computed.
+    const int slot0 = warp * D;
 #pragma unroll
-    for (int i = 0; i < D - 1; ++i)
-        if (ws + i < we) {
-            load(lc, xb[i]);
-            advance(lc);
-        }
+    for (int i = 0; i < D - 1; ++i) {
+        issue(ws + i < we, lc, slot_addr(slot0 + i));
+        if (ws + i < we) advance(lc);
+    }
     __syncthreads();  // the table is complete
     launder(lane8);   // every lookup address derives from lane8: none moves above the barrier
     // Activations, outputs and the workspace may belong to the preceding
@@ -242,7 +288,10 @@ __global__ void __launch_bounds__(NW * 32, 1) q4_gemm_f32_kernel(const Params p)
     if (p.pdl == 2) griddep_wait();
     launder(Aact);  // activations only after the dependency wait
     griddep_launch_dependents();
-    if (ws >= we) return;
+    if (ws >= we) {
+        cp_async_wait<0>();
+        return;
+    }
 
     float acc[R][MP];
 #pragma unroll
@@ -252,7 +301,7 @@ __global__ void __launch_bounds__(NW * 32, 1) q4_gemm_f32_kernel(const Params p)
 
     // acc += this lane's share of the unit at `c`: per 256-k group, 8
     // consecutive k of every row, scaled once by that block's absmax.
-    auto compute = [&](const Cursor& c, const UnitRegs<R>& x) {
+    auto compute = [&](const Cursor& c, uint32_t st) {
         const int k0 = c.kc * kUnitK;
 #pragma unroll
         for (int q = 0; q < 2; ++q) {
@@ -274,16 +323,25 @@ __global__ void __launch_bounds__(NW * 32, 1) q4_gemm_f32_kernel(const Params p)
                     a[m][0] = a[m][1] = a[m][2] = a[m][3] = 0ull;
                 }
             }
+            // this lane's word of every row, and the absmax of the block it lies in
+            uint32_t wq[R];
+            float amq[R];
+            const uint32_t aj = (uint32_t)((256 * q + 8 * lane) >> p.lbs);  // block index inside the unit
+#pragma unroll
+            for (int r = 0; r < R; ++r) {
+                wq[r] = lds_u32(st + (uint32_t)(r * 256 + q * 128 + 4 * lane));
+                amq[r] = lds_f32(st + SL::CODES + (uint32_t)(r * 64) + 4u * aj);
+            }
             // Two running sums per (row, m): even and odd k of the pairs.
             uint64_t t[R][MP];
 #pragma unroll
             for (int j = 0; j < 4; ++j) {  // byte j of the word: k = kq + 2j, kq + 2j + 1
 #pragma unroll
                 for (int r = 0; r < R; ++r) {
-                    const uint64_t cp = j == 0   ? pair_of<0>(x.w[r][q], lane8)
-                                        : j == 1 ? pair_of<1>(x.w[r][q], lane8)
-                                        : j == 2 ? pair_of<2>(x.w[r][q], lane8)
-                                                 : pair_of<3>(x.w[r][q], lane8);
+                    const uint64_t cp = j == 0   ? pair_of<0>(wq[r], lane8)
+                                        : j == 1 ? pair_of<1>(wq[r], lane8)
+                                        : j == 2 ? pair_of<2>(wq[r], lane8)
+                                                 : pair_of<3>(wq[r], lane8);
 #pragma unroll
                     for (int m = 0; m < MP; ++m) t[r][m] = j == 0 ? mul2(a[m][0], cp) : fma2(a[m][j], cp, t[r][m]);
                 }
@@ -292,8 +350,8 @@ __global__ void __launch_bounds__(NW * 32, 1) q4_gemm_f32_kernel(const Params p)
             for (int r = 0; r < R; ++r)
 #pragma unroll
                 for (int m = 0; m < MP; ++m) {
-                    acc[r][m] = fmaf(x.am[r][q], lo_f32(t[r][m]), acc[r][m]);
-                    acc[r][m] = fmaf(x.am[r][q], hi_f32(t[r][m]), acc[r][m]);
+                    acc[r][m] = fmaf(amq[r], lo_f32(t[r][m]), acc[r][m]);
+                    acc[r][m] = fmaf(amq[r], hi_f32(t[r][m]), acc[r][m]);
                 }
         }
     };
@@ -370,26 +428,21 @@ __global__ void __launch_bounds__(NW * 32, 1) q4_gemm_f32_kernel(const Params p)
 #pragma unroll
             for (int m = 0; m < MP; ++m) acc[r][m] = 0.f;
     };
-    auto step = [&](const UnitRegs<R>& x, bool last_of_range) {
-        compute(cc, x);
+    auto step = [&](uint32_t st, bool last_of_range) {
+        compute(cc, st);
         if (cc.kc == p.ku - 1 || last_of_range) finish(cc.rg);
         advance(cc);
     };
 
-    // Unit u sits in buffer (u - ws) % D; before it is computed the loads of
-    // unit u + D - 1 go into the buffer computed last.  The loop is unrolled
-    // D times so that every buffer index is a compile-time constant.
-    for (uint32_t u = ws; u < we; u += D) {
-#pragma unroll
-        for (int i = 0; i < D; ++i) {
-            if (u + i >= we) break;
-            if (u + i + D - 1 < we) {
-                load(lc, xb[(i + D - 1) % D]);
-                advance(lc);
-            }
-            step(xb[i], u + i + 1 == we);
-        }
+    for (uint32_t u = ws; u < we; ++u) {
+        const int i = (int)(u - ws);
+        cp_async_wait<D - 2>();  // this unit's group is complete (one group is committed per unit)
+        __syncwarp();            // and visible to every lane (lanes read words other lanes copied)
+        issue(u + D - 1 < we, lc, slot_addr(slot0 + (i + D - 1) % D));  // refills the slot computed last
+        if (u + D - 1 < we) advance(lc);
+        step(slot_addr(slot0 + i % D), u + 1 == we);
     }
+    cp_async_wait<0>();
 }
 
 // Compiled variants: MP = padded M, R = rows per unit, NW = warps per CTA,
@@ -397,12 +450,14 @@ __global__ void __launch_bounds__(NW * 32, 1) q4_gemm_f32_kernel(const Params p)
 template <int MP, int R, int NW, int D>
 static cudaError_t launch_variant(const Params& p, int ctas, cudaStream_t stream) {
     auto kern = q4_gemm_f32_kernel<MP, R, NW, D>;
-    cudaError_t e = ensure_smem_attr((const void*)kern, kSmemBytes);
+    const int smem = max_smem();
+    if (smem <= 0) return cudaErrorInvalidValue;
+    cudaError_t e = ensure_smem_attr((const void*)kern, (size_t)smem);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)ctas);
     cfg.blockDim = dim3(NW * 32);
-    cfg.dynamicSmemBytes = kSmemBytes;
+    cfg.dynamicSmemBytes = (size_t)smem;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -425,7 +480,7 @@ SimtShape simt_shape(int M) {
     return {16, 2, 8};
 }
 
-size_t simt_smem_bytes() { return simt::kSmemBytes; }
+size_t simt_smem_bytes() { return (size_t)simt::max_smem(); }
 
 cudaError_t simt_launch(const SimtShape& sh, int ctas, const GemmParams& g, int log2_bs, cudaStream_t stream) {
     simt::Params p{};
@@ -448,12 +503,13 @@ cudaError_t simt_launch(const SimtShape& sh, int ctas, const GemmParams& g, int 
     p.warps = (uint32_t)ctas * (uint32_t)sh.warps;
     p.narrow = (uint64_t)p.units * p.warps < ((uint64_t)1 << 32) ? 1 : 0;
     p.a32 = (reinterpret_cast<uintptr_t>(g.A) & 31u) == 0 ? 1 : 0;
+    p.error = g.error;
     switch (sh.m_pad) {
-        case 1: return simt::launch_variant<1, 8, 16, 2>(p, ctas, stream);
-        case 2: return simt::launch_variant<2, 8, 8, 2>(p, ctas, stream);
-        case 4: return simt::launch_variant<4, 8, 8, 2>(p, ctas, stream);
-        case 8: return simt::launch_variant<8, 4, 8, 2>(p, ctas, stream);
-        case 16: return simt::launch_variant<16, 2, 8, 2>(p, ctas, stream);
+        case 1: return simt::launch_variant<1, 8, 16, 4>(p, ctas, stream);
+        case 2: return simt::launch_variant<2, 8, 8, 4>(p, ctas, stream);
+        case 4: return simt::launch_variant<4, 8, 8, 4>(p, ctas, stream);
+        case 8: return simt::launch_variant<8, 4, 8, 4>(p, ctas, stream);
+        case 16: return simt::launch_variant<16, 2, 8, 4>(p, ctas, stream);
         default: return cudaErrorInvalidConfiguration;
     }
 }
