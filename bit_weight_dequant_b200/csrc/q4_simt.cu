@@ -246,24 +246,28 @@ __global__ void __launch_bounds__(NW * 32, 1) q4_gemm_f32_kernel(const Params p)
 
     // Copies the packed words and absmax of the unit at `c` into ring slot
     // `st` and commits them as one group (an empty group past the range).
-    const int nab = (kUnitK >> p.lbs) > 0 ? (kUnitK >> p.lbs) : 1;  // absmax values per row and unit
+    const int lnab = p.lbs < 9 ? 9 - p.lbs : 0;  // log2 of the absmax values per row and unit (512 / bs, at least 1)
+    const int nab = 1 << lnab;
     auto issue = [&](bool valid, const Cursor& c, uint32_t st) {
         if (valid) {
             const int n0 = (int)c.rg * R;
             const int k0 = c.kc * kUnitK;
             // codes: R x 256 B = R x 16 chunks of 16 B; lane l copies chunks l, l + 32, ...
+            // (rows lane / 16 + 2 i, bytes 16 (lane % 16) of the row's 256)
+            const int r0 = lane >> 4, cb = (lane & 15) * 16;
+            const bool kok = k0 + 2 * cb < p.K;   // the chunk's 32 k lie inside the row (K % 32 == 0)
+            const uint8_t* wsrc = Wp + (size_t)(n0 + r0) * row_bytes + (k0 >> 1) + cb;
+            const uint32_t wdst = st + (uint32_t)(r0 * 256 + cb);
 #pragma unroll
             for (int i = 0; i < R / 2; ++i) {
-                const int ch = lane + 32 * i;           // chunk: row ch / 16, bytes 16 (ch % 16)
-                const int r = ch >> 4, cb = (ch & 15) * 16;
-                const int kc0 = k0 + 2 * cb;            // first k of the chunk (32 k per 16 B)
-                const bool ok = (n0 + r < p.N) && (kc0 < p.K);
-                const uint8_t* src = ok ? Wp + (size_t)(n0 + r) * row_bytes + (kc0 >> 1) : Wp;
-                cp_async16(st + (uint32_t)(r * 256 + cb), src, ok ? 16u : 0u);
+                const bool ok = kok && (n0 + r0 + 2 * i < p.N);
+                // R rows of K/2 bytes stay below 2^32 bytes (K < 2^29): 32-bit row offsets
+                cp_async16(wdst + (uint32_t)(512 * i), ok ? wsrc + (uint32_t)(2 * i) * (uint32_t)row_bytes : Wp,
+                           ok ? 16u : 0u);
             }
             // absmax: R rows x nab values; lane l copies values l, l + 32, ...
             for (int v = lane; v < R * nab; v += 32) {
-                const int r = v / nab, j = v - r * nab;
+                const int r = v >> lnab, j = v & (nab - 1);
                 const int kb = k0 + (j << p.lbs);       // first k of block j of the unit
                 const bool ok = (n0 + r < p.N) && (kb < p.K);
                 const float* src = ok ? absmax + (size_t)(n0 + r) * am_row + (kb >> p.lbs) : absmax;
