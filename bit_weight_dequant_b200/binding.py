@@ -57,6 +57,8 @@ def lib() -> ctypes.CDLL:
         L.q4_quantize_blockwise_ex.argtypes = [P, ci, i64, ci, P, P, P, P]
         L.q4_dequantize_blockwise.argtypes = [P, P, P, i64, ci, ci, P, P]
         L.q4_gemm_workspace_size.argtypes = [ci, ci, ci, ci, ci, ctypes.POINTER(sz)]
+        L.q4_gemm_workspace_size_ex.argtypes = [ci, ci, ci, ci, ci, ctypes.POINTER(q4_gemm_plan_t),
+                                                ctypes.POINTER(sz)]
         L.q4_gemm_skinny.argtypes = [P, P, P, P, ci, ci, ci, ci, ci, P, P, sz, P]
         L.q4_gemm_skinny_ex.argtypes = [P, P, P, P, ci, ci, ci, ci, ci, P, P, sz, P, ctypes.POINTER(q4_gemm_plan_t)]
         L.q4_gemm_plan.argtypes = [ci, ci, ci, ci, ci, ci, ctypes.POINTER(q4_gemm_plan_t)]
@@ -69,7 +71,7 @@ def lib() -> ctypes.CDLL:
         L.q4_partition_owner.argtypes = [i64, ci, i64]
         for f in ("q4_quantize_blockwise", "q4_quantize_blockwise_ex", "q4_dequantize_blockwise", "q4_gemm_workspace_size",
                   "q4_gemm_skinny", "q4_gemm_skinny_ex", "q4_gemm_plan", "q4_partition_owner",
-                  "q4_gemm_skinny_noalloc", "q4_gemm_skinny_bias", "q4_gemm_route"):
+                  "q4_gemm_skinny_noalloc", "q4_gemm_skinny_bias", "q4_gemm_route", "q4_gemm_workspace_size_ex"):
             getattr(L, f).restype = ci
         _lib = L
     return _lib
@@ -129,9 +131,10 @@ def q4_gemm_workspace_size(M: int, N: int, K: int, blocksize: int, act_dtype: to
 
 
 @functools.lru_cache(maxsize=4096)
-def _workspace_bytes(M: int, N: int, K: int, blocksize: int, act: int) -> int:
+def _workspace_bytes(M: int, N: int, K: int, blocksize: int, act: int, launch: tuple = ()) -> int:
     v = ctypes.c_size_t(0)
-    _check(lib().q4_gemm_workspace_size(M, N, K, blocksize, act, ctypes.byref(v)), "q4_gemm_workspace_size")
+    ov = _overrides_ref(launch)[1] if launch else None
+    _check(lib().q4_gemm_workspace_size_ex(M, N, K, blocksize, act, ov, ctypes.byref(v)), "q4_gemm_workspace_size")
     return v.value
 
 
@@ -227,10 +230,11 @@ def q4_gemm_skinny(A: torch.Tensor, Wpacked: torch.Tensor, absmax: torch.Tensor,
     if out is None:
         out = torch.empty((M, N), dtype=A.dtype, device=A.device)
     act = _TORCH_TO_Q4[A.dtype]
-    nbytes = _workspace_bytes(M, N, K, blocksize, act)
+    items = tuple(sorted(launch.items())) if launch else ()
+    nbytes = _workspace_bytes(M, N, K, blocksize, act, items)
     stream = torch.cuda.current_stream(A.device).cuda_stream
     ws = (workspace or _default_workspace(A.device, stream)).get(nbytes) if nbytes else None
-    ov_ref = _overrides_ref(tuple(sorted(launch.items())))[1] if launch else None
+    ov_ref = _overrides_ref(items)[1] if launch else None
     if bias is None:
         rc = lib().q4_gemm_skinny_ex(A.data_ptr(), Wpacked.data_ptr(), absmax.data_ptr(), code.data_ptr(), M, N, K,
                                      blocksize, act, out.data_ptr(), ws.data_ptr() if ws is not None else None,
@@ -308,7 +312,7 @@ class Q4Layer:
         self.A, self.Wpacked, self.absmax, self.code, self.bias = A, Wpacked, absmax, code, bias
         self.out = out if out is not None else torch.empty((M, N), dtype=A.dtype, device=A.device)
         assert self.out.dtype == A.dtype and self.out.numel() == M * N and self.out.is_contiguous()
-        nbytes = _workspace_bytes(M, N, K, blocksize, act)
+        nbytes = _workspace_bytes(M, N, K, blocksize, act, tuple(sorted((k, v) for k, v in launch.items() if v)))
         self.workspace = workspace if workspace is not None else Workspace(A.device)
         ws = self.workspace.get(nbytes) if nbytes else None
         self.stream = stream if stream is not None else torch.cuda.current_stream(A.device)

@@ -127,7 +127,12 @@ static int gemm_choose(int M, int N, int K, int blocksize, int act_dtype, int nu
         *ws_bytes = u > 1 ? ws_counter_offset(sms) + align_up((size_t)t64 * sizeof(int), 256) : 0;
         return Q4_OK;
     }
-    if (M > 16 || (ov && (ov->math == 3 || ov->loader == 6))) {
+    // 17 <= M <= 32 runs on the mma.sync kernel with 32-row tiles and 2-unit
+    // stages when its TMA rules hold (and no override asks for tcgen05).
+    const bool want_umma = ov && (ov->math == 3 || ov->loader == 6);
+    const bool mma32 = M > 16 && M <= 32 && !want_umma && blocksize >= 64 && (K / blocksize) % 4 == 0 &&
+                       (int64_t)N * (K / 64) > 1;
+    if ((M > 16 && !mma32) || want_umma) {
         // Tensor-memory kernel (tcgen05): 128-row tiles, 64-k units, 4-unit
         // stages whose absmax box is 4 floats per row.
         if (blocksize < 64 || K % 256 != 0 || (K / blocksize) % 4 != 0) return Q4_ERR_UNSUPPORTED;
@@ -163,16 +168,21 @@ static int gemm_choose(int M, int N, int K, int blocksize, int act_dtype, int nu
     }
     c.math = 1;
     c.sub_block = blocksize < 64 ? blocksize : 64;
-    c.m_pad = M <= 8 ? 8 : 16;
-    c.rows_per_tile = 64;
+    c.m_pad = M <= 8 ? 8 : M <= 16 ? 16 : 32;
+    c.rows_per_tile = M <= 16 ? 64 : 32;
     // The TMA stage ring needs 64-k units and absmax rows that are whole
     // multiples of 16 bytes (a tensor-map stride rule); the pointer itself
     // must also be 16-byte aligned, which the caller checks at launch.
     const bool tma_ok = c.sub_block == 64 && (K / blocksize) % 4 == 0 && (int64_t)N * (K / 64) > 1;
-    c.loader = tma_ok ? 2 : 1;
+    c.loader = mma32 ? 3 : tma_ok ? 2 : 1;
     if (ov && ov->loader > 0) c.loader = ov->loader;
     if (c.loader >= 2 && !tma_ok) return Q4_ERR_UNSUPPORTED;
-    if (c.loader == 2) {
+    if (mma32) {
+        // 32-row tiles: 2-unit stages (64-byte rows), six per warp
+        c.warps = 8;
+        c.depth = 6;
+        c.l2pf = 0;
+    } else if (c.loader == 2) {
         c.warps = 8;
         c.depth = 2;
         c.l2pf = 0;
@@ -301,6 +311,15 @@ int q4_gemm_workspace_size(int M, int N, int K, int blocksize, int act_dtype, si
     return gemm_choose(M, N, K, blocksize, act_dtype, 0, nullptr, &ch, &tiles, &units, bytes, &sms);
 }
 
+int q4_gemm_workspace_size_ex(int M, int N, int K, int blocksize, int act_dtype, const q4_gemm_plan_t* overrides,
+                              size_t* bytes) {
+    if (!bytes) return Q4_ERR_INVALID_ARG;
+    GemmChoice ch;
+    int tiles = 0, sms = 0;
+    int64_t units = 0;
+    return gemm_choose(M, N, K, blocksize, act_dtype, 0, overrides, &ch, &tiles, &units, bytes, &sms);
+}
+
 // The fused GEMM behind every entry point; `bias` may be nullptr.
 static int gemm_entry(const void* A, const uint8_t* Wpacked, const float* absmax, const float* code, const void* bias,
                       int M, int N, int K, int blocksize, int act_dtype, void* out, void* workspace,
@@ -420,10 +439,11 @@ int q4_gemm_route(int M, int N, int K, int blocksize, int act_dtype, int* route)
         return Q4_OK;
     }
     if (rc != Q4_OK) return rc;
-    if (M <= 16) {
+    if (M <= 16 || ch.math == 1) {  // M <= 16, and 17 <= M <= 32 on the 32-row mma.sync kernel
         *route = Q4_ROUTE_FUSED;
         return Q4_OK;
     }
+    // the tensor-memory kernel
     *route = (M <= 64 && (int64_t)N * K >= ((int64_t)1 << 26)) ? Q4_ROUTE_FUSED : Q4_ROUTE_SPLIT;
     return Q4_OK;
 }

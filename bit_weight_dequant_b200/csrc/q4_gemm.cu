@@ -392,12 +392,13 @@ __global__ void __launch_bounds__(S::NW * 32, 1) q4_gemm_mma_kernel(const GemmPa
 // workspace, stops issuing, drains its copies (also bounded) and returns
 // normally (its outputs are then not valid).
 // ===========================================================================
-template <int UPS>
+template <int UPS, int TR = 64>
 struct StageGeom {
     static constexpr uint32_t ROW_BYTES = 32u * UPS;                   // 64 or 128
-    static constexpr uint32_t WEIGHT_BYTES = 64u * ROW_BYTES;          // 4 or 8 KiB
-    static constexpr uint32_t ABSMAX_BYTES = 64u * 4u * 4u;            // 1 KiB
-    static constexpr uint32_t BYTES = WEIGHT_BYTES + ABSMAX_BYTES;     // multiple of 512
+    static constexpr uint32_t WEIGHT_BYTES = (uint32_t)TR * ROW_BYTES; // TR rows of the stage's codes
+    static constexpr uint32_t ABSMAX_BYTES = (uint32_t)TR * 4u * 4u;   // TR rows x 4 floats
+    static constexpr uint32_t COPY_BYTES = WEIGHT_BYTES + ABSMAX_BYTES;  // what the two copies deliver
+    static constexpr uint32_t BYTES = (COPY_BYTES + 1023u) & ~1023u;   // stage stride: swizzled boxes start 1 KiB aligned
     // physical address of 16-byte chunk `chunk` of box row `row` (TMA swizzle)
     __device__ __forceinline__ static uint32_t chunk_addr(uint32_t base, int row, int chunk) {
         if constexpr (UPS == 4)
@@ -485,7 +486,7 @@ template <typename T, class S, int UPS, bool BS64>
 __global__ void __launch_bounds__(S::NW * 32, 1)
     q4_gemm_tma_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_a,
                        const GemmParams p) {
-    using G = StageGeom<UPS>;
+    using G = StageGeom<UPS, S::TR>;
     static_assert(S::NW * S::SLOT_REGS <= 256, "parked partial tiles must fit in the LUT rows");
     extern __shared__ __align__(16) uint8_t smem_ring[];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, tq = lane & 3;
@@ -553,7 +554,7 @@ __global__ void __launch_bounds__(S::NW * 32, 1)
         const uint32_t st = stage_addr(warp * D + k % D);
         const uint32_t bar = bars + (uint32_t)(warp * D + k % D) * 8u;
         if (lane == 0) {
-            mbar_expect_tx(bar, G::BYTES);
+            mbar_expect_tx(bar, G::COPY_BYTES);
             tma_load_2d_hint(st, &tmap_w, kb0 * 32, tile * S::TR, bar, stream_once);
             tma_load_2d(st + G::WEIGHT_BYTES, &tmap_a, (kb0 >> p.am_shift) & ~3, tile * S::TR, bar);
         }
@@ -752,7 +753,7 @@ template <typename T, class S, int UPS, bool BS64>
 __global__ void __launch_bounds__((S::NW + 1) * 32, 1)
     q4_gemm_ws_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_a,
                       const GemmParams p) {
-    using G = StageGeom<UPS>;
+    using G = StageGeom<UPS, S::TR>;
     static_assert(S::NW * S::SLOT_REGS <= 256, "parked partial tiles must fit in the LUT rows");
     static_assert(S::NW <= 32, "one producer lane per consumer warp");
     constexpr int NC = S::NW;     // consumer warps
@@ -826,7 +827,7 @@ __global__ void __launch_bounds__((S::NW + 1) * 32, 1)
                 int tile, kb0, kb, n;
                 next_stage<UPS>(ld, p.kb_per_tile, tile, kb0, kb, n);
                 const uint32_t st = stage_addr(lane * D + slot);
-                mbar_expect_tx(full_bar(lane, slot), G::BYTES);
+                mbar_expect_tx(full_bar(lane, slot), G::COPY_BYTES);
                 tma_load_2d_hint(st, &tmap_w, kb0 * 32, tile * S::TR, full_bar(lane, slot), stream_once);
                 tma_load_2d(st + G::WEIGHT_BYTES, &tmap_a, (kb0 >> p.am_shift) & ~3, tile * S::TR, full_bar(lane, slot));
             }
@@ -1005,15 +1006,15 @@ static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
     return fn;
 }
 
-// Weights: [N rows][K/2 bytes], box 64 rows x (32 * UPS) bytes, 64/128-byte swizzle.
-// Absmax: [N rows][K/bs floats], box 64 rows x 4 floats.
-static cudaError_t make_tensor_maps(const GemmParams& p, int ups, CUtensorMap* tw, CUtensorMap* ta) {
+// Weights: [N rows][K/2 bytes], box `rows` rows x (32 * UPS) bytes, 64/128-byte swizzle.
+// Absmax: [N rows][K/bs floats], box `rows` rows x 4 floats.
+static cudaError_t make_tensor_maps(const GemmParams& p, int ups, int rows, CUtensorMap* tw, CUtensorMap* ta) {
     auto enc = tensor_map_encoder();
     if (!enc) return cudaErrorNotSupported;
     const cuuint32_t estride[2] = {1, 1};
     const cuuint64_t wdim[2] = {(cuuint64_t)(p.K / 2), (cuuint64_t)p.N};
     const cuuint64_t wstride[1] = {(cuuint64_t)(p.K / 2)};
-    const cuuint32_t wbox[2] = {(cuuint32_t)(32 * ups), 64};
+    const cuuint32_t wbox[2] = {(cuuint32_t)(32 * ups), (cuuint32_t)rows};
     if (enc(tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(p.Wp), wdim, wstride, wbox, estride,
             CU_TENSOR_MAP_INTERLEAVE_NONE, ups == 4 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
             // no promotion past the box: a wider L2 fill would take the next
@@ -1023,7 +1024,7 @@ static cudaError_t make_tensor_maps(const GemmParams& p, int ups, CUtensorMap* t
         return cudaErrorInvalidValue;
     const cuuint64_t adim[2] = {(cuuint64_t)p.am_per_row, (cuuint64_t)p.N};
     const cuuint64_t astride[1] = {(cuuint64_t)p.am_per_row * 4};
-    const cuuint32_t abox[2] = {4, 64};
+    const cuuint32_t abox[2] = {4, (cuuint32_t)rows};
     if (enc(ta, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(p.absmax), adim, astride, abox, estride,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
@@ -1044,7 +1045,7 @@ static int max_dynamic_smem() {
 template <typename T, class S, int UPS>
 static cudaError_t launch_tma(const GemmParams& p, cudaStream_t stream) {
     CUtensorMap tw, ta;
-    cudaError_t e = make_tensor_maps(p, UPS, &tw, &ta);
+    cudaError_t e = make_tensor_maps(p, UPS, S::TR, &tw, &ta);
     if (e != cudaSuccess) return e;
     const int smem = max_dynamic_smem();  // the kernel lays out LUT, barriers and stages itself
     if (smem <= 0) return cudaErrorInvalidValue;
@@ -1068,7 +1069,7 @@ static cudaError_t launch_tma(const GemmParams& p, cudaStream_t stream) {
 template <typename T, class S, int UPS>
 static cudaError_t launch_ws(const GemmParams& p, cudaStream_t stream) {
     CUtensorMap tw, ta;
-    cudaError_t e = make_tensor_maps(p, UPS, &tw, &ta);
+    cudaError_t e = make_tensor_maps(p, UPS, S::TR, &tw, &ta);
     if (e != cudaSuccess) return e;
     const int smem = max_dynamic_smem();
     if (smem <= 0) return cudaErrorInvalidValue;
@@ -1107,6 +1108,11 @@ struct Variant {
     Variant {                                                                                 \
         ACT, 2, 64, MP, NW, D, 0, 0, &launch_tma<T, GemmShape<64, MP, 4, NW, D, 0>, 4>         \
     }
+// loader 3 with 32-row tiles (two 16-row MMA tiles per unit): 17 <= M <= 32
+#define Q4_TMA2_R32_VARIANT(ACT, T, MP, NW, D)                                                 \
+    Variant {                                                                                 \
+        ACT, 3, 64, MP, NW, D, 0, 0, &launch_tma<T, GemmShape<64, MP, 2, NW, D, 0>, 2>         \
+    }
 #define Q4_TMA2_VARIANT(ACT, T, MP, NW, D)                                                     \
     Variant {                                                                                 \
         ACT, 3, 64, MP, NW, D, 0, 0, &launch_tma<T, GemmShape<64, MP, 4, NW, D, 0>, 2>         \
@@ -1128,7 +1134,8 @@ struct Variant {
         Q4_VARIANT(ACT, T, 64, 16, 8, 1, 128), Q4_VARIANT(ACT, T, 32, 8, 16, 1, 128),         \
         Q4_VARIANT(ACT, T, 32, 16, 8, 1, 128), Q4_TMA_VARIANT(ACT, T, 8, 8, 2),               \
         Q4_TMA_VARIANT(ACT, T, 16, 8, 2), Q4_TMA2_VARIANT(ACT, T, 8, 16, 2),                  \
-        Q4_TMA2_VARIANT(ACT, T, 16, 8, 4), Q4_WS_VARIANT(ACT, T, 8, 8, 2), Q4_WS_VARIANT(ACT, T, 16, 8, 2)
+        Q4_TMA2_VARIANT(ACT, T, 16, 8, 4), Q4_WS_VARIANT(ACT, T, 8, 8, 2), Q4_WS_VARIANT(ACT, T, 16, 8, 2), \
+        Q4_TMA2_R32_VARIANT(ACT, T, 32, 8, 6)
 
 static const Variant kVariants[] = {
     Q4_VARIANTS_FOR(0, __nv_bfloat16),

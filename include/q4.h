@@ -129,7 +129,9 @@ int q4_gemm_workspace_size(int M, int N, int K, int blocksize, int act_dtype, si
  *   absmax   fp32 [N*K/blocksize], 4-byte aligned
  *   code     fp32 [16], 4-byte aligned
  *   M        0 is a no-op.  bf16/fp16: 1..16 on the mma.sync kernels;
- *            17..128 on the tcgen05 (tensor-memory) kernel, which also
+ *            17..32 on the mma.sync kernel with 32-row tiles when
+ *            blocksize >= 64 and (K / blocksize) % 4 == 0; otherwise (and
+ *            for 33..128) on the tcgen05 (tensor-memory) kernel, which
  *            needs blocksize >= 64, K % 256 == 0, (K / blocksize) % 4 == 0
  *            (else Q4_ERR_UNSUPPORTED) and a 16-byte aligned absmax (else
  *            Q4_ERR_MISALIGNED).  fp32: 1..16.  Larger M ->
@@ -189,9 +191,10 @@ typedef struct {
                        /* (fp32 activations), 3 = tcgen05 with tensor memory     */
     int sub_block;     /* k-width of one work unit: min(blocksize, 64); 512 for  */
                        /* math 2                                                 */
-    int m_pad;         /* M padded to the MMA column count: 8 or 16 (math 1),   */
+    int m_pad;         /* M padded to the MMA column count: 8, 16, 32 (math 1), */
                        /* 32/64/128 (math 3), 1/2/4/8/16 (math 2)                */
-    int rows_per_tile; /* weight rows per work unit                               */
+    int rows_per_tile; /* weight rows per work unit (32 for 17 <= M <= 32 on      */
+                       /* math 1, 64 below, 128 for math 3, R for math 2)        */
     int warps;         /* warps per CTA                                           */
     int ctas;          /* persistent CTAs (<= SM count, <= number of units)       */
     int depth;         /* work units each warp has in flight ahead of its compute */
@@ -219,8 +222,14 @@ int q4_gemm_plan(int M, int N, int K, int blocksize, int act_dtype, int num_sms,
  * depth, l2_prefetch, loader and pdl override the table when > 0 (all
  * other fields are ignored).  A combination that was not compiled returns
  * Q4_ERR_UNSUPPORTED; ctas above the SM count returns Q4_ERR_INVALID_ARG.
- * The workspace size needed does not depend on the overrides.
+ * Overrides that select another kernel (math = 3 below M = 33) change the
+ * workspace layout: size the workspace with q4_gemm_workspace_size_ex.
  */
+/* q4_gemm_workspace_size for a call with launch-table overrides (NULL: the
+ * same as q4_gemm_workspace_size).  Host-only. */
+int q4_gemm_workspace_size_ex(int M, int N, int K, int blocksize, int act_dtype, const q4_gemm_plan_t* overrides,
+                              size_t* bytes);
+
 int q4_gemm_skinny_ex(const void* A, const uint8_t* Wpacked, const float* absmax,
                       const float* code, int M, int N, int K, int blocksize, int act_dtype,
                       void* out, void* workspace, size_t workspace_bytes, void* stream,
@@ -254,7 +263,9 @@ int q4_gemm_skinny_bias(const void* A, const uint8_t* Wpacked, const float* absm
  * The rule, fitted to measurements on B200:
  *   - M <= 16 (bf16, fp16, fp32): fused (2.5-4.9x faster than the split
  *     path for bf16, 1.4-7.7x for fp32);
- *   - 17 <= M <= 64, bf16/fp16, with at least 2^26 weights (N*K): fused (the
+ *   - 17 <= M <= 32, bf16/fp16, blocksize >= 64 and (K / blocksize) % 4 == 0:
+ *     fused, on the mma.sync kernel with 32-row tiles (1.1-2.0x faster);
+ *   - 33 <= M <= 64, bf16/fp16, with at least 2^26 weights (N*K): fused (the
  *     tcgen05 kernel beats the split path there; below it, its fixed
  *     start-up and cross-CTA combine cost more than the split path saves);
  *   - everything else the fused entry rejects (M > 128, fp32 with M > 16,

@@ -93,7 +93,22 @@ def test_gemm_validation_before_cuda():
     assert ex(*args, 1, 64, 4096, 64, 0, ALIGNED, None, 0, None, b.overrides(math=2)) == b.Q4_ERR_UNSUPPORTED
 
 
-@pytest.mark.parametrize("M,N,K", [(17, 4096, 4096), (32, 300, 1024), (64, 28672, 8192), (128, 8192, 28672)])
+@pytest.mark.parametrize("M,N,K", [(17, 4096, 4096), (32, 300, 1024), (31, 8192, 28672)])
+def test_launch_table_m32(M, N, K):
+    """17 <= M <= 32: the mma.sync kernel with 32-row tiles and 2-unit stages."""
+    p = b.q4_gemm_plan(M, N, K, 64, num_sms=148)
+    assert p["math"] == 1 and p["loader"] == 3 and p["rows_per_tile"] == 32 and p["m_pad"] == 32
+    assert p["warps"] == 8 and p["depth"] == 6 and p["sub_block"] == 64
+    tiles = -(-N // 32)
+    assert p["tiles"] == tiles and p["units"] == tiles * (K // 64)
+    assert p["workspace_bytes"] == 256 + 148 * 2 * 4096 + -(-tiles * 4 // 256) * 256
+    # bs = 32 or (K / bs) % 4 != 0: the tensor-memory kernel's rules decide
+    assert b.q4_gemm_plan(24, 256, 4096, 128, num_sms=148)["math"] == 1
+    with pytest.raises(b.Q4Error):
+        b.q4_gemm_plan(24, 256, 4096, 32, num_sms=148)
+
+
+@pytest.mark.parametrize("M,N,K", [(33, 4096, 4096), (48, 300, 1024), (64, 28672, 8192), (128, 8192, 28672)])
 def test_launch_table_tcgen05(M, N, K):
     p = b.q4_gemm_plan(M, N, K, 64, num_sms=148)
     assert p["math"] == 3 and p["loader"] == 6 and p["rows_per_tile"] == 128 and p["sub_block"] == 64
@@ -193,9 +208,10 @@ def test_partition_invariants(total, parts):
 
 
 def test_route_table():
-    """Fused-vs-split advice: fused at M <= 16 (any dtype) and for the
-    tcgen05 kernel's M <= 64 on layers of >= 2^26 weights; split for the rest
-    and for everything the fused entry rejects."""
+    """Fused-vs-split advice: fused at M <= 16 (any dtype), at 17 <= M <= 32
+    on the 32-row mma.sync kernel, and for the tcgen05 kernel's M <= 64 on
+    layers of >= 2^26 weights; split for the rest and for everything the
+    fused entry rejects."""
     import torch
     F, S = b.Q4_ROUTE_FUSED, b.Q4_ROUTE_SPLIT
     cases = {(1, 8192, 8192, 64, torch.bfloat16): F, (16, 5120, 5120, 64, torch.float16): F,
@@ -203,9 +219,10 @@ def test_route_table():
              (17, 5120, 5120, 64, torch.float32): S,                       # fp32 stops at M = 16
              (32, 5120, 17408, 64, torch.bfloat16): F, (64, 5120, 17408, 64, torch.bfloat16): F,
              (65, 5120, 17408, 64, torch.bfloat16): S, (128, 5120, 17408, 64, torch.bfloat16): S,
-             (32, 5120, 5120, 64, torch.bfloat16): S, (32, 8192, 5120, 64, torch.bfloat16): S,
-             (32, 8192, 8192, 64, torch.bfloat16): F,                      # exactly 2^26 weights
-             (32, 5120, 17408, 32, torch.bfloat16): S,                     # tcgen05 needs blocksize >= 64
+             (32, 5120, 5120, 64, torch.bfloat16): F, (17, 8192, 5120, 64, torch.float16): F,  # 32-row mma.sync
+             (48, 5120, 5120, 64, torch.bfloat16): S, (48, 8192, 5120, 64, torch.bfloat16): S,
+             (48, 8192, 8192, 64, torch.bfloat16): F,                      # exactly 2^26 weights
+             (32, 5120, 17408, 32, torch.bfloat16): S,                     # both need blocksize >= 64
              (129, 8192, 8192, 64, torch.bfloat16): S, (4, 64, 4000, 64, torch.bfloat16): S}
     for (M, N, K, bs, dt), want in cases.items():
         assert b.q4_gemm_route(M, N, K, bs, dt) == want, (M, N, K, bs, dt)

@@ -37,8 +37,9 @@ def test_linear_matches_oracle(cuda_device, act, M, N, K, with_bias):
 
 @pytest.mark.parametrize("M", [32, 64])
 def test_linear_fused_tcgen05_route_sampled(cuda_device, M):
-    """A layer large enough for the tcgen05 route (>= 2^26 weights), checked on
-    sampled weight rows against the oracle."""
+    """A large layer on the fused route (M = 32: the 32-row mma.sync kernel;
+    M = 64: the tcgen05 kernel, >= 2^26 weights), checked on sampled weight
+    rows against the oracle."""
     dev = cuda_device
     N, K = 5120, 17408
     assert q4.q4_gemm_route(M, N, K, 64, torch.bfloat16) == q4.Q4_ROUTE_FUSED
