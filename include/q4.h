@@ -264,7 +264,8 @@ int q4_gemm_skinny_bias(const void* A, const uint8_t* Wpacked, const float* absm
  *   - M <= 16 (bf16, fp16, fp32): fused (2.5-4.9x faster than the split
  *     path for bf16, 1.4-7.7x for fp32);
  *   - 17 <= M <= 32, bf16/fp16, blocksize >= 64 and (K / blocksize) % 4 == 0:
- *     fused, on the mma.sync kernel with 32-row tiles (1.1-2.0x faster);
+ *     fused, on the mma.sync kernel with 32-row tiles (parity on 15-24 MB
+ *     layers, 1.9x faster on a 50 MB one);
  *   - 33 <= M <= 64, bf16/fp16, with at least 2^26 weights (N*K): fused (the
  *     tcgen05 kernel beats the split path there; below it, its fixed
  *     start-up and cross-CTA combine cost more than the split path saves);
