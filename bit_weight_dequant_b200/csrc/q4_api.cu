@@ -80,6 +80,19 @@ static size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 static constexpr size_t kWsHeader = 256;
 static size_t ws_counter_offset(int sms) { return kWsHeader + (size_t)sms * 2 * kMaxSlotBytes; }
 
+// With fewer tiles than SMs, one CTA per tile (every tile whole, no
+// cross-CTA fix-up at the end) beats spreading the units over every SM when
+// what the idle SMs would have streamed costs less time than the fix-up
+// saves.  Fitted to B200 measurements: the fix-up (publish, count, read back)
+// costs about 3 us at the end of a launch, and an SM streams about 34 KB/us
+// in the main loop.  Examples: K8192/N8192 (128 tiles, ~10 % faster), K5120/
+// N5120 (80 tiles, ~13 %), but not K28672/N8192 (128 tiles of 0.9 MB each).
+static bool data_parallel_pays(int tiles, int sms, int64_t weights) {
+    const double bytes = (double)weights * 0.5625;                // codes + absmax at blocksize 64
+    const double idle_us = (double)(sms - tiles) * bytes / ((double)tiles * sms * 34400.0);
+    return idle_us < 3.0;
+}
+
 // Validates a GEMM request.  Returns Q4_OK and fills `ch` with the launch
 // table's choice (with `ov` applied) and the problem's unit counts.
 static int gemm_choose(int M, int N, int K, int blocksize, int act_dtype, int num_sms, const q4_gemm_plan_t* ov,
@@ -220,6 +233,7 @@ static int gemm_choose(int M, int N, int K, int blocksize, int act_dtype, int nu
     const int t = N > 0 ? (N + c.rows_per_tile - 1) / c.rows_per_tile : 0;
     const int64_t u = (int64_t)t * (K / c.sub_block);
     int64_t g = (ov && ov->ctas > 0) ? ov->ctas : sms;
+    if (!(ov && ov->ctas > 0) && t >= 1 && t < sms && data_parallel_pays(t, sms, (int64_t)N * K)) g = t;
     if (g > u) g = u;  // every CTA owns at least one unit
     if (g < 1) g = 1;
     c.ctas = (int)g;
