@@ -492,8 +492,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (lds_u32(cw) == 0u) continue;
                     // Up to kFan contributors' values are loaded together before
                     // they are added in CTA order; more (small ranges) go in
-                    // further rounds of the same order.
-                    constexpr int kFan = 4;
+                    // further rounds of the same order.  Five covers a K = 5120
+                    // tile's contributors at 148 CTAs in one round; the 32-column
+                    // build keeps four, where five would spill.
+                    constexpr int kFan = MP == 32 ? 4 : 5;
 #pragma unroll 1
                     for (int m0 = 0; m0 < m16; m0 += 16) {
                         float sum[16];
