@@ -265,12 +265,6 @@ struct Act<__nv_bfloat16> {
         return *reinterpret_cast<uint32_t*>(&h);
     }
     __device__ __forceinline__ static __nv_bfloat16 from_float(float v) { return __float2bfloat16_rn(v); }
-    // Pairwise product of two packed pairs, each rounded once to nearest even.
-    __device__ __forceinline__ static uint32_t mul2(uint32_t a, uint32_t b) {
-        uint32_t d;
-        asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
-        return d;
-    }
 };
 
 // Operand format code of a 16-bit type in a tcgen05 instruction descriptor.
@@ -292,11 +286,6 @@ struct Act<__half> {
         return *reinterpret_cast<uint32_t*>(&h);
     }
     __device__ __forceinline__ static __half from_float(float v) { return __float2half_rn(v); }
-    __device__ __forceinline__ static uint32_t mul2(uint32_t a, uint32_t b) {
-        uint32_t d;
-        asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
-        return d;
-    }
 };
 
 // ---------------------------------------------------------------------------

@@ -159,6 +159,22 @@ __device__ __forceinline__ bool wait_parity(uint32_t bar, uint32_t parity) {
     return false;
 }
 
+// Pairwise product of two packed pairs of T, each rounded once to nearest even.
+template <typename T>
+__device__ __forceinline__ uint32_t mul2(uint32_t a, uint32_t b);
+template <>
+__device__ __forceinline__ uint32_t mul2<__nv_bfloat16>(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+template <>
+__device__ __forceinline__ uint32_t mul2<__half>(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+
 // Table row b (128 B): 32 copies, one per bank, of the pair (code[b >> 4],
 // code[b & 15]) rounded to T, the high nibble's value (the even k) in the
 // low half.  `code` is read once per thread and the pair gathered by
@@ -418,7 +434,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     for (int i = 0; i < 8; ++i)
 #pragma unroll
                         for (int q = 0; q < 4; ++q)
-                            v[4 * i + q] = Act<T>::mul2(lds_u32(lutl + (((words[i] >> (8 * q)) & 0xFFu) << 7)), am2);
+                            v[4 * i + q] = mul2<T>(lds_u32(lutl + (((words[i] >> (8 * q)) & 0xFFu) << 7)), am2);
                     tmem_st32(tbase + lane_bits + kColA + 32u * (uint32_t)b, v);
                     tmem_wait_st();
                     tc_fence_before();
