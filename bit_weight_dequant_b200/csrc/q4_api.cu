@@ -154,7 +154,7 @@ static int gemm_choose(int M, int N, int K, int blocksize, int act_dtype, int nu
         c.m_pad = M <= 32 ? 32 : M <= 64 ? 64 : 128;
         c.rows_per_tile = 128;
         c.loader = 6;
-        c.warps = 6;
+        c.warps = umma_warps();
         c.depth = 0;  // stages: as many as shared memory holds (set at launch)
         c.l2pf = 0;
         c.pdl = (ov && ov->pdl > 0) ? 1 : 0;  // activations and weights are read after the dependency wait

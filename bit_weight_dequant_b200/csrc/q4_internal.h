@@ -35,6 +35,7 @@ size_t gemm_slot_floats(int m_pad);
 // Tensor-memory (tcgen05) GEMM for 17 <= M <= 128 (q4_umma.cu).
 cudaError_t umma_launch(int act_dtype, int m_pad, const GemmParams& p, int smem_bytes, cudaStream_t stream);
 int umma_stages(int m_pad, int smem_bytes);
+int umma_warps();  // warps per CTA: producer, MMA issuer, dequantizing warpgroups
 size_t umma_slot_bytes(int m_pad);
 
 // fp32-activation GEMM on the CUDA cores, M <= 16 (q4_simt.cu): padded M,

@@ -638,6 +638,8 @@ int umma_stages(int mp, int smem_bytes) {
 
 size_t umma_slot_bytes(int mp) { return (size_t)mp * umma::kRows * 4; }
 
+int umma_warps() { return umma::kThreads / 32; }
+
 cudaError_t umma_launch(int act_dtype, int mp, const GemmParams& p, int smem, cudaStream_t stream) {
     if (act_dtype == 0) {
         if (mp == 32) return umma::launch<__nv_bfloat16, 32>(p, smem, stream);

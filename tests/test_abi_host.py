@@ -112,6 +112,7 @@ def test_launch_table_m32(M, N, K):
 def test_launch_table_tcgen05(M, N, K):
     p = b.q4_gemm_plan(M, N, K, 64, num_sms=148)
     assert p["math"] == 3 and p["loader"] == 6 and p["rows_per_tile"] == 128 and p["sub_block"] == 64
+    assert p["warps"] == 10  # producer, MMA issuer, two dequantizing warpgroups
     assert p["m_pad"] == (32 if M <= 32 else 64 if M <= 64 else 128)
     tiles = -(-N // 128)
     assert p["tiles"] == tiles and p["units"] == tiles * (K // 64)
