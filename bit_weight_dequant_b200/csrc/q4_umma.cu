@@ -262,8 +262,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_alloc(tslot, kTmemCols);
         tmem_relinquish();
     }
-    // The code table may be read before the dependency wait only in mode 2.
-    if (p.pdl >= 2) build_pair_table<T>(lut, p.code, tid);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -272,10 +270,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     // grid, and every stage carries activations: wait before any access.
     griddep_wait();
     griddep_launch_dependents();
-    if (p.pdl < 2) {
-        build_pair_table<T>(lut, p.code, tid);
-        __syncthreads();
-    }
+    build_pair_table<T>(lut, p.code, tid);
+    __syncthreads();
 
     const uint32_t cs = part_start(p.units, p.ctas, blockIdx.x);
     const uint32_t ce = part_start(p.units, p.ctas, blockIdx.x + 1);
