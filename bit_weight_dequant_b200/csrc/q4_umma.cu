@@ -19,21 +19,19 @@
 //                mbarriers that release the A buffer, the stage and, at the
 //                end of a tile, the accumulator.
 //   warps 2..9   two warpgroups taking alternate units, one thread per
-//                weight row.  Per 64-k unit the thread looks each of its
-//                row's 32 packed bytes up in a shared-memory table of code
-//                pairs (replicated once per bank, so a warp-wide lookup never
-//                conflicts), scales the pair by the block's absmax with one
-//                paired multiply in the activation type, and stores the 32
-//                pairs into a tensor-memory A buffer (tcgen05.st); at the end
-//                of a tile segment it reads its accumulator row back
-//                (tcgen05.ld) and stores, or publishes a partial.
+//                weight row.  Per 64-k unit the thread builds the 16 products
+//                bf16_rn(code[j] *_fp32 absmax) of its row -- exactly the
+//                values the standalone dequantizer writes, one rounding -- as
+//                byte-plane tables in registers, turns its 32 packed bytes
+//                into 32 bf16 pairs with byte permutes, and stores them into
+//                a tensor-memory A buffer (tcgen05.st); at the end of a tile
+//                segment it reads its accumulator row back (tcgen05.ld) and
+//                stores, or publishes a partial.
 //
-// The weights therefore enter the MMA as T_rn(T(code) * T(absmax)) (T the
-// activation type), within two roundings of T of the standalone
-// dequantizer's T_rn(code *_fp32 absmax).  The earlier per-row byte-permute
-// tables reproduced the latter exactly but made the loop bound by the
-// integer pipe (half rate for byte permutes) at about a third of the rate
-// the table lookups reach.
+// The one rounding matters: a weight rounded three times (a table of codes
+// already rounded to bf16, times a bf16 absmax, rounded again) can be 1.2 %
+// off, and a row of equal codes under one absmax adds those errors with one
+// sign, past the 1e-2 * sum|a w| bound.
 //
 // Work is split stream-K over units of 128 rows x 64 k like the M <= 16
 // kernel: a CTA's contiguous unit range may start and end inside tiles; such
@@ -58,7 +56,6 @@ constexpr int kRows = 128;                  // weight rows per tile = MMA M
 constexpr int kUps = 4;                     // 64-k units per stage
 constexpr uint32_t kWBytes = kRows * 128;   // packed codes of a stage (128 rows x 128 B)
 constexpr uint32_t kAmBytes = kRows * 16;   // absmax of a stage (128 rows x 4 floats)
-constexpr uint32_t kLutBytes = 256u * 128u;  // pair table: 256 byte values x 32 bank copies x 4 B
 constexpr uint32_t kTmemCols = 512;         // the whole tensor memory (one CTA per SM)
 constexpr uint32_t kColD0 = 0, kColD1 = 128, kColA = 256;  // A buffer b at kColA + 32 b
 constexpr int kNA = 8;                                       // A buffers (64-k units in flight)
@@ -159,36 +156,40 @@ __device__ __forceinline__ bool wait_parity(uint32_t bar, uint32_t parity) {
     return false;
 }
 
-// Pairwise product of two packed pairs of T, each rounded once to nearest even.
+// Byte planes of the row's 16 scaled codes: tl[k] / th[k] hold the low /
+// high bytes of values 4k .. 4k+3.
 template <typename T>
-__device__ __forceinline__ uint32_t mul2(uint32_t a, uint32_t b);
-template <>
-__device__ __forceinline__ uint32_t mul2<__nv_bfloat16>(uint32_t a, uint32_t b) {
-    uint32_t d;
-    asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
-    return d;
-}
-template <>
-__device__ __forceinline__ uint32_t mul2<__half>(uint32_t a, uint32_t b) {
-    uint32_t d;
-    asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
-    return d;
+__device__ __forceinline__ void scaled_tables(const float (&c)[16], float am, uint32_t (&tl)[4], uint32_t (&th)[4]) {
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        const uint32_t p0 = Act<T>::pack(__fmul_rn(c[4 * k], am), __fmul_rn(c[4 * k + 1], am));
+        const uint32_t p1 = Act<T>::pack(__fmul_rn(c[4 * k + 2], am), __fmul_rn(c[4 * k + 3], am));
+        tl[k] = prmt<0x6420u>(p0, p1);
+        th[k] = prmt<0x7531u>(p0, p1);
+    }
 }
 
-// Table row b (128 B): 32 copies, one per bank, of the pair (code[b >> 4],
-// code[b & 15]) rounded to T, the high nibble's value (the even k) in the
-// low half.  `code` is read once per thread and the pair gathered by
-// shuffles; the trip count is warp-uniform because kThreads and the 2048
-// 16-byte pieces are both multiples of 32.
-template <typename T>
-__device__ __forceinline__ void build_pair_table(uint32_t lut, const float* code, int tid) {
-    const float cv = __ldg(code + (tid & 15));
-    for (int e = tid; e < 256 * 8; e += kThreads) {
-        const int b = e >> 3;
-        const float hi = __shfl_sync(0xffffffffu, cv, b >> 4);
-        const float lo = __shfl_sync(0xffffffffu, cv, b & 15);
-        const uint32_t v = Act<T>::pack(hi, lo);
-        sts_v4(lut + (uint32_t)b * 128u + (uint32_t)(e & 7) * 16u, v, v, v, v);
+__device__ __forceinline__ uint32_t prmt_r(uint32_t a, uint32_t b, uint32_t sel) {
+    uint32_t r;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(sel));
+    return r;
+}
+
+// The four packed pairs of word w: byte q -> (value[hi nibble] in the low
+// half, value[lo nibble] in the high half), i.e. k = 2q then 2q + 1.
+__device__ __forceinline__ void word_pairs(uint32_t w, const uint32_t (&tl)[4], const uint32_t (&th)[4],
+                                           uint32_t* out) {
+    const uint32_t idx = w & 0x77777777u;          // index inside an 8-entry half
+    const uint32_t half = (w >> 1) & 0x44444444u;  // bit 3 of each nibble as +4 in a selector
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const uint32_t sel = h ? idx >> 16 : idx;
+        const uint32_t pick = (h ? half >> 16 : half) | 0x3210u;
+        const uint32_t l = prmt_r(prmt_r(tl[0], tl[1], sel), prmt_r(tl[2], tl[3], sel), pick);
+        const uint32_t u = prmt_r(prmt_r(th[0], th[1], sel), prmt_r(th[2], th[3], sel), pick);
+        // l / u bytes follow the nibbles lo0 hi0 lo1 hi1 of this half-word
+        out[2 * h] = prmt<0x4051u>(l, u);
+        out[2 * h + 1] = prmt<0x6273u>(l, u);
     }
 }
 
@@ -221,9 +222,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t sraw = smem_addr(smem_umma);
     const uint32_t base = (sraw + 1023u) & ~1023u;
     const int S = nstages;
-    // the pair table after the stages, then barriers and the tensor-memory address
-    const uint32_t lut = base + (uint32_t)S * G::STAGE;
-    const uint32_t bars = lut + kLutBytes;
+    // barriers and the tensor-memory address after the stages
+    const uint32_t bars = base + (uint32_t)S * G::STAGE;
     auto full = [&](int s) { return bars + 8u * (uint32_t)s; };
     auto sfree = [&](int s) { return bars + 8u * (uint32_t)(S + s); };
     const uint32_t aready = bars + 8u * (uint32_t)(2 * S), afree = aready + 8u * kNA;  // [kNA] each
@@ -270,8 +270,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     // grid, and every stage carries activations: wait before any access.
     griddep_wait();
     griddep_launch_dependents();
-    build_pair_table<T>(lut, p.code, tid);
-    __syncthreads();
 
     const uint32_t cs = part_start(p.units, p.ctas, blockIdx.x);
     const uint32_t ce = part_start(p.units, p.ctas, blockIdx.x + 1);
@@ -372,7 +370,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t lane_bits = (uint32_t)(32 * (warp & 3)) << 16;
         const int wg = (warp - 2) >> 2;                      // warpgroup: takes the units u with u % kNWG == wg
         const int ew = (warp - 2) & 3;                       // warp within the warpgroup
-        const uint32_t lutl = lut + (uint32_t)lane * 4u;  // this lane's bank copy
+        float c[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) c[j] = __ldg(p.code + j);
         const T* bias = static_cast<const T*>(p.bias);
         T* out = static_cast<T*>(p.out);
         if (nunits > 0) {
@@ -418,19 +418,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tc_fence_after();
                     const int col = ((kb0 + j) >> p.am_shift) - x0;
                     const float am = col == 0 ? amr[0] : col == 1 ? amr[1] : col == 2 ? amr[2] : amr[3];
-                    const uint32_t am2 = Act<T>::pack(am, am);
+                    uint32_t tl[4], th[4];
+                    scaled_tables<T>(c, am, tl, th);
                     // the row's 32 packed bytes of unit j: 16-byte chunks 2j, 2j+1 (128-byte swizzle)
                     const uint32_t rb = st + (uint32_t)row * 128u;
                     const uint4 w0 = lds_v4(rb + (uint32_t)(((2 * j) ^ (row & 7)) << 4));
                     const uint4 w1 = lds_v4(rb + (uint32_t)(((2 * j + 1) ^ (row & 7)) << 4));
                     const uint32_t words[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
-                    // byte q of word i holds k = 8i + 2q (high nibble) and 8i + 2q + 1: pair 4i + q
                     uint32_t v[32];
 #pragma unroll
-                    for (int i = 0; i < 8; ++i)
-#pragma unroll
-                        for (int q = 0; q < 4; ++q)
-                            v[4 * i + q] = mul2<T>(lds_u32(lutl + (((words[i] >> (8 * q)) & 0xFFu) << 7)), am2);
+                    for (int i = 0; i < 8; ++i) word_pairs(words[i], tl, th, v + 4 * i);
                     tmem_st32(tbase + lane_bits + kColA + 32u * (uint32_t)b, v);
                     tmem_wait_st();
                     tc_fence_before();
@@ -504,10 +501,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (lds_u32(cw) == 0u) continue;
                     // Up to kFan contributors' values are loaded together before
                     // they are added in CTA order; more (small ranges) go in
-                    // further rounds of the same order.  Five covers a K = 5120
-                    // tile's contributors at 148 CTAs in one round; the 32-column
-                    // build keeps four, where five would spill.
-                    constexpr int kFan = MP == 32 ? 4 : 5;
+                    // further rounds of the same order.
+                    constexpr int kFan = 4;
 #pragma unroll 1
                     for (int m0 = 0; m0 < m16; m0 += 16) {
                         float sum[16];
@@ -626,8 +621,8 @@ static cudaError_t launch(const GemmParams& p, int smem, cudaStream_t stream) {
 
 int umma_stages(int mp, int smem_bytes) {
     const int stage = (int)(umma::kWBytes + umma::kAmBytes) + umma::kUps * mp * 128;
-    // 1 KiB alignment slack, the pair table, barriers, tensor-memory slot and handshake words (< 512 B)
-    int s = (smem_bytes - 1024 - (int)umma::kLutBytes - 512) / stage;
+    // 1 KiB alignment slack + barriers, tensor-memory slot and handshake words (< 512 B)
+    int s = (smem_bytes - 1024 - 512) / stage;
     if (s > 6) s = 6;
     return s;
 }

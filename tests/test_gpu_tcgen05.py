@@ -2,10 +2,10 @@
 (and M <= 32 on request, math=3; the launch table sends 17 <= M <= 32 to the
 mma.sync kernel with 32-row tiles where its TMA rules hold): every output element within
 1e-2 * sum_k |a w| + ulp(y) of the oracle.  The weights enter the MMA as
-T_rn(T(code) * T(absmax)) (T = bf16, or fp16 for fp16 activations): a table
-lookup of the code pair and one paired multiply, within about 3 * 2^-9 of
-|w| for bf16; the fp32 accumulation follows.  The operation is the fused
-path of bitsandbytes PR #1920 ("Fused path support for M > 1") at larger M."""
+bf16_rn(code * absmax) (fp16 for fp16 activations), i.e. exactly the values
+the standalone dequantizer writes; the fp32 accumulation follows.  The
+operation is the fused path of bitsandbytes PR #1920 ("Fused path support
+for M > 1") at larger M."""
 import numpy as np
 import pytest
 import torch
