@@ -124,6 +124,18 @@ def weights(N: int, K: int, seed: int, outliers: bool = False) -> np.ndarray:
     return weight_rows(K, seed, 0, N, outliers)
 
 
+def weights_equal_codes(absmax_rows: np.ndarray, K: int, blocksize: int, value: float) -> np.ndarray:
+    """Adversarial W [len(absmax_rows), K] fp32: in every block of row n the
+    first element is absmax_rows[n] and the others are absmax_rows[n] * value
+    (one fp32 product), so each block quantizes to one +1 code and
+    blocksize - 1 copies of the code nearest `value`.  With non-negative
+    activations every weight's rounding error then has the same sign."""
+    am = np.asarray(absmax_rows, dtype=np.float32)
+    W = np.repeat((am * np.float32(value))[:, None], K, axis=1).astype(np.float32)
+    W[:, ::blocksize] = am[:, None]
+    return W
+
+
 def weights_device(N: int, K: int, seed: int, device, outliers: bool = False) -> torch.Tensor:
     """W ~ N(0, 0.02^2) drawn directly on a CUDA device with torch's seeded
     generator (for full-size runs where host generation is too slow).  Rows

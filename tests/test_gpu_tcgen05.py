@@ -123,3 +123,33 @@ def test_tcgen05_then_small_m_share_a_workspace(cuda_device):
                                 torch.from_numpy(absmax).to(cuda_device), torch.from_numpy(code).to(cuda_device),
                                 N, K, 64, workspace=ws, ctas=17)
         check_gemm(bits_of(out.cpu()), y, S, "bf16", f"shared workspace M{M} N{N}")
+
+
+@pytest.mark.parametrize("M", [16, 64])
+def test_equal_codes_under_one_absmax(cuda_device, M):
+    """Rows whose blocks hold one +1 code and 4095 copies of code 1/15 of the
+    uniform table, all-positive activations: the weights' rounding errors
+    share their sign, so the output error is the per-weight error itself.
+    The fused kernels round each weight once (at most 2^-8 for bf16) and stay
+    inside 1e-2 * S; a weight rounded three times (code and absmax each
+    rounded to bf16, then their product) is 1.01 % off at these absmax
+    values and would not.  M = 16 runs the mma.sync kernel, M = 64 the
+    tcgen05 kernel."""
+    dev = cuda_device
+    code = inputs.code_uniform()
+    base = np.float32(0.03308130428195)
+    am = np.array([base * np.float32(2.0 ** k) * np.float32(f) for k in range(-3, 5) for f in (1.0, 1.0001)],
+                  dtype=np.float32)
+    K, bs = 16384, 4096
+    W = inputs.weights_equal_codes(am, K, bs, float(code[8]))
+    N = W.shape[0]
+    packed, absmax = oracle.quantize(W, bs, code)
+    codes = np.stack([packed >> 4, packed & 15], -1).reshape(N, K)
+    assert np.array_equal(absmax, np.repeat(am, K // bs)) and (codes[:, ::bs] == 15).all()
+    assert (np.delete(codes, np.s_[::bs], axis=1) == 8).all()
+    A = torch.ones((M, K), dtype=torch.bfloat16)
+    y, S = oracle.gemm(bits_of(A), ORACLE_ACT["bf16"], packed, absmax, code, M, N, K, bs)
+    out = q4.q4_gemm_skinny(A.to(dev), torch.from_numpy(packed).to(dev), torch.from_numpy(absmax).to(dev),
+                            torch.from_numpy(code).to(dev), N, K, bs)
+    torch.cuda.synchronize(dev)
+    check_gemm(bits_of(out), y, S, "bf16", f"equal codes M{M}")
