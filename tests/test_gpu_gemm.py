@@ -187,7 +187,7 @@ def test_error_paths_leave_no_sticky_error(cuda_device, monkeypatch):
 
 def test_one_hot_activation_selects_dequantized_column(cuda_device):
     """A = e_k: out[0, n] = w[n, k] up to the kernel's rounding of the code to
-    bf16 before the MMA (relative 2^-9) and the final bf16 rounding, i.e.
+    bf16 before the MMA (relative 2^-8, bf16's unit roundoff) and the final bf16 rounding, i.e.
     within one bf16 ulp of the oracle's bf16(w[n, k])."""
     M, N, K, bs = 1, 300, 1024, 64
     code = inputs.code_normal_quantile()
