@@ -120,9 +120,12 @@ int q4_gemm_workspace_size(int M, int N, int K, int blocksize, int act_dtype, si
  * Fused dequantize + skinny matmul (PR #1920's kgemm_4bit_inference_naive
  * generalised to M > 1, "Fused path support for M > 1"):
  *     out[m, n] = round_rn_act( sum_k A[m,k] * code[idx(n,k)] * absmax(n,k) )
- * accumulated in fp32.  bf16/fp16: codes enter the tensor-core contraction
- * rounded to the activation dtype and the per-block absmax scale is applied
- * in fp32.  fp32 (the reply's SIMT kernel, which also takes fp32 inputs):
+ * accumulated in fp32.  bf16/fp16 on the mma.sync kernels (M <= 32): codes
+ * enter the tensor-core contraction rounded to the activation dtype T and the
+ * per-block absmax scale is applied in fp32; on the tcgen05 kernel the
+ * weights enter as T_rn(code *_fp32 absmax).  Either way each weight is
+ * rounded once (at most 2^-8 relative for bf16, 2^-11 for fp16).
+ * fp32 (the reply's SIMT kernel, which also takes fp32 inputs):
  * every product is an fp32 FMA with the exact fp32 code, scaled in fp32.
  *   A        [M, K] act_dtype, row-major contiguous, 16-byte aligned
  *   Wpacked  uint8 [N*K/2] (rows of K/2 bytes), 16-byte aligned
