@@ -78,3 +78,16 @@ def test_three_roundings_can_break_the_contract():
     worst = _max_rel(three, exact)
     assert worst > 1e-2  # a row of such weights under one absmax exceeds the bound
     assert worst <= (1 + u) ** 3 - 1
+
+
+@pytest.mark.parametrize("table", ["normal", "uniform", "fp4"])
+def test_two_roundings_fit_the_contract(table):
+    """The table form that stays admissible: codes rounded to bf16 in the
+    table, the absmax applied in fp32, one rounding of the product.  Two
+    roundings: at most (1 + 2^-8)^2 - 1, about 0.78 %, below 1e-2."""
+    rnd, u, _ = ROUND["bf16"]
+    code, am, exact = _grid(table, "bf16")
+    two = rnd(rnd(code)[None, :] * am[:, None])  # fp32 product of a bf16 code and the fp32 absmax
+    # the fp32 product rounds once more before bf16: at most 2^-24 on top
+    assert _max_rel(two, exact) <= ((1 + u) ** 2 - 1) * (1 + 2.0 ** -20)
+    assert (1 + u) ** 2 - 1 < 1e-2
