@@ -66,7 +66,7 @@ def test_one_rounding_stays_inside_the_contract(table, kind):
     tcgen05 = rnd((code[None, :].astype(np.float32) * am[:, None]))  # T_rn(code *_fp32 absmax)
     mma = rnd(code)[None, :].astype(np.float64) * am[:, None]         # T(code), absmax applied in fp32
     # the fp32 product itself adds at most 2^-24 before the rounding to T
-    assert _max_rel(tcgen05, exact) <= u * (1 + 2.0 ** -20)
+    assert _max_rel(tcgen05, exact) <= (1 + u) * (1 + 2.0 ** -24) - 1
     assert _max_rel(mma, exact) <= u
     assert u < 1e-2
 
@@ -89,5 +89,5 @@ def test_two_roundings_fit_the_contract(table):
     code, am, exact = _grid(table, "bf16")
     two = rnd(rnd(code)[None, :] * am[:, None])  # fp32 product of a bf16 code and the fp32 absmax
     # the fp32 product rounds once more before bf16: at most 2^-24 on top
-    assert _max_rel(two, exact) <= ((1 + u) ** 2 - 1) * (1 + 2.0 ** -20)
+    assert _max_rel(two, exact) <= (1 + u) ** 2 * (1 + 2.0 ** -24) - 1
     assert (1 + u) ** 2 - 1 < 1e-2
