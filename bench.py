@@ -174,7 +174,7 @@ class Layer:
     """One 4-bit linear layer resident on the device, with its C-ABI call
     arguments prepared once (the timed loop only makes the call)."""
 
-    def __init__(self, case: inputs.Case, seed: int, device, pdl: int = 2):
+    def __init__(self, case: inputs.Case, seed: int, device, pdl: int = 2, launch: dict | None = None):
         self.case = case
         dt = TORCH_ACT[case.act]
         code = inputs.CODE_TABLES[case.table]()
@@ -187,7 +187,8 @@ class Layer:
         self.A = self.A_host.to(device)
         self.out = torch.empty((case.M, case.N), dtype=dt, device=device)
         self.out_host = torch.empty((case.M, case.N), dtype=dt).pin_memory()
-        self.ws_bytes = q4.q4_gemm_workspace_size(case.M, case.N, case.K, case.blocksize, dt)
+        self.launch_kw = {k: v for k, v in (launch or {}).items() if v}
+        self.ws_bytes = q4.q4_gemm_workspace_size(case.M, case.N, case.K, case.blocksize, dt, **self.launch_kw)
         self.ws = torch.zeros(max(self.ws_bytes, 16), dtype=torch.uint8, device=device)
         self.act = {"bf16": q4.Q4_BF16, "fp16": q4.Q4_FP16, "fp32": q4.Q4_FP32}[case.act]
         self.plan = q4.q4_gemm_plan(case.M, case.N, case.K, case.blocksize, dt)
@@ -195,7 +196,7 @@ class Layer:
         # Decode-time weights are static model parameters: let each GEMM's
         # prologue and first weight copies overlap the previous kernel.
         self.pdl = pdl
-        self._ov = q4.overrides(pdl=pdl)
+        self._ov = q4.overrides(pdl=pdl, **self.launch_kw)
         self.bytes = case.algorithmic_bytes()
 
     def rebind(self, A: torch.Tensor, out: torch.Tensor):
@@ -409,7 +410,8 @@ def run_ours(args, world, rank, local):
     cases = [(i, c) for i, c in enumerate(wl.cases) if not args.only or c.tag in args.only.split(",")]
     if not cases:
         raise SystemExit(f"--only {args.only!r} matches no case of {args.workload}")
-    layers = [Layer(c, inputs.seed_for(wl.index, c.M) + i, device, args.pdl) for i, c in cases]
+    launch = {"loader": args.loader, "depth": args.depth, "l2_prefetch": args.l2_ahead, "ctas": args.ctas}
+    layers = [Layer(c, inputs.seed_for(wl.index, c.M) + i, device, args.pdl, launch) for i, c in cases]
     host_in, dev_in, host_out, dev_out = bind_step_io(layers, device)
     torch.cuda.synchronize()
     step_bytes = sum(L.bytes for L in layers)
@@ -654,6 +656,10 @@ def main():
     ap.add_argument("--only", default="", help="comma-separated case tags of the workload to run (profiling)")
     ap.add_argument("--split-path", action="store_true",
                     help="also time the split path (dequantize kernel + cuBLAS bf16 GEMM) per layer")
+    ap.add_argument("--loader", type=int, default=0, help="launch-table override: GEMM loader (measurement)")
+    ap.add_argument("--depth", type=int, default=0, help="launch-table override: depth (measurement)")
+    ap.add_argument("--l2-ahead", type=int, default=0, help="launch-table override: l2_prefetch (measurement)")
+    ap.add_argument("--ctas", type=int, default=0, help="launch-table override: CTAs (measurement)")
     ap.add_argument("--pdl", type=int, default=2, choices=[0, 1, 2],
                     help="programmatic dependent launch mode for the GEMMs (2: static weights read early)")
     args = ap.parse_args()

@@ -126,8 +126,10 @@ def q4_dequantize_blockwise(packed: torch.Tensor, absmax: torch.Tensor, code: to
     return out
 
 
-def q4_gemm_workspace_size(M: int, N: int, K: int, blocksize: int, act_dtype: torch.dtype) -> int:
-    return _workspace_bytes(M, N, K, blocksize, _TORCH_TO_Q4[act_dtype])
+def q4_gemm_workspace_size(M: int, N: int, K: int, blocksize: int, act_dtype: torch.dtype, **launch) -> int:
+    """Workspace bytes for a call (with the same launch-table overrides as
+    the call, if any)."""
+    return _workspace_bytes(M, N, K, blocksize, _TORCH_TO_Q4[act_dtype], tuple(sorted(launch.items())))
 
 
 @functools.lru_cache(maxsize=4096)

@@ -64,6 +64,17 @@ static bool injected_failure() {
     return v && v[0] && std::strcmp(v, "0") != 0;
 }
 
+// Test hook for the row-split kernel: Q4_TEST_SKIP_STAGE=<i> makes each
+// CTA's producer leave stage i unloaded, with short wait limits, so the
+// kernel's bounded waits run out and it reports error word 1 (no GPU fault:
+// every wait is bounded, every copy that was issued is waited for).
+static int injected_stage_skip() {
+    const char* v = std::getenv("Q4_TEST_SKIP_STAGE");
+    if (!v || !v[0]) return -1;
+    const int i = std::atoi(v);
+    return i >= 0 ? i : -1;
+}
+
 static int from_cuda(cudaError_t e) {
     if (e == cudaSuccess) return Q4_OK;
     cudaGetLastError();  // drain: leave no error of ours pending
@@ -100,7 +111,7 @@ static int gemm_choose(int M, int N, int K, int blocksize, int act_dtype, int nu
     if (M < 0 || N < 0 || K < 0) return Q4_ERR_INVALID_ARG;
     if (!is_pow2_blocksize(blocksize)) return Q4_ERR_INVALID_ARG;
     if (act_dtype != Q4_BF16 && act_dtype != Q4_FP16 && act_dtype != Q4_FP32) return Q4_ERR_INVALID_ARG;
-    if (ov && (ov->math > 3 || ov->l2_prefetch > 256 || ov->loader > 6 || ov->pdl > 2)) return Q4_ERR_INVALID_ARG;
+    if (ov && (ov->math > 3 || ov->l2_prefetch > 256 || ov->loader > 7 || ov->pdl > 2)) return Q4_ERR_INVALID_ARG;
     if (M > 128 || K % blocksize != 0) return Q4_ERR_UNSUPPORTED;
     GemmChoice c{};
     if (act_dtype == Q4_FP32) {
@@ -187,9 +198,36 @@ static int gemm_choose(int M, int N, int K, int blocksize, int act_dtype, int nu
     // multiples of 16 bytes (a tensor-map stride rule); the pointer itself
     // must also be 16-byte aligned, which the caller checks at launch.
     const bool tma_ok = c.sub_block == 64 && (K / blocksize) % 4 == 0 && (int64_t)N * (K / 64) > 1;
-    c.loader = mma32 ? 3 : tma_ok ? 2 : 1;
+    c.loader = mma32 ? 3 : tma_ok ? 7 : 1;
     if (ov && ov->loader > 0) c.loader = ov->loader;
     if (c.loader >= 2 && !tma_ok) return Q4_ERR_UNSUPPORTED;
+    if (c.loader == 7) {
+        // Row-split kernel: 8-row groups of W split over the CTAs, one shared
+        // stage ring per CTA, no cross-CTA combine (workspace: the error word).
+        if (M > 16) return Q4_ERR_UNSUPPORTED;
+        c.warps = rows_warps();
+        c.depth = (ov && ov->depth > 0) ? ov->depth : 2;  // stage order: 1 round robin, 2 contiguous per warp
+        if (c.depth > 2) return Q4_ERR_UNSUPPORTED;
+        c.l2pf = (ov && ov->l2_prefetch > 1) ? ov->l2_prefetch : 0;
+        c.pdl = (ov && ov->pdl > 0) ? ov->pdl : 0;
+        if (ov && ov->warps > 0 && ov->warps != c.warps) return Q4_ERR_UNSUPPORTED;
+        if (ov && ov->math > 0 && ov->math != 1) return Q4_ERR_UNSUPPORTED;
+        if (!gemm_variant_exists(act_dtype, c)) return Q4_ERR_UNSUPPORTED;
+        int sms = num_sms;
+        if (sms <= 0 && device_sm_count(&sms) != 0) return Q4_ERR_CUDA;
+        if (ov && ov->ctas > sms) return Q4_ERR_INVALID_ARG;
+        const int64_t groups = N > 0 ? ((int64_t)N + 7) / 8 : 0;
+        int64_t g = (ov && ov->ctas > 0) ? ov->ctas : sms;
+        if (g > groups) g = groups;
+        if (g < 1) g = 1;
+        c.ctas = (int)g;
+        *ch = c;
+        *tiles = N > 0 ? (N + 63) / 64 : 0;
+        *units = (int64_t)*tiles * (K / 64);
+        *sms_out = sms;
+        *ws_bytes = kWsHeader;  // the error word only
+        return Q4_OK;
+    }
     if (mma32) {
         // 32-row tiles: 2-unit stages (64-byte rows), six per warp
         c.warps = 8;
@@ -403,6 +441,34 @@ static int gemm_entry(const void* A, const uint8_t* Wpacked, const float* absmax
         int lbs = 0;
         while ((1 << lbs) < blocksize) ++lbs;
         return from_cuda(simt_launch(simt_shape(M), ch.ctas, p, lbs, st));
+    }
+    if (ch.loader == 7) {
+        RowsParams rp{};
+        rp.A = A;
+        rp.out = out;
+        rp.bias = bias;
+        rp.code = code;
+        rp.error = static_cast<int*>(workspace);
+        rp.M = M;
+        rp.N = N;
+        rp.K = K;
+        rp.am_shift = sh;
+        rp.groups = (N + 7) / 8;
+        rp.ctas = ch.ctas;
+        rp.pdl = ch.pdl;
+        rp.l2_ahead = ch.l2pf;
+        rp.contig = ch.depth == 2 ? 1 : 0;
+        rp.wait_limit = kWaitLimit;
+        rp.skip_stage = -1;
+        if (const int skip = injected_stage_skip(); skip >= 0) {
+            rp.skip_stage = skip;
+            rp.wait_limit = 1u << 14;  // run out within microseconds
+        }
+        int smem = 0, dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
+            return from_cuda(cudaGetLastError());
+        return from_cuda(rows_launch(act_dtype, ch.m_pad, rp, Wpacked, absmax, K / blocksize, smem, st));
     }
     if (ch.math == 3) {
         if (workspace)

@@ -7,6 +7,8 @@
 #include <cuda_fp16.h>
 #include <stdint.h>
 
+#include "q4_plan.cuh"
+
 namespace q4 {
 
 // ---------------------------------------------------------------------------
@@ -154,6 +156,16 @@ __device__ __forceinline__ void ldmatrix_x4(uint32_t addr, uint32_t& d0, uint32_
                  : "r"(addr));
 }
 
+// ldmatrix_x4 done only when `on` (warp-uniform); zeros otherwise.
+__device__ __forceinline__ void ldmatrix_x4_if(uint32_t addr, uint32_t on, uint32_t& d0, uint32_t& d1, uint32_t& d2,
+                                               uint32_t& d3) {
+    asm volatile(
+        "{\n .reg .pred p;\n setp.ne.u32 p, %5, 0;\n mov.b32 %0, 0;\n mov.b32 %1, 0;\n mov.b32 %2, 0;\n"
+        " mov.b32 %3, 0;\n @p ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];\n}\n"
+        : "=r"(d0), "=r"(d1), "=r"(d2), "=r"(d3)
+        : "r"(addr), "r"(on));
+}
+
 // ---------------------------------------------------------------------------
 // mbarrier + TMA (bulk tensor copies, no multicast).
 // ---------------------------------------------------------------------------
@@ -199,6 +211,14 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     return ok != 0;
 }
 
+// Every wait on an mbarrier is bounded (kWaitLimit polls by default, see
+// q4_plan.cuh).
+__device__ __forceinline__ bool wait_stage(uint32_t bar, uint32_t parity, uint32_t limit = kWaitLimit) {
+    for (uint32_t it = 0; it < limit; ++it)
+        if (mbar_try_wait(bar, parity)) return true;
+    return false;
+}
+
 // Orders this thread's earlier generic-proxy shared-memory accesses before
 // later async-proxy (TMA) accesses.
 __device__ __forceinline__ void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
@@ -218,6 +238,13 @@ __device__ __forceinline__ void tma_load_2d_hint(uint32_t dst, const void* tmap,
         " [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(dst),
         "l"(tmap), "r"(x), "r"(y), "r"(bar), "l"(policy)
         : "memory");
+}
+
+// Hint that the box at {x, y} of a tensor map will soon be read: the L2
+// fetches it from DRAM now (no shared memory, no completion to wait for).
+__device__ __forceinline__ void tma_prefetch_l2_2d(const void* tmap, int x, int y) {
+    asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(tmap), "r"(x), "r"(y)
+                 : "memory");
 }
 
 // L2 policy for data read exactly once: its lines are the first candidates
@@ -248,6 +275,31 @@ __device__ __forceinline__ uint32_t prmt(uint32_t lo, uint32_t hi) {
     uint32_t r;
     asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(lo), "r"(hi), "n"(SEL));
     return r;
+}
+
+// CTA-scope atomic add on a shared-memory word with acquire-release
+// semantics (publishes this thread's earlier shared writes, observes the
+// writes published by earlier adds).
+__device__ __forceinline__ int atom_add_acq_rel_cta_smem(uint32_t addr, int v) {
+    int old;
+    asm volatile("atom.acq_rel.cta.shared::cta.add.s32 %0, [%1], %2;" : "=r"(old) : "r"(addr), "r"(v) : "memory");
+    return old;
+}
+
+// CTA-scope release add on a shared-memory word (no return value).
+__device__ __forceinline__ void red_add_release_cta_smem(uint32_t addr, uint32_t v) {
+    asm volatile("red.release.cta.shared::cta.add.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+
+// Polls a shared-memory counter (acquire loads) until it reaches `target`;
+// false after `limit` polls.
+__device__ __forceinline__ bool wait_count_at_least(uint32_t addr, uint32_t target, uint32_t limit) {
+    for (uint32_t it = 0; it < limit; ++it) {
+        uint32_t v;
+        asm volatile("ld.acquire.cta.shared::cta.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+        if (v >= target) return true;
+    }
+    return false;
 }
 
 // ---------------------------------------------------------------------------
@@ -318,6 +370,55 @@ __device__ __forceinline__ void mma16816<__half>(float (&d)[4], uint32_t a0, uin
         : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(c[0]), "f"(c[1]), "f"(c[2]),
           "f"(c[3]));
+}
+
+// ---------------------------------------------------------------------------
+// Byte-pair code table in shared memory.
+//
+// Row b (256 bytes) holds 32 copies, one per bank, of the packed pair
+// (code[b >> 4], code[b & 15]) in the activation type -- the first (even)
+// element in the low half -- i.e. exactly one MMA A-fragment register for a
+// packed byte.  Only the lower 128 bytes of a row are the table; the upper
+// halves are free scratch.  The table sits on a 64 KiB boundary of the
+// shared window, so ONE byte permute builds a lookup address
+// (table base | byte << 8 | lane << 2) from a packed word, and a warp-wide
+// lookup never has a bank conflict.
+// ---------------------------------------------------------------------------
+static constexpr uint32_t kLutBytes = 256u * 256u;
+
+// One lookup: byte BYTE of `word` -> packed (code[hi], code[lo]).  `lane4` =
+// table base | lane << 2.
+template <int BYTE>
+__device__ __forceinline__ uint32_t lut_pair(uint32_t word, uint32_t lane4) {
+    // result bytes: [0] = lane4.b0 (lane*4), [1] = word.b<BYTE>, [2..3] = lane4.b2..b3 (table base >> 16)
+    return lds_u32(prmt<0x7604u | (BYTE << 4)>(word, lane4));
+}
+
+// The same lookup, done only when `on` (a warp-uniform flag; 0 otherwise):
+// predicated, so that a block of lookups stays straight-line code.
+template <int BYTE>
+__device__ __forceinline__ uint32_t lut_pair_if(uint32_t word, uint32_t lane4, uint32_t on) {
+    uint32_t v;
+    asm volatile(
+        "{\n .reg .pred p;\n setp.ne.u32 p, %2, 0;\n mov.b32 %0, 0;\n @p ld.shared.b32 %0, [%1];\n}\n"
+        : "=r"(v)
+        : "r"(prmt<0x7604u | (BYTE << 4)>(word, lane4)), "r"(on));
+    return v;
+}
+
+// Builds the table.  `cv` is code[lane & 15] in every lane; the pair is
+// gathered by shuffles, so the table costs one global load per thread.
+// nthreads is a multiple of 32 that divides the 2048 row pieces evenly per
+// warp (the shuffles need whole warps).
+template <typename T>
+__device__ __forceinline__ void build_lut(uint32_t lut, float cv, int tid, int nthreads) {
+    for (int e = tid; e < 256 * 8; e += nthreads) {
+        const int b = e >> 3;
+        const float hi = __shfl_sync(0xffffffffu, cv, b >> 4);
+        const float lo = __shfl_sync(0xffffffffu, cv, b & 15);
+        const uint32_t v = Act<T>::pack(hi, lo);
+        sts_v4(lut + (uint32_t)b * 256u + (uint32_t)(e & 7) * 16u, v, v, v, v);
+    }
 }
 
 }  // namespace q4

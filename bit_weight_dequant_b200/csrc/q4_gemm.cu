@@ -94,13 +94,6 @@ __device__ __forceinline__ void load_unit(Unit<S>& u, const GemmParams& p, int t
     }
 }
 
-// One table lookup: byte BYTE of `word` -> packed (code[hi], code[lo]).
-template <int BYTE>
-__device__ __forceinline__ uint32_t lut_pair(uint32_t word, uint32_t lane4) {
-    // result bytes: [0] = lane4.b0 (lane*4), [1] = word.b<BYTE>, [2..3] = lane4.b2..b3 (table base >> 16)
-    return lds_u32(prmt<0x7604u | (BYTE << 4)>(word, lane4));
-}
-
 template <typename T, class S>
 __device__ __forceinline__ void mma_unit(float (&acc)[S::TW][S::NJ][4], const Unit<S>& u, uint32_t lane4) {
     const float zero[4] = {0.f, 0.f, 0.f, 0.f};
@@ -297,21 +290,6 @@ __device__ __forceinline__ void combine_tiles(const GemmParams& p, uint32_t slot
     }
 }
 
-// Table row b (256 B): 32 copies (one per bank) of the pair (code[b>>4], code[b&15]) as T.
-// `cv` is code[lane & 15] in every lane; the pair is gathered by shuffles, so
-// the table costs one global load per thread.  nthreads is a multiple of 32
-// that divides the 2048 row pieces evenly per warp (the shuffles need whole warps).
-template <typename T>
-__device__ __forceinline__ void build_lut(uint32_t lut, float cv, int tid, int nthreads) {
-    for (int e = tid; e < 256 * 8; e += nthreads) {
-        const int b = e >> 3;
-        const float hi = __shfl_sync(0xffffffffu, cv, b >> 4);
-        const float lo = __shfl_sync(0xffffffffu, cv, b & 15);
-        const uint32_t v = Act<T>::pack(hi, lo);
-        sts_v4(lut + (uint32_t)b * 256u + (uint32_t)(e & 7) * 16u, v, v, v, v);
-    }
-}
-
 template <typename T, class S>
 __global__ void __launch_bounds__(S::NW * 32, 1) q4_gemm_mma_kernel(const GemmParams p) {
     griddep_wait();  // no overlap with a preceding grid in this kernel
@@ -407,10 +385,6 @@ struct StageGeom {
             return base + (uint32_t)row * 64u + (uint32_t)((chunk ^ ((row >> 1) & 3)) << 4);
     }
 };
-static constexpr uint32_t kWaitLimit = 1u << 20;  // try_wait polls before giving up
-
-static constexpr int kErrWaitTimeout = 1;
-static constexpr int kErrNoRoom = 2;
 
 struct StageCursor {
     int tile, kb, left;  // next unit to put in a stage; units of the range still unassigned
@@ -433,12 +407,6 @@ __device__ __forceinline__ void next_stage(StageCursor& c, int kb_per_tile, int&
         c.kb = 0;
         ++c.tile;
     }
-}
-
-__device__ __forceinline__ bool wait_stage(uint32_t bar, uint32_t parity) {
-    for (uint32_t it = 0; it < kWaitLimit; ++it)
-        if (mbar_try_wait(bar, parity)) return true;
-    return false;
 }
 
 // The first partial tile of a warp waits for the combine in the upper half
@@ -991,7 +959,7 @@ static cudaError_t launch_mma(const GemmParams& p, cudaStream_t stream) {
 
 // cuTensorMapEncodeTiled through the runtime's driver entry point (no link
 // against libcuda; the driver is already loaded by the runtime).
-static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
     static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
     static std::once_flag once;
     std::call_once(once, [] {
@@ -1164,9 +1132,19 @@ static const Variant* find_variant(int act, const GemmChoice& ch) {
     return nullptr;
 }
 
-bool gemm_variant_exists(int act_dtype, const GemmChoice& ch) { return find_variant(act_dtype, ch) != nullptr; }
+// Loader 7 is the row-split kernel (q4_rows.cu): bf16/fp16, 64-k units,
+// one or two n8 column tiles, the stage ring sized from shared memory.
+static bool rows_variant(int act_dtype, const GemmChoice& ch) {
+    return ch.loader == 7 && (act_dtype == 0 || act_dtype == 1) && ch.sub_block == 64 &&
+           (ch.m_pad == 8 || ch.m_pad == 16) && ch.warps == rows_warps();
+}
+
+bool gemm_variant_exists(int act_dtype, const GemmChoice& ch) {
+    return rows_variant(act_dtype, ch) || find_variant(act_dtype, ch) != nullptr;
+}
 
 size_t gemm_smem_bytes(int act_dtype, const GemmChoice& ch) {
+    if (rows_variant(act_dtype, ch)) return (size_t)max_dynamic_smem();
     const Variant* v = find_variant(act_dtype, ch);
     if (!v) return 0;
     return v->loader >= 2 ? (size_t)max_dynamic_smem() : v->smem;

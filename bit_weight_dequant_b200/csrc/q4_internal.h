@@ -2,6 +2,8 @@
 // (launchers, launch-table choice, per-device attribute cache).
 #pragma once
 
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -46,6 +48,17 @@ struct SimtShape {
 SimtShape simt_shape(int M);
 size_t simt_smem_bytes();
 cudaError_t simt_launch(const SimtShape& sh, int ctas, const GemmParams& p, int log2_bs, cudaStream_t stream);
+
+// Row-split kernel for M <= 16 with 16-bit activations (q4_rows.cu).
+// act_dtype 0 = bf16, 1 = fp16; m_pad 8 or 16; smem = dynamic shared memory
+// to launch with (the kernel sizes its stage ring from it).
+cudaError_t rows_launch(int act_dtype, int m_pad, const RowsParams& p, const uint8_t* Wp, const float* absmax,
+                        int am_per_row, int smem, cudaStream_t stream);
+int rows_warps();  // warps per CTA
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point, or
+// nullptr when the driver does not provide it.
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder();
 
 cudaError_t quantize_launch(const void* W, int w_dtype, int64_t n, int blocksize, const float* code,
                             uint8_t* packed, float* absmax, cudaStream_t stream);

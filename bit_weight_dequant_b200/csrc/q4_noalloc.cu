@@ -68,10 +68,12 @@ extern "C" int q4_gemm_skinny_noalloc(const void* A, const uint8_t* Wpacked, con
     // allocates nothing); the slots are written before they are read.
     int sms = 0;
     if (q4::device_sm_count(&sms) != 0) return Q4_ERR_CUDA;
+    // (A kernel whose workspace is the header alone -- the row-split kernel --
+    // has no counters to clear.)
     const size_t counters = 256 + (size_t)sms * 2 * q4::kMaxSlotBytes;
     cudaStream_t st = (cudaStream_t)stream;
     if (cudaMemsetAsync(ws, 0, 256, st) != cudaSuccess ||
-        cudaMemsetAsync(static_cast<char*>(ws) + counters, 0, need - counters, st) != cudaSuccess) {
+        (need > counters && cudaMemsetAsync(static_cast<char*>(ws) + counters, 0, need - counters, st) != cudaSuccess)) {
         cudaGetLastError();
         return Q4_ERR_CUDA;
     }

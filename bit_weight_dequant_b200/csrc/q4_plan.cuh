@@ -32,6 +32,13 @@ __host__ __device__ __forceinline__ uint32_t part_owner(uint32_t total, uint32_t
 inline int64_t part_start64(int64_t total, int parts, int p) { return (total * (int64_t)p) / parts; }
 inline int part_owner64(int64_t total, int parts, int64_t u) { return (int)(((u + 1) * (int64_t)parts - 1) / total); }
 
+// Every wait on an mbarrier is bounded: after kWaitLimit polls the kernel
+// records an error word in the workspace, drains what it started (also
+// bounded) and returns; its outputs are then not valid.
+static constexpr uint32_t kWaitLimit = 1u << 20;  // try_wait polls before giving up
+static constexpr int kErrWaitTimeout = 1;         // a bounded wait ran out
+static constexpr int kErrNoRoom = 2;              // the launch gave too little shared memory
+
 // Largest unit count the kernels accept (keeps total * parts below 2^32 for
 // up to 512 parts).
 static constexpr uint32_t kMaxUnits = (1u << 23);
@@ -81,6 +88,31 @@ struct GemmParams {
     int tiles;
     int ctas;
     uint32_t units;    // < kMaxUnits
+};
+
+// Most distinct tile heights (tensor-map pairs) of one row-split launch:
+// two for each of the two group counts a CTA can have.
+static constexpr int kRowsMaxMaps = 4;
+
+// Runtime parameters of one launch of the row-split kernel (q4_rows.cu):
+// CTA c owns a contiguous run of 8-row groups of W and finishes its outputs
+// itself (no workspace besides the error word).
+struct RowsParams {
+    const void* A;
+    void* out;
+    const void* bias;  // [N] activation type, or nullptr
+    const float* code;
+    int* error;        // workspace error word, or nullptr
+    int M, N, K;
+    int am_shift;      // log2(blocksize / 64)
+    int groups;        // ceil(N / 8)
+    int ctas;          // <= groups
+    int pdl;           // dependent launch mode (0, 1, 2), as in GemmParams
+    int l2_ahead;      // stages the producer asks the L2 to fetch beyond the first ring fill
+    uint32_t wait_limit;  // polls before a wait on a stage or a parking buffer gives up
+    int skip_stage;       // test hook: this stage index is never loaded (-1: none)
+    int contig;           // 1: each warp streams a contiguous range of stages (0: round robin)
+    int map_of[10];       // tensor-map pair of tile height h (8 .. 72 rows): map_of[h / 8], filled by the launcher
 };
 
 }  // namespace q4

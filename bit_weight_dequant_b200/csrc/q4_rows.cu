@@ -1,0 +1,616 @@
+// q4_rows.cu -- row-split fused dequantize + skinny GEMM for sm_100a, M <= 16.
+//
+//     out[m, n] = sum_k A[m, k] * code[idx(n, k)] * absmax(n, k)
+//
+// The operation of bitsandbytes PR #1920 ("[ROCm] Optimize
+// kgemm_4bit_inference_naive ...", "Technical details" and "Fused path
+// support for M > 1"), with the same inner step as the stream-K kernel in
+// q4_gemm.cu (byte-pair table lookups feeding mma.sync m16n8k16 with the
+// matrix roles swapped, fp32 absmax applied once per 64-k block), organised
+// so that a launch carries no cross-CTA work at all:
+//
+//  * Rows, not units, are split over the CTAs.  CTA c owns a contiguous run
+//    of whole weight rows (8-row groups; the larger shares go to the lowest
+//    block indices, which the hardware places first), so every output
+//    element is finished inside one CTA: no partial sums in global memory,
+//    no counters, no last-arriver fix-up at the end of the launch.  The
+//    shares differ by at most one 8-row group.
+//  * A CTA's rows form tiles of nearly equal height (at most 72 rows; the
+//    larger heights first).  A stage is one tile's rows x 256 k of packed
+//    codes (128-byte swizzle) plus its absmax box: one TMA box per stage,
+//    one tensor map per height.
+//  * The stages stream through ONE shared ring of D mbarrier-guarded slots,
+//    and warp w computes stages w, w + W, w + 2W, ...  A warp first copies
+//    its stage into registers (code fragments and absmax), then refills the
+//    slot with stage i + D itself -- no producer warp, no "slot free"
+//    barriers, and every slot is prefetch depth, not held during compute.
+//    The warps advance in lockstep (no warp can run ahead of the ring)
+//    instead of each draining its own range at its own pace, so they finish
+//    within about one stage of each other.
+//  * The stages of a tile run in a loop instantiated for the tile's shape
+//    (16-row MMA tiles, half last tile), dispatched once per tile: each
+//    stage is one straight-line block in which the four units' lookup and
+//    MMA chains interleave; rows past a half tile do no lookups.
+//  * Each warp sums its stages of a tile in registers; when it leaves the
+//    tile it parks the partial tile in shared memory, and the last warp to
+//    do so adds the parked partials in stage order (deterministic) and
+//    stores the tile.  Two parking buffers alternate between tiles.
+//  * Under programmatic dependent launch (mode 2) the weights are static:
+//    the ring's first fill (and, optionally, an L2 prefetch of the stages
+//    after it) goes out before the dependency wait, and the table is built
+//    meanwhile.  Activations and outputs are touched only after the wait.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include <type_traits>
+
+#include "q4_device.cuh"
+#include "q4_internal.h"
+#include "q4_plan.cuh"
+
+namespace q4 {
+namespace rows {
+
+constexpr int kW = 8;                // warps per CTA
+constexpr int kThreads = kW * 32;
+constexpr uint32_t kBarBytes = 512;  // mbarriers and small words at the start of the window
+
+// Compile-time shape of the kernel for NJ n8 column tiles (M <= 8 or 16).
+template <int NJ>
+struct Geo {
+    static constexpr int MAX_ROWS = 64;                       // tallest tile
+    static constexpr int MT_MAX = MAX_ROWS / 16;              // 16-row MMA tiles per stage, at most
+    static constexpr uint32_t CODE_BYTES = MAX_ROWS * 128u;   // a stage's codes: rows x 128 B (4 units of 64 k)
+    static constexpr uint32_t AM_BYTES = MAX_ROWS * 16u;      // its absmax box: rows x 4 floats
+    static constexpr uint32_t SLOT = CODE_BYTES + AM_BYTES;   // 9 KiB: every slot stays 1 KiB aligned (swizzle)
+    static constexpr int REGS = MT_MAX * 4 * NJ;              // a warp's partial tile: registers per lane
+    // Ring depth: a compile-time constant, so that slot and phase of a stage
+    // are a mask and a shift.
+    static constexpr int D = 16;
+    static constexpr int R = D / kW;                          // slots per warp when each warp streams its own range
+    // Parking buffers for partial tiles live in the table's free upper row
+    // halves (256 rows of 128 B): two with one column tile, one with two.
+    static constexpr int NB = NJ == 1 ? 2 : 1;
+    static_assert(NB * kW * REGS <= 256, "parking buffers must fit the table's free halves");
+    static_assert(MAX_ROWS / 8 < (int)(sizeof(RowsParams::map_of) / sizeof(int)), "map_of indexes h / 8");
+};
+
+// Position of stage i in the CTA's work: tile `tile` (rows [y, y + h) of the
+// CTA's rows), k-stage `s` (columns [256 s, 256 s + 256)).
+struct Stage {
+    int tile, s, y, h;
+};
+
+// The CTA's share and the order of its stages (identical in every thread):
+// ng 8-row groups in T = ceil(ng / gmax) tiles, the first `extra` tiles one
+// group taller; tile-major, k-stages in order.
+struct Plan {
+    int row0;  // first weight row of the CTA
+    int T, S;  // tiles, k-stages per tile
+    int base, extra;
+    int n_total;
+
+    __device__ __forceinline__ void init(const RowsParams& p, int cta, int gmax) {
+        const int q = p.groups / p.ctas, r = p.groups - q * p.ctas;
+        const int g0 = cta < r ? cta * (q + 1) : r * (q + 1) + (cta - r) * q;
+        const int ng = q + (cta < r ? 1 : 0);
+        row0 = 8 * g0;
+        T = (ng + gmax - 1) / gmax;
+        base = ng / T;
+        extra = ng - base * T;
+        S = p.K >> 8;
+        n_total = T * S;
+    }
+    __device__ __forceinline__ int tile_rows(int t) const { return 8 * (base + (t < extra ? 1 : 0)); }
+    __device__ __forceinline__ int tile_y(int t) const { return 8 * (t * base + min(t, extra)); }
+};
+
+// A warp's position in the stage sequence, advanced by `stride` stages at
+// a time without divisions.
+struct Cur {
+    int i, t, s;
+    __device__ __forceinline__ void init(const Plan& pl, int i0) {
+        i = i0;
+        t = i0 / pl.S;
+        s = i0 - t * pl.S;
+    }
+    __device__ __forceinline__ void step(const Plan& pl, int stride) {
+        i += stride;
+        s += stride;
+        while (s >= pl.S) {
+            s -= pl.S;
+            ++t;
+        }
+    }
+    __device__ __forceinline__ Stage stage(const Plan& pl) const {
+        Stage st;
+        st.tile = t;
+        st.s = s;
+        st.h = pl.tile_rows(t);
+        st.y = pl.tile_y(t);
+        return st;
+    }
+};
+
+// Parking slot of register `r` of warp `w`'s partial tile in buffer `b`:
+// the upper (free) half of table row (b W + w) REGS + r, lane-major.
+template <int NJ>
+__device__ __forceinline__ uint32_t park_addr(uint32_t lut, int b, int w, int r, int lane) {
+    constexpr int REGS = Geo<NJ>::REGS;
+    return lut + (uint32_t)((b * kW + w) * REGS + r) * 256u + 128u + (uint32_t)lane * 4u;
+}
+
+// Tensor maps of the launch: per box height h (8 .. 72 rows), one map of
+// the packed codes (h rows x 128 bytes, 128-byte swizzle) and one of the
+// absmax (h rows x 4 floats); RowsParams::map_of[h / 8] selects the pair.
+struct RowsMaps {
+    CUtensorMap w[kRowsMaxMaps];
+    CUtensorMap a[kRowsMaxMaps];
+};
+
+template <typename T, int NJ, bool BS64>
+__global__ void __launch_bounds__(kThreads, 1)
+    q4_gemm_rows_kernel(const __grid_constant__ RowsMaps maps, const __grid_constant__ RowsParams p) {
+    using G = Geo<NJ>;
+    constexpr int D = G::D, MTM = G::MT_MAX, NB = G::NB;
+    extern __shared__ __align__(16) uint8_t smem_rows[];
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, tq = lane & 3;
+
+    // Shared-memory layout (from the window base, decided at run time):
+    // barriers and small words; ring slots below the 64 KiB-aligned table;
+    // the table (its upper row halves hold the parking buffers); ring slots
+    // above it.
+    const uint32_t sbase = smem_addr(smem_rows);
+    const uint32_t send = sbase + dynamic_smem_size();
+    const uint32_t lut = (sbase + 0xFFFFu) & ~0xFFFFu;
+    // The barriers go below the table when there is room there, else right after it.
+    const bool bars_low = lut >= sbase + kBarBytes;
+    const uint32_t bars = bars_low ? sbase : lut + kLutBytes;
+    const uint32_t a0 = bars_low ? (sbase + kBarBytes + 1023u) & ~1023u : lut;
+    const uint32_t b0 = bars_low ? lut + kLutBytes : lut + kLutBytes + 1024u;
+    const uint32_t na = a0 < lut ? (lut - a0) / G::SLOT : 0u;
+    const uint32_t nb = (send > b0) ? (send - b0) / G::SLOT : 0u;
+    if (b0 > send || na + nb < (uint32_t)D) {  // the host sized the launch wrongly
+        if (tid == 0 && p.error) atomicExch(p.error, kErrNoRoom);
+        return;
+    }
+    auto slot_addr = [&](int k) -> uint32_t {
+        return (uint32_t)k < na ? a0 + (uint32_t)k * G::SLOT : b0 + ((uint32_t)k - na) * G::SLOT;
+    };
+    auto full_bar = [&](int k) -> uint32_t { return bars + (uint32_t)k * 8u; };
+    const uint32_t reduced = bars + (uint32_t)D * 8u;                 // [2] ints: tiles reduced per parking buffer
+    const uint32_t counters = reduced + 8u;                           // [2] ints: parked partials per buffer
+    const uint32_t last_issued = counters + 8u;                       // [D] ints: phase + 1 of the newest copy per slot
+    const uint32_t failed = last_issued + 4u * (uint32_t)D;           // int: a wait of this CTA ran out
+
+    if (p.pdl == 1) griddep_wait();
+    if (tid == 0) {
+        for (int k = 0; k < D; ++k) {
+            mbar_init(full_bar(k), 1);
+            sts_u32(last_issued + 4u * (uint32_t)k, 0u);
+        }
+        sts_u32(reduced, 0u);
+        sts_u32(reduced + 4u, 0u);
+        sts_u32(counters, 0u);
+        sts_u32(counters + 4u, 0u);
+        sts_u32(failed, 0u);
+        mbar_init_fence();
+    }
+    __syncthreads();
+    griddep_launch_dependents();
+
+    Plan pl;
+    pl.init(p, blockIdx.x, G::MAX_ROWS / 8);
+    const uint64_t once = l2_evict_first();  // the codes are read exactly once
+
+    // This warp's stages.  Round robin (the default): stages warp, warp + W,
+    // ... through the shared ring, slot i % D.  Contiguous: the warp's own
+    // balanced range [ws, we) through its own R slots.
+    const bool rr = !p.contig;
+    const int ws = rr ? warp : (int)(((uint32_t)pl.n_total * (uint32_t)warp) / kW);
+    const int we = rr ? pl.n_total : (int)(((uint32_t)pl.n_total * (uint32_t)(warp + 1)) / kW);
+    const int stride = rr ? kW : 1, ahead = rr ? D : G::R;
+    auto slot_of = [&](int i) -> int { return rr ? (i & (D - 1)) : warp * G::R + ((i - ws) & (G::R - 1)); };
+    auto phase_of = [&](int i) -> uint32_t {
+        return rr ? (uint32_t)(i / D) & 1u : (uint32_t)((i - ws) / G::R) & 1u;
+    };
+
+    // Lane 0 of the calling warp loads stage i (at `st`) into its ring slot.
+    auto issue = [&](int i, const Stage& st) {
+        if (i == p.skip_stage) return;  // test hook: this stage's barrier never completes
+        const int k = slot_of(i), mi = p.map_of[st.h >> 3];
+        const uint32_t dst = slot_addr(k);
+        const int y = pl.row0 + st.y;
+        sts_u32(last_issued + 4u * (uint32_t)k, phase_of(i) + 1u);
+        mbar_expect_tx(full_bar(k), (uint32_t)st.h * 144u);
+        tma_load_2d_hint(dst, &maps.w[mi], st.s * 128, y, full_bar(k), once);
+        tma_load_2d(dst + G::CODE_BYTES, &maps.a[mi], ((st.s * 4) >> p.am_shift) & ~3, y, full_bar(k));
+    };
+    // The ring's first fill.  The weights are static, so under dependent
+    // launch mode 2 these copies (and the optional L2 prefetch of the stages
+    // after them) overlap the previous kernel.
+    if (lane == 0) {
+        for (int i = ws, n = 0; i < we && n < (rr ? D : G::R); i += stride, ++n) {
+            if (rr && i >= D) break;
+            Cur c;
+            c.init(pl, i);
+            issue(i, c.stage(pl));
+        }
+        if (warp == 0 && p.l2_ahead > 0) {
+            const int end = min(pl.n_total, D + p.l2_ahead);
+            for (int j = D; j < end; ++j) {
+                Cur c;
+                c.init(pl, j);
+                const Stage sj = c.stage(pl);
+                tma_prefetch_l2_2d(&maps.w[p.map_of[sj.h >> 3]], sj.s * 128, pl.row0 + sj.y);
+            }
+        }
+    }
+    __syncwarp();
+
+    build_lut<T>(lut, __ldg(p.code + (lane & 15)), tid, kW * 32);
+    __syncthreads();
+    if (p.pdl == 2) griddep_wait();  // activations and outputs may belong to the preceding grid
+
+    const uint32_t lane4 = lut | ((uint32_t)lane << 2);
+    const int lm_q = lane >> 3, lm_r = lane & 7;
+    const T* Aact = static_cast<const T*>(p.A);
+    T* out = static_cast<T*>(p.out);
+    const T* bias = static_cast<const T*>(p.bias);
+
+    // Activations of this warp's current stage (4 units x NJ column tiles x
+    // two 16-byte runs); refilled unit by unit with the next stage's.
+    uint32_t aw[4][NJ][2][4];
+    auto load_unit = [&](int kbu, uint32_t(&dst)[NJ][2][4]) {
+#pragma unroll
+        for (int jj = 0; jj < NJ; ++jj) {
+            const int m = 8 * jj + g;
+#pragma unroll
+            for (int ch = 0; ch < 2; ++ch) {
+                if (m < p.M) {
+                    const uint4 v = ldg_v4(Aact + (size_t)m * p.K + kbu * 64 + 32 * ch + 8 * tq);
+                    dst[jj][ch][0] = v.x;
+                    dst[jj][ch][1] = v.y;
+                    dst[jj][ch][2] = v.z;
+                    dst[jj][ch][3] = v.w;
+                } else {
+                    dst[jj][ch][0] = dst[jj][ch][1] = dst[jj][ch][2] = dst[jj][ch][3] = 0u;
+                }
+            }
+        }
+    };
+
+    float acc[MTM][NJ][4];
+#pragma unroll
+    for (int i = 0; i < MTM; ++i)
+#pragma unroll
+        for (int jj = 0; jj < NJ; ++jj)
+#pragma unroll
+            for (int r = 0; r < 4; ++r) acc[i][jj][r] = 0.f;
+
+    // The warps holding a partial of tile t, in stage order: the span
+    // [w_first, w_first + n) modulo W.  Round robin: every warp of the span.
+    // Contiguous: the warps whose (non-empty) ranges meet the tile's stages.
+    auto tile_warps = [&](int t, int& w_first, int& n) {
+        const int f = t * pl.S, l = f + pl.S - 1;
+        if (rr) {
+            w_first = f & (kW - 1);
+            n = min(kW, pl.S);
+        } else {
+            w_first = (int)part_owner((uint32_t)pl.n_total, kW, (uint32_t)f);
+            n = (int)part_owner((uint32_t)pl.n_total, kW, (uint32_t)l) - w_first + 1;
+        }
+    };
+    auto holds_partial = [&](int w) -> bool {  // (within a tile's span)
+        return rr || part_start((uint32_t)pl.n_total, kW, (uint32_t)w) !=
+                         part_start((uint32_t)pl.n_total, kW, (uint32_t)(w + 1));
+    };
+
+    // Leaves tile t: park the partial, and if this warp is the last of the
+    // tile's contributors, add all parked partials in stage order and store.
+    auto flush = [&](int t) -> bool {
+        const int b = NB == 1 ? 0 : (t & 1);
+        // The buffer's previous tile (t - NB) must have been reduced: an
+        // exact count, since a warp that holds no part of the tiles between
+        // may arrive here several reductions ahead (a phase parity would
+        // alias).
+        if (t >= NB && !wait_count_at_least(reduced + 4u * (uint32_t)b, (uint32_t)(t / NB), p.wait_limit))
+            return false;
+#pragma unroll
+        for (int i = 0; i < MTM; ++i)
+#pragma unroll
+            for (int jj = 0; jj < NJ; ++jj)
+#pragma unroll
+                for (int r = 0; r < 4; ++r) {
+                    sts_f32(park_addr<NJ>(lut, b, warp, (i * NJ + jj) * 4 + r, lane), acc[i][jj][r]);
+                    acc[i][jj][r] = 0.f;
+                }
+        __syncwarp();
+        int old = 0;
+        if (lane == 0) old = atom_add_acq_rel_cta_smem(counters + 4u * (uint32_t)b, 1);
+        old = __shfl_sync(0xffffffffu, old, 0);
+        __syncwarp();  // the other lanes read after lane 0's acquire
+        int w0, span, nc = 0;
+        tile_warps(t, w0, span);
+        for (int c = 0; c < span; ++c) nc += holds_partial((w0 + c) & (kW - 1)) ? 1 : 0;
+        if (old != nc - 1) return true;
+        float sum[MTM][NJ][4];
+#pragma unroll
+        for (int i = 0; i < MTM; ++i)
+#pragma unroll
+            for (int jj = 0; jj < NJ; ++jj)
+#pragma unroll
+                for (int r = 0; r < 4; ++r) sum[i][jj][r] = 0.f;
+        for (int c = 0; c < span; ++c) {
+            const int w = (w0 + c) & (kW - 1);
+            if (!holds_partial(w)) continue;
+#pragma unroll
+            for (int i = 0; i < MTM; ++i)
+#pragma unroll
+                for (int jj = 0; jj < NJ; ++jj)
+#pragma unroll
+                    for (int r = 0; r < 4; ++r)
+                        sum[i][jj][r] += lds_f32(park_addr<NJ>(lut, b, w, (i * NJ + jj) * 4 + r, lane));
+        }
+        const int rows_t = pl.tile_rows(t), y_t = pl.tile_y(t);
+#pragma unroll
+        for (int i = 0; i < MTM; ++i)
+#pragma unroll
+            for (int jj = 0; jj < NJ; ++jj)
+#pragma unroll
+                for (int r = 0; r < 4; ++r) {
+                    const int rt = 16 * i + g + ((r & 2) ? 8 : 0);
+                    const int n = pl.row0 + y_t + rt;
+                    const int m = 8 * jj + 2 * tq + (r & 1);
+                    if (rt < rows_t && n < p.N && m < p.M) {
+                        const float bv = bias ? static_cast<float>(bias[n]) : 0.f;  // exact widening
+                        out[(size_t)m * p.N + n] = Act<T>::from_float(sum[i][jj][r] + bv);
+                    }
+                }
+        __syncwarp();
+        if (lane == 0) {
+            sts_u32(counters + 4u * (uint32_t)b, 0u);
+            red_add_release_cta_smem(reduced + 4u * (uint32_t)b, 1u);  // the buffer may be refilled
+        }
+        return true;
+    };
+
+    bool ok = true;
+    Cur cc, ci;  // the stage this warp computes next, and the one it loads into the slot it frees
+    cc.init(pl, ws);
+    ci.init(pl, ws + ahead);
+
+    // This warp's stages of one tile (MT 16-row MMA tiles, the last of them
+    // half when HALF), starting at cc: one tight loop per tile shape.  The
+    // dispatch on the shape happens once per tile, outside the loop, so the
+    // loop body stays one straight-line block in which the four units'
+    // lookup and MMA chains interleave.
+    auto run_tile = [&](auto mt_c, auto half_c) -> bool {
+        constexpr int MT = decltype(mt_c)::value;
+        constexpr bool HALF = decltype(half_c)::value;
+        const int tile = cc.t;
+        while (true) {
+            const int i = cc.i, k = slot_of(i);
+            const int s_cur = cc.s;
+            const uint32_t st_addr = slot_addr(k);
+            if (!wait_stage(full_bar(k), phase_of(i), p.wait_limit)) return false;
+            cc.step(pl, stride);
+            const bool more = cc.i < we;
+            const int s_nxt = more ? cc.s : s_cur;
+            const uint32_t am_st = st_addr + G::CODE_BYTES;
+            const int x0 = ((s_cur * 4) >> p.am_shift) & ~3;
+            float am[MT][2][4];  // absmax of rows 16 ia + g (+ 8 hh), for the stage's 4 units
+#pragma unroll
+            for (int ia = 0; ia < MT; ++ia)
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    if (BS64) {
+                        const uint4 v = lds_v4(am_st + (uint32_t)(16 * ia + 8 * hh + g) * 16u);
+                        am[ia][hh][0] = __uint_as_float(v.x);
+                        am[ia][hh][1] = __uint_as_float(v.y);
+                        am[ia][hh][2] = __uint_as_float(v.z);
+                        am[ia][hh][3] = __uint_as_float(v.w);
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            const int col = ((s_cur * 4 + j) >> p.am_shift) - x0;
+                            am[ia][hh][j] = lds_f32(am_st + (uint32_t)((16 * ia + 8 * hh + g) * 16 + col * 4));
+                        }
+                    }
+                }
+            const float zero[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+#pragma unroll
+                for (int ia = 0; ia < MT; ++ia) {
+                    // d[0 / 1]: rows g / g + 8 of the MMA tile, bytes 4 tq ..
+                    // 4 tq + 3 of the unit (k = 8 tq .. 8 tq + 7); d[2 / 3] the
+                    // same rows 32 k further.  Rows past a half tile look
+                    // nothing up.
+                    uint32_t d[4];
+                    const int row = 16 * ia + 8 * (lm_q & 1) + lm_r, chunk = 2 * j + (lm_q >> 1);
+                    ldmatrix_x4(st_addr + (uint32_t)row * 128u + (uint32_t)((chunk ^ (row & 7)) << 4), d[0], d[1], d[2],
+                                d[3]);
+                    uint32_t q[4][4];
+#pragma unroll
+                    for (int x = 0; x < 4; ++x) {
+                        if (HALF && ia == MT - 1 && (x & 1)) {
+                            q[x][0] = q[x][1] = q[x][2] = q[x][3] = 0u;
+                        } else {
+                            q[x][0] = lut_pair<0>(d[x], lane4);
+                            q[x][1] = lut_pair<1>(d[x], lane4);
+                            q[x][2] = lut_pair<2>(d[x], lane4);
+                            q[x][3] = lut_pair<3>(d[x], lane4);
+                        }
+                    }
+                    float t[NJ][4];
+#pragma unroll
+                    for (int jj = 0; jj < NJ; ++jj)
+                        mma16816<T>(t[jj], q[0][0], q[1][0], q[0][1], q[1][1], aw[j][jj][0][0], aw[j][jj][0][1], zero);
+#pragma unroll
+                    for (int jj = 0; jj < NJ; ++jj)
+                        mma16816<T>(t[jj], q[0][2], q[1][2], q[0][3], q[1][3], aw[j][jj][0][2], aw[j][jj][0][3], t[jj]);
+#pragma unroll
+                    for (int jj = 0; jj < NJ; ++jj)
+                        mma16816<T>(t[jj], q[2][0], q[3][0], q[2][1], q[3][1], aw[j][jj][1][0], aw[j][jj][1][1], t[jj]);
+#pragma unroll
+                    for (int jj = 0; jj < NJ; ++jj)
+                        mma16816<T>(t[jj], q[2][2], q[3][2], q[2][3], q[3][3], aw[j][jj][1][2], aw[j][jj][1][3], t[jj]);
+#pragma unroll
+                    for (int jj = 0; jj < NJ; ++jj) {
+                        acc[ia][jj][0] = fmaf(am[ia][0][j], t[jj][0], acc[ia][jj][0]);
+                        acc[ia][jj][1] = fmaf(am[ia][0][j], t[jj][1], acc[ia][jj][1]);
+                        acc[ia][jj][2] = fmaf(am[ia][1][j], t[jj][2], acc[ia][jj][2]);
+                        acc[ia][jj][3] = fmaf(am[ia][1][j], t[jj][3], acc[ia][jj][3]);
+                    }
+                }
+                load_unit(4 * s_nxt + j, aw[j]);  // the next stage's activations (its own again at the end)
+            }
+            // Refill the slot with the warp's stage `ahead` further on: order
+            // this warp's reads of the slot before the asynchronous write.
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (ci.i < we) {
+                if (lane == 0) issue(ci.i, ci.stage(pl));
+                ci.step(pl, stride);
+            }
+            __syncwarp();
+            if (!more || cc.t != tile) return true;
+        }
+    };
+
+    if (cc.i < we) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) load_unit(4 * cc.s + j, aw[j]);
+        using F = std::false_type;
+        using Tr = std::true_type;
+        while (cc.i < we) {
+            const int tile = cc.t;
+            bool fine;
+            switch (pl.tile_rows(tile) >> 3) {  // rows / 8
+                case 1: fine = run_tile(std::integral_constant<int, 1>{}, Tr{}); break;
+                case 2: fine = run_tile(std::integral_constant<int, 1>{}, F{}); break;
+                case 3: fine = run_tile(std::integral_constant<int, 2>{}, Tr{}); break;
+                case 4: fine = run_tile(std::integral_constant<int, 2>{}, F{}); break;
+                case 5: fine = run_tile(std::integral_constant<int, 3>{}, Tr{}); break;
+                case 6: fine = run_tile(std::integral_constant<int, 3>{}, F{}); break;
+                case 7: fine = run_tile(std::integral_constant<int, 4>{}, Tr{}); break;
+                default: fine = run_tile(std::integral_constant<int, 4>{}, F{}); break;
+            }
+            if (!fine || !flush(tile)) {
+                ok = false;
+                break;
+            }
+        }
+    }
+    if (!ok && lane == 0) {
+        if (p.error) atomicExch(p.error, kErrWaitTimeout);
+        sts_u32(failed, 1u);
+    }
+    __syncthreads();
+    if (tid == 0 && lds_u32(failed)) {
+        // A wait ran out and stages may have been left unread: let every
+        // copy still in flight land before the CTA leaves (bounded).
+        for (int k = 0; k < D; ++k) {
+            const uint32_t ph = lds_u32(last_issued + 4u * (uint32_t)k);
+            if (ph) wait_stage(full_bar(k), ph - 1u);
+        }
+    }
+}
+
+// Weights [N rows][K/2 bytes]: boxes of h rows x 128 bytes, 128-byte
+// swizzle.  Absmax [N rows][K/bs floats]: boxes of h rows x 4 floats.  One
+// pair per distinct tile height of the launch (heights[] in rows).
+static cudaError_t make_maps(const RowsParams& p, const uint8_t* Wp, const float* absmax, int am_per_row,
+                             const int* heights, int nh, RowsMaps* m) {
+    auto enc = tensor_map_encoder();
+    if (!enc) return cudaErrorNotSupported;
+    const cuuint32_t es[2] = {1, 1};
+    const cuuint64_t wdim[2] = {(cuuint64_t)(p.K / 2), (cuuint64_t)p.N};
+    const cuuint64_t wstr[1] = {(cuuint64_t)(p.K / 2)};
+    const cuuint64_t adim[2] = {(cuuint64_t)am_per_row, (cuuint64_t)p.N};
+    const cuuint64_t astr[1] = {(cuuint64_t)am_per_row * 4};
+    for (int v = 0; v < nh; ++v) {
+        const cuuint32_t rows = (cuuint32_t)heights[v];
+        const cuuint32_t wbox[2] = {128, rows};
+        if (enc(&m->w[v], CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(Wp), wdim, wstr, wbox, es,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return cudaErrorInvalidValue;
+        const cuuint32_t abox[2] = {4, rows};
+        if (enc(&m->a[v], CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(absmax), adim, astr, abox, es,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return cudaErrorInvalidValue;
+    }
+    return cudaSuccess;
+}
+
+// Distinct tile heights of a launch (the device's Plan, replayed for the
+// two group counts a CTA can have), and the map index of each height.
+static int stage_heights(const RowsParams& p, int gmax, int* heights, int* map_of) {
+    int nh = 0;
+    auto add = [&](int h) {
+        for (int v = 0; v < nh; ++v)
+            if (heights[v] == h) return;
+        map_of[h >> 3] = nh;
+        heights[nh++] = h;
+    };
+    const int q = p.groups / p.ctas, r = p.groups - q * p.ctas;
+    for (int ng = q; ng <= q + (r ? 1 : 0); ++ng) {
+        if (ng <= 0) continue;
+        const int T = (ng + gmax - 1) / gmax, base = ng / T, extra = ng - base * T;
+        add(8 * base);
+        if (extra) add(8 * (base + 1));
+    }
+    return nh;
+}
+
+template <typename T, int NJ, bool BS64>
+static cudaError_t launch_t(const RowsMaps& m, const RowsParams& p, int smem, cudaStream_t stream) {
+    auto kern = q4_gemm_rows_kernel<T, NJ, BS64>;
+    cudaError_t e = ensure_smem_attr((const void*)kern, (size_t)smem);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)p.ctas);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = (size_t)smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = p.pdl ? 1 : 0;
+    e = cudaLaunchKernelEx(&cfg, kern, m, p);
+    if (e != cudaSuccess) return e;
+    return cudaGetLastError();
+}
+
+}  // namespace rows
+
+int rows_warps() { return rows::kW; }
+
+cudaError_t rows_launch(int act_dtype, int m_pad, const RowsParams& p0, const uint8_t* Wp, const float* absmax,
+                        int am_per_row, int smem, cudaStream_t stream) {
+    RowsParams p = p0;
+    int heights[kRowsMaxMaps];
+    for (int& v : p.map_of) v = 0;
+    const int gmax = (m_pad == 8 ? rows::Geo<1>::MAX_ROWS : rows::Geo<2>::MAX_ROWS) / 8;
+    const int nh = rows::stage_heights(p, gmax, heights, p.map_of);
+    rows::RowsMaps m;
+    cudaError_t e = rows::make_maps(p, Wp, absmax, am_per_row, heights, nh, &m);
+    if (e != cudaSuccess) return e;
+    const bool bs64 = p.am_shift == 0;
+    using namespace rows;
+    if (act_dtype == 0) {
+        if (m_pad == 8) return bs64 ? launch_t<__nv_bfloat16, 1, true>(m, p, smem, stream)
+                                    : launch_t<__nv_bfloat16, 1, false>(m, p, smem, stream);
+        return bs64 ? launch_t<__nv_bfloat16, 2, true>(m, p, smem, stream)
+                    : launch_t<__nv_bfloat16, 2, false>(m, p, smem, stream);
+    }
+    if (m_pad == 8) return bs64 ? launch_t<__half, 1, true>(m, p, smem, stream) : launch_t<__half, 1, false>(m, p, smem, stream);
+    return bs64 ? launch_t<__half, 2, true>(m, p, smem, stream) : launch_t<__half, 2, false>(m, p, smem, stream);
+}
+
+}  // namespace q4

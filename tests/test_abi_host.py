@@ -89,7 +89,12 @@ def test_gemm_validation_before_cuda():
     assert ex(*args, 32, 64, 4096, 32, 0, ALIGNED, None, 0, None, None) == b.Q4_ERR_UNSUPPORTED
     assert ex(*args, 32, 64, 4160, 64, 0, ALIGNED, None, 0, None, None) == b.Q4_ERR_UNSUPPORTED
     assert ex(*args, 12, 64, 4096, 64, 0, ALIGNED, None, 0, None, b.overrides(warps=16)) == b.Q4_ERR_UNSUPPORTED
-    assert ex(*args, 1, 64, 4096, 64, 0, ALIGNED, None, 0, None, b.overrides(depth=7)) == b.Q4_ERR_UNSUPPORTED
+    assert ex(*args, 1, 64, 4096, 64, 0, ALIGNED, None, 0, None, b.overrides(depth=7, loader=2)) == b.Q4_ERR_UNSUPPORTED
+    assert ex(*args, 12, 64, 4096, 64, 0, ALIGNED, None, 0, None, b.overrides(loader=8)) == b.Q4_ERR_INVALID_ARG
+    # the row-split kernel (loader 7): M <= 16, 64-k units, its own warp count
+    assert ex(*args, 20, 64, 4096, 64, 0, ALIGNED, None, 0, None, b.overrides(loader=7)) == b.Q4_ERR_UNSUPPORTED
+    assert ex(*args, 4, 64, 4096, 32, 0, ALIGNED, None, 0, None, b.overrides(loader=7)) == b.Q4_ERR_UNSUPPORTED
+    assert ex(*args, 4, 64, 4096, 64, 0, ALIGNED, None, 0, None, b.overrides(loader=7, warps=9)) == b.Q4_ERR_UNSUPPORTED
     assert ex(*args, 1, 64, 4096, 64, 0, ALIGNED, None, 0, None, b.overrides(math=2)) == b.Q4_ERR_UNSUPPORTED
 
 
@@ -184,12 +189,18 @@ def test_launch_table_invariants(wl):
         assert p["units"] == p["tiles"] * (c.K // p["sub_block"])
         assert 1 <= p["ctas"] <= min(148, p["units"])
         assert p["smem_bytes"] <= 227 * 1024
+        tma_ok = c.blocksize >= 64 and (c.K // c.blocksize) % 4 == 0 and p["units"] > 1
+        assert p["loader"] == (7 if tma_ok else 1)
+        if tma_ok:
+            # row-split kernel: 8-row groups over at most one CTA per SM, the
+            # workspace is the 256-byte error header alone
+            assert p["ctas"] == min(148, -(-c.N // 8)) and p["warps"] == 8 and p["rows_per_tile"] == 64
+            assert p["workspace_bytes"] == 256 and p["depth"] >= 0
+            continue
         # workspace: 2 slots of 4 KiB per SM, then one int per tile (256-B granules)
         want_ws = 0 if p["units"] == 1 else 256 + 148 * 2 * 4096 + -(-p["tiles"] * 4 // 256) * 256
         assert p["workspace_bytes"] == want_ws
         assert p["depth"] >= 1 and p["l2_prefetch"] in (1, 128, 256)
-        tma_ok = c.blocksize >= 64 and (c.K // c.blocksize) % 4 == 0 and p["units"] > 1
-        assert p["loader"] == (2 if tma_ok else 1)
 
 
 @pytest.mark.parametrize("total,parts", [(1, 1), (1, 16), (7, 3), (40, 148), (4096, 148), (57344, 148),

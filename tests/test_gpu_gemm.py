@@ -142,7 +142,7 @@ def test_tma_ring_partitions(cuda_device, ctas, loader):
 def test_tma_error_word_stays_zero(cuda_device):
     ws = q4.Workspace(cuda_device)
     A, P, Am, C, N, K, bs = _problem(cuda_device)
-    for loader in (2, 3, 4, 5):
+    for loader in (2, 3, 4, 5, 7):
         q4.q4_gemm_skinny(A, P, Am, C, N, K, bs, workspace=ws, loader=loader)
     torch.cuda.synchronize()
     assert q4.workspace_error(ws) == 0
@@ -205,7 +205,7 @@ def test_one_hot_activation_selects_dequantized_column(cuda_device):
 
 
 @pytest.mark.parametrize("pdl", [1, 2])
-@pytest.mark.parametrize("loader", [1, 3, 4])
+@pytest.mark.parametrize("loader", [1, 3, 4, 7])
 def test_dependent_launch_chain(cuda_device, pdl, loader):
     """A chain where each GEMM reads the previous GEMM's output as its
     activations: with programmatic dependent launch the second kernel may
