@@ -104,6 +104,24 @@ static bool data_parallel_pays(int tiles, int sms, int64_t weights) {
     return idle_us < 3.0;
 }
 
+// Row-split kernel (loader 7) or stream-K kernel (loader 2) for M <= 16,
+// fitted to B200 measurements of both on the five benchmark configurations
+// (back-to-back launches over distinct weight copies).  The row-split kernel
+// has no cross-CTA fix-up, which is what dominates small and medium layers
+// (K5120/N5120: 7.3 vs 8.2 us; K10240/N320: 5.9 vs 11.2 us; 4096^2: 6.1 vs
+// 6.5 us; K8192/N10240: 13.5 vs 14.7 us).  The stream-K kernel keeps full
+// 64-row tiles, which wins when it already runs one CTA per tile on nearly
+// every SM (N = 8192: 128 tiles), on the largest layers (2^27 weights or
+// more: K8192/N28672 28.8 vs 29.5 us, K2560/N248320 67 vs 96 us) and for
+// M >= 8 on layers of 2^26 weights or more.
+static bool rows_kernel_pays(int M, int N, int K, int sms) {
+    const int64_t tiles = ((int64_t)N + 63) / 64, weights = (int64_t)N * K;
+    if (tiles <= sms && tiles * 5 >= (int64_t)sms * 4) return false;  // one stream-K CTA per tile, >= 80 % of the SMs
+    if (weights >= ((int64_t)1 << 27)) return false;
+    if (M >= 8 && weights >= ((int64_t)1 << 26)) return false;
+    return true;
+}
+
 // Validates a GEMM request.  Returns Q4_OK and fills `ch` with the launch
 // table's choice (with `ov` applied) and the problem's unit counts.
 static int gemm_choose(int M, int N, int K, int blocksize, int act_dtype, int num_sms, const q4_gemm_plan_t* ov,
@@ -198,7 +216,9 @@ static int gemm_choose(int M, int N, int K, int blocksize, int act_dtype, int nu
     // multiples of 16 bytes (a tensor-map stride rule); the pointer itself
     // must also be 16-byte aligned, which the caller checks at launch.
     const bool tma_ok = c.sub_block == 64 && (K / blocksize) % 4 == 0 && (int64_t)N * (K / 64) > 1;
-    c.loader = mma32 ? 3 : tma_ok ? 7 : 1;
+    int sms_hint = num_sms;
+    if (sms_hint <= 0 && device_sm_count(&sms_hint) != 0) sms_hint = 148;  // the choice only; the launch re-queries
+    c.loader = mma32 ? 3 : !tma_ok ? 1 : rows_kernel_pays(M, N, K, sms_hint) ? 7 : 2;
     if (ov && ov->loader > 0) c.loader = ov->loader;
     if (c.loader >= 2 && !tma_ok) return Q4_ERR_UNSUPPORTED;
     if (c.loader == 7) {
@@ -206,7 +226,7 @@ static int gemm_choose(int M, int N, int K, int blocksize, int act_dtype, int nu
         // stage ring per CTA, no cross-CTA combine (workspace: the error word).
         if (M > 16) return Q4_ERR_UNSUPPORTED;
         c.warps = rows_warps();
-        c.depth = (ov && ov->depth > 0) ? ov->depth : 2;  // stage order: 1 round robin, 2 contiguous per warp
+        c.depth = (ov && ov->depth > 0) ? ov->depth : 1;  // stage order: 1 round robin, 2 contiguous per warp
         if (c.depth > 2) return Q4_ERR_UNSUPPORTED;
         c.l2pf = (ov && ov->l2_prefetch > 1) ? ov->l2_prefetch : 0;
         c.pdl = (ov && ov->pdl > 0) ? ov->pdl : 0;

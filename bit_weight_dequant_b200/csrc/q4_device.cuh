@@ -247,6 +247,12 @@ __device__ __forceinline__ void tma_prefetch_l2_2d(const void* tmap, int x, int 
                  : "memory");
 }
 
+// Starts fetching a tensor map (a kernel parameter) into the descriptor
+// cache, so that the first copy through it does not wait for that fetch.
+__device__ __forceinline__ void prefetch_tensormap(const void* tmap) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(tmap) : "memory");
+}
+
 // L2 policy for data read exactly once: its lines are the first candidates
 // for eviction, so they do not push out data that is read again.
 __device__ __forceinline__ uint64_t l2_evict_first() {

@@ -113,6 +113,7 @@ struct RowsParams {
     int skip_stage;       // test hook: this stage index is never loaded (-1: none)
     int contig;           // 1: each warp streams a contiguous range of stages (0: round robin)
     int map_of[10];       // tensor-map pair of tile height h (8 .. 72 rows): map_of[h / 8], filled by the launcher
+    int n_maps;           // tensor-map pairs the launcher encoded
 };
 
 }  // namespace q4

@@ -43,6 +43,7 @@
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
+#include <cstring>
 #include <type_traits>
 
 #include "q4_device.cuh"
@@ -56,23 +57,36 @@ constexpr int kW = 8;                // warps per CTA
 constexpr int kThreads = kW * 32;
 constexpr uint32_t kBarBytes = 512;  // mbarriers and small words at the start of the window
 
-// Compile-time shape of the kernel for NJ n8 column tiles (M <= 8 or 16).
-template <int NJ>
+// Compile-time shape of the kernel for NJ n8 column tiles (M <= 8 or 16)
+// and stage order (CONTIG: each warp streams a contiguous range of stages;
+// else round robin).
+template <int NJ, bool CONTIG>
 struct Geo {
-    static constexpr int MAX_ROWS = 64;                       // tallest tile
-    static constexpr int MT_MAX = MAX_ROWS / 16;              // 16-row MMA tiles per stage, at most
+    // Tallest tile.  Round robin with one column tile: 72 rows (a CTA of
+    // 8q + 1 groups then needs no short tiles).  Contiguous ranges keep
+    // several tiles open at once and need two parking buffers: 64 rows.
+    static constexpr int MAX_ROWS = (NJ == 1 && !CONTIG) ? 72 : 64;
+    static constexpr int MT_MAX = (MAX_ROWS + 15) / 16;       // 16-row MMA tiles per stage, at most
     static constexpr uint32_t CODE_BYTES = MAX_ROWS * 128u;   // a stage's codes: rows x 128 B (4 units of 64 k)
     static constexpr uint32_t AM_BYTES = MAX_ROWS * 16u;      // its absmax box: rows x 4 floats
-    static constexpr uint32_t SLOT = CODE_BYTES + AM_BYTES;   // 9 KiB: every slot stays 1 KiB aligned (swizzle)
+    // With 72-row tiles the codes (9 KiB, 1 KiB aligned for the swizzle) and
+    // the absmax boxes live in separate rings, and the barriers in spare
+    // table rows; otherwise a slot holds both (9 KiB) and the barriers sit
+    // at the start of the window.
+    static constexpr bool SPLIT = MAX_ROWS == 72;
+    static constexpr uint32_t SLOT = CODE_BYTES + AM_BYTES;
     static constexpr int REGS = MT_MAX * 4 * NJ;              // a warp's partial tile: registers per lane
     // Ring depth: a compile-time constant, so that slot and phase of a stage
     // are a mask and a shift.
     static constexpr int D = 16;
-    static constexpr int R = D / kW;                          // slots per warp when each warp streams its own range
-    // Parking buffers for partial tiles live in the table's free upper row
-    // halves (256 rows of 128 B): two with one column tile, one with two.
-    static constexpr int NB = NJ == 1 ? 2 : 1;
-    static_assert(NB * kW * REGS <= 256, "parking buffers must fit the table's free halves");
+    static constexpr int R = D / kW;                          // slots per warp with contiguous ranges
+    // Parking buffers for partial tiles, in the table's free upper row
+    // halves (256 rows of 128 B); with the split layout, rows PARK_ROWS and
+    // PARK_ROWS + 1 hold the barriers and small words.
+    static constexpr int NB = CONTIG ? 2 : 1;
+    static constexpr int PARK_ROWS = NB * kW * REGS;
+    static_assert(PARK_ROWS + (SPLIT ? 2 : 0) <= 256, "parking buffers must fit the table's free halves");
+    static_assert(!SPLIT || D * 8 <= 128, "the full barriers fill one spare row");
     static_assert(MAX_ROWS / 8 < (int)(sizeof(RowsParams::map_of) / sizeof(int)), "map_of indexes h / 8");
 };
 
@@ -135,9 +149,9 @@ struct Cur {
 
 // Parking slot of register `r` of warp `w`'s partial tile in buffer `b`:
 // the upper (free) half of table row (b W + w) REGS + r, lane-major.
-template <int NJ>
+template <class G>
 __device__ __forceinline__ uint32_t park_addr(uint32_t lut, int b, int w, int r, int lane) {
-    constexpr int REGS = Geo<NJ>::REGS;
+    constexpr int REGS = G::REGS;
     return lut + (uint32_t)((b * kW + w) * REGS + r) * 256u + 128u + (uint32_t)lane * 4u;
 }
 
@@ -149,13 +163,20 @@ struct RowsMaps {
     CUtensorMap a[kRowsMaxMaps];
 };
 
-template <typename T, int NJ, bool BS64>
+template <typename T, int NJ, bool BS64, bool CONTIG>
 __global__ void __launch_bounds__(kThreads, 1)
     q4_gemm_rows_kernel(const __grid_constant__ RowsMaps maps, const __grid_constant__ RowsParams p) {
-    using G = Geo<NJ>;
+    using G = Geo<NJ, CONTIG>;
     constexpr int D = G::D, MTM = G::MT_MAX, NB = G::NB;
     extern __shared__ __align__(16) uint8_t smem_rows[];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, tq = lane & 3;
+    // Long-latency first touches go out first: the code table (read by the
+    // table build) and the tensor maps (read by the first copies).
+    const float cv = __ldg(p.code + (lane & 15));
+    if (tid < p.n_maps) {
+        prefetch_tensormap(&maps.w[tid]);
+        prefetch_tensormap(&maps.a[tid]);
+    }
 
     // Shared-memory layout (from the window base, decided at run time):
     // barriers and small words; ring slots below the 64 KiB-aligned table;
@@ -164,22 +185,50 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t sbase = smem_addr(smem_rows);
     const uint32_t send = sbase + dynamic_smem_size();
     const uint32_t lut = (sbase + 0xFFFFu) & ~0xFFFFu;
-    // The barriers go below the table when there is room there, else right after it.
-    const bool bars_low = lut >= sbase + kBarBytes;
-    const uint32_t bars = bars_low ? sbase : lut + kLutBytes;
-    const uint32_t a0 = bars_low ? (sbase + kBarBytes + 1023u) & ~1023u : lut;
-    const uint32_t b0 = bars_low ? lut + kLutBytes : lut + kLutBytes + 1024u;
-    const uint32_t na = a0 < lut ? (lut - a0) / G::SLOT : 0u;
-    const uint32_t nb = (send > b0) ? (send - b0) / G::SLOT : 0u;
-    if (b0 > send || na + nb < (uint32_t)D) {  // the host sized the launch wrongly
+    uint32_t bars, words, a0, b0, na, nb, am_a = 0, am_b = 0, nam_a = 0;
+    bool room;
+    if constexpr (G::SPLIT) {
+        // barriers and words in the spare table rows; codes slots (1 KiB
+        // aligned) below the table, then above it; absmax boxes in what is
+        // left of the two regions.
+        bars = lut + (uint32_t)G::PARK_ROWS * 256u + 128u;
+        words = bars + 256u;
+        a0 = (sbase + 1023u) & ~1023u;
+        b0 = lut + kLutBytes;
+        na = a0 < lut ? min((lut - a0) / G::CODE_BYTES, (uint32_t)D) : 0u;
+        nb = (uint32_t)D - na;
+        am_a = a0 + na * G::CODE_BYTES;
+        nam_a = am_a < lut ? (lut - am_a) / G::AM_BYTES : 0u;
+        am_b = b0 + nb * G::CODE_BYTES;
+        room = am_b <= send && nam_a + (send - am_b) / G::AM_BYTES >= (uint32_t)D;
+    } else {
+        // barriers below the table when there is room there, else right
+        // after it; code + absmax slots below and above the table.
+        const bool bars_low = lut >= sbase + kBarBytes;
+        bars = bars_low ? sbase : lut + kLutBytes;
+        words = bars + (uint32_t)D * 8u;
+        a0 = bars_low ? (sbase + kBarBytes + 1023u) & ~1023u : lut;
+        b0 = bars_low ? lut + kLutBytes : lut + kLutBytes + 1024u;
+        na = a0 < lut ? (lut - a0) / G::SLOT : 0u;
+        nb = (send > b0) ? (send - b0) / G::SLOT : 0u;
+        room = b0 <= send && na + nb >= (uint32_t)D;
+    }
+    if (!room) {  // the host sized the launch wrongly
         if (tid == 0 && p.error) atomicExch(p.error, kErrNoRoom);
         return;
     }
-    auto slot_addr = [&](int k) -> uint32_t {
-        return (uint32_t)k < na ? a0 + (uint32_t)k * G::SLOT : b0 + ((uint32_t)k - na) * G::SLOT;
+    auto slot_addr = [&](int k) -> uint32_t {  // the codes of ring slot k
+        constexpr uint32_t stride = G::SPLIT ? G::CODE_BYTES : G::SLOT;
+        return (uint32_t)k < na ? a0 + (uint32_t)k * stride : b0 + ((uint32_t)k - na) * stride;
+    };
+    auto am_addr = [&](int k) -> uint32_t {  // the absmax box of ring slot k
+        if constexpr (G::SPLIT)
+            return (uint32_t)k < nam_a ? am_a + (uint32_t)k * G::AM_BYTES : am_b + ((uint32_t)k - nam_a) * G::AM_BYTES;
+        else
+            return slot_addr(k) + G::CODE_BYTES;
     };
     auto full_bar = [&](int k) -> uint32_t { return bars + (uint32_t)k * 8u; };
-    const uint32_t reduced = bars + (uint32_t)D * 8u;                 // [2] ints: tiles reduced per parking buffer
+    const uint32_t reduced = words;                                   // [2] ints: tiles reduced per parking buffer
     const uint32_t counters = reduced + 8u;                           // [2] ints: parked partials per buffer
     const uint32_t last_issued = counters + 8u;                       // [D] ints: phase + 1 of the newest copy per slot
     const uint32_t failed = last_issued + 4u * (uint32_t)D;           // int: a wait of this CTA ran out
@@ -207,7 +256,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // This warp's stages.  Round robin (the default): stages warp, warp + W,
     // ... through the shared ring, slot i % D.  Contiguous: the warp's own
     // balanced range [ws, we) through its own R slots.
-    const bool rr = !p.contig;
+    constexpr bool rr = !CONTIG;
     const int ws = rr ? warp : (int)(((uint32_t)pl.n_total * (uint32_t)warp) / kW);
     const int we = rr ? pl.n_total : (int)(((uint32_t)pl.n_total * (uint32_t)(warp + 1)) / kW);
     const int stride = rr ? kW : 1, ahead = rr ? D : G::R;
@@ -225,19 +274,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         sts_u32(last_issued + 4u * (uint32_t)k, phase_of(i) + 1u);
         mbar_expect_tx(full_bar(k), (uint32_t)st.h * 144u);
         tma_load_2d_hint(dst, &maps.w[mi], st.s * 128, y, full_bar(k), once);
-        tma_load_2d(dst + G::CODE_BYTES, &maps.a[mi], ((st.s * 4) >> p.am_shift) & ~3, y, full_bar(k));
+        tma_load_2d(am_addr(k), &maps.a[mi], ((st.s * 4) >> p.am_shift) & ~3, y, full_bar(k));
     };
     // The ring's first fill.  The weights are static, so under dependent
     // launch mode 2 these copies (and the optional L2 prefetch of the stages
     // after them) overlap the previous kernel.
-    if (lane == 0) {
-        for (int i = ws, n = 0; i < we && n < (rr ? D : G::R); i += stride, ++n) {
-            if (rr && i >= D) break;
+    {
+        // lane j issues the warp's j-th stage of the fill
+        const int i = ws + lane * stride;
+        if (lane < (rr ? D / kW : G::R) && i < we && i < (rr ? D : we)) {
             Cur c;
             c.init(pl, i);
             issue(i, c.stage(pl));
         }
-        if (warp == 0 && p.l2_ahead > 0) {
+        if (warp == 0 && lane == 0 && p.l2_ahead > 0) {
             const int end = min(pl.n_total, D + p.l2_ahead);
             for (int j = D; j < end; ++j) {
                 Cur c;
@@ -249,7 +299,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     __syncwarp();
 
-    build_lut<T>(lut, __ldg(p.code + (lane & 15)), tid, kW * 32);
+    build_lut<T>(lut, cv, tid, kW * 32);
     __syncthreads();
     if (p.pdl == 2) griddep_wait();  // activations and outputs may belong to the preceding grid
 
@@ -323,7 +373,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int jj = 0; jj < NJ; ++jj)
 #pragma unroll
                 for (int r = 0; r < 4; ++r) {
-                    sts_f32(park_addr<NJ>(lut, b, warp, (i * NJ + jj) * 4 + r, lane), acc[i][jj][r]);
+                    sts_f32(park_addr<G>(lut, b, warp, (i * NJ + jj) * 4 + r, lane), acc[i][jj][r]);
                     acc[i][jj][r] = 0.f;
                 }
         __syncwarp();
@@ -351,7 +401,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int jj = 0; jj < NJ; ++jj)
 #pragma unroll
                     for (int r = 0; r < 4; ++r)
-                        sum[i][jj][r] += lds_f32(park_addr<NJ>(lut, b, w, (i * NJ + jj) * 4 + r, lane));
+                        sum[i][jj][r] += lds_f32(park_addr<G>(lut, b, w, (i * NJ + jj) * 4 + r, lane));
         }
         const int rows_t = pl.tile_rows(t), y_t = pl.tile_y(t);
 #pragma unroll
@@ -398,7 +448,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             cc.step(pl, stride);
             const bool more = cc.i < we;
             const int s_nxt = more ? cc.s : s_cur;
-            const uint32_t am_st = st_addr + G::CODE_BYTES;
+            const uint32_t am_st = am_addr(k);
             const int x0 = ((s_cur * 4) >> p.am_shift) & ~3;
             float am[MT][2][4];  // absmax of rows 16 ia + g (+ 8 hh), for the stage's 4 units
 #pragma unroll
@@ -496,7 +546,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                 case 5: fine = run_tile(std::integral_constant<int, 3>{}, Tr{}); break;
                 case 6: fine = run_tile(std::integral_constant<int, 3>{}, F{}); break;
                 case 7: fine = run_tile(std::integral_constant<int, 4>{}, Tr{}); break;
-                default: fine = run_tile(std::integral_constant<int, 4>{}, F{}); break;
+                case 8: fine = run_tile(std::integral_constant<int, 4>{}, F{}); break;
+                default:
+                    if constexpr (MTM >= 5) {
+                        fine = run_tile(std::integral_constant<int, 5>{}, Tr{});  // 72 rows
+                    } else {
+                        fine = false;
+                    }
+                    break;
             }
             if (!fine || !flush(tile)) {
                 ok = false;
@@ -567,9 +624,9 @@ static int stage_heights(const RowsParams& p, int gmax, int* heights, int* map_o
     return nh;
 }
 
-template <typename T, int NJ, bool BS64>
+template <typename T, int NJ, bool BS64, bool CONTIG>
 static cudaError_t launch_t(const RowsMaps& m, const RowsParams& p, int smem, cudaStream_t stream) {
-    auto kern = q4_gemm_rows_kernel<T, NJ, BS64>;
+    auto kern = q4_gemm_rows_kernel<T, NJ, BS64, CONTIG>;
     cudaError_t e = ensure_smem_attr((const void*)kern, (size_t)smem);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
@@ -594,23 +651,36 @@ int rows_warps() { return rows::kW; }
 cudaError_t rows_launch(int act_dtype, int m_pad, const RowsParams& p0, const uint8_t* Wp, const float* absmax,
                         int am_per_row, int smem, cudaStream_t stream) {
     RowsParams p = p0;
+    if (m_pad != 8) p.contig = 0;  // two column tiles: round robin only (the partial tiles fill the parking space)
     int heights[kRowsMaxMaps];
     for (int& v : p.map_of) v = 0;
-    const int gmax = (m_pad == 8 ? rows::Geo<1>::MAX_ROWS : rows::Geo<2>::MAX_ROWS) / 8;
-    const int nh = rows::stage_heights(p, gmax, heights, p.map_of);
+    const int max_rows = (m_pad == 8 && !p.contig) ? rows::Geo<1, false>::MAX_ROWS : rows::Geo<1, true>::MAX_ROWS;
+    const int nh = rows::stage_heights(p, max_rows / 8, heights, p.map_of);
     rows::RowsMaps m;
+    memset(&m, 0, sizeof(m));
+    p.n_maps = nh;
     cudaError_t e = rows::make_maps(p, Wp, absmax, am_per_row, heights, nh, &m);
     if (e != cudaSuccess) return e;
     const bool bs64 = p.am_shift == 0;
     using namespace rows;
     if (act_dtype == 0) {
-        if (m_pad == 8) return bs64 ? launch_t<__nv_bfloat16, 1, true>(m, p, smem, stream)
-                                    : launch_t<__nv_bfloat16, 1, false>(m, p, smem, stream);
-        return bs64 ? launch_t<__nv_bfloat16, 2, true>(m, p, smem, stream)
-                    : launch_t<__nv_bfloat16, 2, false>(m, p, smem, stream);
+        if (m_pad == 8) {
+            if (p.contig)
+                return bs64 ? launch_t<__nv_bfloat16, 1, true, true>(m, p, smem, stream)
+                            : launch_t<__nv_bfloat16, 1, false, true>(m, p, smem, stream);
+            return bs64 ? launch_t<__nv_bfloat16, 1, true, false>(m, p, smem, stream)
+                        : launch_t<__nv_bfloat16, 1, false, false>(m, p, smem, stream);
+        }
+        return bs64 ? launch_t<__nv_bfloat16, 2, true, false>(m, p, smem, stream)
+                    : launch_t<__nv_bfloat16, 2, false, false>(m, p, smem, stream);
     }
-    if (m_pad == 8) return bs64 ? launch_t<__half, 1, true>(m, p, smem, stream) : launch_t<__half, 1, false>(m, p, smem, stream);
-    return bs64 ? launch_t<__half, 2, true>(m, p, smem, stream) : launch_t<__half, 2, false>(m, p, smem, stream);
+    if (m_pad == 8) {
+        if (p.contig)
+            return bs64 ? launch_t<__half, 1, true, true>(m, p, smem, stream)
+                        : launch_t<__half, 1, false, true>(m, p, smem, stream);
+        return bs64 ? launch_t<__half, 1, true, false>(m, p, smem, stream) : launch_t<__half, 1, false, false>(m, p, smem, stream);
+    }
+    return bs64 ? launch_t<__half, 2, true, false>(m, p, smem, stream) : launch_t<__half, 2, false, false>(m, p, smem, stream);
 }
 
 }  // namespace q4

@@ -190,8 +190,10 @@ def test_launch_table_invariants(wl):
         assert 1 <= p["ctas"] <= min(148, p["units"])
         assert p["smem_bytes"] <= 227 * 1024
         tma_ok = c.blocksize >= 64 and (c.K // c.blocksize) % 4 == 0 and p["units"] > 1
-        assert p["loader"] == (7 if tma_ok else 1)
-        if tma_ok:
+        tiles, weights = -(-c.N // 64), c.N * c.K
+        rows = not (tiles <= 148 and tiles * 5 >= 148 * 4) and weights < 2**27 and not (c.M >= 8 and weights >= 2**26)
+        assert p["loader"] == ((7 if rows else 2) if tma_ok else 1), (wl, c)
+        if tma_ok and rows:
             # row-split kernel: 8-row groups over at most one CTA per SM, the
             # workspace is the 256-byte error header alone
             assert p["ctas"] == min(148, -(-c.N // 8)) and p["warps"] == 8 and p["rows_per_tile"] == 64
@@ -201,6 +203,8 @@ def test_launch_table_invariants(wl):
         want_ws = 0 if p["units"] == 1 else 256 + 148 * 2 * 4096 + -(-p["tiles"] * 4 // 256) * 256
         assert p["workspace_bytes"] == want_ws
         assert p["depth"] >= 1 and p["l2_prefetch"] in (1, 128, 256)
+        if tma_ok:
+            assert p["warps"] == 8 and p["depth"] == 2  # stream-K TMA kernel
 
 
 @pytest.mark.parametrize("total,parts", [(1, 1), (1, 16), (7, 3), (40, 148), (4096, 148), (57344, 148),
