@@ -68,8 +68,8 @@ def kernel_name(plan: dict) -> str:
         return "q4_gemm_f32_kernel"
     if plan["math"] == 3:
         return "q4_gemm_umma_kernel"
-    return {1: "q4_gemm_mma_kernel", 2: "q4_gemm_tma_kernel", 3: "q4_gemm_tma_kernel"}.get(plan["loader"],
-                                                                                            "q4_gemm_ws_kernel")
+    return {1: "q4_gemm_mma_kernel", 2: "q4_gemm_tma_kernel", 3: "q4_gemm_tma_kernel",
+            7: "q4_gemm_rows_kernel"}.get(plan["loader"], "q4_gemm_ws_kernel")
 
 
 def ncu_traffic(workload: str):
@@ -232,10 +232,16 @@ def crossover_estimates(layers, per_shape, peak_gbs: float) -> list:
     """Per weight shape measured at several M: the smallest M at which the
     split path's HBM-peak time undercuts the measured fused time, taken
     from the measured points or, past them, from a line through the last two."""
+    return crossover_from_points([(L.case, ps["us_serialized"]) for L, ps in zip(layers, per_shape)], peak_gbs)
+
+
+def crossover_from_points(points, peak_gbs: float) -> list:
+    """crossover_estimates over (case, measured fused us) pairs."""
     by_shape = {}
-    for L, ps in zip(layers, per_shape):
-        c = L.case
-        by_shape.setdefault((c.N, c.K, c.blocksize), []).append((c.M, ps["us_serialized"], c))
+    for c, us in points:
+        if c.act != "bf16" or c.table != "normal" or c.outliers:
+            continue
+        by_shape.setdefault((c.N, c.K, c.blocksize), []).append((c.M, us, c))
     res = []
     for (N, K, bs), pts in by_shape.items():
         pts.sort(key=lambda x: x[0])
@@ -296,6 +302,122 @@ def measure_split_path(layers, device, stream, reps: int = 20) -> list:
         out.append({"tag": c.tag, "dequant_us": round(times[0], 2), "gemm_us": round(times[1], 2),
                     "us": round(times[0] + times[1], 2), "timing": f"CUDA graph of {reps} launches per half, best of 3"})
     return out
+
+
+CONFIGS = ("square4096", "decode70b", "msweep", "variants", "aspect")
+
+
+def copies_for(weight_bytes: int) -> int:
+    """Distinct weight copies a back-to-back timing cycles through so that
+    the bytes it reads exceed three times the L2: max(2, ceil(3 L2 / bytes)),
+    at most 64 and at most about 6 GB in all."""
+    need = max(2, -(-3 * L2_BYTES // max(1, weight_bytes)))
+    return int(max(1, min(need, 64, (6 << 30) // max(1, weight_bytes))))
+
+
+def measure_configs(device, peak: float, stream, reps: int = 3) -> list:
+    """Every case of the five configurations, one at a time: device time per
+    launch of back-to-back fused GEMMs (CUDA graph, dependent launch mode 2)
+    through the C ABI, cycling over distinct weight copies so that the
+    weights come from HBM, not L2 (the copies read more than 3x the L2)."""
+    import ctypes
+    P = ctypes.c_void_p
+    L = q4.lib()
+    rows = []
+    for name in CONFIGS:
+        wl = inputs.workloads()[name]
+        for i, c in enumerate(wl.cases):
+            seed = inputs.seed_for(wl.index, c.M) + i
+            dt = TORCH_ACT[c.act]
+            code = torch.from_numpy(inputs.CODE_TABLES[c.table]()).to(device)
+            W = inputs.weights_device(c.N, c.K, seed, device, c.outliers)
+            packed, absmax = q4.q4_quantize_blockwise(W.reshape(-1), c.blocksize, code)
+            del W
+            wbytes = packed.numel() + 4 * absmax.numel()
+            n = copies_for(wbytes)
+            copies = [(packed, absmax)] + [(packed.clone(), absmax.clone()) for _ in range(n - 1)]
+            A = inputs.activations(c.M, c.K, dt, seed).to(device)
+            out = torch.empty((c.M, c.N), dtype=dt, device=device)
+            ws_bytes = q4.q4_gemm_workspace_size(c.M, c.N, c.K, c.blocksize, dt)
+            ws = torch.zeros(max(ws_bytes, 16), dtype=torch.uint8, device=device)
+            act = {"bf16": q4.Q4_BF16, "fp16": q4.Q4_FP16, "fp32": q4.Q4_FP32}[c.act]
+            ov = q4.overrides(pdl=2)
+            args = [(P(A.data_ptr()), P(pk.data_ptr()), P(am.data_ptr()), P(code.data_ptr()), c.M, c.N, c.K,
+                     c.blocksize, act, P(out.data_ptr()), P(ws.data_ptr()), ws.numel()) for pk, am in copies]
+            R = max(20, n)
+
+            def run(s):
+                for r in range(R):
+                    rc = L.q4_gemm_skinny_ex(*args[r % n], P(s.cuda_stream), ctypes.byref(ov))
+                    if rc != 0:
+                        raise q4.Q4Error(rc, "q4_gemm_skinny_ex")
+
+            with torch.cuda.stream(stream):
+                run(stream)
+            stream.synchronize()
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream, capture_error_mode="relaxed"):
+                run(torch.cuda.current_stream())
+            best = float("inf")
+            for _ in range(reps):
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                with torch.cuda.stream(stream):
+                    e0.record(stream)
+                    g.replay()
+                    e1.record(stream)
+                stream.synchronize()
+                best = min(best, e0.elapsed_time(e1) * 1e3 / R)
+            del g, copies, packed, absmax
+            torch.cuda.empty_cache()
+            plan = q4.q4_gemm_plan(c.M, c.N, c.K, c.blocksize, dt)
+            b = c.algorithmic_bytes()
+            gbs = b / (best * 1e-6) / 1e9
+            e = 4 if c.act == "fp32" else 2
+            rows.append({
+                "config": name, "case": c.tag, "M": c.M, "N": c.N, "K": c.K, "blocksize": c.blocksize, "act": c.act,
+                "table": c.table, "outliers": c.outliers, "us": round(best, 3), "GB/s": round(gbs, 1),
+                "frac_of_peak": round(gbs / peak, 4), "bytes": b,
+                "bf16_weight_roofline_us": round((c.M * c.K * e + 2 * c.N * c.K + c.M * c.N * e) / (peak * 1e3), 3),
+                "t_split_est_us": round(split_time_est_us(c, peak), 3),
+                "weight_copies": n, "l2": "from HBM" if n * wbytes > L2_BYTES else "fits L2 (not HBM-bound)",
+                "kernel": kernel_name(plan), "loader": plan["loader"], "ctas": plan["ctas"]})
+            log(f"per_config {name} {c.tag}: {best:.2f} us, {gbs:.0f} GB/s, {n} copies, {kernel_name(plan)}")
+    return rows
+
+
+def oracle_per_config(rows: list, seconds: float) -> None:
+    """The oracle (as it stands) on a sample of each per_config case's
+    weight rows, one thread and all of this process's cores (row slices on
+    threads; the C oracle releases the GIL), scaled to the full layer."""
+    import concurrent.futures as cf
+    import oracle
+    cores = len(os.sched_getaffinity(0))
+    budget = seconds / max(1, len(rows))
+    with cf.ThreadPoolExecutor(max_workers=cores) as pool:
+        for r in rows:
+            c = inputs.Case(r["M"], r["N"], r["K"], r["blocksize"], r["act"], r["table"], r["outliers"], r["case"])
+            per_row = _oracle_time(c, 2, _oracle_sample(c, 2, 1)) / 2
+            nrows = int(max(cores, min(c.N, 4096, budget / max(per_row, 1e-9))))
+            prep = _oracle_sample(c, nrows, 1)
+            t1 = _oracle_time(c, nrows, prep)
+            a, packed, absmax, code = prep
+            rb, ab = c.K // 2, c.K // c.blocksize
+            bounds = [nrows * t // cores for t in range(cores + 1)]
+
+            def part(t):
+                lo, hi = bounds[t], bounds[t + 1]
+                if hi <= lo:
+                    return 0.0
+                sub = (a, packed[lo * rb:hi * rb], absmax[lo * ab:hi * ab], code)
+                return _oracle_time(c, hi - lo, sub)
+
+            t0 = time.perf_counter()
+            list(pool.map(part, range(cores)))
+            tall = time.perf_counter() - t0
+            r["oracle_us_1core"] = round(t1 / nrows * c.N * 1e6, 1)
+            r["oracle_us_all_cores"] = round(tall / nrows * c.N * 1e6, 1)
+            r["oracle_cores"] = cores
+            r["oracle_sample_rows"] = nrows
 
 
 def run_e2e(layers, device, steps: int, world: int) -> float:
@@ -504,6 +626,7 @@ def run_ours(args, world, rank, local):
     # dequantize kernel into a bf16 weight matrix, then a cuBLAS bf16 GEMM.
     split_path = measure_split_path(layers, device, stream) if args.split_path else None
 
+
     # End to end through the public Python API: per step, one H2D copy of all
     # of the step's activations from pinned memory, the layer calls, one D2H
     # copy of all of its outputs.  Two buffer sets alternate between steps and
@@ -519,10 +642,21 @@ def run_ours(args, world, rank, local):
     h2d = host_in.numel()
     d2h = host_out.numel()
 
+    # Every case of the five configurations, each timed from HBM (outside
+    # the timed region; single-GPU runs).
+    total_weight_bytes = sum(L.packed.numel() + 4 * L.absmax.numel() for L in layers)
+    per_config = None
+    if not args.no_per_config and world == 1:
+        for L in layers:  # hand the step's weights back before the per-case layers are built
+            L.packed = L.absmax = None
+        torch.cuda.empty_cache()
+        per_config = measure_configs(device, peak, stream)
+
     if rank != 0:
         return None
     cpu = cpu_baseline(wl, args.cpu_seconds) if (world == 1 and not args.no_cpu_baseline) else None
-    total_weight_bytes = sum(L.packed.numel() + 4 * L.absmax.numel() for L in layers)
+    if per_config is not None and not args.no_cpu_baseline:
+        oracle_per_config(per_config, args.cpu_seconds)
     act_dtype = "+".join(sorted({ {"bf16": "bf16", "fp16": "f16", "fp32": "f32"}[L.case.act] for L in layers}))
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
@@ -530,8 +664,12 @@ def run_ours(args, world, rank, local):
         "vs_baseline": None, "dtype": act_dtype, "data": "synthetic",
         "config": {"workload": wl.name + (f" [only {args.only}]" if args.only else ""), "M": sorted({c.M for c in wl.cases}), "blocksize": 64,
                    "code_table": "normal-quantile", "activations": f"{act_dtype} ~N(0,1)", "weights": "N(0,0.02^2) fp32 -> 4-bit",
-                   "l2": f"inputs larger than L2: {total_weight_bytes / 1e6:.0f} MB of packed weights per step "
-                         f"vs {L2_BYTES / 2**20:.0f} MiB L2, no flush",
+                   "l2": (f"inputs larger than L2: {total_weight_bytes / 1e6:.0f} MB of packed weights per step "
+                          f"vs {L2_BYTES / 2**20:.0f} MiB L2, no flush" if total_weight_bytes * args.steps > 3 * L2_BYTES
+                          and total_weight_bytes > L2_BYTES else
+                          f"{total_weight_bytes / 1e6:.1f} MB of packed weights per step fit the "
+                          f"{L2_BYTES / 2**20:.0f} MiB L2: this step's figure is L2-fed, not HBM-bound "
+                          f"(per_config times every case from HBM)"),
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                    "timing": f"CUDA graphs of {chunk} steps, CUDA events, device time",
                    "dependent_launch": args.pdl},
@@ -541,7 +679,11 @@ def run_ours(args, world, rank, local):
                      "per_unit": "0.5 B per weight (codes) + 4/bs B (absmax) + A and C once",
                      "duration": "average launch = timed-region device time / launches (all launches are this kernel)"},
         "per_shape": per_shape,
-        "crossover": crossover_estimates(layers, per_shape, peak),
+        "crossover": crossover_estimates(layers, per_shape, peak) or (
+            crossover_from_points([(inputs.Case(r["M"], r["N"], r["K"], r["blocksize"], r["act"], r["table"],
+                                                r["outliers"]), r["us"]) for r in per_config
+                                   if r["config"] == "msweep"], peak) if per_config else []),
+        "per_config": per_config,
         "split_path": split_path if args.split_path else None,
         "e2e": {"value": round(e2e_value, 2) if e2e_value else None, "unit": "GB/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "steps": e2e_steps,
@@ -588,23 +730,49 @@ def _oracle_time(case, rows, prepared):
     return time.perf_counter() - t0
 
 
+def _oracle_parallel(case, rows, prepared, pool, cores) -> float:
+    """Seconds for the oracle's GEMM over `rows` weight rows split into
+    `cores` row slices run on threads (the C oracle releases the GIL)."""
+    a, packed, absmax, code = prepared
+    rb, ab = case.K // 2, case.K // case.blocksize
+    bounds = [rows * t // cores for t in range(cores + 1)]
+
+    def part(t):
+        lo, hi = bounds[t], bounds[t + 1]
+        return _oracle_time(case, hi - lo, (a, packed[lo * rb:hi * rb], absmax[lo * ab:hi * ab], code)) if hi > lo else 0.0
+
+    t0 = time.perf_counter()
+    list(pool.map(part, range(cores)))
+    return time.perf_counter() - t0
+
+
 def cpu_baseline(wl, seconds: float) -> dict:
-    """The oracle's GEMM as it stands (plain C loops, one thread), on the
-    first rows of each layer, called repeatedly for about `seconds` in all."""
-    tot_bytes = tot_s = 0.0
+    """The oracle's GEMM as it stands (plain C loops) on the first rows of
+    each layer: on all of this process's cores (row slices on threads; the
+    value) and on one thread, called repeatedly for about `seconds` in all."""
+    import concurrent.futures as cf
+    cores = len(os.sched_getaffinity(0))
+    res = {}
     desc = []
-    for i, c in enumerate(wl.cases):
-        rows = min(c.N, SAMPLE_ROWS_MAX)
-        prep = _oracle_sample(c, rows, inputs.seed_for(wl.index, c.M) + i)
-        spent, reps = 0.0, 0
-        while reps == 0 or spent < seconds / len(wl.cases):
-            spent += _oracle_time(c, rows, prep)
-            reps += 1
-        tot_s += spent
-        tot_bytes += reps * inputs.Case(c.M, rows, c.K, c.blocksize, act=c.act).algorithmic_bytes()
-        desc.append(f"{reps}x {rows}/{c.N} rows of K{c.K}N{c.N}")
-    return {"value": round(tot_bytes / tot_s / 1e9, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
-            "sample": "; ".join(desc) + f" (M={wl.cases[0].M}; {tot_s:.1f} s single-threaded)"}
+    with cf.ThreadPoolExecutor(max_workers=cores) as pool:
+        for mode, n_thr in (("1", 1), ("all", cores)):
+            tot_bytes = tot_s = 0.0
+            for i, c in enumerate(wl.cases):
+                rows = min(c.N, SAMPLE_ROWS_MAX * n_thr)
+                prep = _oracle_sample(c, rows, inputs.seed_for(wl.index, c.M) + i)
+                spent, reps = 0.0, 0
+                while reps == 0 or spent < seconds / 2 / len(wl.cases):
+                    spent += _oracle_time(c, rows, prep) if n_thr == 1 else _oracle_parallel(c, rows, prep, pool, n_thr)
+                    reps += 1
+                tot_s += spent
+                tot_bytes += reps * inputs.Case(c.M, rows, c.K, c.blocksize, act=c.act).algorithmic_bytes()
+                if mode == "all":
+                    desc.append(f"{reps}x {rows}/{c.N} rows of K{c.K}N{c.N}")
+            res[mode] = tot_bytes / tot_s / 1e9
+    return {"value": round(res["all"], 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
+            "single_thread_value": round(res["1"], 4),
+            "sample": "; ".join(desc) + f" per all-core run (M={wl.cases[0].M}; row slices on {cores} threads, "
+                      f"and the same layers one thread at a time; about {seconds:.0f} s in all)"}
 
 
 def run_reference(args, world, rank):
@@ -613,22 +781,26 @@ def run_reference(args, world, rank):
     whole run takes about --reference-seconds."""
     if rank != 0:
         return None
+    import concurrent.futures as cf
     wl = inputs.workloads()[args.workload]
+    cores = len(os.sched_getaffinity(0))
+    pool = cf.ThreadPoolExecutor(max_workers=cores)
     per_row = []
     for i, c in enumerate(wl.cases):
         prep = _oracle_sample(c, 2, inputs.seed_for(wl.index, c.M) + i)
         per_row.append(_oracle_time(c, 2, prep) / 2)
     step_s = args.reference_seconds / max(1, args.steps + args.warmup)
-    rows = [int(max(1, min(c.N, SAMPLE_ROWS_MAX, step_s / len(wl.cases) / max(pr, 1e-9))))
+    rows = [int(max(cores, min(c.N, SAMPLE_ROWS_MAX * cores, cores * step_s / len(wl.cases) / max(pr, 1e-9))))
             for c, pr in zip(wl.cases, per_row)]
     preps = [_oracle_sample(c, r, inputs.seed_for(wl.index, c.M) + i) for i, (c, r) in enumerate(zip(wl.cases, rows))]
     for _ in range(args.warmup):
         for c, r, p in zip(wl.cases, rows, preps):
-            _oracle_time(c, r, p)
+            _oracle_parallel(c, r, p, pool, cores)
     tot_s = 0.0
     for _ in range(args.steps):
         for c, r, p in zip(wl.cases, rows, preps):
-            tot_s += _oracle_time(c, r, p)
+            tot_s += _oracle_parallel(c, r, p, pool, cores)
+    pool.shutdown()
     step_bytes = sum(inputs.Case(c.M, r, c.K, c.blocksize, act=c.act).algorithmic_bytes()
                      for c, r in zip(wl.cases, rows))
     value = step_bytes * args.steps / tot_s / 1e9
@@ -636,8 +808,8 @@ def run_reference(args, world, rank):
     return {"impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(tot_s / args.steps * 1e3, 4),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": wl.name, "parallelism": "CPU oracle, one thread"},
-            "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "config": {"workload": wl.name, "parallelism": f"CPU oracle, row slices on {cores} threads"},
+            "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
                              "sample": sample + " per step"},
             "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
@@ -653,6 +825,7 @@ def main():
     ap.add_argument("--reference-seconds", type=float, default=60.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end leg (profiling runs)")
+    ap.add_argument("--no-per-config", action="store_true", help="skip timing every case of the five configurations")
     ap.add_argument("--only", default="", help="comma-separated case tags of the workload to run (profiling)")
     ap.add_argument("--split-path", action="store_true",
                     help="also time the split path (dequantize kernel + cuBLAS bf16 GEMM) per layer")

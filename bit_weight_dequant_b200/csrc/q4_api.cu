@@ -109,15 +109,16 @@ static bool data_parallel_pays(int tiles, int sms, int64_t weights) {
 // (back-to-back launches over distinct weight copies).  The row-split kernel
 // has no cross-CTA fix-up, which is what dominates small and medium layers
 // (K5120/N5120: 7.3 vs 8.2 us; K10240/N320: 5.9 vs 11.2 us; 4096^2: 6.1 vs
-// 6.5 us; K8192/N10240: 13.5 vs 14.7 us).  The stream-K kernel keeps full
-// 64-row tiles, which wins when it already runs one CTA per tile on nearly
-// every SM (N = 8192: 128 tiles), on the largest layers (2^27 weights or
-// more: K8192/N28672 28.8 vs 29.5 us, K2560/N248320 67 vs 96 us) and for
-// M >= 8 on layers of 2^26 weights or more.
+// 6.5 us; K8192/N10240: 13.5 vs 14.7 us), and a chain of layers runs best on
+// one kernel throughout (the 70B-class decode step: 83.5 us on the row-split
+// kernel, 84.8 us on stream-K, 86.7 us mixing them per layer).  The
+// stream-K kernel stays where the row-split kernel's tiles hold few k-stages
+// and every CTA has many of them (K2560/N248320: 67 vs 96 us), and for
+// M >= 8 on layers of 2^26 weights or more (K17408/N5120 at M = 16: 21 vs
+// 26 us).
 static bool rows_kernel_pays(int M, int N, int K, int sms) {
     const int64_t tiles = ((int64_t)N + 63) / 64, weights = (int64_t)N * K;
-    if (tiles <= sms && tiles * 5 >= (int64_t)sms * 4) return false;  // one stream-K CTA per tile, >= 80 % of the SMs
-    if (weights >= ((int64_t)1 << 27)) return false;
+    if (K < 4096 && tiles > 4 * (int64_t)sms) return false;
     if (M >= 8 && weights >= ((int64_t)1 << 26)) return false;
     return true;
 }

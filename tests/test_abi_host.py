@@ -191,7 +191,7 @@ def test_launch_table_invariants(wl):
         assert p["smem_bytes"] <= 227 * 1024
         tma_ok = c.blocksize >= 64 and (c.K // c.blocksize) % 4 == 0 and p["units"] > 1
         tiles, weights = -(-c.N // 64), c.N * c.K
-        rows = not (tiles <= 148 and tiles * 5 >= 148 * 4) and weights < 2**27 and not (c.M >= 8 and weights >= 2**26)
+        rows = not (c.K < 4096 and tiles > 4 * 148) and not (c.M >= 8 and weights >= 2**26)
         assert p["loader"] == ((7 if rows else 2) if tma_ok else 1), (wl, c)
         if tma_ok and rows:
             # row-split kernel: 8-row groups over at most one CTA per SM, the
