@@ -192,6 +192,7 @@ class Layer:
         self.ws = torch.zeros(max(self.ws_bytes, 16), dtype=torch.uint8, device=device)
         self.act = {"bf16": q4.Q4_BF16, "fp16": q4.Q4_FP16, "fp32": q4.Q4_FP32}[case.act]
         self.plan = q4.q4_gemm_plan(case.M, case.N, case.K, case.blocksize, dt)
+        self.plan.update({k: v for k, v in self.launch_kw.items() if k in ("math", "loader")})
         self.rebind(self.A, self.out)
         # Decode-time weights are static model parameters: let each GEMM's
         # prologue and first weight copies overlap the previous kernel.
@@ -532,7 +533,8 @@ def run_ours(args, world, rank, local):
     cases = [(i, c) for i, c in enumerate(wl.cases) if not args.only or c.tag in args.only.split(",")]
     if not cases:
         raise SystemExit(f"--only {args.only!r} matches no case of {args.workload}")
-    launch = {"loader": args.loader, "depth": args.depth, "l2_prefetch": args.l2_ahead, "ctas": args.ctas}
+    launch = {"loader": args.loader, "depth": args.depth, "l2_prefetch": args.l2_ahead, "ctas": args.ctas,
+              "math": args.math}
     layers = [Layer(c, inputs.seed_for(wl.index, c.M) + i, device, args.pdl, launch) for i, c in cases]
     host_in, dev_in, host_out, dev_out = bind_step_io(layers, device)
     torch.cuda.synchronize()
@@ -833,6 +835,8 @@ def main():
     ap.add_argument("--depth", type=int, default=0, help="launch-table override: depth (measurement)")
     ap.add_argument("--l2-ahead", type=int, default=0, help="launch-table override: l2_prefetch (measurement)")
     ap.add_argument("--ctas", type=int, default=0, help="launch-table override: CTAs (measurement)")
+    ap.add_argument("--math", type=int, default=0, choices=[0, 1, 2, 3],
+                    help="launch-table override: math (2: the CUDA-core kernel; measurement)")
     ap.add_argument("--pdl", type=int, default=2, choices=[0, 1, 2],
                     help="programmatic dependent launch mode for the GEMMs (2: static weights read early)")
     args = ap.parse_args()

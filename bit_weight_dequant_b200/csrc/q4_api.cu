@@ -133,9 +133,10 @@ static int gemm_choose(int M, int N, int K, int blocksize, int act_dtype, int nu
     if (ov && (ov->math > 3 || ov->l2_prefetch > 256 || ov->loader > 7 || ov->pdl > 2)) return Q4_ERR_INVALID_ARG;
     if (M > 128 || K % blocksize != 0) return Q4_ERR_UNSUPPORTED;
     GemmChoice c{};
-    if (act_dtype == Q4_FP32) {
-        // fp32 activations: the CUDA-core kernel (M <= 16), units of R rows x
-        // 512 k split over every warp of the grid.
+    if (act_dtype == Q4_FP32 || (ov && ov->math == 2)) {
+        // The CUDA-core kernel (M <= 16), units of R rows x 512 k split over
+        // every warp of the grid: fp32 activations always; bf16 / fp16 on
+        // request (math = 2), widened exactly to fp32 on load.
         if (M > 16) return Q4_ERR_UNSUPPORTED;
         if (ov && ((ov->math > 0 && ov->math != 2) || ov->loader > 1)) return Q4_ERR_UNSUPPORTED;
         const SimtShape sh = simt_shape(M);
@@ -461,7 +462,7 @@ static int gemm_entry(const void* A, const uint8_t* Wpacked, const float* absmax
     if (ch.math == 2) {
         int lbs = 0;
         while ((1 << lbs) < blocksize) ++lbs;
-        return from_cuda(simt_launch(simt_shape(M), ch.ctas, p, lbs, st));
+        return from_cuda(simt_launch(simt_shape(M), ch.ctas, p, lbs, act_dtype, st));
     }
     if (ch.loader == 7) {
         RowsParams rp{};

@@ -47,7 +47,9 @@ struct SimtShape {
 };
 SimtShape simt_shape(int M);
 size_t simt_smem_bytes();
-cudaError_t simt_launch(const SimtShape& sh, int ctas, const GemmParams& p, int log2_bs, cudaStream_t stream);
+// act_dtype: 0 bf16, 1 fp16 (widened exactly to fp32 on load), 2 fp32.
+cudaError_t simt_launch(const SimtShape& sh, int ctas, const GemmParams& p, int log2_bs, int act_dtype,
+                        cudaStream_t stream);
 
 // Row-split kernel for M <= 16 with 16-bit activations (q4_rows.cu).
 // act_dtype 0 = bf16, 1 = fp16; m_pad 8 or 16; smem = dynamic shared memory

@@ -1,15 +1,18 @@
-// q4_simt.cu -- fused blockwise 4-bit dequantize + skinny GEMM with fp32
-// activations, on the CUDA cores, for sm_100a:
+// q4_simt.cu -- fused blockwise 4-bit dequantize + skinny GEMM on the CUDA
+// cores, for sm_100a:
 //
 //     out[m, n] = [bias[n]] + sum_k A[m, k] * code[idx(n, k)] * absmax(n, k)
-//     M <= 16, A / out / bias fp32.
+//     M <= 16; A / out / bias fp32, or bf16 / fp16.
 //
 // The maintainer's reply in bitsandbytes PR #1920 ("[ROCm] Optimize
-// kgemm_4bit_inference_naive ...") describes the replacement kernels: the
-// tensor-core versions take fp16/bf16, the SIMT kernel also takes fp32, and
-// all accumulate in fp32.  This is that fp32 case.  Every product is an fp32
-// FMA of the activation with the exact fp32 code value; nothing is rounded
-// to 16 bits.
+// kgemm_4bit_inference_naive ...") describes the replacement kernels: a SIMT
+// kernel for the smallest batches and tensor-core (MMA) versions past them,
+// the SIMT kernel also taking fp32, all accumulating in fp32.  This is the
+// SIMT kernel.  Every product is an fp32 FMA of the activation (16-bit
+// activations widened exactly) with the exact fp32 code value; nothing is
+// rounded to 16 bits before the single rounding of the output.  For 16-bit
+// activations the launch table keeps the tensor-core kernels (measured
+// faster at every M); this kernel serves them on request (math = 2).
 //
 // Design for B200:
 //  * HBM-bound at M = 1 (0.5625 B per weight at blocksize 64), so the code
@@ -57,12 +60,12 @@ static int max_smem() {
 }
 
 struct Params {
-    const float* A;        // [M, K]
+    const void* A;         // [M, K] activations: fp32, or bf16/fp16 (widened exactly to fp32 on load)
     const uint8_t* Wp;     // [N, K/2]
     const float* absmax;   // [N * K / blocksize]
     const float* code;     // [16]
-    float* out;            // [M, N]
-    const float* bias;     // [N] or nullptr
+    void* out;             // [M, N] in the activation type
+    const void* bias;      // [N] in the activation type, or nullptr
     float* partials;       // [warps][2][R * MP]
     int* counters;         // [row groups], zero between calls
     int M, N, K;
@@ -177,7 +180,35 @@ struct Slot {
 
 static constexpr int kErrNoRoom = 2;
 
-template <int MP, int R, int NW, int D>
+// Activation types: fp32 as given; bf16 / fp16 widened exactly to fp32
+// (four pairs from one 16-byte load), the output rounded once to the type.
+template <typename TA>
+struct ActIO;
+template <>
+struct ActIO<float> {
+    __device__ __forceinline__ static float widen(float v) { return v; }
+    __device__ __forceinline__ static float narrow(float v) { return v; }
+};
+template <>
+struct ActIO<__nv_bfloat16> {
+    __device__ __forceinline__ static float widen(__nv_bfloat16 v) { return __bfloat162float(v); }
+    __device__ __forceinline__ static __nv_bfloat16 narrow(float v) { return __float2bfloat16_rn(v); }
+    // packed pair (first value in the low half) -> the float pair, exactly
+    __device__ __forceinline__ static uint64_t pair(uint32_t w) {
+        return (uint64_t)(w << 16) | ((uint64_t)(w & 0xFFFF0000u) << 32);
+    }
+};
+template <>
+struct ActIO<__half> {
+    __device__ __forceinline__ static float widen(__half v) { return __half2float(v); }
+    __device__ __forceinline__ static __half narrow(float v) { return __float2half_rn(v); }
+    __device__ __forceinline__ static uint64_t pair(uint32_t w) {
+        const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w));
+        return (uint64_t)__float_as_uint(f.x) | ((uint64_t)__float_as_uint(f.y) << 32);
+    }
+};
+
+template <typename TA, int MP, int R, int NW, int D>
 __global__ void __launch_bounds__(NW * 32, 1) q4_gemm_f32_kernel(const Params p) {
     extern __shared__ __align__(16) uint8_t smem[];
     const uint32_t sbase = smem_addr(smem);
@@ -186,7 +217,7 @@ __global__ void __launch_bounds__(NW * 32, 1) q4_gemm_f32_kernel(const Params p)
     uint32_t lane8 = table | ((uint32_t)(lane & 15) << 3);
     const uint8_t* Wp = p.Wp;
     const float* absmax = p.absmax;
-    const float* Aact = p.A;
+    const TA* Aact = static_cast<const TA*>(p.A);
 
     if (p.pdl != 2) griddep_wait();
     // The loads are plain asm the compiler may move: each one takes its
@@ -316,12 +347,18 @@ __global__ void __launch_bounds__(NW * 32, 1) q4_gemm_f32_kernel(const Params p)
 #pragma unroll
             for (int m = 0; m < MP; ++m) {
                 if (m < p.M) {
-                    const float* src = Aact + (size_t)m * p.K + kq;
-                    if (p.a32) {
-                        ldg_pairs8(src, a[m]);
+                    const TA* src = Aact + (size_t)m * p.K + kq;
+                    if constexpr (sizeof(TA) == 2) {
+                        const uint4 v = ldg_v4(src);  // 8 values, 16-byte aligned (K % 32 == 0, A 16-byte aligned)
+                        a[m][0] = ActIO<TA>::pair(v.x);
+                        a[m][1] = ActIO<TA>::pair(v.y);
+                        a[m][2] = ActIO<TA>::pair(v.z);
+                        a[m][3] = ActIO<TA>::pair(v.w);
+                    } else if (p.a32) {
+                        ldg_pairs8(reinterpret_cast<const float*>(src), a[m]);
                     } else {
-                        ldg_pairs(src, a[m][0], a[m][1]);
-                        ldg_pairs(src + 4, a[m][2], a[m][3]);
+                        ldg_pairs(reinterpret_cast<const float*>(src), a[m][0], a[m][1]);
+                        ldg_pairs(reinterpret_cast<const float*>(src) + 4, a[m][2], a[m][3]);
                     }
                 } else {
                     a[m][0] = a[m][1] = a[m][2] = a[m][3] = 0ull;
@@ -364,7 +401,10 @@ __global__ void __launch_bounds__(NW * 32, 1) q4_gemm_f32_kernel(const Params p)
     auto store = [&](uint32_t rg, int e, float v) {
         const int r = e % R, m = e / R;
         const int n = (int)rg * R + r;
-        if (n < p.N && m < p.M) p.out[(size_t)m * p.N + n] = p.bias ? v + p.bias[n] : v;
+        if (n < p.N && m < p.M) {
+            const TA* bias = static_cast<const TA*>(p.bias);
+            static_cast<TA*>(p.out)[(size_t)m * p.N + n] = ActIO<TA>::narrow(bias ? v + ActIO<TA>::widen(bias[n]) : v);
+        }
     };
     constexpr int RM = R * MP;
 
@@ -451,9 +491,9 @@ __global__ void __launch_bounds__(NW * 32, 1) q4_gemm_f32_kernel(const Params p)
 
 // Compiled variants: MP = padded M, R = rows per unit, NW = warps per CTA,
 // D = register buffers per warp.
-template <int MP, int R, int NW, int D>
+template <typename TA, int MP, int R, int NW, int D>
 static cudaError_t launch_variant(const Params& p, int ctas, cudaStream_t stream) {
-    auto kern = q4_gemm_f32_kernel<MP, R, NW, D>;
+    auto kern = q4_gemm_f32_kernel<TA, MP, R, NW, D>;
     const int smem = max_smem();
     if (smem <= 0) return cudaErrorInvalidValue;
     cudaError_t e = ensure_smem_attr((const void*)kern, (size_t)smem);
@@ -486,14 +526,27 @@ SimtShape simt_shape(int M) {
 
 size_t simt_smem_bytes() { return (size_t)simt::max_smem(); }
 
-cudaError_t simt_launch(const SimtShape& sh, int ctas, const GemmParams& g, int log2_bs, cudaStream_t stream) {
+template <typename TA>
+static cudaError_t simt_launch_t(const SimtShape& sh, int ctas, const simt::Params& p, cudaStream_t stream) {
+    switch (sh.m_pad) {
+        case 1: return simt::launch_variant<TA, 1, 8, 16, 4>(p, ctas, stream);
+        case 2: return simt::launch_variant<TA, 2, 8, 8, 4>(p, ctas, stream);
+        case 4: return simt::launch_variant<TA, 4, 8, 8, 4>(p, ctas, stream);
+        case 8: return simt::launch_variant<TA, 8, 4, 8, 4>(p, ctas, stream);
+        case 16: return simt::launch_variant<TA, 16, 2, 8, 4>(p, ctas, stream);
+        default: return cudaErrorInvalidConfiguration;
+    }
+}
+
+cudaError_t simt_launch(const SimtShape& sh, int ctas, const GemmParams& g, int log2_bs, int act_dtype,
+                        cudaStream_t stream) {
     simt::Params p{};
-    p.A = static_cast<const float*>(g.A);
+    p.A = g.A;
     p.Wp = g.Wp;
     p.absmax = g.absmax;
     p.code = g.code;
-    p.out = static_cast<float*>(g.out);
-    p.bias = static_cast<const float*>(g.bias);
+    p.out = g.out;
+    p.bias = g.bias;
     p.partials = g.partials;
     p.counters = g.counters;
     p.M = g.M;
@@ -508,14 +561,9 @@ cudaError_t simt_launch(const SimtShape& sh, int ctas, const GemmParams& g, int 
     p.narrow = (uint64_t)p.units * p.warps < ((uint64_t)1 << 32) ? 1 : 0;
     p.a32 = (reinterpret_cast<uintptr_t>(g.A) & 31u) == 0 ? 1 : 0;
     p.error = g.error;
-    switch (sh.m_pad) {
-        case 1: return simt::launch_variant<1, 8, 16, 4>(p, ctas, stream);
-        case 2: return simt::launch_variant<2, 8, 8, 4>(p, ctas, stream);
-        case 4: return simt::launch_variant<4, 8, 8, 4>(p, ctas, stream);
-        case 8: return simt::launch_variant<8, 4, 8, 4>(p, ctas, stream);
-        case 16: return simt::launch_variant<16, 2, 8, 4>(p, ctas, stream);
-        default: return cudaErrorInvalidConfiguration;
-    }
+    if (act_dtype == 0) return simt_launch_t<__nv_bfloat16>(sh, ctas, p, stream);
+    if (act_dtype == 1) return simt_launch_t<__half>(sh, ctas, p, stream);
+    return simt_launch_t<float>(sh, ctas, p, stream);
 }
 
 }  // namespace q4

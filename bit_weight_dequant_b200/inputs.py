@@ -240,6 +240,10 @@ def workloads() -> dict:
     w["msweep_f32"] = Workload("fp32 activations, M 1,2,4,8,16 on K5120/N5120, K17408/N5120", 8, f32)
     w["longk_f32"] = Workload("M=1 K=131072 N=2048 bs64 fp32 activations (main-loop profiling shape)", 9,
                               [Case(1, 2048, 131072, act="fp32", tag="longk")])
+    # Not one of the five: the decode gate_up shape at M = 1, 2, 4, for the
+    # CUDA-core against tensor-core comparison.
+    w["gate_up_m"] = Workload("M 1,2,4 on K8192/N28672 bs64 bf16 normal-table", 10,
+                              [Case(M, 28672, 8192, tag=f"gate_upM{M}") for M in (1, 2, 4)])
     # Not one of the five: one long-K layer whose launch is almost all main
     # loop (start-up and tail are a few percent), for profiling the loop.
     w["longk"] = Workload("M=1 K=131072 N=8192 bs64 bf16 normal-table (main-loop profiling shape)", 5,

@@ -97,9 +97,12 @@ def run_case(case: inputs.Case, seed: int, device, check_quantizer: bool = True,
 
 
 def sample_rows(N: int, extra: int = 40, seed: int = 0) -> np.ndarray:
-    """Rows to check at full size: both ends, tile edges, the middle and a
-    seeded random spread."""
-    rows = {0, 1, N // 2, N - 2, N - 1, 63, 64, 127, 128, N - 65, N - 64}
+    """Rows to check at full size: the first and last row of every 64-row
+    tile and of the 8-row group after its first, both ends, the middle and a
+    seeded random spread (about 1 row in 16)."""
+    rows = {0, 1, N // 2, N - 2, N - 1, N - 65, N - 64}
+    for r in range(0, N, 64):
+        rows |= {r, r + 7, r + 8, r + 63}
     rng = np.random.default_rng(seed)
     rows |= set(rng.integers(0, N, extra).tolist())
     return np.array(sorted(r for r in rows if 0 <= r < N), dtype=np.int64)

@@ -95,7 +95,9 @@ def test_gemm_validation_before_cuda():
     assert ex(*args, 20, 64, 4096, 64, 0, ALIGNED, None, 0, None, b.overrides(loader=7)) == b.Q4_ERR_UNSUPPORTED
     assert ex(*args, 4, 64, 4096, 32, 0, ALIGNED, None, 0, None, b.overrides(loader=7)) == b.Q4_ERR_UNSUPPORTED
     assert ex(*args, 4, 64, 4096, 64, 0, ALIGNED, None, 0, None, b.overrides(loader=7, warps=9)) == b.Q4_ERR_UNSUPPORTED
-    assert ex(*args, 1, 64, 4096, 64, 0, ALIGNED, None, 0, None, b.overrides(math=2)) == b.Q4_ERR_UNSUPPORTED
+    # the CUDA-core kernel takes 16-bit activations on request, M <= 16
+    assert ex(*args, 17, 64, 4096, 64, 0, ALIGNED, None, 0, None, b.overrides(math=2)) == b.Q4_ERR_UNSUPPORTED
+    assert ex(*args, 4, 64, 4096, 64, 1, ALIGNED, None, 0, None, b.overrides(math=2, loader=2)) == b.Q4_ERR_UNSUPPORTED
 
 
 @pytest.mark.parametrize("M,N,K", [(17, 4096, 4096), (32, 300, 1024), (31, 8192, 28672)])

@@ -152,3 +152,31 @@ def test_f32_full_size_sampled(cuda_device, M, N, K):
     p_ref, a_ref = oracle.quantize(Wr, 64, code)
     y, S = oracle.gemm_f32(A, p_ref, a_ref, code, M, rows.size, K, 64)
     check_f32(out[:, rows_d], y, S, K, f"f32 full M{M} N{N} K{K}")
+
+
+@pytest.mark.parametrize("act", ["bf16", "fp16"])
+@pytest.mark.parametrize("M", [1, 2, 3, 4, 7, 16])
+@pytest.mark.parametrize("N,K,bs", [(300, 1024, 64), (513, 2560, 64), (61, 1088, 32), (190, 4096, 256)])
+def test_simt_16bit_activations(cuda_device, act, M, N, K, bs):
+    """The same kernel on bf16 / fp16 activations (override math = 2): the
+    activations are widened exactly, every product is an fp32 FMA and the
+    output is rounded once to the activation type."""
+    from parity import run_case
+    run_case(inputs.Case(M, N, K, blocksize=bs, act=act), seed=4700 + M + N, device=cuda_device,
+             check_quantizer=False, math=2)
+
+
+@pytest.mark.parametrize("ctas", [1, 3, 37])
+def test_simt_16bit_split_groups_and_bias(cuda_device, ctas):
+    """Row groups cut by warp boundaries and the bias epilogue, bf16."""
+    M, N, K, bs = 3, 700, 3072, 64
+    code, packed, absmax, _ = _problem(M, N, K, bs, 4800 + ctas)
+    A = inputs.activations(M, K, torch.bfloat16, 4801 + ctas)
+    bias = inputs.activations(1, N, torch.bfloat16, 4802).reshape(N)
+    dev = cuda_device
+    out = q4.q4_gemm_skinny(A.to(dev), torch.from_numpy(packed).to(dev), torch.from_numpy(absmax).to(dev),
+                            torch.from_numpy(code).to(dev), N, K, bs, bias=bias.to(dev), math=2, ctas=ctas)
+    torch.cuda.synchronize(dev)
+    from parity import bits_of, check_gemm
+    y, S = oracle.gemm(bits_of(A), oracle.BF16, packed, absmax, code, M, N, K, bs, bias_bits=bits_of(bias))
+    check_gemm(bits_of(out), y, S, "bf16", f"simt bf16 bias ctas {ctas}")
