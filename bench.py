@@ -56,7 +56,7 @@ def hbm_peak():
 
 def gemm_kernel_hash() -> str:
     h = hashlib.sha256()
-    for f in ("q4_gemm.cu", "q4_device.cuh", "q4_plan.cuh"):
+    for f in ("q4_gemm.cu", "q4_rows.cu", "q4_device.cuh", "q4_plan.cuh"):
         with open(os.path.join(ROOT, "bit_weight_dequant_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]

@@ -272,6 +272,7 @@ __device__ __forceinline__ void combine_tiles(const GemmParams& p, uint32_t slot
         int prev = 0;
         if (lane == 0) prev = atom_add_acq_rel_gpu(p.counters + t, 1);
         prev = __shfl_sync(0xffffffffu, prev, 0);
+        __syncwarp();  // the other lanes read the partials after lane 0's acquire
         const int cf = (int)part_owner(p.units, p.ctas, t0), cl = (int)part_owner(p.units, p.ctas, t1 - 1);
         if (prev != cl - cf) continue;
         zero_acc<S>(sum);

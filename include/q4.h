@@ -1,9 +1,10 @@
 /*
  * q4.h -- C ABI of libq4: blockwise 4-bit weight quantization,
  * dequantization and the fused dequantize + skinny matmul
- *     C[M,N] = A[M,K] . dequant(W)[N,K]^T,   1 <= M <= 16,
- * the decode-time hot path of a 4-bit quantized linear layer, hand-written
- * for NVIDIA B200 (sm_100a).
+ *     C[M,N] = A[M,K] . dequant(W)[N,K]^T,   1 <= M <= 128,
+ * the decode-time hot path of a 4-bit quantized linear layer (M <= 16;
+ * 17..128 on the larger-batch kernels), hand-written for NVIDIA B200
+ * (sm_100a).
  *
  * Source of the method: bitsandbytes PR #1920, "[ROCm] Optimize
  * kgemm_4bit_inference_naive for ROCm, use it for batch sizes other than 1":
@@ -56,7 +57,8 @@ extern "C" {
 typedef enum {
     Q4_OK = 0,
     Q4_ERR_INVALID_ARG = 1, /* null pointer, negative size, bad blocksize or dtype */
-    Q4_ERR_UNSUPPORTED = 2, /* M > 16, K % blocksize != 0, fp32 activations     */
+    Q4_ERR_UNSUPPORTED = 2, /* M > 128, K % blocksize != 0, fp32 with M > 16,   */
+                            /* a shape or override no compiled kernel takes     */
     Q4_ERR_MISALIGNED = 3,  /* a pointer misses the alignment stated below      */
     Q4_ERR_CUDA = 4,        /* a CUDA call or kernel launch failed              */
     Q4_ERR_WORKSPACE = 5    /* GEMM workspace missing or smaller than required  */
@@ -126,7 +128,9 @@ int q4_gemm_workspace_size(int M, int N, int K, int blocksize, int act_dtype, si
  * weights enter as T_rn(code *_fp32 absmax).  Either way each weight is
  * rounded once (at most 2^-8 relative for bf16, 2^-11 for fp16).
  * fp32 (the reply's SIMT kernel, which also takes fp32 inputs):
- * every product is an fp32 FMA with the exact fp32 code, scaled in fp32.
+ * every product is an fp32 FMA with the exact fp32 code, scaled in fp32;
+ * bf16/fp16 run on that kernel on request (override math = 2), widened
+ * exactly to fp32 on load.
  *   A        [M, K] act_dtype, row-major contiguous, 16-byte aligned
  *   Wpacked  uint8 [N*K/2] (rows of K/2 bytes), 16-byte aligned
  *   absmax   fp32 [N*K/blocksize], 4-byte aligned
@@ -150,6 +154,8 @@ int q4_gemm_workspace_size(int M, int N, int K, int blocksize, int act_dtype, si
  *            fixed-size region of partial sums (scratch), then one counter
  *            per weight tile (every call returns the counters it used to
  *            zero), so one workspace serves every problem size on a device.
+ *            Some kernels need the header alone (q4_gemm_workspace_size
+ *            then returns 256).
  *            The error word stays 0 unless a kernel gave up a bounded wait
  *            for its own asynchronous copies (1; outputs of that call are
  *            not valid) or found too little shared memory (2); the caller
@@ -180,6 +186,13 @@ int q4_gemm_skinny(const void* A, const uint8_t* Wpacked, const float* absmax, c
  *   - Every call shares the one array and clears its error word and tile
  *     counters with cudaMemsetAsync on `stream` before the kernel; calls that
  *     overlap on the GPU (other streams, other threads) race on it.
+ *   - The array's error word (see q4_gemm_skinny) is not reported: a call
+ *     whose kernel gave up a bounded wait returns Q4_OK with outputs that
+ *     are not valid, and the next call clears the word.  Callers that must
+ *     see such failures use q4_gemm_skinny with their own workspace.
+ *   - The cached address belongs to the CUDA context that was current at
+ *     the first call; after cudaDeviceReset on that device, do not call
+ *     this entry again in the same process.
  */
 #define Q4_NOALLOC_WORKSPACE_BYTES (2u << 20) /* 2 MiB */
 
@@ -191,7 +204,8 @@ int q4_gemm_skinny_noalloc(const void* A, const uint8_t* Wpacked, const float* a
  * tests).  `num_sms` <= 0 means "the current device's SM count". */
 typedef struct {
     int math;          /* 1 = tensor-core (mma.sync m16n8k16), 2 = CUDA-core FMA  */
-                       /* (fp32 activations), 3 = tcgen05 with tensor memory     */
+                       /* (fp32 activations; bf16/fp16 on request, M <= 16),     */
+                       /* 3 = tcgen05 with tensor memory                         */
     int sub_block;     /* k-width of one work unit: min(blocksize, 64); 512 for  */
                        /* math 2                                                 */
     int m_pad;         /* M padded to the MMA column count: 8, 16, 32 (math 1), */
@@ -201,9 +215,17 @@ typedef struct {
     int warps;         /* warps per CTA                                           */
     int ctas;          /* persistent CTAs (<= SM count, <= number of units)       */
     int depth;         /* work units each warp has in flight ahead of its compute */
+                       /* (loader 7: stage order, 1 round robin over the warps,  */
+                       /* 2 a contiguous range of stages per warp)               */
     int l2_prefetch;   /* L2 fetch-size hint on weight loads: 1 none, 128, 256 B  */
+                       /* (loader 7: 0 none, else stages fetched into L2 ahead   */
+                       /* of the shared-memory ring)                             */
     int loader;        /* 1 = per-lane global loads; TMA shared-memory ring with  */
-                       /* 2 = 4-unit (128-byte) or 3 = 2-unit (64-byte) stages   */
+                       /* 2 = 4-unit (128-byte) or 3 = 2-unit (64-byte) stages,  */
+                       /* units split over CTAs (stream-K); 7 = row-split: 8-row */
+                       /* groups of W split over the CTAs, every output finished */
+                       /* inside one CTA (M <= 16; default where it measured     */
+                       /* faster)                                                */
     int pdl;           /* programmatic dependent launch: 0 off; 1 on, the kernel  */
                        /* touches global memory only after the preceding grid    */
                        /* completed; 2 on, and code/Wpacked/absmax may be read   */

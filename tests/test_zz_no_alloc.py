@@ -28,7 +28,9 @@ def _ptr(t):
     return ctypes.c_void_p(t.data_ptr())
 
 
-@pytest.mark.parametrize("M,N,K", [(1, 1000, 4096), (5, 3000, 2560), (16, 700, 1024)])
+# (2, 40000, 2048) runs on the stream-K kernel, whose tile counters the entry
+# point clears; the others need the 256-byte header alone.
+@pytest.mark.parametrize("M,N,K", [(1, 1000, 4096), (5, 3000, 2560), (16, 700, 1024), (2, 40000, 2048)])
 def test_noalloc_matches_regular_entry_point_twice(cuda_device, M, N, K):
     bs = 64
     code = inputs.code_normal_quantile()
