@@ -98,22 +98,26 @@ static constexpr int kRowsMaxMaps = 4;
 // CTA c owns a contiguous run of 8-row groups of W and finishes its outputs
 // itself (no workspace besides the error word).
 struct RowsParams {
+    // What the prologue reads comes first, so that it shares the first
+    // cache lines of the parameter block.
+    int groups;        // ceil(N / 8)
+    int ctas;          // <= groups
+    int K;
+    int am_shift;      // log2(blocksize / 64)
+    int pdl;           // dependent launch mode (0, 1, 2), as in GemmParams
+    int l2_ahead;      // stages the producer asks the L2 to fetch beyond the first ring fill
+    int skip_stage;    // test hook: this stage index is never loaded (-1: none)
+    int contig;        // 1: each warp streams a contiguous range of stages (0: round robin)
+    int n_maps;        // tensor-map pairs the launcher encoded
+    uint32_t map_bits; // tensor-map pair of tile height h (8 .. 72 rows): bits 2 (h / 8) .. 2 (h / 8) + 1,
+                       // filled by the launcher (a uniform word, not an indexed array)
+    uint32_t wait_limit;  // polls before a wait on a stage or a parking buffer gives up
+    int M, N;
     const void* A;
     void* out;
     const void* bias;  // [N] activation type, or nullptr
     const float* code;
     int* error;        // workspace error word, or nullptr
-    int M, N, K;
-    int am_shift;      // log2(blocksize / 64)
-    int groups;        // ceil(N / 8)
-    int ctas;          // <= groups
-    int pdl;           // dependent launch mode (0, 1, 2), as in GemmParams
-    int l2_ahead;      // stages the producer asks the L2 to fetch beyond the first ring fill
-    uint32_t wait_limit;  // polls before a wait on a stage or a parking buffer gives up
-    int skip_stage;       // test hook: this stage index is never loaded (-1: none)
-    int contig;           // 1: each warp streams a contiguous range of stages (0: round robin)
-    int map_of[10];       // tensor-map pair of tile height h (8 .. 72 rows): map_of[h / 8], filled by the launcher
-    int n_maps;           // tensor-map pairs the launcher encoded
 };
 
 }  // namespace q4

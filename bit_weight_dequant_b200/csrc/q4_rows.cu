@@ -87,8 +87,11 @@ struct Geo {
     static constexpr int PARK_ROWS = NB * kW * REGS;
     static_assert(PARK_ROWS + (SPLIT ? 2 : 0) <= 256, "parking buffers must fit the table's free halves");
     static_assert(!SPLIT || D * 8 <= 128, "the full barriers fill one spare row");
-    static_assert(MAX_ROWS / 8 < (int)(sizeof(RowsParams::map_of) / sizeof(int)), "map_of indexes h / 8");
+    static_assert(2 * (MAX_ROWS / 8) + 2 <= 32 && kRowsMaxMaps <= 4, "map_bits holds a 2-bit pair index per h / 8");
 };
+
+// Tensor-map pair of tile height h.
+__device__ __forceinline__ int map_index(const RowsParams& p, int h) { return (int)((p.map_bits >> (2 * (h >> 3))) & 3u); }
 
 // Position of stage i in the CTA's work: tile `tile` (rows [y, y + h) of the
 // CTA's rows), k-stage `s` (columns [256 s, 256 s + 256)).
@@ -157,7 +160,7 @@ __device__ __forceinline__ uint32_t park_addr(uint32_t lut, int b, int w, int r,
 
 // Tensor maps of the launch: per box height h (8 .. 72 rows), one map of
 // the packed codes (h rows x 128 bytes, 128-byte swizzle) and one of the
-// absmax (h rows x 4 floats); RowsParams::map_of[h / 8] selects the pair.
+// absmax (h rows x 4 floats); map_index(p, h) selects the pair.
 struct RowsMaps {
     CUtensorMap w[kRowsMaxMaps];
     CUtensorMap a[kRowsMaxMaps];
@@ -165,7 +168,7 @@ struct RowsMaps {
 
 template <typename T, int NJ, bool BS64, bool CONTIG>
 __global__ void __launch_bounds__(kThreads, 1)
-    q4_gemm_rows_kernel(const __grid_constant__ RowsMaps maps, const __grid_constant__ RowsParams p) {
+    q4_gemm_rows_kernel(const __grid_constant__ RowsParams p, const __grid_constant__ RowsMaps maps) {
     using G = Geo<NJ, CONTIG>;
     constexpr int D = G::D, MTM = G::MT_MAX, NB = G::NB;
     extern __shared__ __align__(16) uint8_t smem_rows[];
@@ -234,20 +237,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t failed = last_issued + 4u * (uint32_t)D;           // int: a wait of this CTA ran out
 
     if (p.pdl == 1) griddep_wait();
-    if (tid == 0) {
-        for (int k = 0; k < D; ++k) {
-            mbar_init(full_bar(k), 1);
-            sts_u32(last_issued + 4u * (uint32_t)k, 0u);
-        }
-        sts_u32(reduced, 0u);
-        sts_u32(reduced + 4u, 0u);
-        sts_u32(counters, 0u);
-        sts_u32(counters + 4u, 0u);
-        sts_u32(failed, 0u);
-        mbar_init_fence();
-    }
-    __syncthreads();
-    griddep_launch_dependents();
 
     Plan pl;
     pl.init(p, blockIdx.x, G::MAX_ROWS / 8);
@@ -268,7 +257,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // Lane 0 of the calling warp loads stage i (at `st`) into its ring slot.
     auto issue = [&](int i, const Stage& st) {
         if (i == p.skip_stage) return;  // test hook: this stage's barrier never completes
-        const int k = slot_of(i), mi = p.map_of[st.h >> 3];
+        const int k = slot_of(i), mi = map_index(p, st.h);
         const uint32_t dst = slot_addr(k);
         const int y = pl.row0 + st.y;
         sts_u32(last_issued + 4u * (uint32_t)k, phase_of(i) + 1u);
@@ -278,22 +267,39 @@ __global__ void __launch_bounds__(kThreads, 1)
     };
     // The ring's first fill.  The weights are static, so under dependent
     // launch mode 2 these copies (and the optional L2 prefetch of the stages
-    // after them) overlap the previous kernel.
+    // after them) overlap the previous kernel.  Every slot belongs to one
+    // warp (round robin: slots w and w + W; contiguous: the warp's R slots),
+    // so lane j of each warp sets up its j-th slot and loads the warp's j-th
+    // stage into it at once, with no CTA-wide barrier in between; the
+    // barrier after the table build publishes the rest.
     {
-        // lane j issues the warp's j-th stage of the fill
         const int i = ws + lane * stride;
-        if (lane < (rr ? D / kW : G::R) && i < we && i < (rr ? D : we)) {
-            Cur c;
-            c.init(pl, i);
-            issue(i, c.stage(pl));
+        if (lane < (rr ? D / kW : G::R)) {
+            const int k = rr ? warp + kW * lane : warp * G::R + lane;  // = slot_of(i)
+            mbar_init(full_bar(k), 1);
+            sts_u32(last_issued + 4u * (uint32_t)k, 0u);
+            mbar_init_fence();
+            if (i < we && i < (rr ? D : we)) {
+                Cur c;
+                c.init(pl, i);
+                issue(i, c.stage(pl));
+            }
         }
+        if (tid == 0) {
+            sts_u32(reduced, 0u);
+            sts_u32(reduced + 4u, 0u);
+            sts_u32(counters, 0u);
+            sts_u32(counters + 4u, 0u);
+            sts_u32(failed, 0u);
+        }
+        griddep_launch_dependents();
         if (warp == 0 && lane == 0 && p.l2_ahead > 0) {
             const int end = min(pl.n_total, D + p.l2_ahead);
             for (int j = D; j < end; ++j) {
                 Cur c;
                 c.init(pl, j);
                 const Stage sj = c.stage(pl);
-                tma_prefetch_l2_2d(&maps.w[p.map_of[sj.h >> 3]], sj.s * 128, pl.row0 + sj.y);
+                tma_prefetch_l2_2d(&maps.w[map_index(p, sj.h)], sj.s * 128, pl.row0 + sj.y);
             }
         }
     }
@@ -606,12 +612,13 @@ static cudaError_t make_maps(const RowsParams& p, const uint8_t* Wp, const float
 
 // Distinct tile heights of a launch (the device's Plan, replayed for the
 // two group counts a CTA can have), and the map index of each height.
-static int stage_heights(const RowsParams& p, int gmax, int* heights, int* map_of) {
+static int stage_heights(const RowsParams& p, int gmax, int* heights, uint32_t* map_bits) {
     int nh = 0;
+    *map_bits = 0;
     auto add = [&](int h) {
         for (int v = 0; v < nh; ++v)
             if (heights[v] == h) return;
-        map_of[h >> 3] = nh;
+        *map_bits |= (uint32_t)nh << (2 * (h >> 3));
         heights[nh++] = h;
     };
     const int q = p.groups / p.ctas, r = p.groups - q * p.ctas;
@@ -639,7 +646,7 @@ static cudaError_t launch_t(const RowsMaps& m, const RowsParams& p, int smem, cu
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = p.pdl ? 1 : 0;
-    e = cudaLaunchKernelEx(&cfg, kern, m, p);
+    e = cudaLaunchKernelEx(&cfg, kern, p, m);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
@@ -653,9 +660,8 @@ cudaError_t rows_launch(int act_dtype, int m_pad, const RowsParams& p0, const ui
     RowsParams p = p0;
     if (m_pad != 8) p.contig = 0;  // two column tiles: round robin only (the partial tiles fill the parking space)
     int heights[kRowsMaxMaps];
-    for (int& v : p.map_of) v = 0;
     const int max_rows = (m_pad == 8 && !p.contig) ? rows::Geo<1, false>::MAX_ROWS : rows::Geo<1, true>::MAX_ROWS;
-    const int nh = rows::stage_heights(p, max_rows / 8, heights, p.map_of);
+    const int nh = rows::stage_heights(p, max_rows / 8, heights, &p.map_bits);
     rows::RowsMaps m;
     memset(&m, 0, sizeof(m));
     p.n_maps = nh;
