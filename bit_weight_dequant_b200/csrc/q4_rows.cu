@@ -315,9 +315,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     T* out = static_cast<T*>(p.out);
     const T* bias = static_cast<const T*>(p.bias);
 
-    // Activations of this warp's current stage (4 units x NJ column tiles x
-    // two 16-byte runs); refilled unit by unit with the next stage's.
-    uint32_t aw[4][NJ][2][4];
+    // Activations of AU units of this warp's stages (NJ column tiles x two
+    // 16-byte runs each), refilled unit by unit with the unit AU further
+    // on: the whole stage ahead with one column tile; half a stage with two,
+    // whose activation registers would otherwise crowd out the accumulators
+    // (spills).
+    constexpr int AU = NJ == 1 ? 4 : 2;
+    uint32_t aw[AU][NJ][2][4];
     auto load_unit = [&](int kbu, uint32_t(&dst)[NJ][2][4]) {
 #pragma unroll
         for (int jj = 0; jj < NJ; ++jj) {
@@ -503,16 +507,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                     float t[NJ][4];
 #pragma unroll
                     for (int jj = 0; jj < NJ; ++jj)
-                        mma16816<T>(t[jj], q[0][0], q[1][0], q[0][1], q[1][1], aw[j][jj][0][0], aw[j][jj][0][1], zero);
+                        mma16816<T>(t[jj], q[0][0], q[1][0], q[0][1], q[1][1], aw[j % AU][jj][0][0], aw[j % AU][jj][0][1], zero);
 #pragma unroll
                     for (int jj = 0; jj < NJ; ++jj)
-                        mma16816<T>(t[jj], q[0][2], q[1][2], q[0][3], q[1][3], aw[j][jj][0][2], aw[j][jj][0][3], t[jj]);
+                        mma16816<T>(t[jj], q[0][2], q[1][2], q[0][3], q[1][3], aw[j % AU][jj][0][2], aw[j % AU][jj][0][3], t[jj]);
 #pragma unroll
                     for (int jj = 0; jj < NJ; ++jj)
-                        mma16816<T>(t[jj], q[2][0], q[3][0], q[2][1], q[3][1], aw[j][jj][1][0], aw[j][jj][1][1], t[jj]);
+                        mma16816<T>(t[jj], q[2][0], q[3][0], q[2][1], q[3][1], aw[j % AU][jj][1][0], aw[j % AU][jj][1][1], t[jj]);
 #pragma unroll
                     for (int jj = 0; jj < NJ; ++jj)
-                        mma16816<T>(t[jj], q[2][2], q[3][2], q[2][3], q[3][3], aw[j][jj][1][2], aw[j][jj][1][3], t[jj]);
+                        mma16816<T>(t[jj], q[2][2], q[3][2], q[2][3], q[3][3], aw[j % AU][jj][1][2], aw[j % AU][jj][1][3], t[jj]);
 #pragma unroll
                     for (int jj = 0; jj < NJ; ++jj) {
                         acc[ia][jj][0] = fmaf(am[ia][0][j], t[jj][0], acc[ia][jj][0]);
@@ -521,7 +525,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                         acc[ia][jj][3] = fmaf(am[ia][1][j], t[jj][3], acc[ia][jj][3]);
                     }
                 }
-                load_unit(4 * s_nxt + j, aw[j]);  // the next stage's activations (its own again at the end)
+                // The unit AU further on, in this stage or the next (the
+                // warp's own stage again at the end).
+                load_unit(j + AU < 4 ? 4 * s_cur + j + AU : 4 * s_nxt + j + AU - 4, aw[j % AU]);
             }
             // Refill the slot with the warp's stage `ahead` further on: order
             // this warp's reads of the slot before the asynchronous write.
@@ -538,7 +544,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (cc.i < we) {
 #pragma unroll
-        for (int j = 0; j < 4; ++j) load_unit(4 * cc.s + j, aw[j]);
+        for (int j = 0; j < AU; ++j) load_unit(4 * cc.s + j, aw[j]);
         using F = std::false_type;
         using Tr = std::true_type;
         while (cc.i < we) {
