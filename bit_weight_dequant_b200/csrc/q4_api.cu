@@ -220,13 +220,17 @@ static int gemm_choose(int M, int N, int K, int blocksize, int act_dtype, int nu
     const bool tma_ok = c.sub_block == 64 && (K / blocksize) % 4 == 0 && (int64_t)N * (K / 64) > 1;
     int sms_hint = num_sms;
     if (sms_hint <= 0 && device_sm_count(&sms_hint) != 0) sms_hint = 148;  // the choice only; the launch re-queries
-    c.loader = mma32 ? 3 : !tma_ok ? 1 : rows_kernel_pays(M, N, K, sms_hint) ? 7 : 2;
+    // The row-split kernel also takes blocksize 32 (two absmax per 64-k unit,
+    // an 8-float box per stage): K a multiple of its 256-k stage.
+    const bool rows_ok = tma_ok || (blocksize == 32 && K % 256 == 0 && (int64_t)N * (K / 64) > 1);
+    c.loader = mma32 ? 3 : (rows_ok && rows_kernel_pays(M, N, K, sms_hint)) ? 7 : !tma_ok ? 1 : 2;
     if (ov && ov->loader > 0) c.loader = ov->loader;
-    if (c.loader >= 2 && !tma_ok) return Q4_ERR_UNSUPPORTED;
+    if (c.loader == 7 ? !rows_ok : (c.loader >= 2 && !tma_ok)) return Q4_ERR_UNSUPPORTED;
     if (c.loader == 7) {
         // Row-split kernel: 8-row groups of W split over the CTAs, one shared
         // stage ring per CTA, no cross-CTA combine (workspace: the error word).
         if (M > 16) return Q4_ERR_UNSUPPORTED;
+        c.sub_block = 64;  // 64-k units at every blocksize (two absmax per unit at blocksize 32)
         c.warps = rows_warps();
         c.depth = (ov && ov->depth > 0) ? ov->depth : 1;  // stage order: 1 round robin, 2 contiguous per warp
         if (c.depth > 2) return Q4_ERR_UNSUPPORTED;

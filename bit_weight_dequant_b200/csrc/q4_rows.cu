@@ -57,24 +57,32 @@ constexpr int kW = 8;                // warps per CTA
 constexpr int kThreads = kW * 32;
 constexpr uint32_t kBarBytes = 512;  // mbarriers and small words at the start of the window
 
-// Compile-time shape of the kernel for NJ n8 column tiles (M <= 8 or 16)
-// and stage order (CONTIG: each warp streams a contiguous range of stages;
-// else round robin).
-template <int NJ, bool CONTIG>
+// Absmax granularity of a kernel instance: one block per stage or more
+// (blocksize >= 128), one per 64-k unit (blocksize 64), two per unit
+// (blocksize 32).
+enum : int { kAmShared = 0, kAm64 = 1, kAm32 = 2 };
+
+// Compile-time shape of the kernel for NJ n8 column tiles (M <= 8 or 16),
+// stage order (CONTIG: each warp streams a contiguous range of stages;
+// else round robin) and absmax granularity AMK.
+template <int NJ, bool CONTIG, int AMK>
 struct Geo {
     // Tallest tile.  Round robin with one column tile: 72 rows (a CTA of
     // 8q + 1 groups then needs no short tiles).  Contiguous ranges keep
     // several tiles open at once and need two parking buffers: 64 rows.
-    static constexpr int MAX_ROWS = (NJ == 1 && !CONTIG) ? 72 : 64;
+    // Blocksize 32 doubles the absmax box: 56 rows keep 16 slots in the
+    // window.
+    static constexpr int MAX_ROWS = AMK == kAm32 ? 56 : (NJ == 1 && !CONTIG) ? 72 : 64;
     static constexpr int MT_MAX = (MAX_ROWS + 15) / 16;       // 16-row MMA tiles per stage, at most
+    static constexpr uint32_t AMW = AMK == kAm32 ? 32u : 16u; // absmax bytes per row and stage (8 or 4 floats)
     static constexpr uint32_t CODE_BYTES = MAX_ROWS * 128u;   // a stage's codes: rows x 128 B (4 units of 64 k)
-    static constexpr uint32_t AM_BYTES = MAX_ROWS * 16u;      // its absmax box: rows x 4 floats
+    static constexpr uint32_t AM_BYTES = MAX_ROWS * AMW;      // its absmax box
     // With 72-row tiles the codes (9 KiB, 1 KiB aligned for the swizzle) and
     // the absmax boxes live in separate rings, and the barriers in spare
-    // table rows; otherwise a slot holds both (9 KiB) and the barriers sit
-    // at the start of the window.
+    // table rows; otherwise a slot holds both (padded to 1 KiB: 9 KiB) and
+    // the barriers sit at the start of the window.
     static constexpr bool SPLIT = MAX_ROWS == 72;
-    static constexpr uint32_t SLOT = CODE_BYTES + AM_BYTES;
+    static constexpr uint32_t SLOT = (CODE_BYTES + AM_BYTES + 1023u) & ~1023u;
     static constexpr int REGS = MT_MAX * 4 * NJ;              // a warp's partial tile: registers per lane
     // Ring depth: a compile-time constant, so that slot and phase of a stage
     // are a mask and a shift.
@@ -166,10 +174,10 @@ struct RowsMaps {
     CUtensorMap a[kRowsMaxMaps];
 };
 
-template <typename T, int NJ, bool BS64, bool CONTIG>
+template <typename T, int NJ, int AMK, bool CONTIG>
 __global__ void __launch_bounds__(kThreads, 1)
     q4_gemm_rows_kernel(const __grid_constant__ RowsParams p, const __grid_constant__ RowsMaps maps) {
-    using G = Geo<NJ, CONTIG>;
+    using G = Geo<NJ, CONTIG, AMK>;
     constexpr int D = G::D, MTM = G::MT_MAX, NB = G::NB;
     extern __shared__ __align__(16) uint8_t smem_rows[];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, tq = lane & 3;
@@ -261,9 +269,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t dst = slot_addr(k);
         const int y = pl.row0 + st.y;
         sts_u32(last_issued + 4u * (uint32_t)k, phase_of(i) + 1u);
-        mbar_expect_tx(full_bar(k), (uint32_t)st.h * 144u);
+        mbar_expect_tx(full_bar(k), (uint32_t)st.h * (128u + G::AMW));
         tma_load_2d_hint(dst, &maps.w[mi], st.s * 128, y, full_bar(k), once);
-        tma_load_2d(am_addr(k), &maps.a[mi], ((st.s * 4) >> p.am_shift) & ~3, y, full_bar(k));
+        tma_load_2d(am_addr(k), &maps.a[mi], AMK == kAm32 ? st.s * 8 : ((st.s * 4) >> p.am_shift) & ~3, y,
+                    full_bar(k));
     };
     // The ring's first fill.  The weights are static, so under dependent
     // launch mode 2 these copies (and the optional L2 prefetch of the stages
@@ -317,10 +326,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     // Activations of AU units of this warp's stages (NJ column tiles x two
     // 16-byte runs each), refilled unit by unit with the unit AU further
-    // on: the whole stage ahead with one column tile; half a stage with two,
-    // whose activation registers would otherwise crowd out the accumulators
-    // (spills).
-    constexpr int AU = NJ == 1 ? 4 : 2;
+    // on: the whole stage ahead with one column tile; half a stage with two
+    // (or at blocksize 32), whose registers would otherwise crowd out the
+    // accumulators (spills).
+    constexpr int AU = (NJ == 1 && AMK != kAm32) ? 4 : 2;
     uint32_t aw[AU][NJ][2][4];
     auto load_unit = [&](int kbu, uint32_t(&dst)[NJ][2][4]) {
 #pragma unroll
@@ -459,19 +468,21 @@ __global__ void __launch_bounds__(kThreads, 1)
             const bool more = cc.i < we;
             const int s_nxt = more ? cc.s : s_cur;
             const uint32_t am_st = am_addr(k);
-            const int x0 = ((s_cur * 4) >> p.am_shift) & ~3;
-            float am[MT][2][4];  // absmax of rows 16 ia + g (+ 8 hh), for the stage's 4 units
+            [[maybe_unused]] float am[MT][2][4];  // absmax of rows 16 ia + g (+ 8 hh), the stage's 4 units (unused at blocksize 32)
 #pragma unroll
             for (int ia = 0; ia < MT; ++ia)
 #pragma unroll
                 for (int hh = 0; hh < 2; ++hh) {
-                    if (BS64) {
+                    if constexpr (AMK == kAm32) {
+                        // two per unit: loaded unit by unit below
+                    } else if constexpr (AMK == kAm64) {
                         const uint4 v = lds_v4(am_st + (uint32_t)(16 * ia + 8 * hh + g) * 16u);
                         am[ia][hh][0] = __uint_as_float(v.x);
                         am[ia][hh][1] = __uint_as_float(v.y);
                         am[ia][hh][2] = __uint_as_float(v.z);
                         am[ia][hh][3] = __uint_as_float(v.w);
                     } else {
+                        const int x0 = ((s_cur * 4) >> p.am_shift) & ~3;
 #pragma unroll
                         for (int j = 0; j < 4; ++j) {
                             const int col = ((s_cur * 4 + j) >> p.am_shift) - x0;
@@ -504,25 +515,65 @@ __global__ void __launch_bounds__(kThreads, 1)
                             q[x][3] = lut_pair<3>(d[x], lane4);
                         }
                     }
-                    float t[NJ][4];
+                    if constexpr (AMK == kAm32) {
+                        // Blocksize 32: the first two MMAs cover k 0..31 of the
+                        // unit, the last two k 32..63; each half is scaled by
+                        // its own block's absmax.
+                        float2 a2[2];
 #pragma unroll
-                    for (int jj = 0; jj < NJ; ++jj)
-                        mma16816<T>(t[jj], q[0][0], q[1][0], q[0][1], q[1][1], aw[j % AU][jj][0][0], aw[j % AU][jj][0][1], zero);
+                        for (int hh = 0; hh < 2; ++hh)
+                            a2[hh] = lds_f32x2(am_st + (uint32_t)(16 * ia + 8 * hh + g) * G::AMW + (uint32_t)j * 8u);
+                        float tl[NJ][4], th[NJ][4];
 #pragma unroll
-                    for (int jj = 0; jj < NJ; ++jj)
-                        mma16816<T>(t[jj], q[0][2], q[1][2], q[0][3], q[1][3], aw[j % AU][jj][0][2], aw[j % AU][jj][0][3], t[jj]);
+                        for (int jj = 0; jj < NJ; ++jj) {
+                            mma16816<T>(tl[jj], q[0][0], q[1][0], q[0][1], q[1][1], aw[j % AU][jj][0][0],
+                                        aw[j % AU][jj][0][1], zero);
+                            mma16816<T>(th[jj], q[2][0], q[3][0], q[2][1], q[3][1], aw[j % AU][jj][1][0],
+                                        aw[j % AU][jj][1][1], zero);
+                        }
 #pragma unroll
-                    for (int jj = 0; jj < NJ; ++jj)
-                        mma16816<T>(t[jj], q[2][0], q[3][0], q[2][1], q[3][1], aw[j % AU][jj][1][0], aw[j % AU][jj][1][1], t[jj]);
+                        for (int jj = 0; jj < NJ; ++jj) {
+                            mma16816<T>(tl[jj], q[0][2], q[1][2], q[0][3], q[1][3], aw[j % AU][jj][0][2],
+                                        aw[j % AU][jj][0][3], tl[jj]);
+                            mma16816<T>(th[jj], q[2][2], q[3][2], q[2][3], q[3][3], aw[j % AU][jj][1][2],
+                                        aw[j % AU][jj][1][3], th[jj]);
+                        }
 #pragma unroll
-                    for (int jj = 0; jj < NJ; ++jj)
-                        mma16816<T>(t[jj], q[2][2], q[3][2], q[2][3], q[3][3], aw[j % AU][jj][1][2], aw[j % AU][jj][1][3], t[jj]);
+                        for (int jj = 0; jj < NJ; ++jj) {
+                            acc[ia][jj][0] = fmaf(a2[0].x, tl[jj][0], acc[ia][jj][0]);
+                            acc[ia][jj][1] = fmaf(a2[0].x, tl[jj][1], acc[ia][jj][1]);
+                            acc[ia][jj][2] = fmaf(a2[1].x, tl[jj][2], acc[ia][jj][2]);
+                            acc[ia][jj][3] = fmaf(a2[1].x, tl[jj][3], acc[ia][jj][3]);
+                            acc[ia][jj][0] = fmaf(a2[0].y, th[jj][0], acc[ia][jj][0]);
+                            acc[ia][jj][1] = fmaf(a2[0].y, th[jj][1], acc[ia][jj][1]);
+                            acc[ia][jj][2] = fmaf(a2[1].y, th[jj][2], acc[ia][jj][2]);
+                            acc[ia][jj][3] = fmaf(a2[1].y, th[jj][3], acc[ia][jj][3]);
+                        }
+                    } else {
+                        float t[NJ][4];
 #pragma unroll
-                    for (int jj = 0; jj < NJ; ++jj) {
-                        acc[ia][jj][0] = fmaf(am[ia][0][j], t[jj][0], acc[ia][jj][0]);
-                        acc[ia][jj][1] = fmaf(am[ia][0][j], t[jj][1], acc[ia][jj][1]);
-                        acc[ia][jj][2] = fmaf(am[ia][1][j], t[jj][2], acc[ia][jj][2]);
-                        acc[ia][jj][3] = fmaf(am[ia][1][j], t[jj][3], acc[ia][jj][3]);
+                        for (int jj = 0; jj < NJ; ++jj)
+                            mma16816<T>(t[jj], q[0][0], q[1][0], q[0][1], q[1][1], aw[j % AU][jj][0][0],
+                                        aw[j % AU][jj][0][1], zero);
+#pragma unroll
+                        for (int jj = 0; jj < NJ; ++jj)
+                            mma16816<T>(t[jj], q[0][2], q[1][2], q[0][3], q[1][3], aw[j % AU][jj][0][2],
+                                        aw[j % AU][jj][0][3], t[jj]);
+#pragma unroll
+                        for (int jj = 0; jj < NJ; ++jj)
+                            mma16816<T>(t[jj], q[2][0], q[3][0], q[2][1], q[3][1], aw[j % AU][jj][1][0],
+                                        aw[j % AU][jj][1][1], t[jj]);
+#pragma unroll
+                        for (int jj = 0; jj < NJ; ++jj)
+                            mma16816<T>(t[jj], q[2][2], q[3][2], q[2][3], q[3][3], aw[j % AU][jj][1][2],
+                                        aw[j % AU][jj][1][3], t[jj]);
+#pragma unroll
+                        for (int jj = 0; jj < NJ; ++jj) {
+                            acc[ia][jj][0] = fmaf(am[ia][0][j], t[jj][0], acc[ia][jj][0]);
+                            acc[ia][jj][1] = fmaf(am[ia][0][j], t[jj][1], acc[ia][jj][1]);
+                            acc[ia][jj][2] = fmaf(am[ia][1][j], t[jj][2], acc[ia][jj][2]);
+                            acc[ia][jj][3] = fmaf(am[ia][1][j], t[jj][3], acc[ia][jj][3]);
+                        }
                     }
                 }
                 // The unit AU further on, in this stage or the next (the
@@ -589,9 +640,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // Weights [N rows][K/2 bytes]: boxes of h rows x 128 bytes, 128-byte
-// swizzle.  Absmax [N rows][K/bs floats]: boxes of h rows x 4 floats.  One
-// pair per distinct tile height of the launch (heights[] in rows).
-static cudaError_t make_maps(const RowsParams& p, const uint8_t* Wp, const float* absmax, int am_per_row,
+// swizzle.  Absmax [N rows][K/bs floats]: boxes of h rows x `am_box` floats
+// (4; 8 at blocksize 32).  One pair per distinct tile height of the launch
+// (heights[] in rows).
+static cudaError_t make_maps(const RowsParams& p, const uint8_t* Wp, const float* absmax, int am_per_row, int am_box,
                              const int* heights, int nh, RowsMaps* m) {
     auto enc = tensor_map_encoder();
     if (!enc) return cudaErrorNotSupported;
@@ -607,7 +659,7 @@ static cudaError_t make_maps(const RowsParams& p, const uint8_t* Wp, const float
                 CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return cudaErrorInvalidValue;
-        const cuuint32_t abox[2] = {4, rows};
+        const cuuint32_t abox[2] = {(cuuint32_t)am_box, rows};
         if (enc(&m->a[v], CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(absmax), adim, astr, abox, es,
                 CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
@@ -637,9 +689,9 @@ static int stage_heights(const RowsParams& p, int gmax, int* heights, uint32_t* 
     return nh;
 }
 
-template <typename T, int NJ, bool BS64, bool CONTIG>
+template <typename T, int NJ, int AMK, bool CONTIG>
 static cudaError_t launch_t(const RowsMaps& m, const RowsParams& p, int smem, cudaStream_t stream) {
-    auto kern = q4_gemm_rows_kernel<T, NJ, BS64, CONTIG>;
+    auto kern = q4_gemm_rows_kernel<T, NJ, AMK, CONTIG>;
     cudaError_t e = ensure_smem_attr((const void*)kern, (size_t)smem);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
@@ -661,38 +713,48 @@ static cudaError_t launch_t(const RowsMaps& m, const RowsParams& p, int smem, cu
 
 int rows_warps() { return rows::kW; }
 
+// The kernel instance for an activation type and absmax granularity:
+// one column tile (round robin or contiguous ranges) or two.
+template <typename T, int AMK>
+static cudaError_t launch_for(int m_pad, const rows::RowsMaps& m, const RowsParams& p, int smem, cudaStream_t stream) {
+    using namespace rows;
+    if (m_pad != 8) return launch_t<T, 2, AMK, false>(m, p, smem, stream);
+    if constexpr (AMK != kAm32) {
+        if (p.contig) return launch_t<T, 1, AMK, true>(m, p, smem, stream);
+    }
+    return launch_t<T, 1, AMK, false>(m, p, smem, stream);
+}
+
+template <typename T>
+static cudaError_t launch_am(int amk, int m_pad, const rows::RowsMaps& m, const RowsParams& p, int smem,
+                             cudaStream_t stream) {
+    using namespace rows;
+    if (amk == kAm32) return launch_for<T, kAm32>(m_pad, m, p, smem, stream);
+    if (amk == kAm64) return launch_for<T, kAm64>(m_pad, m, p, smem, stream);
+    return launch_for<T, kAmShared>(m_pad, m, p, smem, stream);
+}
+
 cudaError_t rows_launch(int act_dtype, int m_pad, const RowsParams& p0, const uint8_t* Wp, const float* absmax,
                         int am_per_row, int smem, cudaStream_t stream) {
+    using namespace rows;
     RowsParams p = p0;
-    if (m_pad != 8) p.contig = 0;  // two column tiles: round robin only (the partial tiles fill the parking space)
+    // blocksize = K / am_per_row: 32, 64, or larger (am_shift = log2(bs / 64))
+    const int amk = (int64_t)am_per_row * 32 == p.K ? kAm32 : p.am_shift == 0 ? kAm64 : kAmShared;
+    // Two column tiles or blocksize 32: round robin only (the partial tiles
+    // fill the parking space; blocksize 32 has no contiguous instance).
+    if (m_pad != 8 || amk == kAm32) p.contig = 0;
     int heights[kRowsMaxMaps];
-    const int max_rows = (m_pad == 8 && !p.contig) ? rows::Geo<1, false>::MAX_ROWS : rows::Geo<1, true>::MAX_ROWS;
-    const int nh = rows::stage_heights(p, max_rows / 8, heights, &p.map_bits);
-    rows::RowsMaps m;
+    const int max_rows = amk == kAm32 ? Geo<1, false, kAm32>::MAX_ROWS
+                         : (m_pad == 8 && !p.contig) ? Geo<1, false, kAm64>::MAX_ROWS
+                                                     : Geo<1, true, kAm64>::MAX_ROWS;
+    const int nh = stage_heights(p, max_rows / 8, heights, &p.map_bits);
+    RowsMaps m;
     memset(&m, 0, sizeof(m));
     p.n_maps = nh;
-    cudaError_t e = rows::make_maps(p, Wp, absmax, am_per_row, heights, nh, &m);
+    cudaError_t e = make_maps(p, Wp, absmax, am_per_row, amk == kAm32 ? 8 : 4, heights, nh, &m);
     if (e != cudaSuccess) return e;
-    const bool bs64 = p.am_shift == 0;
-    using namespace rows;
-    if (act_dtype == 0) {
-        if (m_pad == 8) {
-            if (p.contig)
-                return bs64 ? launch_t<__nv_bfloat16, 1, true, true>(m, p, smem, stream)
-                            : launch_t<__nv_bfloat16, 1, false, true>(m, p, smem, stream);
-            return bs64 ? launch_t<__nv_bfloat16, 1, true, false>(m, p, smem, stream)
-                        : launch_t<__nv_bfloat16, 1, false, false>(m, p, smem, stream);
-        }
-        return bs64 ? launch_t<__nv_bfloat16, 2, true, false>(m, p, smem, stream)
-                    : launch_t<__nv_bfloat16, 2, false, false>(m, p, smem, stream);
-    }
-    if (m_pad == 8) {
-        if (p.contig)
-            return bs64 ? launch_t<__half, 1, true, true>(m, p, smem, stream)
-                        : launch_t<__half, 1, false, true>(m, p, smem, stream);
-        return bs64 ? launch_t<__half, 1, true, false>(m, p, smem, stream) : launch_t<__half, 1, false, false>(m, p, smem, stream);
-    }
-    return bs64 ? launch_t<__half, 2, true, false>(m, p, smem, stream) : launch_t<__half, 2, false, false>(m, p, smem, stream);
+    return act_dtype == 0 ? launch_am<__nv_bfloat16>(amk, m_pad, m, p, smem, stream)
+                          : launch_am<__half>(amk, m_pad, m, p, smem, stream);
 }
 
 }  // namespace q4

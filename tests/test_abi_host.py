@@ -91,9 +91,11 @@ def test_gemm_validation_before_cuda():
     assert ex(*args, 12, 64, 4096, 64, 0, ALIGNED, None, 0, None, b.overrides(warps=16)) == b.Q4_ERR_UNSUPPORTED
     assert ex(*args, 1, 64, 4096, 64, 0, ALIGNED, None, 0, None, b.overrides(depth=7, loader=2)) == b.Q4_ERR_UNSUPPORTED
     assert ex(*args, 12, 64, 4096, 64, 0, ALIGNED, None, 0, None, b.overrides(loader=8)) == b.Q4_ERR_INVALID_ARG
-    # the row-split kernel (loader 7): M <= 16, 64-k units, its own warp count
+    # the row-split kernel (loader 7): M <= 16, 64-k units (blocksize 32 only with K % 256 == 0), its own
+    # warp count
     assert ex(*args, 20, 64, 4096, 64, 0, ALIGNED, None, 0, None, b.overrides(loader=7)) == b.Q4_ERR_UNSUPPORTED
-    assert ex(*args, 4, 64, 4096, 32, 0, ALIGNED, None, 0, None, b.overrides(loader=7)) == b.Q4_ERR_UNSUPPORTED
+    assert ex(*args, 4, 64, 4160, 32, 0, ALIGNED, None, 0, None, b.overrides(loader=7)) == b.Q4_ERR_UNSUPPORTED
+    assert ex(*args, 4, 64, 4096, 32, 0, ALIGNED, None, 0, None, b.overrides(loader=7, depth=3)) == b.Q4_ERR_UNSUPPORTED
     assert ex(*args, 4, 64, 4096, 64, 0, ALIGNED, None, 0, None, b.overrides(loader=7, warps=9)) == b.Q4_ERR_UNSUPPORTED
     # the CUDA-core kernel takes 16-bit activations on request, M <= 16
     assert ex(*args, 17, 64, 4096, 64, 0, ALIGNED, None, 0, None, b.overrides(math=2)) == b.Q4_ERR_UNSUPPORTED
@@ -185,17 +187,19 @@ def test_launch_table_invariants(wl):
             continue  # tensor-memory and fp32 tables: test_launch_table_tcgen05, test_launch_table_f32
         p = b.q4_gemm_plan(c.M, c.N, c.K, c.blocksize, num_sms=148)
         assert p["math"] == 1
-        assert p["sub_block"] == min(c.blocksize, 64)
         assert p["m_pad"] == (8 if c.M <= 8 else 16)
         assert p["tiles"] == -(-c.N // p["rows_per_tile"])
         assert p["units"] == p["tiles"] * (c.K // p["sub_block"])
         assert 1 <= p["ctas"] <= min(148, p["units"])
         assert p["smem_bytes"] <= 227 * 1024
-        tma_ok = c.blocksize >= 64 and (c.K // c.blocksize) % 4 == 0 and p["units"] > 1
+        tma_ok = c.blocksize >= 64 and (c.K // c.blocksize) % 4 == 0 and c.N * (c.K // 64) > 1
+        # the row-split kernel also takes blocksize 32 when K is a multiple of its 256-k stage
+        rows_ok = tma_ok or (c.blocksize == 32 and c.K % 256 == 0 and c.N * (c.K // 64) > 1)
         tiles, weights = -(-c.N // 64), c.N * c.K
-        rows = not (c.K < 4096 and tiles > 4 * 148) and not (c.M >= 8 and weights >= 2**26)
-        assert p["loader"] == ((7 if rows else 2) if tma_ok else 1), (wl, c)
-        if tma_ok and rows:
+        rows = rows_ok and not (c.K < 4096 and tiles > 4 * 148) and not (c.M >= 8 and weights >= 2**26)
+        assert p["loader"] == (7 if rows else 2 if tma_ok else 1), (wl, c)
+        assert p["sub_block"] == (64 if rows else min(c.blocksize, 64))
+        if rows:
             # row-split kernel: 8-row groups over at most one CTA per SM, the
             # workspace is the 256-byte error header alone
             assert p["ctas"] == min(148, -(-c.N // 8)) and p["warps"] == 8 and p["rows_per_tile"] == 64

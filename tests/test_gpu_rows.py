@@ -1,13 +1,14 @@
 """GPU parity of the row-split fused kernel (launch-table loader 7, the
 default for M <= 16 with 16-bit activations when blocksize >= 64 and
-(K / blocksize) % 4 == 0) against the oracle: every output element within
+(K / blocksize) % 4 == 0, or blocksize 32 and K % 256 == 0) against the
+oracle: every output element within
 |gpu - y| <= 1e-2 * sum_k |a w| + ulp(y).
 
 The kernel splits 8-row groups of W over the CTAs and finishes every output
 inside one CTA; the cases below cover the shapes of that split (one CTA,
 CTAs with one group, ragged last groups past N, groups that leave partial
 64-row tiles), tiles of every height up to 72 rows, the L2 prefetch ahead of the stage
-ring, every blocksize the tensor maps take, fp16,
+ring, every blocksize from 32 to 4096, fp16,
 the code tables, the bias epilogue, dependent-launch chains, determinism,
 and a bounded wait that is made to run out.  The operation is the fused path
 of bitsandbytes PR #1920 ("Fused path support for M > 1")."""
@@ -82,10 +83,27 @@ def test_rows_l2_prefetch(cuda_device, ahead):
 
 
 @pytest.mark.parametrize("M", [1, 6, 16])
-@pytest.mark.parametrize("bs,K", [(64, 1280), (128, 1536), (256, 4096), (512, 2048), (1024, 8192), (4096, 16384)])
+@pytest.mark.parametrize("bs,K", [(32, 1280), (32, 4096), (64, 1280), (128, 1536), (256, 4096), (512, 2048),
+                                  (1024, 8192), (4096, 16384)])
 def test_rows_blocksizes(cuda_device, M, bs, K):
     run_case(Case(M, 333, K, blocksize=bs), seed=11400 + bs + M, device=cuda_device, check_quantizer=False,
              loader=7)
+
+
+@pytest.mark.parametrize("M", [1, 9])
+@pytest.mark.parametrize("ctas,depth", [(1, 0), (3, 0), (37, 2), (148, 0)])
+@pytest.mark.parametrize("N", [300, 1003])
+def test_rows_blocksize32(cuda_device, M, ctas, depth, N):
+    """Blocksize 32: two absmax per 64-k unit (8-float boxes per stage, tiles
+    of at most 56 rows), each half of the unit's MMAs scaled by its own
+    block; a request for contiguous ranges falls back to round robin."""
+    if ctas > (N + 7) // 8:
+        pytest.skip("more CTAs than 8-row groups")
+    kw = {"ctas": ctas}
+    if depth:
+        kw["depth"] = depth
+    run_case(Case(M, N, 2560, blocksize=32, outliers=(N == 1003)), seed=11450 + M + ctas + N, device=cuda_device,
+             check_quantizer=False, loader=7, **kw)
 
 
 @pytest.mark.parametrize("M", [1, 4, 11])
