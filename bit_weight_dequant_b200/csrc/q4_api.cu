@@ -180,6 +180,7 @@ static int gemm_choose(int M, int N, int K, int blocksize, int act_dtype, int nu
         // Tensor-memory kernel (tcgen05): 128-row tiles, 64-k units, 4-unit
         // stages whose absmax box is 4 floats per row.
         if (blocksize < 64 || K % 256 != 0 || (K / blocksize) % 4 != 0) return Q4_ERR_UNSUPPORTED;
+        if (ov && ov->loader > 0 && ov->loader != 6) return Q4_ERR_UNSUPPORTED;  // another kernel's loader
         c.math = 3;
         c.sub_block = 64;
         c.m_pad = M <= 32 ? 32 : M <= 64 ? 64 : 128;
@@ -229,8 +230,9 @@ static int gemm_choose(int M, int N, int K, int blocksize, int act_dtype, int nu
     if (c.loader == 7) {
         // Row-split kernel: 8-row groups of W split over the CTAs, one shared
         // stage ring per CTA, no cross-CTA combine (workspace: the error word).
-        if (M > 16) return Q4_ERR_UNSUPPORTED;
+        if (M > 32 || (M > 16 && !tma_ok)) return Q4_ERR_UNSUPPORTED;
         c.sub_block = 64;  // 64-k units at every blocksize (two absmax per unit at blocksize 32)
+        c.rows_per_tile = 64;
         c.warps = rows_warps();
         c.depth = (ov && ov->depth > 0) ? ov->depth : 1;  // stage order: 1 round robin, 2 contiguous per warp
         if (c.depth > 2) return Q4_ERR_UNSUPPORTED;

@@ -1134,10 +1134,10 @@ static const Variant* find_variant(int act, const GemmChoice& ch) {
 }
 
 // Loader 7 is the row-split kernel (q4_rows.cu): bf16/fp16, 64-k units,
-// one or two n8 column tiles, the stage ring sized from shared memory.
+// one, two or four n8 column tiles, the stage ring sized from shared memory.
 static bool rows_variant(int act_dtype, const GemmChoice& ch) {
     return ch.loader == 7 && (act_dtype == 0 || act_dtype == 1) && ch.sub_block == 64 &&
-           (ch.m_pad == 8 || ch.m_pad == 16) && ch.warps == rows_warps();
+           (ch.m_pad == 8 || ch.m_pad == 16 || ch.m_pad == 32) && ch.warps == rows_warps();
 }
 
 bool gemm_variant_exists(int act_dtype, const GemmChoice& ch) {

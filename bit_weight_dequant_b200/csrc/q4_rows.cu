@@ -71,8 +71,9 @@ struct Geo {
     // 8q + 1 groups then needs no short tiles).  Contiguous ranges keep
     // several tiles open at once and need two parking buffers: 64 rows.
     // Blocksize 32 doubles the absmax box: 56 rows keep 16 slots in the
-    // window.
-    static constexpr int MAX_ROWS = AMK == kAm32 ? 56 : (NJ == 1 && !CONTIG) ? 72 : 64;
+    // window.  Four column tiles (17 <= M <= 32): 32 rows, so that the
+    // partial tiles (32 registers a warp) still fit the parking space.
+    static constexpr int MAX_ROWS = NJ == 4 ? 32 : AMK == kAm32 ? 56 : (NJ == 1 && !CONTIG) ? 72 : 64;
     static constexpr int MT_MAX = (MAX_ROWS + 15) / 16;       // 16-row MMA tiles per stage, at most
     static constexpr uint32_t AMW = AMK == kAm32 ? 32u : 16u; // absmax bytes per row and stage (8 or 4 floats)
     static constexpr uint32_t CODE_BYTES = MAX_ROWS * 128u;   // a stage's codes: rows x 128 B (4 units of 64 k)
@@ -718,6 +719,10 @@ int rows_warps() { return rows::kW; }
 template <typename T, int AMK>
 static cudaError_t launch_for(int m_pad, const rows::RowsMaps& m, const RowsParams& p, int smem, cudaStream_t stream) {
     using namespace rows;
+    if (m_pad == 32) {
+        if constexpr (AMK != kAm32) return launch_t<T, 4, AMK, false>(m, p, smem, stream);
+        return cudaErrorInvalidValue;  // M > 16 needs blocksize >= 64
+    }
     if (m_pad != 8) return launch_t<T, 2, AMK, false>(m, p, smem, stream);
     if constexpr (AMK != kAm32) {
         if (p.contig) return launch_t<T, 1, AMK, true>(m, p, smem, stream);
@@ -740,11 +745,13 @@ cudaError_t rows_launch(int act_dtype, int m_pad, const RowsParams& p0, const ui
     RowsParams p = p0;
     // blocksize = K / am_per_row: 32, 64, or larger (am_shift = log2(bs / 64))
     const int amk = (int64_t)am_per_row * 32 == p.K ? kAm32 : p.am_shift == 0 ? kAm64 : kAmShared;
-    // Two column tiles or blocksize 32: round robin only (the partial tiles
-    // fill the parking space; blocksize 32 has no contiguous instance).
+    // Two or four column tiles or blocksize 32: round robin only (the
+    // partial tiles fill the parking space; blocksize 32 has no contiguous
+    // instance).
     if (m_pad != 8 || amk == kAm32) p.contig = 0;
     int heights[kRowsMaxMaps];
-    const int max_rows = amk == kAm32 ? Geo<1, false, kAm32>::MAX_ROWS
+    const int max_rows = m_pad == 32     ? Geo<4, false, kAm64>::MAX_ROWS
+                         : amk == kAm32 ? Geo<1, false, kAm32>::MAX_ROWS
                          : (m_pad == 8 && !p.contig) ? Geo<1, false, kAm64>::MAX_ROWS
                                                      : Geo<1, true, kAm64>::MAX_ROWS;
     const int nh = stage_heights(p, max_rows / 8, heights, &p.map_bits);

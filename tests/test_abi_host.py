@@ -91,9 +91,10 @@ def test_gemm_validation_before_cuda():
     assert ex(*args, 12, 64, 4096, 64, 0, ALIGNED, None, 0, None, b.overrides(warps=16)) == b.Q4_ERR_UNSUPPORTED
     assert ex(*args, 1, 64, 4096, 64, 0, ALIGNED, None, 0, None, b.overrides(depth=7, loader=2)) == b.Q4_ERR_UNSUPPORTED
     assert ex(*args, 12, 64, 4096, 64, 0, ALIGNED, None, 0, None, b.overrides(loader=8)) == b.Q4_ERR_INVALID_ARG
-    # the row-split kernel (loader 7): M <= 16, 64-k units (blocksize 32 only with K % 256 == 0), its own
-    # warp count
-    assert ex(*args, 20, 64, 4096, 64, 0, ALIGNED, None, 0, None, b.overrides(loader=7)) == b.Q4_ERR_UNSUPPORTED
+    # the row-split kernel (loader 7): M <= 32 (blocksize >= 64 past 16), 64-k units (blocksize 32 only with
+    # K % 256 == 0), its own warp count
+    assert ex(*args, 33, 64, 4096, 64, 0, ALIGNED, None, 0, None, b.overrides(loader=7)) == b.Q4_ERR_UNSUPPORTED
+    assert ex(*args, 20, 64, 4096, 32, 0, ALIGNED, None, 0, None, b.overrides(loader=7)) == b.Q4_ERR_UNSUPPORTED
     assert ex(*args, 4, 64, 4160, 32, 0, ALIGNED, None, 0, None, b.overrides(loader=7)) == b.Q4_ERR_UNSUPPORTED
     assert ex(*args, 4, 64, 4096, 32, 0, ALIGNED, None, 0, None, b.overrides(loader=7, depth=3)) == b.Q4_ERR_UNSUPPORTED
     assert ex(*args, 4, 64, 4096, 64, 0, ALIGNED, None, 0, None, b.overrides(loader=7, warps=9)) == b.Q4_ERR_UNSUPPORTED

@@ -210,3 +210,23 @@ def test_rows_bounded_wait_runs_out(cuda_device, monkeypatch, skip):
     assert q4.workspace_error(ws) == 0
     y, S = oracle.gemm(bits_of(A), oracle.BF16, packed, absmax, code, M, N, K, 64)
     check_gemm(bits_of(out), y, S, "bf16", "after the time-out")
+
+
+@pytest.mark.parametrize("M", [17, 24, 32])
+@pytest.mark.parametrize("N,K,act", [(300, 1024, "bf16"), (1000, 2560, "fp16"), (77, 4096, "bf16"), (4100, 768, "bf16")])
+def test_rows_four_column_tiles(cuda_device, M, N, K, act):
+    """17 <= M <= 32 on the row-split kernel (four n8 column tiles, tiles of
+    at most 32 rows, half a stage of activations in flight)."""
+    run_case(Case(M, N, K, act=act), seed=12200 + M + N, device=cuda_device, check_quantizer=False, loader=7)
+
+
+def test_rows_four_column_tiles_bias_and_partitions(cuda_device):
+    M, N, K = 29, 1500, 2048
+    P, Am, C, packed, absmax, code = _layer(cuda_device, N, K, 12300)
+    A = inputs.activations(M, K, torch.bfloat16, 12301)
+    bias = inputs.activations(1, N, torch.bfloat16, 12302).reshape(N)
+    y, S = oracle.gemm(bits_of(A), oracle.BF16, packed, absmax, code, M, N, K, 64, bias_bits=bits_of(bias))
+    for ctas in (1, 7, 148):
+        out = q4.q4_gemm_skinny(A.to(cuda_device), P, Am, C, N, K, 64, bias=bias.to(cuda_device), loader=7, ctas=ctas)
+        torch.cuda.synchronize()
+        check_gemm(bits_of(out), y, S, "bf16", f"rows M29 bias ctas {ctas}")
