@@ -65,17 +65,21 @@ extern "C" int q4_gemm_skinny_noalloc(const void* A, const uint8_t* Wpacked, con
     // The array keeps the previous call's contents.  Clear what must start
     // at zero -- the 256-byte header with the error word, and the tile
     // counters after the partial-sum slots -- with cudaMemsetAsync (which
-    // allocates nothing); the slots are written before they are read.
-    int sms = 0;
-    if (q4::device_sm_count(&sms) != 0) return Q4_ERR_CUDA;
-    // (A kernel whose workspace is the header alone -- the row-split kernel --
-    // has no counters to clear.)
-    const size_t counters = 256 + (size_t)sms * 2 * q4::kMaxSlotBytes;
+    // allocates nothing); the slots are written before they are read.  A
+    // kernel whose workspace is the header alone (the row-split kernel) only
+    // ever writes the error word, which this entry does not report, so it
+    // gets no memset: each one costs 3-4 us of stream time in a graph.
     cudaStream_t st = (cudaStream_t)stream;
-    if (cudaMemsetAsync(ws, 0, 256, st) != cudaSuccess ||
-        (need > counters && cudaMemsetAsync(static_cast<char*>(ws) + counters, 0, need - counters, st) != cudaSuccess)) {
-        cudaGetLastError();
-        return Q4_ERR_CUDA;
+    if (need > 256) {
+        int sms = 0;
+        if (q4::device_sm_count(&sms) != 0) return Q4_ERR_CUDA;
+        const size_t counters = 256 + (size_t)sms * 2 * q4::kMaxSlotBytes;
+        if (cudaMemsetAsync(ws, 0, 256, st) != cudaSuccess ||
+            (need > counters &&
+             cudaMemsetAsync(static_cast<char*>(ws) + counters, 0, need - counters, st) != cudaSuccess)) {
+            cudaGetLastError();
+            return Q4_ERR_CUDA;
+        }
     }
     return q4_gemm_skinny(A, Wpacked, absmax, code, M, N, K, blocksize, act_dtype, out, ws, need, stream);
 }

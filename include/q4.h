@@ -184,7 +184,8 @@ int q4_gemm_skinny(const void* A, const uint8_t* Wpacked, const float* absmax, c
  *     with that device current (cudaGetSymbolAddress); make that first call
  *     before capturing a stream into a CUDA graph.
  *   - Every call shares the one array and clears its error word and tile
- *     counters with cudaMemsetAsync on `stream` before the kernel; calls that
+ *     counters with cudaMemsetAsync on `stream` before the kernel (not when
+ *     the kernel's workspace is the 256-byte header alone); calls that
  *     overlap on the GPU (other streams, other threads) race on it.
  *   - The array's error word (see q4_gemm_skinny) is not reported: a call
  *     whose kernel gave up a bounded wait returns Q4_OK with outputs that

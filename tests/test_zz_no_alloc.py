@@ -54,6 +54,30 @@ def test_noalloc_matches_regular_entry_point_twice(cuda_device, M, N, K):
         assert np.all(np.abs(got - y) <= tol), f"call {call}: outside the oracle tolerance"
 
 
+@pytest.mark.parametrize("M,N,K", [(1, 3000, 4096), (9, 700, 1024)])
+def test_noalloc_fp32_activations_twice(cuda_device, M, N, K):
+    """The CUDA-core kernel (fp32 activations) through the built-in array,
+    whose row-group counters the entry point clears before each call."""
+    bs = 64
+    code = inputs.code_normal_quantile()
+    packed, absmax = oracle.quantize(inputs.weights(N, K, 4343 + N), bs, code)
+    a = inputs.activations_fp32(M, K, 4344)
+    A = torch.from_numpy(a).to(cuda_device)
+    P, Am, C = (torch.from_numpy(x).to(cuda_device) for x in (packed, absmax, code))
+    y, S = oracle.gemm_f32(a, packed, absmax, code, M, N, K, bs)
+    L = q4.lib()
+    stream = ctypes.c_void_p(torch.cuda.current_stream(cuda_device).cuda_stream)
+    for call in range(2):
+        out = torch.full((M, N), float("nan"), dtype=torch.float32, device=cuda_device)
+        rc = L.q4_gemm_skinny_noalloc(_ptr(A), _ptr(P), _ptr(Am), _ptr(C), M, N, K, bs, q4.Q4_FP32, _ptr(out),
+                                      stream)
+        assert rc == q4.Q4_OK, q4.status_string(rc)
+        torch.cuda.synchronize()
+        got = out.cpu().numpy().astype(np.float64)
+        assert np.all(np.abs(got - y) <= 1e-2 * S + np.spacing(np.abs(y).astype(np.float32)).astype(np.float64)), \
+            f"call {call}: outside the oracle tolerance"
+
+
 def test_noalloc_rejects_problems_beyond_its_scratch(cuda_device):
     # the workspace grows with the tile count: find an N whose need exceeds the array
     limit = 2 << 20
