@@ -34,6 +34,14 @@ def test_rows_shapes(cuda_device, M, N, K):
     run_case(Case(M, N, K), seed=11000 + 7 * M + N + K, device=cuda_device, check_quantizer=False, loader=7)
 
 
+@pytest.mark.parametrize("M", [1, 16, 32])
+@pytest.mark.parametrize("N,K", [(1, 256), (3, 512), (7, 768), (5, 256), (9, 256)])
+def test_rows_tiny_layers(cuda_device, M, N, K):
+    """Fewer rows than one 8-row group and fewer k-stages than warps: one CTA,
+    one short tile, most warps idle."""
+    run_case(Case(M, N, K), seed=12400 + 31 * M + N + K, device=cuda_device, check_quantizer=False, loader=7)
+
+
 @pytest.mark.parametrize("ctas", [1, 2, 3, 7, 33, 148])
 @pytest.mark.parametrize("M", [1, 5, 12])
 def test_rows_partitions(cuda_device, ctas, M):
