@@ -316,60 +316,82 @@ def copies_for(weight_bytes: int) -> int:
     return int(max(1, min(need, 64, (6 << 30) // max(1, weight_bytes))))
 
 
-def measure_configs(device, peak: float, stream, reps: int = 3) -> list:
-    """Every case of the five configurations, one at a time: device time per
-    launch of back-to-back fused GEMMs (CUDA graph, dependent launch mode 2)
-    through the C ABI, cycling over distinct weight copies so that the
-    weights come from HBM, not L2 (the copies read more than 3x the L2)."""
+def time_case(c, seed: int, device, stream, reps: int = 3):
+    """Device time per launch of back-to-back fused GEMMs for one case (CUDA
+    graph, dependent launch mode 2) through the C ABI, cycling over distinct
+    weight copies so that the weights come from HBM, not L2 (the copies read
+    more than 3x the L2).  Returns (us, copies, weight bytes)."""
     import ctypes
     P = ctypes.c_void_p
     L = q4.lib()
+    dt = TORCH_ACT[c.act]
+    code = torch.from_numpy(inputs.CODE_TABLES[c.table]()).to(device)
+    W = inputs.weights_device(c.N, c.K, seed, device, c.outliers)
+    packed, absmax = q4.q4_quantize_blockwise(W.reshape(-1), c.blocksize, code)
+    del W
+    wbytes = packed.numel() + 4 * absmax.numel()
+    n = copies_for(wbytes)
+    copies = [(packed, absmax)] + [(packed.clone(), absmax.clone()) for _ in range(n - 1)]
+    A = inputs.activations(c.M, c.K, dt, seed).to(device)
+    out = torch.empty((c.M, c.N), dtype=dt, device=device)
+    ws_bytes = q4.q4_gemm_workspace_size(c.M, c.N, c.K, c.blocksize, dt)
+    ws = torch.zeros(max(ws_bytes, 16), dtype=torch.uint8, device=device)
+    act = {"bf16": q4.Q4_BF16, "fp16": q4.Q4_FP16, "fp32": q4.Q4_FP32}[c.act]
+    ov = q4.overrides(pdl=2)
+    args = [(P(A.data_ptr()), P(pk.data_ptr()), P(am.data_ptr()), P(code.data_ptr()), c.M, c.N, c.K,
+             c.blocksize, act, P(out.data_ptr()), P(ws.data_ptr()), ws.numel()) for pk, am in copies]
+    R = max(20, n)
+
+    def run(s):
+        for r in range(R):
+            rc = L.q4_gemm_skinny_ex(*args[r % n], P(s.cuda_stream), ctypes.byref(ov))
+            if rc != 0:
+                raise q4.Q4Error(rc, "q4_gemm_skinny_ex")
+
+    with torch.cuda.stream(stream):
+        run(stream)
+    stream.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream, capture_error_mode="relaxed"):
+        run(torch.cuda.current_stream())
+    best = float("inf")
+    for _ in range(reps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            g.replay()
+            e1.record(stream)
+        stream.synchronize()
+        best = min(best, e0.elapsed_time(e1) * 1e3 / R)
+    del g, copies, packed, absmax
+    torch.cuda.empty_cache()
+    return best, n, wbytes
+
+
+# The smallest layer the row-split kernel takes (one 8-row group, one
+# 256-k stage): timed like every case, its per-launch time is the fixed cost
+# of one link in a chain of dependent launches, the floor for tiny layers.
+FLOOR_CASE = inputs.Case(1, 8, 256, tag="floor")
+
+
+def measure_latency_floor(device, stream) -> dict:
+    us, _, _ = time_case(FLOOR_CASE, 12345, device, stream)
+    plan = q4.q4_gemm_plan(FLOOR_CASE.M, FLOOR_CASE.N, FLOOR_CASE.K, FLOOR_CASE.blocksize, torch.bfloat16)
+    log(f"latency floor (M1 N8 K256): {us:.2f} us")
+    return {"case": "M1 N8 K256 bs64 bf16", "us": round(us, 3), "kernel": kernel_name(plan),
+            "how": "per-launch time of the smallest layer, timed like per_config: the fixed cost of one "
+                   "dependent launch in a chain"}
+
+
+def measure_configs(device, peak: float, stream, reps: int = 3) -> list:
+    """Every case of the five configurations, one at a time (time_case)."""
     rows = []
     for name in CONFIGS:
         wl = inputs.workloads()[name]
         for i, c in enumerate(wl.cases):
             seed = inputs.seed_for(wl.index, c.M) + i
             dt = TORCH_ACT[c.act]
-            code = torch.from_numpy(inputs.CODE_TABLES[c.table]()).to(device)
-            W = inputs.weights_device(c.N, c.K, seed, device, c.outliers)
-            packed, absmax = q4.q4_quantize_blockwise(W.reshape(-1), c.blocksize, code)
-            del W
-            wbytes = packed.numel() + 4 * absmax.numel()
-            n = copies_for(wbytes)
-            copies = [(packed, absmax)] + [(packed.clone(), absmax.clone()) for _ in range(n - 1)]
-            A = inputs.activations(c.M, c.K, dt, seed).to(device)
-            out = torch.empty((c.M, c.N), dtype=dt, device=device)
-            ws_bytes = q4.q4_gemm_workspace_size(c.M, c.N, c.K, c.blocksize, dt)
-            ws = torch.zeros(max(ws_bytes, 16), dtype=torch.uint8, device=device)
-            act = {"bf16": q4.Q4_BF16, "fp16": q4.Q4_FP16, "fp32": q4.Q4_FP32}[c.act]
-            ov = q4.overrides(pdl=2)
-            args = [(P(A.data_ptr()), P(pk.data_ptr()), P(am.data_ptr()), P(code.data_ptr()), c.M, c.N, c.K,
-                     c.blocksize, act, P(out.data_ptr()), P(ws.data_ptr()), ws.numel()) for pk, am in copies]
-            R = max(20, n)
-
-            def run(s):
-                for r in range(R):
-                    rc = L.q4_gemm_skinny_ex(*args[r % n], P(s.cuda_stream), ctypes.byref(ov))
-                    if rc != 0:
-                        raise q4.Q4Error(rc, "q4_gemm_skinny_ex")
-
-            with torch.cuda.stream(stream):
-                run(stream)
-            stream.synchronize()
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g, stream=stream, capture_error_mode="relaxed"):
-                run(torch.cuda.current_stream())
-            best = float("inf")
-            for _ in range(reps):
-                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                with torch.cuda.stream(stream):
-                    e0.record(stream)
-                    g.replay()
-                    e1.record(stream)
-                stream.synchronize()
-                best = min(best, e0.elapsed_time(e1) * 1e3 / R)
-            del g, copies, packed, absmax
-            torch.cuda.empty_cache()
+            best, n, wbytes = time_case(c, seed, device, stream, reps)
             plan = q4.q4_gemm_plan(c.M, c.N, c.K, c.blocksize, dt)
             b = c.algorithmic_bytes()
             gbs = b / (best * 1e-6) / 1e9
@@ -654,12 +676,13 @@ def run_ours(args, world, rank, local):
     # Every case of the five configurations, each timed from HBM (outside
     # the timed region; single-GPU runs).
     total_weight_bytes = sum(L.packed.numel() + 4 * L.absmax.numel() for L in layers)
-    per_config = None
+    per_config = latency_floor = None
     if not args.no_per_config and world == 1:
         for L in layers:  # hand the step's weights back before the per-case layers are built
             L.packed = L.absmax = None
         torch.cuda.empty_cache()
         per_config = measure_configs(device, peak, stream)
+        latency_floor = measure_latency_floor(device, stream)
 
     if rank != 0:
         return None
@@ -693,6 +716,7 @@ def run_ours(args, world, rank, local):
                                                 r["outliers"]), r["us"]) for r in per_config
                                    if r["config"] == "msweep"], peak) if per_config else []),
         "per_config": per_config,
+        "latency_floor": latency_floor,
         "split_path": split_path if args.split_path else None,
         "e2e": {"value": round(e2e_value, 2) if e2e_value else None, "unit": "GB/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "steps": e2e_steps,
