@@ -55,10 +55,15 @@ def hbm_peak():
 
 
 def gemm_kernel_hash() -> str:
+    """Hash of the GEMM kernels' source with line comments and blank lines
+    removed: a comment edit does not invalidate counters taken on the code."""
     h = hashlib.sha256()
     for f in ("q4_gemm.cu", "q4_rows.cu", "q4_device.cuh", "q4_plan.cuh"):
-        with open(os.path.join(ROOT, "bit_weight_dequant_b200", "csrc", f), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(ROOT, "bit_weight_dequant_b200", "csrc", f), encoding="utf-8") as fh:
+            for line in fh:
+                code = line.split("//", 1)[0].rstrip()
+                if code:
+                    h.update(code.encode() + b"\n")
     return h.hexdigest()[:16]
 
 

@@ -1,4 +1,5 @@
-// q4_rows.cu -- row-split fused dequantize + skinny GEMM for sm_100a, M <= 16.
+// q4_rows.cu -- row-split fused dequantize + skinny GEMM for sm_100a, M <= 16
+// (the launch table's default there), and up to 32 on request.
 //
 //     out[m, n] = sum_k A[m, k] * code[idx(n, k)] * absmax(n, k)
 //
@@ -6,8 +7,9 @@
 // kgemm_4bit_inference_naive ...", "Technical details" and "Fused path
 // support for M > 1"), with the same inner step as the stream-K kernel in
 // q4_gemm.cu (byte-pair table lookups feeding mma.sync m16n8k16 with the
-// matrix roles swapped, fp32 absmax applied once per 64-k block), organised
-// so that a launch carries no cross-CTA work at all:
+// matrix roles swapped, fp32 absmax applied once per 64-k block, or per
+// 32-k half at blocksize 32), organised so that a launch carries no
+// cross-CTA work at all:
 //
 //  * Rows, not units, are split over the CTAs.  CTA c owns a contiguous run
 //    of whole weight rows (8-row groups; the larger shares go to the lowest
@@ -15,30 +17,34 @@
 //    element is finished inside one CTA: no partial sums in global memory,
 //    no counters, no last-arriver fix-up at the end of the launch.  The
 //    shares differ by at most one 8-row group.
-//  * A CTA's rows form tiles of nearly equal height (at most 72 rows; the
-//    larger heights first).  A stage is one tile's rows x 256 k of packed
-//    codes (128-byte swizzle) plus its absmax box: one TMA box per stage,
-//    one tensor map per height.
-//  * The stages stream through ONE shared ring of D mbarrier-guarded slots,
-//    and warp w computes stages w, w + W, w + 2W, ...  A warp first copies
-//    its stage into registers (code fragments and absmax), then refills the
-//    slot with stage i + D itself -- no producer warp, no "slot free"
-//    barriers, and every slot is prefetch depth, not held during compute.
-//    The warps advance in lockstep (no warp can run ahead of the ring)
-//    instead of each draining its own range at its own pace, so they finish
-//    within about one stage of each other.
+//  * A CTA's rows form tiles of nearly equal height (the larger heights
+//    first; at most 72 rows with one MMA column tile, 64 with two or with
+//    contiguous ranges, 56 at blocksize 32, 32 with four column tiles).  A
+//    stage is one tile's rows x 256 k of packed codes (128-byte swizzle)
+//    plus its absmax box: one TMA box each, one tensor-map pair per height.
+//  * The stages stream through one ring of D = 16 mbarrier-guarded slots.
+//    Round robin (the default): warp w computes stages w, w + 8, w + 16, ...
+//    from slots w and w + 8, and after copying a stage into registers (code
+//    fragments and absmax) refills the slot with the stage 16 further on,
+//    which is its own again -- no producer warp, no "slot free" barriers,
+//    every slot is prefetch depth.  Each warp's first two copies are issued
+//    by its own lanes right after they set up its slots' barriers.
 //  * The stages of a tile run in a loop instantiated for the tile's shape
 //    (16-row MMA tiles, half last tile), dispatched once per tile: each
 //    stage is one straight-line block in which the four units' lookup and
 //    MMA chains interleave; rows past a half tile do no lookups.
 //  * Each warp sums its stages of a tile in registers; when it leaves the
-//    tile it parks the partial tile in shared memory, and the last warp to
-//    do so adds the parked partials in stage order (deterministic) and
-//    stores the tile.  Two parking buffers alternate between tiles.
+//    tile it parks the partial tile in shared memory (the lookup table's
+//    free row halves), and the last warp to do so adds the parked partials
+//    in stage order (deterministic) and stores the tile.  An exact count of
+//    reduced tiles guards the reuse of the parking space (two buffers with
+//    contiguous ranges, one with round robin).
 //  * Under programmatic dependent launch (mode 2) the weights are static:
 //    the ring's first fill (and, optionally, an L2 prefetch of the stages
 //    after it) goes out before the dependency wait, and the table is built
 //    meanwhile.  Activations and outputs are touched only after the wait.
+//  * Every wait is bounded; on time-out the kernel sets the workspace error
+//    word, waits (bounded) for the copies it issued and returns.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
