@@ -135,7 +135,9 @@ int q4_gemm_workspace_size(int M, int N, int K, int blocksize, int act_dtype, si
  *   Wpacked  uint8 [N*K/2] (rows of K/2 bytes), 16-byte aligned
  *   absmax   fp32 [N*K/blocksize], 4-byte aligned
  *   code     fp32 [16], 4-byte aligned
- *   M        0 is a no-op.  bf16/fp16: 1..16 on the mma.sync kernels;
+ *   M        0 is a no-op.  bf16/fp16: 1..16 on the mma.sync kernels
+ *            (the row-split kernel by default, the stream-K kernel on
+ *            head-like layers and for M >= 8 on layers of >= 2^26 weights);
  *            17..32 on the mma.sync kernel with 32-row tiles when
  *            blocksize >= 64 and (K / blocksize) % 4 == 0; otherwise (and
  *            for 33..128) on the tcgen05 (tensor-memory) kernel, which
@@ -225,8 +227,9 @@ typedef struct {
                        /* 2 = 4-unit (128-byte) or 3 = 2-unit (64-byte) stages,  */
                        /* units split over CTAs (stream-K); 7 = row-split: 8-row */
                        /* groups of W split over the CTAs, every output finished */
-                       /* inside one CTA (M <= 16; default where it measured     */
-                       /* faster)                                                */
+                       /* inside one CTA (the default at M <= 16 where it        */
+                       /* measured faster; blocksize 32 with K % 256 == 0 too;   */
+                       /* 17 <= M <= 32 on request, blocksize >= 64)             */
     int pdl;           /* programmatic dependent launch: 0 off; 1 on, the kernel  */
                        /* touches global memory only after the preceding grid    */
                        /* completed; 2 on, and code/Wpacked/absmax may be read   */
