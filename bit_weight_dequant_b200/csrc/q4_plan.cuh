@@ -108,7 +108,6 @@ struct RowsParams {
     int l2_ahead;      // stages the producer asks the L2 to fetch beyond the first ring fill
     int skip_stage;    // test hook: this stage index is never loaded (-1: none)
     int contig;        // 1: each warp streams a contiguous range of stages (0: round robin)
-    int n_maps;        // tensor-map pairs the launcher encoded
     uint32_t map_bits; // tensor-map pair of tile height h (8 .. 72 rows): bits 2 (h / 8) .. 2 (h / 8) + 1,
                        // filled by the launcher (a uniform word, not an indexed array)
     uint32_t wait_limit;  // polls before a wait on a stage or a parking buffer gives up

@@ -188,13 +188,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     constexpr int D = G::D, MTM = G::MT_MAX, NB = G::NB;
     extern __shared__ __align__(16) uint8_t smem_rows[];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, tq = lane & 3;
-    // Long-latency first touches go out first: the code table (read by the
-    // table build) and the tensor maps (read by the first copies).
-    const float cv = __ldg(p.code + (lane & 15));
-    if (tid < p.n_maps) {
+    // Long-latency first touches go out first: the tensor maps (read by the
+    // first copies; every slot holds a valid map, so no parameter has to
+    // arrive before the prefetch) and the code table (read by the table
+    // build).
+    if (tid < kRowsMaxMaps) {
         prefetch_tensormap(&maps.w[tid]);
         prefetch_tensormap(&maps.a[tid]);
     }
+    const float cv = __ldg(p.code + (lane & 15));
 
     // Shared-memory layout (from the window base, decided at run time):
     // barriers and small words; ring slots below the 64 KiB-aligned table;
@@ -763,9 +765,12 @@ cudaError_t rows_launch(int act_dtype, int m_pad, const RowsParams& p0, const ui
     const int nh = stage_heights(p, max_rows / 8, heights, &p.map_bits);
     RowsMaps m;
     memset(&m, 0, sizeof(m));
-    p.n_maps = nh;
     cudaError_t e = make_maps(p, Wp, absmax, am_per_row, amk == kAm32 ? 8 : 4, heights, nh, &m);
     if (e != cudaSuccess) return e;
+    for (int v = nh; v < kRowsMaxMaps; ++v) {  // unused slots repeat a valid map (the kernel prefetches all)
+        m.w[v] = m.w[0];
+        m.a[v] = m.a[0];
+    }
     return act_dtype == 0 ? launch_am<__nv_bfloat16>(amk, m_pad, m, p, smem, stream)
                           : launch_am<__half>(amk, m_pad, m, p, smem, stream);
 }
