@@ -110,7 +110,7 @@ static bool data_parallel_pays(int tiles, int sms, int64_t weights) {
 // has no cross-CTA fix-up, which is what dominates small and medium layers
 // (K5120/N5120: 7.3 vs 8.2 us; K10240/N320: 5.9 vs 11.2 us; 4096^2: 6.1 vs
 // 6.5 us; K8192/N10240: 13.5 vs 14.7 us), and a chain of layers runs best on
-// one kernel throughout (the 70B-class decode step: 83.5 us on the row-split
+// one kernel throughout (the 70B-class decode step: 82.6 us on the row-split
 // kernel, 84.8 us on stream-K, 86.7 us mixing them per layer).  The
 // stream-K kernel stays where the row-split kernel's tiles hold few k-stages
 // and every CTA has many of them (K2560/N248320: 67 vs 96 us), and for
