@@ -174,6 +174,27 @@ static int gemm_choose(int M, int N, int K, int blocksize, int act_dtype, int nu
     // 17 <= M <= 32 runs on the mma.sync kernel with 32-row tiles and 2-unit
     // stages when its TMA rules hold (and no override asks for tcgen05).
     const bool want_umma = ov && (ov->math == 3 || ov->loader == 6);
+    // 33 <= M <= 64 under the same rules: row chunks of 32 on the mma.sync
+    // kernels, one launch each (every chunk streams the weights again).
+    // Measured faster than the tcgen05 kernel on every shape of the M sweep
+    // at these M; M > 64 stays on tcgen05.
+    if (M > 32 && M <= 64 && !want_umma && blocksize >= 64 && (K / blocksize) % 4 == 0 &&
+        (int64_t)N * (K / 64) > 1) {
+        GemmChoice first{}, rest{};
+        int t1 = 0, t2 = 0, s1 = 0, s2 = 0;
+        int64_t u1 = 0, u2 = 0;
+        size_t w1 = 0, w2 = 0;
+        int rc = gemm_choose(32, N, K, blocksize, act_dtype, num_sms, ov, &first, &t1, &u1, &w1, &s1);
+        if (rc == Q4_OK) rc = gemm_choose(M - 32, N, K, blocksize, act_dtype, num_sms, ov, &rest, &t2, &u2, &w2, &s2);
+        if (rc != Q4_OK) return rc;
+        first.chunk_rows = 32;
+        *ch = first;
+        *tiles = t1;
+        *units = u1;
+        *ws_bytes = w1 > w2 ? w1 : w2;  // the chunks run one after another on one workspace
+        *sms_out = s1;
+        return Q4_OK;
+    }
     const bool mma32 = M > 16 && M <= 32 && !want_umma && blocksize >= 64 && (K / blocksize) % 4 == 0 &&
                        (int64_t)N * (K / 64) > 1;
     if ((M > 16 && !mma32) || want_umma) {
@@ -419,6 +440,20 @@ static int gemm_entry(const void* A, const uint8_t* Wpacked, const float* absmax
         return Q4_ERR_MISALIGNED;
     if (need > 0 && (!workspace || workspace_bytes < need)) return Q4_ERR_WORKSPACE;
     if (workspace && !aligned(workspace, 16)) return Q4_ERR_MISALIGNED;
+    if (ch.chunk_rows > 0) {
+        // Row chunks: each is a call of its own (its own launch-table entry,
+        // alignment fallback included) on the rows of A and out it covers,
+        // one after another on the caller's stream and workspace.
+        const size_t esize = act_dtype == Q4_FP32 ? 4 : 2;
+        for (int r0 = 0; r0 < M; r0 += ch.chunk_rows) {
+            const int mc = M - r0 < ch.chunk_rows ? M - r0 : ch.chunk_rows;
+            rc = gemm_entry(static_cast<const char*>(A) + (size_t)r0 * K * esize, Wpacked, absmax, code, bias, mc, N,
+                            K, blocksize, act_dtype, static_cast<char*>(out) + (size_t)r0 * N * esize, workspace,
+                            workspace_bytes, stream, overrides);
+            if (rc != Q4_OK) return rc;
+        }
+        return Q4_OK;
+    }
     if (ch.math == 3 && !aligned(absmax, 16)) return Q4_ERR_MISALIGNED;  // tensor-map base
     if (ch.math != 3 && ch.loader >= 2 && !aligned(absmax, 16)) {  // the tensor map needs a 16-byte aligned base
         if (overrides && overrides->loader >= 2) return Q4_ERR_MISALIGNED;
@@ -547,11 +582,12 @@ int q4_gemm_route(int M, int N, int K, int blocksize, int act_dtype, int* route)
         return Q4_OK;
     }
     if (rc != Q4_OK) return rc;
-    if (M <= 16 || ch.math == 1) {  // M <= 16, and 17 <= M <= 32 on the 32-row mma.sync kernel
+    if (M <= 16 || (ch.math == 1 && ch.chunk_rows == 0)) {  // M <= 16, and 17 <= M <= 32 on the 32-row kernel
         *route = Q4_ROUTE_FUSED;
         return Q4_OK;
     }
-    // the tensor-memory kernel
+    // 33 <= M <= 64 (row chunks on the mma.sync kernels) and the tensor-memory
+    // kernel: fused only on layers of 2^26 weights or more
     *route = (M <= 64 && (int64_t)N * K >= ((int64_t)1 << 26)) ? Q4_ROUTE_FUSED : Q4_ROUTE_SPLIT;
     return Q4_OK;
 }

@@ -24,6 +24,8 @@ struct GemmChoice {
     int l2pf;       // L2 fetch-size hint on weight loads: 0 (none), 128, 256 (loader 1)
     int loader;     // 1 = per-lane global loads, 2/3 = TMA stage ring of 4/2-unit stages, 6 = tcgen05 kernel
     int pdl;        // programmatic dependent launch mode (0, 1, 2)
+    int chunk_rows; // > 0: the call runs as ceil(M / chunk_rows) launches of at most chunk_rows
+                    // activation rows each (this entry describes the first)
 };
 
 // Sets cudaFuncAttributeMaxDynamicSharedMemorySize once per (kernel, device).

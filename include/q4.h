@@ -139,8 +139,11 @@ int q4_gemm_workspace_size(int M, int N, int K, int blocksize, int act_dtype, si
  *            (the row-split kernel by default, the stream-K kernel on
  *            head-like layers and for M >= 8 on layers of >= 2^26 weights);
  *            17..32 on the mma.sync kernel with 32-row tiles when
- *            blocksize >= 64 and (K / blocksize) % 4 == 0; otherwise (and
- *            for 33..128) on the tcgen05 (tensor-memory) kernel, which
+ *            blocksize >= 64 and (K / blocksize) % 4 == 0, and 33..64 under
+ *            the same rules as ceil(M / 32) launches of at most 32 rows each
+ *            on the stream (every launch streams the weights again; the
+ *            plan describes the first); otherwise (and for 65..128) on the
+ *            tcgen05 (tensor-memory) kernel, which
  *            needs blocksize >= 64, K % 256 == 0, (K / blocksize) % 4 == 0
  *            (else Q4_ERR_UNSUPPORTED) and a 16-byte aligned absmax (else
  *            Q4_ERR_MISALIGNED).  fp32: 1..16.  Larger M ->
@@ -295,9 +298,9 @@ int q4_gemm_skinny_bias(const void* A, const uint8_t* Wpacked, const float* absm
  *   - 17 <= M <= 32, bf16/fp16, blocksize >= 64 and (K / blocksize) % 4 == 0:
  *     fused, on the mma.sync kernel with 32-row tiles (parity on 15-24 MB
  *     layers, 1.9x faster on a 50 MB one);
- *   - 33 <= M <= 64, bf16/fp16, with at least 2^26 weights (N*K): fused (the
- *     tcgen05 kernel beats the split path there; below it, its fixed
- *     start-up and cross-CTA combine cost more than the split path saves);
+ *   - 33 <= M <= 64, bf16/fp16, with at least 2^26 weights (N*K): fused (row
+ *     chunks of 32 on the mma.sync kernels, or the tcgen05 kernel, beat the
+ *     split path there; below it the split path is faster);
  *   - everything else the fused entry rejects (M > 128, fp32 with M > 16,
  *     the tcgen05 kernel's shape rules) or loses on: split.
  * Argument errors as q4_gemm_skinny (Q4_ERR_INVALID_ARG); route NULL ->

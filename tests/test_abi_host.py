@@ -91,9 +91,9 @@ def test_gemm_validation_before_cuda():
     assert ex(*args, 12, 64, 4096, 64, 0, ALIGNED, None, 0, None, b.overrides(warps=16)) == b.Q4_ERR_UNSUPPORTED
     assert ex(*args, 1, 64, 4096, 64, 0, ALIGNED, None, 0, None, b.overrides(depth=7, loader=2)) == b.Q4_ERR_UNSUPPORTED
     assert ex(*args, 12, 64, 4096, 64, 0, ALIGNED, None, 0, None, b.overrides(loader=8)) == b.Q4_ERR_INVALID_ARG
-    # the row-split kernel (loader 7): M <= 32 (blocksize >= 64 past 16), 64-k units (blocksize 32 only with
+    # the row-split kernel (loader 7): M <= 32 (blocksize >= 64 past 16; 33..64 in row chunks), 64-k units (blocksize 32 only with
     # K % 256 == 0), its own warp count
-    assert ex(*args, 33, 64, 4096, 64, 0, ALIGNED, None, 0, None, b.overrides(loader=7)) == b.Q4_ERR_UNSUPPORTED
+    assert ex(*args, 65, 64, 4096, 64, 0, ALIGNED, None, 0, None, b.overrides(loader=7)) == b.Q4_ERR_UNSUPPORTED
     assert ex(*args, 20, 64, 4096, 32, 0, ALIGNED, None, 0, None, b.overrides(loader=7)) == b.Q4_ERR_UNSUPPORTED
     assert ex(*args, 4, 64, 4160, 32, 0, ALIGNED, None, 0, None, b.overrides(loader=7)) == b.Q4_ERR_UNSUPPORTED
     assert ex(*args, 4, 64, 4096, 32, 0, ALIGNED, None, 0, None, b.overrides(loader=7, depth=3)) == b.Q4_ERR_UNSUPPORTED
@@ -118,7 +118,19 @@ def test_launch_table_m32(M, N, K):
         b.q4_gemm_plan(24, 256, 4096, 32, num_sms=148)
 
 
-@pytest.mark.parametrize("M,N,K", [(33, 4096, 4096), (48, 300, 1024), (64, 28672, 8192), (128, 8192, 28672)])
+@pytest.mark.parametrize("M,N,K", [(33, 4096, 4096), (48, 300, 1024), (64, 28672, 8192)])
+def test_launch_table_row_chunks(M, N, K):
+    """33 <= M <= 64: row chunks of 32 on the mma.sync kernels; the plan is
+    the first chunk's (the 32-row kernel), the workspace the largest chunk's."""
+    p = b.q4_gemm_plan(M, N, K, 64, num_sms=148)
+    p32 = b.q4_gemm_plan(32, N, K, 64, num_sms=148)
+    prest = b.q4_gemm_plan(M - 32, N, K, 64, num_sms=148)
+    assert p["math"] == 1 and p["loader"] == 3 and p["m_pad"] == 32
+    assert {k: p[k] for k in p if k != "workspace_bytes"} == {k: p32[k] for k in p32 if k != "workspace_bytes"}
+    assert p["workspace_bytes"] == max(p32["workspace_bytes"], prest["workspace_bytes"])
+
+
+@pytest.mark.parametrize("M,N,K", [(65, 4096, 4096), (96, 300, 1024), (128, 8192, 28672)])
 def test_launch_table_tcgen05(M, N, K):
     p = b.q4_gemm_plan(M, N, K, 64, num_sms=148)
     assert p["math"] == 3 and p["loader"] == 6 and p["rows_per_tile"] == 128 and p["sub_block"] == 64

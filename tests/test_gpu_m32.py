@@ -77,3 +77,34 @@ def test_m32_deterministic(cuda_device):
     a = q4.q4_gemm_skinny(*args, ctas=37).clone()
     b = q4.q4_gemm_skinny(*args, ctas=37).clone()
     assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+
+
+@pytest.mark.parametrize("M", [33, 40, 48, 49, 63, 64])
+@pytest.mark.parametrize("N,K,act", [(300, 1024, "bf16"), (513, 2048, "fp16"), (1000, 512, "bf16"),
+                                     (65, 4096, "bf16")])
+def test_row_chunks_33_to_64(cuda_device, M, N, K, act):
+    """33 <= M <= 64: row chunks of 32 on the mma.sync kernels (the last
+    chunk of M - 32 rows on its own kernel: the row-split kernel for up to 16
+    rows, the 32-row kernel above), one after another on one workspace."""
+    p = _plan(M, N, K)
+    assert p["math"] == 1 and p["loader"] == 3 and p["m_pad"] == 32
+    run_case(Case(M, N, K, act=act), seed=8600 + M * 3 + N + K, device=cuda_device, check_quantizer=False)
+
+
+def test_row_chunks_bias_and_partitions(cuda_device):
+    import oracle
+    from bit_weight_dequant_b200 import inputs
+    from parity import bits_of, check_gemm
+    M, N, K = 57, 700, 2048
+    code = inputs.code_normal_quantile()
+    packed, absmax = oracle.quantize(inputs.weights(N, K, 8700), 64, code)
+    A = inputs.activations(M, K, torch.bfloat16, 8701)
+    bias = inputs.activations(1, N, torch.bfloat16, 8702).reshape(N)
+    y, S = oracle.gemm(bits_of(A), oracle.BF16, packed, absmax, code, M, N, K, 64, bias_bits=bits_of(bias))
+    dev = cuda_device
+    P, C = torch.from_numpy(packed).to(dev), torch.from_numpy(code).to(dev)
+    Am = torch.from_numpy(absmax).to(dev)
+    for kw in ({}, {"ctas": 5}, {"pdl": 2}):
+        out = q4.q4_gemm_skinny(A.to(dev), P, Am, C, N, K, 64, bias=bias.to(dev), **kw)
+        torch.cuda.synchronize()
+        check_gemm(bits_of(out), y, S, "bf16", f"row chunks M57 {kw}")

@@ -38,7 +38,7 @@ def test_linear_matches_oracle(cuda_device, act, M, N, K, with_bias):
 @pytest.mark.parametrize("M", [32, 64])
 def test_linear_fused_tcgen05_route_sampled(cuda_device, M):
     """A large layer on the fused route (M = 32: the 32-row mma.sync kernel;
-    M = 64: the tcgen05 kernel, >= 2^26 weights), checked on sampled weight
+    M = 64: two row chunks of 32 on it, >= 2^26 weights), checked on sampled weight
     rows against the oracle."""
     dev = cuda_device
     N, K = 5120, 17408

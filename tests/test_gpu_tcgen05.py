@@ -1,6 +1,7 @@
-"""GPU parity of the tensor-memory (tcgen05) kernel that serves 33 <= M <= 128
-(and M <= 32 on request, math=3; the launch table sends 17 <= M <= 32 to the
-mma.sync kernel with 32-row tiles where its TMA rules hold): every output element within
+"""GPU parity of the tensor-memory (tcgen05) kernel that serves 65 <= M <= 128
+(and M <= 64 on request, math=3; the launch table sends 17 <= M <= 64 to the
+mma.sync kernels, in row chunks of 32 above M = 32, where their TMA rules
+hold): every output element within
 1e-2 * sum_k |a w| + ulp(y) of the oracle.  The weights enter the MMA as
 bf16_rn(code * absmax) (fp16 for fp16 activations), i.e. exactly the values
 the standalone dequantizer writes; the fp32 accumulation follows.  The
@@ -23,20 +24,21 @@ pytestmark = pytest.mark.gpu
 @pytest.mark.parametrize("N,K", [(128, 256), (300, 1024), (513, 2048), (1000, 512)])
 def test_tcgen05_bf16(cuda_device, M, N, K):
     run_case(Case(M, N, K), seed=7000 + M * 3 + N + K, device=cuda_device, check_quantizer=False,
-             **({"math": 3} if M <= 32 else {}))
+             **({"math": 3} if M <= 64 else {}))
 
 
 @pytest.mark.parametrize("M", [20, 64, 128])
 @pytest.mark.parametrize("act,table", [("fp16", "normal"), ("bf16", "uniform"), ("bf16", "fp4"), ("fp16", "fp4")])
 def test_tcgen05_dtypes_tables(cuda_device, M, act, table):
     run_case(Case(M, 384, 1536, act=act, table=table), seed=7100 + M, device=cuda_device, check_quantizer=False,
-             **({"math": 3} if M <= 32 else {}))
+             **({"math": 3} if M <= 64 else {}))
 
 
 @pytest.mark.parametrize("M", [40, 128])
 @pytest.mark.parametrize("bs", [128, 256, 1024])
 def test_tcgen05_blocksizes(cuda_device, M, bs):
-    run_case(Case(M, 256, 4096, blocksize=bs), seed=7200 + bs + M, device=cuda_device, check_quantizer=False)
+    run_case(Case(M, 256, 4096, blocksize=bs), seed=7200 + bs + M, device=cuda_device, check_quantizer=False,
+             **({"math": 3} if M <= 64 else {}))
 
 
 @pytest.mark.parametrize("ctas", [1, 2, 3, 7, 33, 148])
@@ -44,7 +46,7 @@ def test_tcgen05_blocksizes(cuda_device, M, bs):
 def test_tcgen05_partitions(cuda_device, ctas, M):
     """Tiles cut between CTAs (workspace fix-up) at every CTA count."""
     run_case(Case(M, 640, 2048), seed=7300 + ctas, device=cuda_device, check_quantizer=False, ctas=ctas,
-             **({"math": 3} if M <= 32 else {}))
+             **({"math": 3} if M <= 64 else {}))
 
 
 @pytest.mark.parametrize("M", [1, 5, 16])
@@ -53,7 +55,7 @@ def test_tcgen05_small_m_on_request(cuda_device, M):
 
 
 def test_tcgen05_outliers(cuda_device):
-    run_case(Case(64, 256, 2048, outliers=True), seed=7500, device=cuda_device, check_quantizer=False)
+    run_case(Case(64, 256, 2048, outliers=True), seed=7500, device=cuda_device, check_quantizer=False, math=3)
 
 
 @pytest.mark.parametrize("ctas", [5, 37])
@@ -65,7 +67,7 @@ def test_tcgen05_deterministic_and_counters_left_zero(cuda_device, ctas):
     A = inputs.activations(M, K, torch.bfloat16, 9).to(cuda_device)
     P, Am, C = (torch.from_numpy(x).to(cuda_device) for x in (packed, absmax, code))
     ws = q4.Workspace(cuda_device)
-    outs = [q4.q4_gemm_skinny(A, P, Am, C, N, K, 64, workspace=ws, ctas=ctas) for _ in range(3)]
+    outs = [q4.q4_gemm_skinny(A, P, Am, C, N, K, 64, workspace=ws, ctas=ctas, math=3) for _ in range(3)]
     torch.cuda.synchronize()
     for o in outs[1:]:
         assert torch.equal(o.view(torch.int16), outs[0].view(torch.int16))
@@ -77,7 +79,7 @@ def test_tcgen05_deterministic_and_counters_left_zero(cuda_device, ctas):
 
 
 @pytest.mark.parametrize("act", ["bf16", "fp16"])
-@pytest.mark.parametrize("launch", [{}, {"ctas": 9}])
+@pytest.mark.parametrize("launch", [{"math": 3}, {"ctas": 9, "math": 3}])
 def test_tcgen05_bias(cuda_device, act, launch):
     M, N, K = 50, 300, 1024
     code = inputs.code_normal_quantile()
@@ -121,7 +123,7 @@ def test_tcgen05_then_small_m_share_a_workspace(cuda_device):
         y, S = oracle.gemm(bits_of(A), oracle.BF16, packed, absmax, code, M, N, K, 64)
         out = q4.q4_gemm_skinny(A.to(cuda_device), torch.from_numpy(packed).to(cuda_device),
                                 torch.from_numpy(absmax).to(cuda_device), torch.from_numpy(code).to(cuda_device),
-                                N, K, 64, workspace=ws, ctas=17)
+                                N, K, 64, workspace=ws, ctas=17, **({"math": 3} if M > 16 else {}))
         check_gemm(bits_of(out.cpu()), y, S, "bf16", f"shared workspace M{M} N{N}")
 
 
@@ -150,6 +152,6 @@ def test_equal_codes_under_one_absmax(cuda_device, M):
     A = torch.ones((M, K), dtype=torch.bfloat16)
     y, S = oracle.gemm(bits_of(A), ORACLE_ACT["bf16"], packed, absmax, code, M, N, K, bs)
     out = q4.q4_gemm_skinny(A.to(dev), torch.from_numpy(packed).to(dev), torch.from_numpy(absmax).to(dev),
-                            torch.from_numpy(code).to(dev), N, K, bs)
+                            torch.from_numpy(code).to(dev), N, K, bs, **({"math": 3} if M > 16 else {}))
     torch.cuda.synchronize(dev)
     check_gemm(bits_of(out), y, S, "bf16", f"equal codes M{M}")
