@@ -162,16 +162,6 @@ __device__ __forceinline__ void ldmatrix_x4(uint32_t addr, uint32_t& d0, uint32_
                  : "r"(addr));
 }
 
-// ldmatrix_x4 done only when `on` (warp-uniform); zeros otherwise.
-__device__ __forceinline__ void ldmatrix_x4_if(uint32_t addr, uint32_t on, uint32_t& d0, uint32_t& d1, uint32_t& d2,
-                                               uint32_t& d3) {
-    asm volatile(
-        "{\n .reg .pred p;\n setp.ne.u32 p, %5, 0;\n mov.b32 %0, 0;\n mov.b32 %1, 0;\n mov.b32 %2, 0;\n"
-        " mov.b32 %3, 0;\n @p ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];\n}\n"
-        : "=r"(d0), "=r"(d1), "=r"(d2), "=r"(d3)
-        : "r"(addr), "r"(on));
-}
-
 // ---------------------------------------------------------------------------
 // mbarrier + TMA (bulk tensor copies, no multicast).
 // ---------------------------------------------------------------------------
@@ -404,18 +394,6 @@ template <int BYTE>
 __device__ __forceinline__ uint32_t lut_pair(uint32_t word, uint32_t lane4) {
     // result bytes: [0] = lane4.b0 (lane*4), [1] = word.b<BYTE>, [2..3] = lane4.b2..b3 (table base >> 16)
     return lds_u32(prmt<0x7604u | (BYTE << 4)>(word, lane4));
-}
-
-// The same lookup, done only when `on` (a warp-uniform flag; 0 otherwise):
-// predicated, so that a block of lookups stays straight-line code.
-template <int BYTE>
-__device__ __forceinline__ uint32_t lut_pair_if(uint32_t word, uint32_t lane4, uint32_t on) {
-    uint32_t v;
-    asm volatile(
-        "{\n .reg .pred p;\n setp.ne.u32 p, %2, 0;\n mov.b32 %0, 0;\n @p ld.shared.b32 %0, [%1];\n}\n"
-        : "=r"(v)
-        : "r"(prmt<0x7604u | (BYTE << 4)>(word, lane4)), "r"(on));
-    return v;
 }
 
 // Builds the table.  `cv` is code[lane & 15] in every lane; the pair is
